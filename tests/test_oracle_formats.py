@@ -1,0 +1,207 @@
+"""Pins of the oracle's number formats and quantizers against hand-worked
+examples, exhaustive code tables, an independent library (torch's
+float8_e4m3fn cast) and the error bounds the formats guarantee."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+
+
+def _group(values, K=128):
+    w = np.zeros((1, K), np.float32)
+    for k, v in values.items():
+        w[0, int(k)] = v
+    return w
+
+
+# ---------------------------------------------------------------- INT4 ----
+
+def test_int4_worked_example(golden):
+    g = golden["int4"]
+    w = _group(g["group_values"])
+    codes, s = O.quantize_int4(w)
+    assert float(s[0, 0]) == g["scale"]["value_num"] * 2.0 ** g["scale"]["value_exp"]
+    u = O.unpack_int4(codes)[0]
+    for k, c in g["codes"].items():
+        assert u[int(k)] == c
+    assert np.all(np.delete(u, [int(k) for k in g["codes"]]) == 8)
+    deq = O.dequantize_int4(codes, s)[0]
+    for k, v in g["dequant"].items():
+        assert deq[int(k)] == v
+
+
+def test_int4_ties_round_half_even(golden):
+    t = golden["int4"]["ties"]
+    w = np.zeros((1, 128), np.float32)
+    w[0, :len(t["w"])] = t["w"]
+    codes, s = O.quantize_int4(w)
+    assert float(s[0, 0]) == t["scale"]
+    q = O.unpack_int4(codes)[0, :len(t["w"])].astype(int) - 8
+    assert list(q) == t["q"]
+
+
+def test_int4_nibble_packing_and_table():
+    # every nibble value in every position parity, decoded as (u - 8) * s
+    u = np.tile(np.arange(16, dtype=np.uint8), 8)[None, :]            # [1,128]
+    codes = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+    assert codes[0, 0] == 0x10 and codes[0, 7] == 0xFE
+    s = np.array([[0.25]], np.float16)
+    deq = O.dequantize_int4(codes, s)[0]
+    assert np.array_equal(deq, (np.arange(128) % 16 - 8) * 0.25)
+
+
+def test_int4_zero_group_and_error_bound():
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    w[3, 128:256] = 0.0
+    codes, s = O.quantize_int4(w)
+    assert s[3, 1] == 0 and np.all(O.unpack_int4(codes)[3, 128:256] == 8)
+    deq = O.dequantize_int4(codes, s)
+    sf = np.repeat(s.astype(np.float64), 128, axis=1)
+    # |w - deq| <= s/2, up to the fp16 rounding of the scale at the clamp
+    assert np.all(np.abs(w - deq) <= sf * 0.5 * (1 + 2.0 ** -8) + 1e-30)
+    q = O.unpack_int4(codes).astype(int) - 8
+    assert q.min() >= -8 and q.max() <= 7
+
+
+# ---------------------------------------------------------------- INT2 ----
+
+def test_int2_worked_example(golden):
+    g = golden["int2"]
+    w = _group(g["group_values"], K=128)
+    w = np.repeat(w, 4, axis=0)                     # N must be a multiple of 4
+    codes, s, zeros = O.quantize_int2(w)
+    assert float(s[0, 0]) == g["scale"]["value_num"] * 2.0 ** g["scale"]["value_exp"]
+    z = O.unpack_int2_zeros(zeros)
+    assert np.all(z[:, 0] == g["zero"])
+    u = O.unpack_int2(codes)[0]
+    for k, c in g["codes"].items():
+        assert u[int(k)] == c
+    assert np.all(u[4:] == 1)                       # zeros quantize to the zero point
+    deq = O.dequantize_int2(codes, s, zeros)[0]
+    for k, v in g["dequant"].items():
+        assert deq[int(k)] == v
+
+
+def test_int2_symmetric_special_case(golden):
+    sc = golden["int2"]["symmetric_case"]
+    w = np.zeros((4, 128), np.float32)
+    w[:, 0], w[:, 1] = sc["min"], sc["max"]
+    codes, s, zeros = O.quantize_int2(w)
+    assert float(s[0, 0]) == sc["scale"]
+    assert np.all(O.unpack_int2_zeros(zeros) == sc["zero"])
+
+
+def test_int2_one_sided_groups():
+    w = np.zeros((4, 256), np.float32)
+    w[:, :128] = np.linspace(0.01, 0.3, 128)        # all positive: min forced to 0
+    w[:, 128:] = -np.linspace(0.01, 0.3, 128)       # all negative: max forced to 0
+    codes, s, zeros = O.quantize_int2(w)
+    z = O.unpack_int2_zeros(zeros)
+    assert np.all(z[:, 0] == 0) and np.all(z[:, 1] == 3)
+
+
+def test_int2_crumb_and_zero_tables():
+    # all 4 codes x all 4 zeros, codes in every position of the byte
+    u = np.tile(np.arange(4, dtype=np.uint8), 32)[None, :].repeat(4, axis=0)   # [4,128]
+    codes = (u[:, 0::4] | (u[:, 1::4] << 2) | (u[:, 2::4] << 4) | (u[:, 3::4] << 6)).astype(np.uint8)
+    assert codes[0, 0] == 0b11100100
+    zrow = np.arange(4, dtype=np.uint8)                                       # row n has zero n
+    zeros = (zrow[0::4] | (zrow[1::4] << 2) | (zrow[2::4] << 4) | (zrow[3::4] << 6)).astype(np.uint8)[:, None]
+    s = np.full((4, 1), 0.5, np.float16)
+    deq = O.dequantize_int2(codes, s, zeros)
+    for n in range(4):
+        assert np.array_equal(deq[n], (np.arange(128) % 4 - n) * 0.5)
+
+
+def test_int2_error_bound():
+    rng = np.random.default_rng(2)
+    w = (rng.standard_normal((64, 384)) * 0.02).astype(np.float32)
+    codes, s, zeros = O.quantize_int2(w)
+    deq = O.dequantize_int2(codes, s, zeros)
+    sf = np.repeat(s.astype(np.float64), 128, axis=1)
+    g = w.reshape(64, 3, 128)
+    lo = np.repeat(np.minimum(g.min(axis=2), 0), 128, axis=1)
+    hi = np.repeat(np.maximum(g.max(axis=2), 0), 128, axis=1)
+    inside = (w >= lo) & (w <= hi)
+    err = np.abs(w - deq)
+    # inside the representable range [(0-z)s, (3-z)s] the error is <= s/2; the
+    # range itself can miss [min,max] by the rounding of z and of the scale
+    zf = np.repeat(O.unpack_int2_zeros(zeros).astype(np.float64), 128, axis=1)
+    rep = (w >= -zf * sf) & (w <= (3 - zf) * sf)
+    assert np.all(err[inside & rep] <= sf[inside & rep] * 0.5 * (1 + 2.0 ** -8))
+    assert np.all(err[inside] <= sf[inside] * 1.0 + 1e-12)
+
+
+# ------------------------------------------------------------ FP8 / FP4 ----
+
+def test_e4m3_decode_matches_torch_all_bytes():
+    b = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = O.e4m3_decode(np.arange(256, dtype=np.uint8))
+    assert np.array_equal(np.isnan(ref), np.isnan(mine))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ref[ok], mine[ok])
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x38] == 1.0
+
+
+def test_e4m3_rounding_matches_torch():
+    rng = np.random.default_rng(3)
+    finite = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))          # 0 .. 448 ascending
+    mids = ((finite[1:] + finite[:-1]) / 2).astype(np.float32)       # exact ties
+    rnd = np.exp2(rng.uniform(-12, 9.5, 20000)).astype(np.float32)
+    v = np.concatenate([finite.astype(np.float32), mids, rnd, np.float32([0.0, 1e-30, 500.0, 1e6])])
+    v = np.concatenate([v, -v])
+    mine = O.e4m3_rne_satfinite(v)
+    clamped = torch.from_numpy(np.clip(v, -448, 448))
+    ref = clamped.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    nz = O.e4m3_decode(ref) != 0                                      # torch may drop -0 sign
+    assert np.array_equal(mine[nz], ref[nz])
+    assert np.all(O.e4m3_decode(mine[~nz]) == 0)
+
+
+def test_e2m1_grid_and_midpoints():
+    vals = O.e2m1_decode(np.arange(16, dtype=np.uint8))
+    assert list(vals[:8]) == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    assert list(vals[8:]) == [-0.0, -0.5, -1, -1.5, -2, -3, -4, -6]
+    mid = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6, 6.0: 7, 7.0: 7, 100.0: 7}
+    for v, c in mid.items():
+        assert O.e2m1_rne_satfinite(np.float32(v)) == c, v
+        assert O.e2m1_rne_satfinite(np.float32(-v)) == c | 8, -v
+    # every grid value round-trips
+    assert np.array_equal(O.e2m1_rne_satfinite(vals.astype(np.float32)), np.arange(16))
+
+
+def test_nvfp4_worked_blocks(golden):
+    g = golden["nvfp4"]
+    w = np.zeros((3, 32), np.float32)
+    w[0, :16] = g["blocks"][0]["values"]
+    w[1, :16] = g["blocks"][1]["values"]
+    w[2, 20] = g["matrix_amax"]
+    gs = O.nvfp4_global_scale(np.abs(w).max())
+    assert gs == np.float32(g["global_scale"])
+    codes, sb = O.quantize_nvfp4(w, gs)
+    q = O.unpack_nvfp4(codes)
+    for r in range(2):
+        blk = g["blocks"][r]
+        assert sb[r, 0] == blk["block_scale_byte"]
+        assert O.e4m3_decode(sb[r, 0]) == blk["block_scale"]
+        assert list(q[r, :16]) == blk["codes"]
+    deq = O.dequantize_nvfp4(codes, sb, gs)
+    assert deq[2, 20] == 2688.0
+
+
+def test_nvfp4_error_bound_random():
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((32, 256)) * 0.02).astype(np.float32)
+    gs = O.nvfp4_global_scale(np.abs(w).max())
+    codes, sb = O.quantize_nvfp4(w, gs)
+    deq = O.dequantize_nvfp4(codes, sb, gs)
+    unit = np.repeat(O.e4m3_decode(sb) * float(gs), 16, axis=1)
+    # worst grid spacing is 2 (in [4, 6]) -> error <= 1 unit, plus scale rounding
+    assert np.all(np.abs(w - deq) <= unit * 1.0 + 1e-12)
+    amax_b = np.abs(w.reshape(32, 16, 16)).max(axis=2)
+    # the block scale maps the block amax near the top of the E2M1 range
+    ratio = amax_b / (O.e4m3_decode(sb) * float(gs))
+    assert np.all((ratio > 6 / 1.07) & (ratio < 6 * 1.07))
