@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Throughput of the routed-expert MoE layer on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle arm
+
+A step is one pass of the whole layer (router, top-k, expert GEMVs/GEMMs,
+combine) over one batch of seeded synthetic tokens of the workload.  Default
+workload: decode batch 1, W4A16 INT4 experts (T=1, H=2048, I=512, E=512,
+top-10 plus one bf16 shared expert), 100 seeded tokens cycled over the steps.
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent
+replica on its own tokens (the layer is per-token, so there is no exchange),
+and the slowest rank's device time defines the whole-job throughput.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "decode-b1-int4"
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 roofline"
+UNIT = "tokens/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded oracle sample length")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-mb", type=int, default=512)
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------- clock sampling
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv", dir=out_dir)
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.25)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9 or parts[0] != str(self.idx):
+                        continue
+                    try:
+                        sm.append(float(parts[1]))
+                        smax.append(float(parts[2]))
+                    except ValueError:
+                        continue
+                    for n, v in zip(names, parts[5:9]):
+                        if v.lower() == "active":
+                            reasons.add(n)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- oracle arm
+def oracle_tokens_per_s(wl, seconds, rank_offset=0):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload:
+    whole decode steps (router, top-k, expert SwiGLU from the packed weights,
+    combine) until `seconds` of work are done.  Quantization of the weights
+    is set-up, as on the GPU, and is not timed."""
+    from threadpoolctl import threadpool_info
+
+    from bit_quantized_mixture_b200 import synth
+    from oracle import moe_oracle as O
+
+    xs = synth.activations_bf16(wl)
+    wr = synth.router_bf16(wl)
+    shared = tuple(O.bf16_bits_to_f64(m) for m in synth.shared_bf16(wl)) if wl.shared else None
+    q = {}
+
+    def quantized(e):
+        if e not in q:
+            mats = synth.expert_fp32(wl, e)
+            ew = {}
+            for name, m in zip(("gate", "up", "down"), mats):
+                if wl.quant == "int4":
+                    c, s = O.quantize_int4(m)
+                    ew[name] = {"codes": c, "scales": s}
+                elif wl.quant == "int2":
+                    c, s, z = O.quantize_int2(m)
+                    ew[name] = {"codes": c, "scales": s, "zeros": z}
+                else:
+                    raise ValueError("oracle timing covers the W4A16/W2A16 decode workloads")
+            q[e] = ew
+        return q[e]
+
+    # prepare (untimed) the experts of the first steps, then time whole steps
+    n_steps = wl.steps
+    spent, tokens, steps_done = 0.0, 0, 0
+    while spent < seconds and steps_done < n_steps:
+        i = (rank_offset + steps_done) % n_steps
+        x = xs[i * wl.T:(i + 1) * wl.T]
+        ids_probe, _ = O.route_topk(O.router_logits(x, wr), wl.k)
+        for e in np.unique(ids_probe):
+            quantized(int(e))
+        t0 = time.perf_counter()
+        ids, w = O.route_topk(O.router_logits(x, wr), wl.k)
+        O.moe_forward(x, ids, w, wl.quant, lambda e: O.dequantize_expert(wl.quant, quantized(e)), shared=shared)
+        spent += time.perf_counter() - t0
+        tokens += wl.T
+        steps_done += 1
+    threads = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+    return tokens / spent, {"cores": int(threads), "sample": f"{steps_done} steps x {wl.T} tokens of {wl.name}",
+                            "seconds": spent}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from bit_quantized_mixture_b200 import synth
+    wl = synth.workload(args.workload)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
+    vals = []
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(wl, per_step / 4)
+    info = None
+    for s in range(args.steps):
+        v, info = oracle_tokens_per_s(wl, per_step, rank_offset=s)
+        vals.append(v)
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.T / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                       "quant": wl.quant, "shared": wl.shared},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                             "sample": info["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def expert_bytes(wl):
+    """Packed bytes of one routed expert's gate+up and down matrices."""
+    H, I = wl.H, wl.I
+    if wl.quant == "int4":
+        gu = 2 * (I * H // 2 + I * (H // 128) * 2)
+        dn = H * I // 2 + H * (I // 128) * 2
+    elif wl.quant == "int2":
+        gu = 2 * (I * H // 4 + I * (H // 128) * 2 + I * (H // 128))
+        dn = H * I // 4 + H * (I // 128) * 2 + H * (I // 128)
+    else:
+        gu = 2 * (I * H // 2 + I * (H // 16))
+        dn = H * I // 2 + H * (I // 16)
+    return gu, dn
+
+
+def run_decode(args, wl, dev, rank, world):
+    import torch
+
+    from bit_quantized_mixture_b200 import synth
+    from bit_quantized_mixture_b200.layer import build_layer
+
+    layer, _ = build_layer(wl, dev.index, max_tokens=wl.T)
+    xs_host = synth.activations_bf16(wl)
+    xs = torch.from_numpy(xs_host.view(np.int16)).to(dev).view(torch.bfloat16)
+    T, k = wl.T, wl.k
+    nsteps = wl.steps
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(args.flush_mb * (1 << 20) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    off = rank * 37  # replicas work on different tokens
+
+    # one CUDA graph per seeded token batch: route + forward
+    graphs = []
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(nsteps):       # eager pass first (also a warm-up of every path)
+            xi = xs[i * T:(i + 1) * T]
+            layer.route(xi, ids, w)
+            layer.forward(xi, ids, w, y)
+    stream.synchronize()
+    for i in range(nsteps):
+        g = torch.cuda.CUDAGraph()
+        xi = xs[i * T:(i + 1) * T]
+        with torch.cuda.graph(g, stream=stream):
+            layer.route(xi, ids, w)
+            layer.forward(xi, ids, w, y)
+        graphs.append(g)
+    torch.cuda.synchronize(dev)
+
+    def step_index(s):
+        return (off + s) % nsteps
+
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            flush.zero_()
+            graphs[step_index(s)].replay()
+    stream.synchronize()
+
+    # ---- timed region: device time of K steps, L2 flushed between steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    with clocks:
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                flush.zero_()
+                ev0[s].record(stream)
+                graphs[step_index(s)].replay()
+                ev1[s].record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    total_ms = float(sum(step_ms))
+    total_ms_max = allreduce_max(total_ms, dev, world)
+
+    # ---- per-kernel breakdown (events between the library's kernels)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    uniq_per_step = []
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            i = step_index(s)
+            xi = xs[i * T:(i + 1) * T]
+            flush.zero_()
+            layer.set_profile_events(pev[s])
+            layer.route(xi, ids, w)
+            layer.forward(xi, ids, w, y)
+    layer.set_profile_events(None)
+    stream.synchronize()
+    k_route = [p[0].elapsed_time(p[1]) for p in pev]
+    k_gu = [p[2].elapsed_time(p[3]) for p in pev]
+    k_dn = [p[3].elapsed_time(p[4]) for p in pev]
+    # distinct experts per step (from the seeded routing, recomputed on device)
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            i = step_index(s)
+            layer.route(xs[i * T:(i + 1) * T], ids, w)
+            uniq_per_step.append(torch.unique(ids).numel())
+    stream.synchronize()
+
+    # ---- end to end through the public API with host buffers
+    x_pin = torch.from_numpy(xs_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_stage = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        layer.route(x_stage, ids, w)
+        layer.forward(x_stage, ids, w, y)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            i = step_index(s)
+            flush.zero_()
+            e0[s].record(stream)
+            x_stage.copy_(x_pin[i * T:(i + 1) * T], non_blocking=True)
+            g_e2e.replay()
+            y_pin.copy_(y, non_blocking=True)
+            e1[s].record(stream)
+    stream.synchronize()
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
+    e2e_ms_max = allreduce_max(e2e_ms, dev, world)
+
+    # ---- roofline of the dominant kernel (gate/up GEMV over the experts)
+    gu_b, dn_b = expert_bytes(wl)
+    H, I = wl.H, wl.I
+    sh_gu = 2 * I * H * 2 if wl.shared else 0
+    sh_dn = H * I * 2 if wl.shared else 0
+    kern = {"route": float(np.mean(k_route)), "gateup": float(np.mean(k_gu)), "down": float(np.mean(k_dn))}
+    mean_uniq = float(np.mean(uniq_per_step))
+    bytes_gu = mean_uniq * gu_b + sh_gu + T * H * 2 + (T * k + T) * I * 4
+    bytes_dn = mean_uniq * dn_b + sh_dn + (T * k + T) * I * 4 + T * H * 2 + (T * k + T) * H * 4 * 2
+    bytes_rt = wl.E * H * 2 + T * H * 2 + T * wl.E * 4
+    per_kernel = {"route": bytes_rt, "gateup": bytes_gu, "down": bytes_dn}
+    dom = max(kern, key=kern.get)
+    peaks, peak_kind = measured_peaks()
+    achieved = per_kernel[dom] / (kern[dom] * 1e-3) / 1e9
+    traffic = load_traffic(dom, wl.name)
+    step_bytes = bytes_rt + bytes_gu + bytes_dn
+    layer.close()
+    return {
+        "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
+        "clocks": clocks.summary(), "kernels_ms": kern, "dominant": dom,
+        "roofline": {"bound": "hbm", "kernel": f"k_dec_{dom}", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": per_kernel[dom], "peak_source": peak_kind},
+        "layer_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
+        "launches_per_step": 3, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
+    }
+
+
+def load_traffic(kernel, workload):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary, only if
+    the kernel source has not changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    import hashlib
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{workload}:{kernel}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "bit_quantized_mixture_b200", "csrc", ent["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["sha256"]:
+        return None
+    return ent["dram_bytes_per_launch"]
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(v, dev, world):
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+
+    from bit_quantized_mixture_b200 import synth
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.workload(args.workload)
+    if wl.T > 4:
+        raise SystemExit("this bench times the decode workloads (T <= 4)")
+    r = run_decode(args, wl, dev, rank, world)
+    tokens_all = r["steps_tokens"] * world
+    value = tokens_all / (r["total_ms"] * 1e-3)
+    e2e = tokens_all / (r["e2e_ms"] * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "quant": wl.quant,
+                   "shared": wl.shared, "parallelism": f"replicas x{world}",
+                   "l2": f"flushed ({args.flush_mb} MB write) between timed steps",
+                   "cuda_graph": True},
+        "roofline": r["roofline"],
+        "kernels_ms": r["kernels_ms"],
+        "layer_hbm_gbs": r["layer_gbs"],
+        "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, info = oracle_tokens_per_s(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                                "sample": info["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,94 @@
+// Device helpers shared by the MoE kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MOE_DEV __device__ __forceinline__
+
+namespace moe {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------- reductions
+MOE_DEV float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+MOE_DEV float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+MOE_DEV float warp_min(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// ---------------------------------------------------------------- bf16 bits
+MOE_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+MOE_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+MOE_DEV float bf16_to_f(__nv_bfloat16 h) { return __bfloat162float(h); }
+
+// Two fp32 -> packed bf16x2 (round to nearest even); lo goes to the low half.
+MOE_DEV uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ------------------------------------------------------------- fp8 / fp4 cvt
+// fp32 -> E4M3FN byte, round to nearest even, saturating to +-448.
+MOE_DEV uint32_t f32_to_e4m3(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xffu;
+}
+// E4M3FN byte -> fp32 (exact).
+MOE_DEV float e4m3_to_f32(uint32_t b) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(b & 0xffu);
+    asm("{ .reg .b16 t; mov.b16 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
+}
+// Two fp32 -> two E2M1 nibbles (lo in bits 0-3), RNE, saturating to +-6.
+MOE_DEV uint32_t f32x2_to_e2m1(float lo, float hi) {
+    uint32_t r;
+    asm("{ .reg .b8 b0, b1, b2, b3;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n"
+        "  mov.b32 %0, {b0, b1, b2, b3}; }"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r & 0xffu;
+}
+// E2M1 code (low nibble) -> fp32 value (exact).
+MOE_DEV float e2m1_to_f32(uint32_t c) {
+    // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 scaled by 2 fit in a nibble each
+    const uint32_t twice = 0xC8643210u;   // nibble i = 2 * magnitude(i)
+    float m = 0.5f * (float)((twice >> (4 * (c & 7u))) & 0xfu);
+    return (c & 8u) ? -m : m;
+}
+
+// ------------------------------------------------------------ memory access
+MOE_DEV uint4 ldg_nc_v4(const void* p) {
+    uint4 r;
+    asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+MOE_DEV uint4 ldg_stream_v4(const void* p) {   // read once: do not keep in L1
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+// Programmatic dependent launch: wait for the previous grid's results / let
+// the next grid start its prologue.
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace moe

@@ -1,0 +1,70 @@
+// Host-side launchers of the MoE kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.cuh"
+
+namespace moe {
+
+// quantize.cu
+cudaError_t launch_quantize(int quant, const float* w, int N, int K, float g, void* codes, void* scales,
+                            void* zeros, cudaStream_t st);
+cudaError_t launch_quantize_act_nvfp4(const void* x, int T, int K, float g, void* codes, void* scales,
+                                      cudaStream_t st);
+cudaError_t launch_absmax(const float* x, long long n, float* out, cudaStream_t st);
+cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const uint8_t* src_scales,
+                            const uint8_t* src_zeros, uint8_t* dst_codes, uint8_t* dst_scales,
+                            uint8_t* dst_zeros, cudaStream_t st);
+cudaError_t launch_unpack(const MatGeom& gm, const uint8_t* dev_codes, const uint8_t* dev_scales,
+                          const uint8_t* dev_zeros, uint8_t* codes, uint8_t* scales, uint8_t* zeros,
+                          cudaStream_t st);
+
+// route.cu
+struct RouteArgs {
+    const void* x;          // bf16 [T, H]
+    const void* wr;         // bf16 [E, H]
+    const float* logits_in; // fp32 [T, E] (route from logits) or null
+    float* logits;          // fp32 [T, E] workspace or caller buffer
+    int32_t* ids;           // [T, k]
+    float* w;               // [T, k]
+    unsigned int* counter;  // zero-initialised grid counter (decode router)
+    int T, H, E, k;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+// permute.cu
+cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm, int32_t* inv, int32_t* chunk_scratch, cudaStream_t st);
+size_t permute_scratch_ints(int slots, int E);
+
+// decode.cu (small-T path) and segment path
+struct ExpertArgs {
+    MatView gate, up, down;        // routed experts (device layout)
+    const uint8_t* sh_gate;        // shared expert bf16 device layout, or null
+    const uint8_t* sh_up;
+    const uint8_t* sh_down;
+    const float* g_gate;           // NVFP4 per-expert global scales, [E]
+    const float* g_down;
+    float g_x, g_a;                // NVFP4 activation global scales
+    int quant, H, I, E, k;
+};
+struct DecodeArgs {
+    ExpertArgs ex;
+    const void* x;                 // bf16 [T, H]
+    const int32_t* ids;            // [T, k]
+    const float* w;                // [T, k]
+    void* y;                       // bf16 [T, H]
+    float* a;                      // workspace fp32 [T*k, I]
+    float* a_sh;                   // workspace fp32 [T, I]
+    float* part;                   // workspace fp32 [T*k, H]
+    float* part_sh;                // workspace fp32 [T, H]
+    unsigned int* counters;        // workspace, H/32 zero-initialised counters
+    int T;
+    cudaEvent_t ev_mid;            // optional: recorded between the two kernels
+};
+bool decode_supported(int T, int k);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace moe

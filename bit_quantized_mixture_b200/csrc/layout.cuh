@@ -1,0 +1,74 @@
+// Device layout of the expert weights held in a layer's arena.
+//
+// Every matrix W [N, K] is cut into blocks of 128 rows x 64 columns
+// (nb = N/128 row blocks, kb = K/64 column blocks), stored block after block
+// (row block major).  Inside a block the packed codes of one row occupy
+// 32 bytes (INT4, NVFP4), 16 bytes (INT2) or 128 bytes (bf16):
+//
+//   INT4 / NVFP4 / INT2 : [16-byte chunk c][row r (128)][16 bytes]
+//       so 32 consecutive rows of one chunk are 512 contiguous bytes (one
+//       coalesced warp load).  Inside each 32-bit word the codes of eight
+//       (INT4/NVFP4) or sixteen (INT2) consecutive columns are stored in the
+//       order that lets one shift-and-mask pull out two neighbouring columns
+//       into the two 16-bit halves of a register:
+//         INT4  nibble p of the word holds column 2*(p%4) + p/4
+//         INT2  crumb  p of the word holds column 2*(p%8) + p/8
+//       Chunk c of an INT4/NVFP4 row covers columns [32c, 32c+32); word w of
+//       a chunk covers [8w, 8w+8) (INT4) or [16w, 16w+16) (INT2, one chunk).
+//   bf16 : the 16 KB image of a 128x64 K-major tile in the 128-byte swizzle
+//       the tensor cores read: row r, 16-byte chunk c (columns 8c..8c+7) at
+//       byte (r/8)*1024 + (r%8)*128 + ((c ^ (r%8)) * 16).
+//
+// Scales (INT4/INT2): fp16 [nb][K/128][128 rows]; zeros (INT2): uint8, one
+// zero per byte, [nb][K/128][128]; NVFP4 block scales: E4M3 bytes
+// [nb][kb][128 rows][4] (the four 16-column blocks of the 64-column block).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kBlkN = 128;      // rows per block
+constexpr int kBlkK = 64;       // columns per block
+constexpr int kGroup = 128;     // INT4/INT2 quantization group
+constexpr int kFp4Blk = 16;     // NVFP4 scale block
+
+enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3 };
+
+__host__ __device__ constexpr int row_bytes_per_kblock(int q) {
+    return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : 32);
+}
+
+struct MatGeom {
+    int N = 0, K = 0, quant = 0;
+    __host__ __device__ int nb() const { return N / kBlkN; }
+    __host__ __device__ int kbs() const { return K / kBlkK; }
+    __host__ __device__ int groups() const { return K / kGroup; }
+    __host__ __device__ size_t block_bytes() const { return (size_t)kBlkN * row_bytes_per_kblock(quant); }
+    __host__ __device__ size_t codes_bytes() const { return (size_t)nb() * kbs() * block_bytes(); }
+    __host__ __device__ size_t scales_bytes() const {
+        if (quant == Q_INT4 || quant == Q_INT2) return (size_t)N * groups() * 2;
+        if (quant == Q_NVFP4) return (size_t)N * (K / kFp4Blk);
+        return 0;
+    }
+    __host__ __device__ size_t zeros_bytes() const { return quant == Q_INT2 ? (size_t)N * groups() : 0; }
+};
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// One matrix kind (gate, up or down) of every routed expert.
+struct MatView {
+    const uint8_t* codes;   // expert e at codes + e * stride
+    const uint8_t* scales;  // expert e at scales + e * stride
+    const uint8_t* zeros;   // expert e at zeros + e * stride (INT2)
+    size_t stride;          // bytes between consecutive experts
+    int N, K;
+};
+
+// byte offset of block (rb, kb) inside the codes of one matrix
+__host__ __device__ inline size_t block_offset(const MatGeom& g, int rb, int kb) {
+    return ((size_t)rb * g.kbs() + kb) * g.block_bytes();
+}
+
+}  // namespace moe

@@ -1,0 +1,178 @@
+// Router: logits = x Wr^T (bf16 inputs, fp32 accumulation), softmax and
+// top-k with renormalised weights.
+//
+// Ten of 512 experts are selected per token ("Qwen3.8-Flash-Next on one 24 GB
+// GPU", "What the patch does"); the router stays bf16 because a small logit
+// perturbation changes routing on near-ties ("Qwen3.8-Flash-Next-FP6-INT8",
+// "Precision map").  Order: logit descending, expert index ascending on
+// equal logits.  Weights: w_j = exp(l_j - l_max) / sum_selected exp(l - l_max),
+// which equals the full softmax renormalised over the selected experts.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kRouteMaxTSmall = 16;   // decode router: tokens staged in smem
+constexpr size_t kRouteMaxSmem = 160 * 1024;
+constexpr int kMaxK = 32;
+
+// One warp selects the top-k of one token's logits (row of E <= 1024 values,
+// read through L2).  Writes ids/w for that token.
+MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                       float* __restrict__ wout) {
+    const int lane = threadIdx.x & 31;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? __ldcg(row + e) : -FLT_MAX;
+    }
+    uint32_t removed = 0;
+    float my_val = 0.0f;
+    int my_idx = 0;
+    float lmax = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        float best = -INFINITY;
+        int bidx = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = lane + 32 * i;
+            const bool live = (e < E) && !((removed >> i) & 1u);
+            if (live && (v[i] > best || (v[i] == best && e < bidx))) { best = v[i]; bidx = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+            if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+        }
+        if ((bidx & 31) == lane) removed |= 1u << (bidx >> 5);
+        if (j == 0) lmax = best;
+        if (lane == j) { my_val = best; my_idx = bidx; }
+    }
+    const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
+    const float sum = warp_sum(ex);
+    if (lane < k) {
+        ids[lane] = my_idx;
+        wout[lane] = __fdiv_rn(ex, sum);
+    }
+}
+
+// Decode router (T <= 16): one warp per expert row, a grid-wide ticket lets
+// the last CTA to finish run the top-k of every token (no waiting).
+__global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
+    extern __shared__ float xs[];          // [T][H] fp32
+    __shared__ int s_last;
+    const int H = a.H, T = a.T;
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    for (int i = threadIdx.x; i < T * H; i += blockDim.x) xs[i] = __bfloat162float(x[i]);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 4 + warp;
+    if (e < a.E) {
+        const uint8_t* row = reinterpret_cast<const uint8_t*>(a.wr) + (size_t)e * H * 2;
+        float acc[kRouteMaxTSmall];
+#pragma unroll
+        for (int t = 0; t < kRouteMaxTSmall; ++t) acc[t] = 0.0f;
+        for (int c = lane; c < H / 8; c += 32) {
+            const uint4 q = ldg_stream_v4(row + (size_t)c * 16);
+            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int t = 0; t < kRouteMaxTSmall; ++t) {
+                if (t < T) {
+                    const float* xr = xs + t * H + c * 8;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[t] = fmaf(bf16_lo(wv[i]), xr[2 * i], acc[t]);
+                        acc[t] = fmaf(bf16_hi(wv[i]), xr[2 * i + 1], acc[t]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kRouteMaxTSmall; ++t) {
+            if (t < T) {
+                const float s = warp_sum(acc[t]);
+                if (lane == 0) a.logits[(size_t)t * a.E + e] = s;
+            }
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int t = warp; t < T; t += 4)
+        warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
+    __syncthreads();
+    if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
+}
+
+// Router GEMM for larger T on CUDA cores: 64 tokens x 64 experts per CTA.
+__global__ void __launch_bounds__(256) k_router_gemm(RouteArgs a) {
+    __shared__ float As[32][65];
+    __shared__ float Bs[32][65];
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.wr);
+    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < a.H; k0 += 32) {
+        for (int i = threadIdx.x; i < 64 * 32; i += 256) {
+            const int r = i / 32, c = i % 32;
+            const int t = t0 + r, e = e0 + r;
+            As[c][r] = (t < a.T) ? __bfloat162float(x[(size_t)t * a.H + k0 + c]) : 0.0f;
+            Bs[c][r] = (e < a.E) ? __bfloat162float(wr[(size_t)e * a.H + k0 + c]) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int c = 0; c < 32; ++c) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { av[i] = As[c][ty * 4 + i]; bv[i] = Bs[c][tx * 4 + i]; }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+            if (t < a.T && e < a.E) a.logits[(size_t)t * a.E + e] = acc[i][j];
+        }
+}
+
+__global__ void __launch_bounds__(256) k_topk(RouteArgs a) {
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    const float* row = (a.logits_in ? a.logits_in : a.logits) + (size_t)t * a.E;
+    warp_topk(row, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
+}
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
+    if (a.logits_in == nullptr) {
+        const size_t smem = (size_t)a.T * a.H * sizeof(float);
+        if (a.T <= kRouteMaxTSmall && smem <= kRouteMaxSmem) {
+            cudaError_t e = cudaFuncSetAttribute(k_router_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kRouteMaxSmem);
+            if (e != cudaSuccess) return e;
+            k_router_small<<<(a.E + 3) / 4, 128, smem, st>>>(a);
+            return cudaGetLastError();
+        }
+        dim3 grid((a.E + 63) / 64, (a.T + 63) / 64);
+        k_router_gemm<<<grid, 256, 0, st>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    k_topk<<<(a.T + 7) / 8, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

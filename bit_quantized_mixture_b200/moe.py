@@ -1,0 +1,217 @@
+"""Python binding of libmoe_b200.so (argument marshalling only).
+
+Every name mirrors an entry point of include/moe_b200.h.  Tensors are torch
+CUDA tensors (device memory and streams come from PyTorch); host-side inputs
+of the load calls may also be numpy arrays.  There is no fallback: if the
+library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_STATE, MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(7)
+QUANT = {"int4": 0, "int2": 1, "nvfp4": 2, "bf16": 3}
+SHARED = -1
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"[{status}] {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("hidden", "inter", "num_experts", "top_k", "quant", "has_shared", "max_tokens", "device")]
+
+
+class QMatrix(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("global_scale", ctypes.c_float)]
+
+
+class ExpertWeights(ctypes.Structure):
+    _fields_ = [("gate", QMatrix), ("up", QMatrix), ("down", QMatrix)]
+
+
+_lib = None
+
+
+def lib():
+    """Load the CUDA library once; raise if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m bit_quantized_mixture_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+        sig = {
+            "moe_create": [ctypes.POINTER(Config), ctypes.POINTER(vp)],
+            "moe_destroy": [vp],
+            "moe_load_router": [vp, vp, vp],
+            "moe_load_expert_weights": [vp, i32, ctypes.POINTER(ExpertWeights), vp],
+            "moe_set_act_global_scales": [vp, f32, f32],
+            "moe_route": [vp, vp, i32, vp, vp, vp, vp],
+            "moe_route_from_logits": [vp, vp, i32, vp, vp, vp],
+            "moe_forward": [vp, vp, i32, vp, vp, vp, vp],
+            "moe_quantize": [i32, vp, i32, i32, f32, vp, vp, vp, vp],
+            "moe_absmax": [vp, i64, vp, vp],
+            "moe_quantize_act_nvfp4": [vp, i32, i32, f32, vp, vp, vp],
+            "moe_permute": [vp, i32, i32, i32, vp, vp, vp, vp, vp],
+            "moe_debug_unpack_matrix": [vp, i32, i32, vp, vp, vp, vp, vp],
+            "moe_set_profile_events": [vp, ctypes.POINTER(vp), i32],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.moe_status_str.argtypes = [ctypes.c_int]
+        L.moe_status_str.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = [vp]
+        L.moe_last_error.restype = ctypes.c_char_p
+        L.moe_nvfp4_global_scale.argtypes = [f32]
+        L.moe_nvfp4_global_scale.restype = f32
+        _lib = L
+    return _lib
+
+
+def _check(status, handle=None):
+    if status != MOE_OK:
+        raise MoeError(status, lib().moe_last_error(handle).decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    if isinstance(t, np.ndarray):
+        assert t.flags["C_CONTIGUOUS"]
+        return t.ctypes.data
+    raise TypeError(type(t))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def nvfp4_global_scale(amax: float) -> float:
+    return float(lib().moe_nvfp4_global_scale(float(amax)))
+
+
+class MoeLayer:
+    """One MoE layer: owns the weight arena and workspace on one device."""
+
+    def __init__(self, hidden, inter, num_experts, top_k, quant, has_shared, max_tokens, device=0):
+        self.cfg = Config(hidden, inter, num_experts, top_k, QUANT[quant], int(bool(has_shared)), max_tokens, device)
+        self.quant = quant
+        h = ctypes.c_void_p()
+        _check(lib().moe_create(ctypes.byref(self.cfg), ctypes.byref(h)))
+        self.h = h
+        self._keep = []            # host arrays that must outlive asynchronous copies
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def load_router(self, w_bf16, stream=None):
+        _check(lib().moe_load_router(self.h, _ptr(w_bf16), _stream(stream)), self.h)
+
+    def load_expert(self, expert, mats, stream=None):
+        """mats: {'gate'|'up'|'down': {'codes', 'scales', 'zeros', 'g'}} arrays in
+        interchange layout (torch tensors or numpy arrays)."""
+        ew = ExpertWeights()
+        for name in ("gate", "up", "down"):
+            m = mats[name]
+            q = getattr(ew, name)
+            q.codes = _ptr(m["codes"])
+            q.scales = _ptr(m.get("scales"))
+            q.zeros = _ptr(m.get("zeros"))
+            q.global_scale = float(m.get("g", 0.0))
+        _check(lib().moe_load_expert_weights(self.h, int(expert), ctypes.byref(ew), _stream(stream)), self.h)
+
+    def set_act_global_scales(self, g_x, g_a):
+        _check(lib().moe_set_act_global_scales(self.h, float(g_x), float(g_a)), self.h)
+
+    def route(self, x, ids, w, logits=None, stream=None):
+        _check(lib().moe_route(self.h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(logits), _stream(stream)), self.h)
+
+    def route_from_logits(self, logits, ids, w, stream=None):
+        _check(lib().moe_route_from_logits(self.h, _ptr(logits), logits.shape[0], _ptr(ids), _ptr(w),
+                                           _stream(stream)), self.h)
+
+    def forward(self, x, ids, w, y, stream=None):
+        _check(lib().moe_forward(self.h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(y), _stream(stream)), self.h)
+
+    def set_profile_events(self, events):
+        """events: 5 torch.cuda.Event(enable_timing=True) or None."""
+        if events is None:
+            _check(lib().moe_set_profile_events(self.h, None, 0), self.h)
+            return
+        arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+        _check(lib().moe_set_profile_events(self.h, arr, len(events)), self.h)
+
+    def debug_unpack(self, expert, which, codes, scales=None, zeros=None, global_scale=None, stream=None):
+        _check(lib().moe_debug_unpack_matrix(self.h, int(expert), int(which), _ptr(codes), _ptr(scales),
+                                             _ptr(zeros), _ptr(global_scale), _stream(stream)), self.h)
+
+
+def quantize(quant, w, global_scale=0.0, stream=None):
+    """w: CUDA fp32 [N, K] -> (codes, scales, zeros) CUDA uint8/fp16 tensors."""
+    N, K = w.shape
+    dev = w.device
+    q = QUANT[quant]
+    zeros = None
+    if quant == "int4":
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 128), dtype=torch.float16, device=dev)
+    elif quant == "int2":
+        codes = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 128), dtype=torch.float16, device=dev)
+        zeros = torch.empty((N // 4, K // 128), dtype=torch.uint8, device=dev)
+    else:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_quantize(q, _ptr(w), N, K, float(global_scale), _ptr(codes), _ptr(scales), _ptr(zeros),
+                              _stream(stream)))
+    return codes, scales, zeros
+
+
+def absmax(x, out, stream=None):
+    _check(lib().moe_absmax(_ptr(x), x.numel(), _ptr(out), _stream(stream)))
+
+
+def quantize_act_nvfp4(x, g, stream=None):
+    T, K = x.shape
+    codes = torch.empty((T, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((T, K // 16), dtype=torch.uint8, device=x.device)
+    _check(lib().moe_quantize_act_nvfp4(_ptr(x), T, K, float(g), _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def permute(ids, num_experts, stream=None):
+    T, k = ids.shape
+    dev = ids.device
+    counts = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _check(lib().moe_permute(_ptr(ids), T, k, num_experts, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                             _stream(stream)))
+    return counts, offsets, perm, inv

@@ -1,0 +1,220 @@
+/*
+ * moe_b200.h - C ABI of the B200 (sm_100a) routed-expert MoE layer.
+ *
+ * The layer is the mixture-of-experts block of a sparse MoE LLM whose routed
+ * experts are stored with low-bit group quantization:
+ *   1. router logits x Wr^T (bf16 router, fp32 logits), softmax and top-k
+ *      with the k weights renormalised to sum to one
+ *      ("Qwen3.8-Flash-Next on one 24 GB GPU", "What the patch does": ten of
+ *      512 experts per token; "Qwen3.8-Flash-Next-FP6-INT8", "Precision map":
+ *      routers stay bf16);
+ *   2. token-to-expert permutation;
+ *   3. each selected expert's SwiGLU MLP a = silu(x Wg^T) * (x Wu^T),
+ *      o = a Wd^T, with dequantization fused into the products, in three
+ *      weight formats: INT4 symmetric group-128 W4A16
+ *      ("albucino/Qwen3.8-Flash-Next-W4A16-FP8PLE", "Composition"), INT2
+ *      group-128 with fp16 scale and 2-bit zero ("Qwen3.8-Flash-Next on one
+ *      24 GB GPU", "Hardware and software requirements"), and NVFP4 W4A4
+ *      E2M1 with one E4M3 scale per 16 elements
+ *      ("meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", "Format");
+ *   4. y_t = sum_j w_tj o_tj + shared(x_t), the bf16 shared expert added
+ *      with weight one (same NVFP4 card, "Format": shared experts stay BF16).
+ *
+ * Conventions for every entry point
+ *   - Pointers named *_dev are device pointers of the handle's device.
+ *     Pointers named *_any may be host or device memory (copied with
+ *     cudaMemcpyDefault).  All other data pointers are device pointers.
+ *   - All calls are asynchronous on the given stream unless stated.
+ *     Argument and state errors are detected on the host before any work is
+ *     enqueued and return without side effects.  A failed launch returns
+ *     MOE_ERR_CUDA; moe_last_error() gives the text.
+ *   - A handle is not reentrant: calls on one handle must not overlap in
+ *     host threads.  Device work of one handle must not overlap in time
+ *     (the handle owns one workspace), i.e. use one stream per handle or
+ *     order the streams.
+ *   - bf16 tensors are row-major, 16-byte aligned, with rows of H (or I)
+ *     contiguous elements.
+ *
+ * Interchange formats (the layout the load and quantize calls exchange).
+ * A matrix W is [N, K] (output rows, input columns); groups run along K.
+ *   INT4  codes  uint8 [N, K/2]; element k = 2j in the low nibble of byte j;
+ *                stored code u = q + 8 with q = clamp(rne(w/s), -8, 7)
+ *         scales fp16  [N, K/128]; s = fp16(amax/7)
+ *   INT2  codes  uint8 [N, K/4]; element k = 4j + i at bits 2i..2i+1;
+ *                u = clamp(rne(w/s) + z, 0, 3)
+ *         scales fp16  [N, K/128]; s = fp16((max - min)/3), min <= 0 <= max
+ *         zeros  uint8 [N/4, K/128]; zero of row n at bits 2(n%4) of byte
+ *                (n/4, group); z = clamp(rne(-min/s), 0, 3)
+ *   NVFP4 codes  uint8 [N, K/2]; low nibble = even k; E2M1 sign-magnitude
+ *         scales uint8 [N, K/16]; E4M3FN block scale per 16 elements
+ *         global fp32 g per matrix (gate and up share one); w ~ e2m1 * s * g
+ *   BF16  codes  bf16 [N, K] (shared expert only)
+ * Every rounding is round-half-to-even; every code decision is taken in IEEE
+ * fp32.  The library re-lays loaded weights into its own tiled device layout;
+ * moe_debug_unpack_matrix() returns them in the interchange layout.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or index */
+    MOE_ERR_UNSUPPORTED = 2,   /* shape or format this build does not handle */
+    MOE_ERR_STATE = 3,         /* e.g. forward before the weights are loaded */
+    MOE_ERR_OOM = 4,           /* device allocation failed in moe_create     */
+    MOE_ERR_CUDA = 5,          /* a CUDA call or launch failed               */
+    MOE_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up         */
+} moe_status;
+
+typedef enum {
+    MOE_Q_INT4 = 0,            /* INT4 symmetric, group 128, fp16 scales (W4A16) */
+    MOE_Q_INT2 = 1,            /* INT2 asymmetric, group 128, fp16 scale + 2-bit zero (W2A16) */
+    MOE_Q_NVFP4 = 2,           /* E2M1 + E4M3 per-16 scale + fp32 global (W4A4) */
+    MOE_Q_BF16 = 3             /* unquantized bf16 (shared expert) */
+} moe_quant;
+
+#define MOE_SHARED_EXPERT (-1)
+
+typedef struct {
+    int32_t hidden;        /* H: multiple of 128 */
+    int32_t inter;         /* I: multiple of 128 */
+    int32_t num_experts;   /* E: 1 .. 1024 */
+    int32_t top_k;         /* k: 1 .. min(E, 32) */
+    int32_t quant;         /* moe_quant of the routed experts (not BF16) */
+    int32_t has_shared;    /* 1: one always-on bf16 shared expert of width I */
+    int32_t max_tokens;    /* largest T any call will pass; sizes the workspace */
+    int32_t device;        /* CUDA device ordinal */
+} moe_config;
+
+typedef struct moe_layer* moe_handle;
+
+/* One quantized matrix in interchange layout (see above). */
+typedef struct {
+    const void* codes;     /* required */
+    const void* scales;    /* INT4/INT2: fp16; NVFP4: E4M3 bytes; BF16: NULL */
+    const void* zeros;     /* INT2 only, else NULL */
+    float global_scale;    /* NVFP4 only */
+} moe_qmatrix;
+
+typedef struct {
+    moe_qmatrix gate;      /* [I, H] */
+    moe_qmatrix up;        /* [I, H] */
+    moe_qmatrix down;      /* [H, I] */
+} moe_expert_weights;
+
+/* ------------------------------------------------------------------ setup */
+
+/* Validate cfg, allocate the weight arena and the workspace for max_tokens on
+ * cfg->device.  On success *out owns all device memory until moe_destroy.
+ * Errors: INVALID_ARG (bad cfg/null), UNSUPPORTED (shape), OOM, CUDA. */
+moe_status moe_create(const moe_config* cfg, moe_handle* out);
+
+/* Synchronize the handle's device, free everything; NULL is a no-op. */
+moe_status moe_destroy(moe_handle h);
+
+/* Copy the bf16 router matrix Wr [E, H] (host or device) into the arena. */
+moe_status moe_load_router(moe_handle h, const void* w_router_any, moe_stream_t stream);
+
+/* Copy one expert's three matrices (host or device, interchange layout) into
+ * the arena, re-laid for the kernels.  expert in [0, E) takes the routed
+ * format of the handle; MOE_SHARED_EXPERT takes BF16 codes.  The caller may
+ * free its arrays once the stream has passed this call.  Errors:
+ * INVALID_ARG (index, null codes/scales/zeros for the format). */
+moe_status moe_load_expert_weights(moe_handle h, int32_t expert,
+                                   const moe_expert_weights* w, moe_stream_t stream);
+
+/* NVFP4 (W4A4) only: the static per-layer fp32 global scales of the input
+ * activations (g_x) and of the SwiGLU intermediate (g_a), each amax/(6*448)
+ * of a calibration pass. */
+moe_status moe_set_act_global_scales(moe_handle h, float g_x, float g_a);
+
+/* ---------------------------------------------------------------- hot path */
+
+/* Router: logits = x Wr^T (fp32), then per token the k largest logits in
+ * order (logit descending, expert index ascending on ties) and weights
+ * w_j = exp(l_j - l_max) / sum_selected exp(l - l_max).
+ *   x          bf16 [T, H]           topk_ids int32 [T, k]
+ *   topk_w     fp32 [T, k]           logits_out fp32 [T, E] or NULL
+ * 1 <= T <= max_tokens.  Errors: INVALID_ARG, STATE (router not loaded). */
+moe_status moe_route(moe_handle h, const void* x, int32_t T, int32_t* topk_ids,
+                     float* topk_w, float* logits_out, moe_stream_t stream);
+
+/* The softmax/top-k half of moe_route on caller-supplied fp32 logits [T, E]. */
+moe_status moe_route_from_logits(moe_handle h, const float* logits, int32_t T,
+                                 int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* Expert computation and combine:
+ *   y_t = sum_{j<k} topk_w[t,j] * Expert_{topk_ids[t,j]}(x_t) + Shared(x_t)
+ * x bf16 [T, H] in, y bf16 [T, H] out (single rounding of the fp32 sum).
+ * Every id must lie in [0, E); ids of one token should be distinct.
+ * Errors: INVALID_ARG, STATE (experts/shared/scales not loaded). */
+moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* topk_ids,
+                       const float* topk_w, void* y, moe_stream_t stream);
+
+/* ------------------------------------------------- format kernels (no handle) */
+
+/* Quantize W fp32 [N, K] (device) into interchange layout (device outputs).
+ * quant INT4/INT2/NVFP4; global_scale is used for NVFP4 only.
+ * INT4/INT2 need K % 128 == 0 (INT2 also N % 4 == 0); NVFP4 K % 16 == 0. */
+moe_status moe_quantize(int32_t quant, const float* w, int32_t N, int32_t K, float global_scale,
+                        void* codes, void* scales, void* zeros, moe_stream_t stream);
+
+/* *amax_inout_dev = max(*amax_inout_dev, max_i |x_i|) over n fp32 values. */
+moe_status moe_absmax(const float* x, int64_t n, float* amax_inout_dev, moe_stream_t stream);
+
+/* NVFP4 global scale of a tensor with the given amax: amax / (6 * 448) in
+ * fp32 (host function, no device work). */
+float moe_nvfp4_global_scale(float amax);
+
+/* NVFP4 activation quantization of bf16 rows x [T, K] with global scale g:
+ * codes uint8 [T, K/2], scales uint8 [T, K/16] (interchange layout). */
+moe_status moe_quantize_act_nvfp4(const void* x, int32_t T, int32_t K, float g,
+                                  void* codes, void* scales, moe_stream_t stream);
+
+/* Token permutation of the flat slots s = t*k + j into expert-major order,
+ * stable in s: counts int32 [E], offsets int32 [E+1], perm int32 [T*k]
+ * (slot at each permuted position), inv int32 [T*k] (position of each slot).
+ * ids must lie in [0, E).  Uses no handle; deterministic. */
+moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       moe_stream_t stream);
+
+/* ---------------------------------------------------------------- debug */
+
+/* Write loaded matrix `which` (0 gate, 1 up, 2 down) of `expert` back in
+ * interchange layout into device buffers sized as above (NVFP4: the global
+ * scale is written to *global_scale_out when non-NULL). */
+moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
+                                   void* codes, void* scales, void* zeros,
+                                   float* global_scale_out, moe_stream_t stream);
+
+/* Profiling aid: when events != NULL, every later moe_route records
+ * events[0] before and events[1] after its kernels, and every later
+ * moe_forward records events[2] before the expert kernels, events[3] between
+ * the gate/up and the down kernel (decode path) and events[4] after the last
+ * kernel, all on the call's stream.  events are cudaEvent_t handles created
+ * by the caller (n >= 5); NULL turns recording off.  Recording an event
+ * between two kernels removes their launch overlap, so time the layer itself
+ * with recording off. */
+moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n);
+
+/* Static text of a status code. */
+const char* moe_status_str(moe_status s);
+
+/* Text of the last error on this handle (or of the last handle-free call
+ * made by this host thread when h is NULL). */
+const char* moe_last_error(moe_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */
