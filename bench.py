@@ -281,6 +281,11 @@ def run_decode(args, wl, dev, rank, world):
 
     # ---- per-kernel breakdown (events between the library's kernels)
     pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for evs in pev:            # torch creates the CUDA event on first record
+            for ev in evs:
+                ev.record(stream)
+    stream.synchronize()
     uniq_per_step = []
     with torch.cuda.stream(stream):
         for s in range(args.steps):

@@ -34,15 +34,18 @@ bool decode_supported(int T, int k) { return T >= 1 && T <= kDecMaxT && T * k <=
 
 struct Plan {
     int n_unique;
+    int ids[kDecMaxSlots];       // the launch's expert ids (flat slots)
     int first[kDecMaxSlots];     // first slot of each distinct expert
     unsigned char is_first[kDecMaxSlots];
 };
 
 MOE_DEV void build_plan(const int32_t* __restrict__ ids, int n, Plan& p) {
+    for (int s = threadIdx.x; s < n; s += blockDim.x) p.ids[s] = __ldcg(ids + s);
+    __syncthreads();
     for (int s = threadIdx.x; s < n; s += blockDim.x) {
-        const int e = __ldcg(ids + s);
+        const int e = p.ids[s];
         bool f = true;
-        for (int q = 0; q < s && f; ++q) f = (__ldcg(ids + q) != e);
+        for (int q = 0; q < s; ++q) f = f && (p.ids[q] != e);
         p.is_first[s] = f;
     }
     __syncthreads();
@@ -65,11 +68,11 @@ MOE_DEV void build_plan(const int32_t* __restrict__ ids, int n, Plan& p) {
 // With valid input (distinct ids per token) there are at most T <= kDecMaxT;
 // repeated ids within a token are invalid input: the extra slots are dropped
 // so that no buffer is overrun.
-MOE_DEV int item_tokens(const int32_t* __restrict__ ids, int n, int k, int s0, int* tok, int* slot) {
-    const int e0 = __ldcg(ids + s0);
+MOE_DEV int item_tokens(const int* __restrict__ ids, int n, int k, int s0, int* tok, int* slot) {
+    const int e0 = ids[s0];
     int c = 0;
     for (int s = s0; s < n && c < kDecMaxT; ++s) {
-        if (__ldcg(ids + s) == e0) {
+        if (ids[s] == e0) {
             if (threadIdx.x == 0) { tok[c] = s / k; slot[c] = s; }
             ++c;
         }
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
         m = T;
         if (threadIdx.x < T) { tok[threadIdx.x] = threadIdx.x; slot_of[threadIdx.x] = threadIdx.x; }
     } else {
-        m = min(item_tokens(a.ids, n, k, plan.first[u], tok, slot_of), MT);
+        m = min(item_tokens(plan.ids, n, k, plan.first[u], tok, slot_of), MT);
     }
     float* xs = smem;                                // [m][H] fp32
     float* red = smem + MT * H;                      // [8][2][MT][32]
@@ -310,7 +313,7 @@ __global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
         const MatPtr mats[2] = {{ex.sh_gate, nullptr, nullptr}, {ex.sh_up, nullptr, nullptr}};
         warp_rows_dot<Q_BF16, MT, 2>(acc, mats, nb, r, KB, G, warp, kGuThreads / 32, xs, H, m);
     } else {
-        e = __ldcg(a.ids + plan.first[u]);
+        e = plan.ids[plan.first[u]];
         if (e >= 0 && e < ex.E) {        // an id outside [0, E) contributes zero
             const MatPtr mats[2] = {expert_mat(ex.gate, e), expert_mat(ex.up, e)};
             warp_rows_dot<Q, MT, 2>(acc, mats, nb, r, KB, G, warp, kGuThreads / 32, xs, H, m);
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kDnThreads) k_dec_down(DecodeArgs a) {
         m = T;
         if (threadIdx.x < T) { tok[threadIdx.x] = threadIdx.x; slot_of[threadIdx.x] = threadIdx.x; }
     } else {
-        m = min(item_tokens(a.ids, n, k, plan.first[u], tok, slot_of), MT);
+        m = min(item_tokens(plan.ids, n, k, plan.first[u], tok, slot_of), MT);
     }
     float* as = smem;                                // [m][I]
     float* red = smem + MT * I;                      // [4][MT][32]
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(kDnThreads) k_dec_down(DecodeArgs a) {
         const MatPtr mats[1] = {{ex.sh_down, nullptr, nullptr}};
         warp_rows_dot<Q_BF16, MT, 1>(acc, mats, nb, r, KB, G, warp, kDnThreads / 32, as, I, m);
     } else {
-        e = __ldcg(a.ids + plan.first[u]);
+        e = plan.ids[plan.first[u]];
         if (e >= 0 && e < ex.E) {        // an id outside [0, E) contributes zero
             const MatPtr mats[1] = {expert_mat(ex.down, e)};
             warp_rows_dot<Q, MT, 1>(acc, mats, nb, r, KB, G, warp, kDnThreads / 32, as, I, m);
@@ -427,8 +430,12 @@ __global__ void __launch_bounds__(kDnThreads) k_dec_down(DecodeArgs a) {
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.y);
     for (int i = threadIdx.x; i < T * 32; i += blockDim.x) {
         const int t = i / 32, h = hb * 32 + i % 32;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (j < k) ? __ldcg(a.part + (size_t)(t * k + j) * H + h) : 0.0f;
         float s = 0.0f;
-        for (int j = 0; j < k; ++j) s += __ldcg(a.part + (size_t)(t * k + j) * H + h);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s += v[j];          // fixed order j = 0 .. k-1
         if (ex.sh_down) s += __ldcg(a.part_sh + (size_t)t * H + h);
         y[(size_t)t * H + h] = __float2bfloat16_rn(s);
     }

@@ -60,6 +60,85 @@ MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __r
     }
 }
 
+// Top-k of one token by the 4 warps of a CTA: each warp selects the k best
+// of its quarter of the experts, then warp 0 selects the k best of those
+// 4k candidates.  Same order and weights as warp_topk.
+MOE_DEV void cta4_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                       float* __restrict__ wout, float* cand_v, int* cand_i) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = (E + 3) / 4, e0 = warp * q, e1 = min(E, e0 + q);
+    float v[8];
+    int vi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = e0 + lane + 32 * i;
+        vi[i] = e;
+        v[i] = (e < e1) ? __ldcg(row + e) : -INFINITY;
+    }
+    uint32_t removed = 0;
+    for (int j = 0; j < k; ++j) {
+        float best = -INFINITY;
+        int bidx = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool live = (vi[i] < e1) && !((removed >> i) & 1u);
+            if (live && (v[i] > best || (v[i] == best && vi[i] < bidx))) { best = v[i]; bidx = vi[i]; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+            if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+        }
+        if (bidx != 0x7fffffff && ((bidx - e0) & 31) == lane) removed |= 1u << ((bidx - e0) >> 5);
+        if (lane == 0) { cand_v[warp * kMaxK + j] = best; cand_i[warp * kMaxK + j] = bidx; }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // 4k <= 128 candidates, 4 per lane
+        float cv[4];
+        int ci[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = lane + 32 * i, w = c / kMaxK, jj = c % kMaxK;
+            const bool ok = jj < k;
+            cv[i] = ok ? cand_v[w * kMaxK + jj] : -INFINITY;
+            ci[i] = ok ? cand_i[w * kMaxK + jj] : 0x7fffffff;
+        }
+        uint32_t rem = 0;
+        float my_val = 0.0f, lmax = 0.0f;
+        int my_idx = 0;
+        for (int j = 0; j < k; ++j) {
+            float best = -INFINITY;
+            int bidx = 0x7fffffff, bslot = -1;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const bool live = !((rem >> i) & 1u) && ci[i] != 0x7fffffff;
+                if (live && (cv[i] > best || (cv[i] == best && ci[i] < bidx))) { best = cv[i]; bidx = ci[i]; bslot = i; }
+            }
+            int owner = (bslot >= 0) ? lane : 32;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+                const int oo = __shfl_xor_sync(0xffffffffu, owner, o);
+                const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
+                if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; owner = oo; bslot = os; }
+            }
+            if (owner == lane) rem |= 1u << bslot;
+            if (j == 0) lmax = best;
+            if (lane == j) { my_val = best; my_idx = bidx; }
+        }
+        const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
+        const float sum = warp_sum(ex);
+        if (lane < k) {
+            ids[lane] = my_idx;
+            wout[lane] = __fdiv_rn(ex, sum);
+        }
+    }
+    __syncthreads();
+}
+
 // Decode router (T <= 16): one warp per expert row, a grid-wide ticket lets
 // the last CTA to finish run the top-k of every token (no waiting).
 __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
@@ -71,22 +150,34 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 4 + warp;
+    pdl_launch_dependents();                 // let the expert kernel get resident
     if (e < a.E) {
         const uint8_t* row = reinterpret_cast<const uint8_t*>(a.wr) + (size_t)e * H * 2;
         float acc[kRouteMaxTSmall];
 #pragma unroll
         for (int t = 0; t < kRouteMaxTSmall; ++t) acc[t] = 0.0f;
-        for (int c = lane; c < H / 8; c += 32) {
-            const uint4 q = ldg_stream_v4(row + (size_t)c * 16);
-            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+        for (int c0 = 0; c0 < H / 8; c0 += 32 * 8) {
+            uint4 q[8];
 #pragma unroll
-            for (int t = 0; t < kRouteMaxTSmall; ++t) {
-                if (t < T) {
-                    const float* xr = xs + t * H + c * 8;
+            for (int u = 0; u < 8; ++u) {          // 8 loads in flight per lane
+                const int c = c0 + lane + 32 * u;
+                q[u] = (c < H / 8) ? ldg_stream_v4(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        acc[t] = fmaf(bf16_lo(wv[i]), xr[2 * i], acc[t]);
-                        acc[t] = fmaf(bf16_hi(wv[i]), xr[2 * i + 1], acc[t]);
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + lane + 32 * u;
+                if (c < H / 8) {
+                    const uint32_t wv[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+                    for (int t = 0; t < kRouteMaxTSmall; ++t) {
+                        if (t < T) {
+                            const float* xr = xs + t * H + c * 8;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                acc[t] = fmaf(bf16_lo(wv[i]), xr[2 * i], acc[t]);
+                                acc[t] = fmaf(bf16_hi(wv[i]), xr[2 * i + 1], acc[t]);
+                            }
+                        }
                     }
                 }
             }
@@ -105,9 +196,13 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int t = warp; t < T; t += 4)
-        warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
-    __syncthreads();
+    __shared__ float cand_v[4 * kMaxK];
+    __shared__ int cand_i[4 * kMaxK];
+    if (a.E <= 1024) {
+        for (int t = 0; t < T; ++t)
+            cta4_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k,
+                      cand_v, cand_i);
+    }
     if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
 }
 
