@@ -1,6 +1,7 @@
 // Host-side launchers of the MoE kernels (internal to the library).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -66,5 +67,32 @@ struct DecodeArgs {
 };
 bool decode_supported(int T, int k);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+// grouped_gemm.cu (prefill path)
+struct GemmTile {
+    int expert;   // routed expert, or -1 for the shared expert
+    int rb;       // 128-row block of the weight matrix
+    int seg;      // first row of the segment (permuted position, or token for shared)
+    int count;    // tokens in this tile
+};
+struct PrefillArgs {
+    ExpertArgs ex;
+    const void* x;                 // bf16 [T, H]
+    const int32_t* ids;            // [T, k]
+    const float* w;                // [T, k]
+    void* y;                       // bf16 [T, H]
+    int T;
+    int32_t *counts, *offsets, *perm, *inv, *perm_scratch;
+    GemmTile* tiles;
+    int* num_tiles;
+    __nv_bfloat16* xq;             // NVFP4: [T, H] dequantized W4A4 activations
+    __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order
+    __nv_bfloat16* a_sh;           // [T, I] shared-expert intermediate
+    __nv_bfloat16* o;              // [T*k, H] weighted expert outputs by slot
+    __nv_bfloat16* o_sh;           // [T, H] shared-expert output
+    int* err;                      // device error word (bounded waits)
+};
+size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I);
+cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st);
 
 }  // namespace moe

@@ -38,6 +38,12 @@ struct moe_layer {
     unsigned int* dec_counters = nullptr;   // [H/32]
     uint8_t* staging = nullptr;    // interchange copy of one matrix
     size_t staging_bytes = 0;
+    // prefill path
+    int32_t *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr, *perm_scratch = nullptr;
+    GemmTile* tiles = nullptr;
+    int* num_tiles = nullptr;
+    int* dev_err = nullptr;
+    __nv_bfloat16 *xq = nullptr, *a_perm = nullptr, *a_sh = nullptr, *o = nullptr, *o_sh = nullptr;
     // state
     bool router_loaded = false;
     bool shared_loaded = false;
@@ -162,6 +168,20 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 32));
     h->staging_bytes = (size_t)2 * H * I + 65536;
     const size_t o_stage = carve(h->staging_bytes);
+    const size_t Tm = (size_t)c.max_tokens, slots = Tm * k;
+    const size_t o_counts = carve(sizeof(int32_t) * E);
+    const size_t o_offsets = carve(sizeof(int32_t) * (E + 1));
+    const size_t o_perm = carve(sizeof(int32_t) * slots);
+    const size_t o_inv = carve(sizeof(int32_t) * slots);
+    const size_t o_pscr = carve(sizeof(int32_t) * permute_scratch_ints((int)slots, E));
+    const size_t o_tiles = carve(sizeof(GemmTile) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
+    const size_t o_ntiles = carve(sizeof(int));
+    const size_t o_err = carve(sizeof(int));
+    const size_t o_xq = carve(c.quant == MOE_Q_NVFP4 ? Tm * H * 2 : 0);
+    const size_t o_aperm = carve(slots * I * 2);
+    const size_t o_ash16 = carve(c.has_shared ? Tm * I * 2 : 0);
+    const size_t o_o = carve(slots * H * 2);
+    const size_t o_osh = carve(c.has_shared ? Tm * H * 2 : 0);
     h->ws_bytes = w;
     if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -177,6 +197,19 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->dec_part_sh = reinterpret_cast<float*>(h->ws + o_psh);
     h->dec_counters = reinterpret_cast<unsigned int*>(h->ws + o_cnt);
     h->staging = h->ws + o_stage;
+    h->counts = reinterpret_cast<int32_t*>(h->ws + o_counts);
+    h->offsets = reinterpret_cast<int32_t*>(h->ws + o_offsets);
+    h->perm = reinterpret_cast<int32_t*>(h->ws + o_perm);
+    h->inv = reinterpret_cast<int32_t*>(h->ws + o_inv);
+    h->perm_scratch = reinterpret_cast<int32_t*>(h->ws + o_pscr);
+    h->tiles = reinterpret_cast<GemmTile*>(h->ws + o_tiles);
+    h->num_tiles = reinterpret_cast<int*>(h->ws + o_ntiles);
+    h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
+    h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
+    h->a_perm = reinterpret_cast<__nv_bfloat16*>(h->ws + o_aperm);
+    h->a_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_ash16);
+    h->o = reinterpret_cast<__nv_bfloat16*>(h->ws + o_o);
+    h->o_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_osh);
     cudaError_t e1 = cudaMemset(h->ws, 0, h->ws_bytes);
     cudaError_t e2 = cudaMemset(h->arena, 0, h->arena_bytes);
     if (e1 != cudaSuccess || e2 != cudaSuccess) {
@@ -392,6 +425,21 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         return fail(h, MOE_ERR_STATE, "moe_forward: NVFP4 activation global scales not set");
     DeviceGuard dg(c.device);
     cudaStream_t st = (cudaStream_t)stream;
+    if (!decode_supported(T, c.top_k)) {       // more tokens than the GEMV path takes
+        PrefillArgs p{};
+        p.ex = expert_args(h);
+        p.x = x; p.ids = topk_ids; p.w = topk_w; p.y = y; p.T = T;
+        p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
+        p.perm_scratch = h->perm_scratch;
+        p.tiles = h->tiles; p.num_tiles = h->num_tiles;
+        p.xq = h->xq; p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
+        p.err = h->dev_err;
+        if (h->prof[2]) cudaEventRecord(h->prof[2], st);
+        cudaError_t e = launch_prefill(p, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "moe_forward (grouped GEMM path)");
+        if (h->prof[4]) cudaEventRecord(h->prof[4], st);
+        return MOE_OK;
+    }
     DecodeArgs a{};
     a.ex = expert_args(h);
     a.a = h->dec_a;
@@ -414,6 +462,22 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         t0 += tc;
     }
     if (h->prof[4]) cudaEventRecord(h->prof[4], st);
+    return MOE_OK;
+}
+
+moe_status moe_sync_status(moe_handle h, moe_stream_t stream) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_sync_status: null handle");
+    DeviceGuard dg(h->cfg.device);
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_sync_status");
+    int code = 0;
+    e = cudaMemcpy(&code, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_sync_status");
+    if (code) {
+        const int zero = 0;
+        cudaMemcpy(h->dev_err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(h, MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (site %d); outputs are invalid", code);
+    }
     return MOE_OK;
 }
 

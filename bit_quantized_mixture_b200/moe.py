@@ -67,6 +67,7 @@ def lib():
             "moe_permute": [vp, i32, i32, i32, vp, vp, vp, vp, vp],
             "moe_debug_unpack_matrix": [vp, i32, i32, vp, vp, vp, vp, vp],
             "moe_set_profile_events": [vp, ctypes.POINTER(vp), i32],
+            "moe_sync_status": [vp, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -158,6 +159,10 @@ class MoeLayer:
 
     def forward(self, x, ids, w, y, stream=None):
         _check(lib().moe_forward(self.h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(y), _stream(stream)), self.h)
+
+    def sync_status(self, stream=None):
+        """Synchronize the stream; raise on a device-side timeout or CUDA error."""
+        _check(lib().moe_sync_status(self.h, _stream(stream)), self.h)
 
     def set_profile_events(self, events):
         """events: 5 torch.cuda.Event(enable_timing=True) or None."""

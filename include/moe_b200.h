@@ -206,6 +206,12 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
  * with recording off. */
 moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n);
 
+/* Synchronize `stream` and report device-side failures of earlier calls on
+ * this handle: MOE_ERR_TIMEOUT when a kernel gave up a bounded wait (the
+ * kernel stopped and its outputs are invalid; the flag is cleared), or
+ * MOE_ERR_CUDA for an asynchronous CUDA error.  MOE_OK otherwise. */
+moe_status moe_sync_status(moe_handle h, moe_stream_t stream);
+
 /* Static text of a status code. */
 const char* moe_status_str(moe_status s);
 

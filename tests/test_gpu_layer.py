@@ -223,3 +223,82 @@ def test_errors_are_reported_without_device_work():
         layer.set_act_global_scales(1.0, 1.0)        # not an NVFP4 layer
     assert ei.value.status == moe.MOE_ERR_STATE
     layer.close()
+
+
+# ------------------------------------------------ grouped GEMM (prefill) path
+MID = {
+    "int4": synth.custom("tiny-int4", H=512, I=384, E=24, k=6, shared=True),
+    "int2": synth.custom("tiny-int4", quant="int2", H=512, I=384, E=24, k=6, shared=True),
+    "nvfp4": synth.custom("tiny-int4", quant="nvfp4", H=512, I=384, E=24, k=6, shared=True),
+}
+
+
+@pytest.mark.parametrize("quant", ["int4", "int2", "nvfp4"])
+@pytest.mark.parametrize("T", [5, 37, 300])
+def test_prefill_matches_oracle(quant, T):
+    """T > 4 runs the permutation + tcgen05 grouped GEMMs: several 128-row
+    weight blocks, several 64-column K blocks, token tiles with ragged tails
+    and the shared expert's tiles."""
+    y, y_ref, layer, _ = _forward_case(MID[quant], T)
+    layer.sync_status()
+    assert_close_output(y, y_ref)
+
+
+def test_prefill_one_expert_takes_many_tokens():
+    """All tokens on the same experts: segments of several 128-token tiles."""
+    wl = MID["int4"]
+    T = 700
+    ox = OracleExperts(wl)
+    layer = get_layer(wl, T)
+    x = synth.activations_bf16(wl, steps=T // wl.T + 1)[:T]
+    ids = np.tile(np.array([3, 7, 0, 23, 11, 5], np.int32), (T, 1))
+    w = np.tile(np.array([0.3, 0.2, 0.15, 0.15, 0.1, 0.1]), (T, 1))
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+    layer.forward(bf16_tensor(x, DEV), torch.from_numpy(ids).to(DEV), torch.from_numpy(w.astype(np.float32)).to(DEV), y)
+    layer.sync_status()
+    y_ref = O.moe_forward(x, ids, w, "int4", ox, shared=ox.shared())
+    assert_close_output(to_bits(y), y_ref)
+
+
+def test_prefill_is_deterministic():
+    wl = MID["int2"]
+    y1, _, _, _ = _forward_case(wl, 300)
+    y2, _, _, _ = _forward_case(wl, 300)
+    assert np.array_equal(y1, y2)
+
+
+def _full_size_sampled(wl_name, sample):
+    wl = synth.workload(wl_name)
+    layer = get_layer(wl, wl.T)
+    ox = OracleExperts(wl)
+    x = synth.activations_bf16(wl)
+    L = synth.routing_logits(wl)
+    ids_d = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
+    w_d = torch.empty((wl.T, wl.k), dtype=torch.float32, device=DEV)
+    layer.route_from_logits(torch.from_numpy(L).to(DEV), ids_d, w_d)
+    ids, w = ids_d.cpu().numpy(), w_d.cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(wl.T, sample, replace=False))
+    act = None
+    if wl.quant == "nvfp4":
+        xf = O.bf16_bits_to_f32(x)
+        g_x = O.nvfp4_global_scale(np.abs(xf).max())
+        # the intermediate scale is a calibration input of both sides; the
+        # amax of a token sample serves (values above it saturate to 6 * s_b)
+        g_a = O.nvfp4_global_scale(O.intermediate_amax(x[toks], ids[toks], "nvfp4", ox, g_x))
+        act = (g_x, g_a)
+        layer.set_act_global_scales(g_x, g_a)
+    y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=DEV)
+    layer.forward(bf16_tensor(x, DEV), ids_d, w_d, y)
+    layer.sync_status()
+    y_ref = O.moe_forward(x[toks], ids[toks], w[toks], wl.quant, ox, shared=ox.shared(), act_scales=act)
+    assert_close_output(to_bits(y)[toks], y_ref)
+    return layer
+
+
+def test_prefill_zipf_int4_full_size_sampled_tokens():
+    _full_size_sampled("prefill-int4-zipf", 12)
+
+
+def test_prefill_nvfp4_full_size_sampled_tokens():
+    _full_size_sampled("prefill-nvfp4", 8)
