@@ -61,7 +61,7 @@ struct DecodeArgs {
     float* a_sh;                   // workspace fp32 [T, I]
     float* part;                   // workspace fp32 [T*k, H]
     float* part_sh;                // workspace fp32 [T, H]
-    unsigned int* counters;        // workspace, H/32 zero-initialised counters
+    unsigned int* counters;        // workspace, H/16 zero-initialised counters
     int T;
     cudaEvent_t ev_mid;            // optional: recorded between the two kernels
 };

@@ -31,11 +31,11 @@ struct moe_layer {
     size_t ws_bytes = 0;
     float* logits = nullptr;       // [max_tokens, E]
     unsigned int* route_counter = nullptr;
-    float* dec_a = nullptr;        // [4*k, I]
-    float* dec_a_sh = nullptr;     // [4, I]
-    float* dec_part = nullptr;     // [4*k, H]
-    float* dec_part_sh = nullptr;  // [4, H]
-    unsigned int* dec_counters = nullptr;   // [H/32]
+    float* dec_a = nullptr;        // [8*k, I]
+    float* dec_a_sh = nullptr;     // [8, I]
+    float* dec_part = nullptr;     // [8*k, H]
+    float* dec_part_sh = nullptr;  // [8, H]
+    unsigned int* dec_counters = nullptr;   // [H/16]
     uint8_t* staging = nullptr;    // interchange copy of one matrix
     size_t staging_bytes = 0;
     // prefill path
@@ -156,7 +156,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->g_down = h->g_gate + E;
 
     // workspace
-    const int MT = 4;   // tokens per decode launch
+    const int MT = 8;   // tokens per decode launch
     size_t w = 0;
     auto carve = [&](size_t bytes) { size_t o = w; w = align_up(w + bytes, 256); return o; };
     const size_t o_logits = carve(sizeof(float) * (size_t)c.max_tokens * E);
@@ -165,7 +165,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_ash = carve(sizeof(float) * (size_t)MT * I);
     const size_t o_part = carve(sizeof(float) * (size_t)MT * k * H);
     const size_t o_psh = carve(sizeof(float) * (size_t)MT * H);
-    const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 32));
+    const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 16));
     h->staging_bytes = (size_t)2 * H * I + 65536;
     const size_t o_stage = carve(h->staging_bytes);
     const size_t Tm = (size_t)c.max_tokens, slots = Tm * k;
@@ -450,7 +450,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
     a.ev_mid = h->prof[3];
     if (h->prof[2]) cudaEventRecord(h->prof[2], st);
     for (int t0 = 0; t0 < T;) {
-        int tc = T - t0 < 4 ? T - t0 : 4;
+        int tc = T - t0 < 8 ? T - t0 : 8;
         while (!decode_supported(tc, c.top_k)) --tc;
         a.x = reinterpret_cast<const uint8_t*>(x) + (size_t)t0 * c.hidden * 2;
         a.ids = topk_ids + (size_t)t0 * c.top_k;
