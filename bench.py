@@ -280,26 +280,36 @@ def run_decode(args, wl, dev, rank, world):
     total_ms_max = allreduce_max(total_ms, dev, world)
 
     # ---- per-kernel breakdown (events between the library's kernels)
-    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # Each step's kernels are captured in a graph with event-record nodes
+    # between them (no host gaps); the events split the step per kernel.
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nsteps)]
     with torch.cuda.stream(stream):
         for evs in pev:            # torch creates the CUDA event on first record
             for ev in evs:
                 ev.record(stream)
     stream.synchronize()
-    uniq_per_step = []
-    with torch.cuda.stream(stream):
-        for s in range(args.steps):
-            i = step_index(s)
-            xi = xs[i * T:(i + 1) * T]
-            flush.zero_()
-            layer.set_profile_events(pev[s])
+    pgraphs = []
+    for i in range(nsteps):
+        g = torch.cuda.CUDAGraph()
+        xi = xs[i * T:(i + 1) * T]
+        layer.set_profile_events(pev[i])
+        with torch.cuda.graph(g, stream=stream):
             layer.route(xi, ids, w)
             layer.forward(xi, ids, w, y)
+        pgraphs.append(g)
     layer.set_profile_events(None)
-    stream.synchronize()
-    k_route = [p[0].elapsed_time(p[1]) for p in pev]
-    k_gu = [p[2].elapsed_time(p[3]) for p in pev]
-    k_dn = [p[3].elapsed_time(p[4]) for p in pev]
+    k_route, k_gu, k_dn = [], [], []
+    for s in range(args.steps):
+        i = step_index(s)
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            pgraphs[i].replay()
+        stream.synchronize()
+        p = pev[i]
+        k_route.append(p[0].elapsed_time(p[1]))
+        k_gu.append(p[2].elapsed_time(p[3]))
+        k_dn.append(p[3].elapsed_time(p[4]))
+    uniq_per_step = []
     # distinct experts per step (from the seeded routing, recomputed on device)
     with torch.cuda.stream(stream):
         for s in range(args.steps):

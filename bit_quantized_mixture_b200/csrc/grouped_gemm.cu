@@ -75,6 +75,7 @@ struct GemmArgs {
     const float* g_w;         // NVFP4 per-expert weight global scale, or null
     float g_act;              // NVFP4 activation global scale of the B operand
     float g_req;              // NVFP4: global scale of the requantized intermediate (mode 0)
+    const float* tok_scale;   // mode 0, INT4/INT2: power of two of each token's fp16 activations
     int* err;
 };
 
@@ -87,6 +88,48 @@ MOE_DEV void store_chunk(uint8_t* a_tile, int r, int c8, uint32_t w0, uint32_t w
 }
 
 MOE_DEV uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+MOE_DEV uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+// INT4 / INT2 codes -> fp16 (u - 8) * s or (u - z) * s: the integer is exact
+// in fp16 and so is the fp16 scale, so each weight is rounded once (2^-12).
+MOE_DEV void dequant_row_f16(int quant, const uint8_t* stg, uint8_t* a_tile, int r) {
+    if (quant == Q_INT4) {
+        const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(stg + 4096)[r]);
+        const __half2 off = __float2half2_rn(1032.0f);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(stg + (c * kBlkN + r) * 16);
+            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + u
+                    o[j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
+                }
+                store_chunk(a_tile, r, c * 4 + w, o[0], o[1], o[2], o[3]);
+            }
+        }
+    } else {
+        const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(stg + 2048)[r]);
+        const __half2 off = __float2half2_rn(1024.0f + (float)stg[2048 + 256 + r]);
+        const uint4 q = *reinterpret_cast<const uint4*>(stg + r * 16);
+        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t t = ((wv[w] >> (2 * j)) & 0x00030003u) | 0x64006400u;   // 1024 + u
+                o[j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
+            }
+            store_chunk(a_tile, r, 2 * w, o[0], o[1], o[2], o[3]);
+            store_chunk(a_tile, r, 2 * w + 1, o[4], o[5], o[6], o[7]);
+        }
+    }
+}
 
 MOE_DEV void dequant_row(int quant, const uint8_t* stg, uint8_t* a_tile, int r) {
     if (quant == Q_INT4) {
@@ -264,7 +307,8 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
         for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x, ++local) {
             const GemmTile t = a.tiles[ti];
             const int n_mma = (t.count + 15) & ~15;
-            const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+            const bool f16 = MODE == 0 && a.tok_scale != nullptr && t.expert >= 0;
+            const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
             const int ab = local & 1;
             if (!mbar_wait(&acc_empty[ab], ((uint32_t)(local >> 1) & 1u) ^ 1u, &abort_flag, a.err, 2)) break;
             tc_fence_after();
@@ -308,8 +352,12 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                 if (t.expert >= 0) {
                     uint8_t* A = smem + L::A + s * NMAT * kATile;
                     const uint8_t* stg = smem + L::STG + s * NMAT * kStgMat;
+                    const bool f16 = MODE == 0 && a.tok_scale != nullptr;
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) dequant_row(a.quant, stg + m * kStgMat, A + m * kATile, r);
+                    for (int m = 0; m < NMAT; ++m) {
+                        if (f16) dequant_row_f16(a.quant, stg + m * kStgMat, A + m * kATile, r);
+                        else dequant_row(a.quant, stg + m * kStgMat, A + m * kATile, r);
+                    }
                     fence_proxy_async_smem();
                 }
                 mbar_arrive(&full[s]);
@@ -340,7 +388,10 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                     tmem_ld16(taddr + 128, v1);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float gg = v0[i] * gsc, uu = v1[i] * gsc;
+                        float tsc = gsc;
+                        if (!shared && a.tok_scale && c0 + i < t.count)
+                            tsc = __ldg(a.tok_scale + __ldg(a.perm + t.seg + c0 + i) / a.k_top);
+                        const float gg = v0[i] * tsc, uu = v1[i] * tsc;
                         float act = gg / (1.0f + expf(-gg)) * uu;
                         if (!shared && a.quant == Q_NVFP4) {
                             // W4A4: requantize the intermediate per 16 consecutive rows
@@ -464,6 +515,40 @@ __global__ void k_combine(const __nv_bfloat16* __restrict__ O, const __nv_bfloat
     *reinterpret_cast<uint4*>(y + (size_t)t * H + c) = out;
 }
 
+// INT4 / INT2 gate/up operand: each token row of x scaled by a power of two
+// 2^-p (exact) so that its largest magnitude lies in [2^14, 2^15), stored as
+// fp16 (exact: bf16 has 8 significant bits); scale[t] = 2^p undoes it in the
+// GEMM epilogue.  One warp per token row.
+__global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, int T, int H, __half* __restrict__ x16,
+                           float* __restrict__ scale) {
+    const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    float amax = 0.0f;
+    for (int c = lane; c < H / 8; c += 32) {
+        const uint4 q = src[c];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    }
+    amax = warp_max(amax);
+    int e = 0;
+    if (amax > 0.0f) frexpf(amax, &e);         // amax in [2^(e-1), 2^e)
+    const int p = (amax > 0.0f) ? e - 15 : 0;  // amax * 2^-p in [2^14, 2^15)
+    const float down = ldexpf(1.0f, -p);
+    for (int c = lane; c < H / 8; c += 32) {
+        const uint4 q = src[c];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = h2_bits(__floats2half2_rn(bf16_lo(w[i]) * down, bf16_hi(w[i]) * down));
+        reinterpret_cast<uint4*>(x16 + (size_t)t * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) scale[t] = ldexpf(1.0f, p);
+}
+
 // NVFP4 activations: x -> bf16 values q * s_b (the global scale is applied in
 // the GEMM epilogue); one thread per 16-element block.
 __global__ void k_act_fp4_values(const __nv_bfloat16* __restrict__ x, int T, int H, float g,
@@ -509,15 +594,16 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D bf16 map over [rows, cols] (cols contiguous), box 64 x box_rows, 128-byte swizzle
-static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2D 16-bit map over [rows, cols] (cols contiguous), box 64 x box_rows, 128-byte swizzle
+static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -546,16 +632,23 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     const bool fp4 = ex.quant == Q_NVFP4;
     const void* xin = p.x;
+    CUtensorMapDataType xdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (fp4) {
         const long long nblk = (long long)T * (H / kFp4Blk);
         k_act_fp4_values<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)p.x, T, H, ex.g_x,
                                                                          p.xq);
         xin = p.xq;
+    } else {
+        k_x_to_f16<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, T, H, reinterpret_cast<__half*>(p.xq),
+                                                 p.tok_scale);
+        xin = p.xq;
+        xdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     }
     const bool has_sh = ex.sh_gate != nullptr;
     CUtensorMap m_routed, m_shared;
     // ---- gate / up
-    if (!make_map(&m_routed, xin, (uint64_t)T, (uint64_t)H, 1) || !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, 1))
+    if (!make_map(&m_routed, xin, (uint64_t)T, (uint64_t)H, 1, xdt) ||
+        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, 1))
         return cudaErrorInvalidValue;
     k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
     GemmArgs g{};
@@ -575,6 +668,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.g_w = fp4 ? ex.g_gate : nullptr;
     g.g_act = fp4 ? ex.g_x : 1.0f;
     g.g_req = ex.g_a;
+    g.tok_scale = fp4 ? nullptr : p.tok_scale;
     g.err = p.err;
     const int grid = num_sms();
     err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<0>::ALLOC);
@@ -598,6 +692,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.topk_w = p.w;
     g.g_w = fp4 ? ex.g_down : nullptr;
     g.g_act = fp4 ? ex.g_a : 1.0f;
+    g.tok_scale = nullptr;
     err = cudaFuncSetAttribute(k_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<1>::ALLOC);
     if (err != cudaSuccess) return err;
     k_grouped_gemm<1><<<grid, kGemmThreads, SmemLayout<1>::ALLOC, st>>>(m_routed, m_shared, g);

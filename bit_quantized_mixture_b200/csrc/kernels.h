@@ -85,7 +85,8 @@ struct PrefillArgs {
     int32_t *counts, *offsets, *perm, *inv, *perm_scratch;
     GemmTile* tiles;
     int* num_tiles;
-    __nv_bfloat16* xq;             // NVFP4: [T, H] dequantized W4A4 activations
+    __nv_bfloat16* xq;             // [T, H]: NVFP4 W4A4 activation values, else fp16 scaled x
+    float* tok_scale;              // [T]: power of two of each token's fp16 activations
     __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order
     __nv_bfloat16* a_sh;           // [T, I] shared-expert intermediate
     __nv_bfloat16* o;              // [T*k, H] weighted expert outputs by slot

@@ -44,6 +44,7 @@ struct moe_layer {
     int* num_tiles = nullptr;
     int* dev_err = nullptr;
     __nv_bfloat16 *xq = nullptr, *a_perm = nullptr, *a_sh = nullptr, *o = nullptr, *o_sh = nullptr;
+    float* tok_scale = nullptr;
     // state
     bool router_loaded = false;
     bool shared_loaded = false;
@@ -177,7 +178,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_tiles = carve(sizeof(GemmTile) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
     const size_t o_ntiles = carve(sizeof(int));
     const size_t o_err = carve(sizeof(int));
-    const size_t o_xq = carve(c.quant == MOE_Q_NVFP4 ? Tm * H * 2 : 0);
+    const size_t o_xq = carve(Tm * H * 2);
+    const size_t o_tsc = carve(Tm * sizeof(float));
     const size_t o_aperm = carve(slots * I * 2);
     const size_t o_ash16 = carve(c.has_shared ? Tm * I * 2 : 0);
     const size_t o_o = carve(slots * H * 2);
@@ -206,6 +208,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->num_tiles = reinterpret_cast<int*>(h->ws + o_ntiles);
     h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
     h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
+    h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
     h->a_perm = reinterpret_cast<__nv_bfloat16*>(h->ws + o_aperm);
     h->a_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_ash16);
     h->o = reinterpret_cast<__nv_bfloat16*>(h->ws + o_o);
@@ -432,7 +435,8 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
         p.perm_scratch = h->perm_scratch;
         p.tiles = h->tiles; p.num_tiles = h->num_tiles;
-        p.xq = h->xq; p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
+        p.xq = h->xq; p.tok_scale = h->tok_scale;
+        p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_prefill(p, st);

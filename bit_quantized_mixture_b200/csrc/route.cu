@@ -145,14 +145,40 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     extern __shared__ float xs[];          // [T][H] fp32
     __shared__ int s_last;
     const int H = a.H, T = a.T;
-    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
-    for (int i = threadIdx.x; i < T * H; i += blockDim.x) xs[i] = __bfloat162float(x[i]);
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 4 + warp;
     pdl_launch_dependents();                 // let the expert kernel get resident
+    const uint8_t* row = reinterpret_cast<const uint8_t*>(a.wr) + (size_t)(e < a.E ? e : 0) * H * 2;
+    // first batch of router-row loads goes out before the activations are staged
+    uint4 q0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int c = lane + 32 * u;
+        q0[u] = (e < a.E && c < H / 8) ? ldg_stream_v4(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+    }
+    {   // stage x as fp32: 16-byte loads, four in flight per thread
+        const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+        const int nchunks = T * H / 8;
+        for (int i0 = threadIdx.x; i0 < nchunks; i0 += 4 * blockDim.x) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * blockDim.x;
+                v[u] = (i < nchunks) ? xv[i] : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * blockDim.x;
+                if (i < nchunks) {
+                    float4* d = reinterpret_cast<float4*>(xs + (size_t)i * 8);
+                    d[0] = make_float4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y));
+                    d[1] = make_float4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w));
+                }
+            }
+        }
+    }
+    __syncthreads();
     if (e < a.E) {
-        const uint8_t* row = reinterpret_cast<const uint8_t*>(a.wr) + (size_t)e * H * 2;
         float acc[kRouteMaxTSmall];
 #pragma unroll
         for (int t = 0; t < kRouteMaxTSmall; ++t) acc[t] = 0.0f;
@@ -161,7 +187,7 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {          // 8 loads in flight per lane
                 const int c = c0 + lane + 32 * u;
-                q[u] = (c < H / 8) ? ldg_stream_v4(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0);
+                q[u] = (c0 == 0) ? q0[u] : ((c < H / 8) ? ldg_stream_v4(row + (size_t)c * 16) : make_uint4(0, 0, 0, 0));
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
