@@ -280,35 +280,29 @@ def run_decode(args, wl, dev, rank, world):
     total_ms_max = allreduce_max(total_ms, dev, world)
 
     # ---- per-kernel breakdown (events between the library's kernels)
-    # Each step's kernels are captured in a graph with event-record nodes
-    # between them (no host gaps); the events split the step per kernel.
-    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nsteps)]
+    # Per-kernel breakdown: eager launches with the library's profiling
+    # events between its kernels (events inside graphs cannot be timed).  The
+    # 512 MB flush before each step keeps the host ahead of the GPU, so the
+    # intervals hold the kernels and their launch latency, not host gaps.
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for evs in pev:            # torch creates the CUDA event on first record
             for ev in evs:
                 ev.record(stream)
     stream.synchronize()
-    pgraphs = []
-    for i in range(nsteps):
-        g = torch.cuda.CUDAGraph()
-        xi = xs[i * T:(i + 1) * T]
-        layer.set_profile_events(pev[i])
-        with torch.cuda.graph(g, stream=stream):
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            i = step_index(s)
+            xi = xs[i * T:(i + 1) * T]
+            flush.zero_()
+            layer.set_profile_events(pev[s])
             layer.route(xi, ids, w)
             layer.forward(xi, ids, w, y)
-        pgraphs.append(g)
     layer.set_profile_events(None)
-    k_route, k_gu, k_dn = [], [], []
-    for s in range(args.steps):
-        i = step_index(s)
-        with torch.cuda.stream(stream):
-            flush.zero_()
-            pgraphs[i].replay()
-        stream.synchronize()
-        p = pev[i]
-        k_route.append(p[0].elapsed_time(p[1]))
-        k_gu.append(p[2].elapsed_time(p[3]))
-        k_dn.append(p[3].elapsed_time(p[4]))
+    stream.synchronize()
+    k_route = [p[0].elapsed_time(p[1]) for p in pev]
+    k_gu = [p[2].elapsed_time(p[3]) for p in pev]
+    k_dn = [p[3].elapsed_time(p[4]) for p in pev]
     uniq_per_step = []
     # distinct experts per step (from the seeded routing, recomputed on device)
     with torch.cuda.stream(stream):
@@ -362,12 +356,15 @@ def run_decode(args, wl, dev, rank, world):
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "dominant": dom,
-        "roofline": {"bound": "hbm", "kernel": f"k_dec_{dom}", "achieved": achieved, "peak": peaks["hbm_gbs"],
+        "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes_per_launch": per_kernel[dom], "peak_source": peak_kind},
         "layer_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
         "launches_per_step": 3, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
     }
+
+
+KERNEL_NAMES = {"route": "k_router_small", "gateup": "k_dec_gateup", "down": "k_dec_down"}
 
 
 def load_traffic(kernel, workload):

@@ -69,8 +69,10 @@ struct GemmArgs {
     int K;                    // reduction length (H or I)
     int k_top;
     int out_ld;               // row length of the outputs (I or H)
-    __nv_bfloat16* out;       // mode 0: A_perm [slots, I]; mode 1: O [slots, H] by slot id
-    __nv_bfloat16* out_sh;    // shared expert output [T, out_ld]
+    __nv_bfloat16* out;       // mode 0: A_perm [slots, I] (bf16)
+    __nv_bfloat16* out_sh;    // mode 0: shared expert intermediate [T, I] (bf16)
+    __half* o16;              // mode 1: O [slots, H] by slot id (fp16)
+    __half* o16_sh;           // mode 1: shared expert output [T, H] (fp16)
     const float* topk_w;      // mode 1: routing weight of each slot
     const float* g_w;         // NVFP4 per-expert weight global scale, or null
     float g_act;              // NVFP4 activation global scale of the B operand
@@ -90,6 +92,7 @@ MOE_DEV void store_chunk(uint8_t* a_tile, int r, int c8, uint32_t w0, uint32_t w
 MOE_DEV uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 MOE_DEV uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+MOE_DEV __half f16_sat(float v) { return __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f)); }
 
 // INT4 / INT2 codes -> fp16 (u - 8) * s or (u - z) * s: the integer is exact
 // in fp16 and so is the fp16 scale, so each weight is rounded once (2^-12).
@@ -414,16 +417,18 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                         }
                     }
                 } else {
+                    // per-slot outputs are fp16 (saturating at +-65504): their
+                    // rounding error stays well below the final bf16 one
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int col = c0 + i;
                         if (col < t.count) {
                             if (shared) {
-                                a.out_sh[((size_t)t.seg + col) * a.out_ld + col_out] = __float2bfloat16_rn(v0[i]);
+                                a.o16_sh[((size_t)t.seg + col) * a.out_ld + col_out] = f16_sat(v0[i]);
                             } else {
                                 const int slot = __ldg(a.perm + t.seg + col);
                                 const float o = v0[i] * gsc * __ldg(a.topk_w + slot);
-                                a.out[(size_t)slot * a.out_ld + col_out] = __float2bfloat16_rn(o);
+                                a.o16[(size_t)slot * a.out_ld + col_out] = f16_sat(o);
                             }
                         }
                     }
@@ -488,8 +493,11 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
 
 // --------------------------------------------------------------- combine
 // y[t] = sum_{j<k} O[t*k + j] + S[t], fp32 sum in fixed j order, one bf16 rounding.
-__global__ void k_combine(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ S, int T, int H,
-                          int k, __nv_bfloat16* __restrict__ y) {
+MOE_DEV float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
+MOE_DEV float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+
+__global__ void k_combine(const __half* __restrict__ O, const __half* __restrict__ S, int T, int H, int k,
+                          __nv_bfloat16* __restrict__ y) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one thread per 8 columns
     const int per_row = H / 8;
     if (i >= (long long)T * per_row) return;
@@ -499,13 +507,13 @@ __global__ void k_combine(const __nv_bfloat16* __restrict__ O, const __nv_bfloat
         const uint4 q = *reinterpret_cast<const uint4*>(O + ((size_t)t * k + j) * H + c);
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) { acc[2 * p] += bf16_lo(w[p]); acc[2 * p + 1] += bf16_hi(w[p]); }
+        for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
     }
     if (S) {
         const uint4 q = *reinterpret_cast<const uint4*>(S + (size_t)t * H + c);
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) { acc[2 * p] += bf16_lo(w[p]); acc[2 * p + 1] += bf16_hi(w[p]); }
+        for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
     }
     uint4 out;
     out.x = pack_bf16x2(acc[0], acc[1]);
@@ -687,8 +695,10 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.sh1 = nullptr;
     g.K = I;
     g.out_ld = H;
-    g.out = p.o;
-    g.out_sh = p.o_sh;
+    g.out = nullptr;
+    g.out_sh = nullptr;
+    g.o16 = p.o;
+    g.o16_sh = p.o_sh;
     g.topk_w = p.w;
     g.g_w = fp4 ? ex.g_down : nullptr;
     g.g_act = fp4 ? ex.g_a : 1.0f;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -89,8 +90,8 @@ struct PrefillArgs {
     float* tok_scale;              // [T]: power of two of each token's fp16 activations
     __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order
     __nv_bfloat16* a_sh;           // [T, I] shared-expert intermediate
-    __nv_bfloat16* o;              // [T*k, H] weighted expert outputs by slot
-    __nv_bfloat16* o_sh;           // [T, H] shared-expert output
+    __half* o;                     // [T*k, H] weighted expert outputs by slot (fp16)
+    __half* o_sh;                  // [T, H] shared-expert output (fp16)
     int* err;                      // device error word (bounded waits)
 };
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I);

@@ -43,7 +43,8 @@ struct moe_layer {
     GemmTile* tiles = nullptr;
     int* num_tiles = nullptr;
     int* dev_err = nullptr;
-    __nv_bfloat16 *xq = nullptr, *a_perm = nullptr, *a_sh = nullptr, *o = nullptr, *o_sh = nullptr;
+    __nv_bfloat16 *xq = nullptr, *a_perm = nullptr, *a_sh = nullptr;
+    __half *o = nullptr, *o_sh = nullptr;
     float* tok_scale = nullptr;
     // state
     bool router_loaded = false;
@@ -211,8 +212,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
     h->a_perm = reinterpret_cast<__nv_bfloat16*>(h->ws + o_aperm);
     h->a_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_ash16);
-    h->o = reinterpret_cast<__nv_bfloat16*>(h->ws + o_o);
-    h->o_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_osh);
+    h->o = reinterpret_cast<__half*>(h->ws + o_o);
+    h->o_sh = reinterpret_cast<__half*>(h->ws + o_osh);
     cudaError_t e1 = cudaMemset(h->ws, 0, h->ws_bytes);
     cudaError_t e2 = cudaMemset(h->arena, 0, h->arena_bytes);
     if (e1 != cudaSuccess || e2 != cudaSuccess) {
