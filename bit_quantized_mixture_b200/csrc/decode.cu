@@ -375,7 +375,7 @@ MOE_DEV MatPtr expert_mat(const MatView& v, int e) {
 
 // ------------------------------------------------------------- gate / up
 template <int Q>
-__global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
+__global__ void __launch_bounds__(kGuThreads, 3) k_dec_gateup(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ Plan plan;
     __shared__ int tok[kDecMaxT];
@@ -386,26 +386,34 @@ __global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
     const int rb_per_exp = I / 16;
     const int u = blockIdx.x / rb_per_exp;          // distinct expert, or the shared one when u == n
     const int rb16 = blockIdx.x % rb_per_exp;
-
-    pdl_wait();                                      // ids come from the router
-    pdl_launch_dependents();
-    build_plan(a.ids, n, plan);
     const bool is_shared = (u == n);
-    if (!is_shared && u >= plan.n_unique) return;
-    int m;
-    if (is_shared) {
-        m = T;
-        if (threadIdx.x < T) { tok[threadIdx.x] = threadIdx.x; slot_of[threadIdx.x] = threadIdx.x; }
-    } else {
-        m = item_tokens(plan.ids, n, k, plan.first[u], tok, slot_of);
-    }
+
+    // The activations do not depend on the routing: stage all T token rows
+    // (row t = token t, rows T..8 zero) before waiting for the router.
     const int ldx = H + kXPad;
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem_raw);                   // [8][ldx]
-    float* red = reinterpret_cast<float*>(smem_raw + (size_t)kDecMaxT * ldx * 2);      // [8][2][16][8]
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem_raw);                   // [9][ldx]
+    float* red = reinterpret_cast<float*>(smem_raw + (size_t)(kDecMaxT + 1) * ldx * 2);   // [8][2][16][8]
+    if (threadIdx.x < kDecMaxT) tok[threadIdx.x] = threadIdx.x;
     __syncthreads();
     const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
-    if (Q == Q_NVFP4 && !is_shared) stage_rows_fp4_from_bf16(xs, ldx, x, H, tok, m, ex.g_x);
-    else stage_rows_bf16(xs, ldx, x, H, tok, m);
+    if (Q == Q_NVFP4 && !is_shared) stage_rows_fp4_from_bf16(xs, ldx, x, H, tok, T, ex.g_x);
+    else stage_rows_bf16(xs, ldx, x, H, tok, T);
+    for (int i = threadIdx.x; i < ldx / 8; i += blockDim.x)
+        reinterpret_cast<uint4*>(xs + kDecMaxT * ldx)[i] = make_uint4(0, 0, 0, 0);
+
+    int m;
+    if (is_shared) {
+        // the shared expert needs nothing from the router
+        m = T;
+        if (threadIdx.x < T) slot_of[threadIdx.x] = threadIdx.x;
+        pdl_launch_dependents();
+    } else {
+        pdl_wait();                                  // ids come from the router
+        pdl_launch_dependents();
+        build_plan(a.ids, n, plan);
+        if (u >= plan.n_unique) return;
+        m = item_tokens(plan.ids, n, k, plan.first[u], tok, slot_of);
+    }
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -413,7 +421,7 @@ __global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
     const int KB = H / kBlkK, G = H / kGroup;
     const int r0 = rb16 * 16;
     const int nb = r0 / kBlkN, rl = r0 % kBlkN + g;
-    const __nv_bfloat16* xrow = xs + g * ldx;
+    const __nv_bfloat16* xrow = xs + (g < m ? tok[g] : kDecMaxT) * ldx;     // item column g = token tok[g]
     float acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
     int e = 0;
     if (is_shared) {
@@ -459,7 +467,7 @@ __global__ void __launch_bounds__(kGuThreads) k_dec_gateup(DecodeArgs a) {
 
 // ------------------------------------------------------- down + combine
 template <int Q>
-__global__ void __launch_bounds__(kDnThreads) k_dec_down(DecodeArgs a) {
+__global__ void __launch_bounds__(kDnThreads, 10) k_dec_down(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ Plan plan;
     __shared__ int tok[kDecMaxT];
@@ -535,12 +543,14 @@ __global__ void __launch_bounds__(kDnThreads) k_dec_down(DecodeArgs a) {
         }
     }
     // the last item of this row block to finish combines
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(a.counters + hb, 1u) == (unsigned)items_per_rb - 1u);
+    if (threadIdx.x == 0) {
+        __threadfence();                      // this CTA's partials before its ticket
+        s_last = (atomicAdd(a.counters + hb, 1u) == (unsigned)items_per_rb - 1u);
+        if (s_last) __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.y);
     for (int i = threadIdx.x; i < T * 16; i += blockDim.x) {
         const int t = i / 16, h = h0 + i % 16;
@@ -563,7 +573,7 @@ static cudaError_t launch_decode_q(const DecodeArgs& a, cudaStream_t st) {
     const int n = a.T * ex.k;
     const int items_gu = (n + (ex.sh_gate ? 1 : 0)) * (ex.I / 16);
     const int items_dn = (n + (ex.sh_down ? 1 : 0)) * (ex.H / 16);
-    const size_t smem_gu = (size_t)kDecMaxT * (ex.H + kXPad) * 2 + 8 * 2 * 16 * 8 * sizeof(float);
+    const size_t smem_gu = (size_t)(kDecMaxT + 1) * (ex.H + kXPad) * 2 + 8 * 2 * 16 * 8 * sizeof(float);
     const size_t smem_dn = (size_t)kDecMaxT * (ex.I + kXPad) * 2 + 4 * 16 * 8 * sizeof(float);
     cudaError_t err = cudaFuncSetAttribute(k_dec_gateup<Q>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_gu);
     if (err != cudaSuccess) return err;

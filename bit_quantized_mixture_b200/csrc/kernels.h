@@ -36,6 +36,9 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 
+// moe_api.cu: text returned by moe_last_error(NULL) on this host thread
+void set_thread_error(const char* msg);
+
 // permute.cu
 cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* inv, int32_t* chunk_scratch, cudaStream_t st);

@@ -69,6 +69,8 @@ static moe_status fail(moe_layer* h, moe_status s, const char* fmt, ...) {
     return s;
 }
 
+void moe::set_thread_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+
 static moe_status cuda_fail(moe_layer* h, cudaError_t e, const char* where) {
     return fail(h, MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }

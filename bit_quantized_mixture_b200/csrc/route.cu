@@ -14,43 +14,49 @@
 
 namespace moe {
 
-constexpr int kRouteMaxTSmall = 16;   // decode router: tokens staged in smem
+constexpr int kRouteMaxTSmall = 8;    // decode router: tokens staged in smem
 constexpr size_t kRouteMaxSmem = 160 * 1024;
 constexpr int kMaxK = 32;
 
-// One warp selects the top-k of one token's logits (row of E <= 1024 values,
-// read through L2).  Writes ids/w for that token.
+// Order-preserving key of an fp32 value (larger value -> larger key).
+MOE_DEV uint32_t order_key(float v) {
+    const uint32_t b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One warp selects the top-k of one token's logits (E <= 1024 values read
+// through L2, expert e held by lane e % 32) and writes ids / weights.  Each
+// round takes the largest remaining key with one warp max-reduction and,
+// among equal keys, the smallest expert index with one min-reduction.
 MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
                        float* __restrict__ wout) {
     const int lane = threadIdx.x & 31;
-    float v[32];
+    uint32_t key[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldcg(row + e) : -FLT_MAX;
+        key[i] = (e < E) ? order_key(__ldcg(row + e)) : 0u;
     }
-    uint32_t removed = 0;
-    float my_val = 0.0f;
+    uint32_t live = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
+    float my_val = 0.0f, lmax = 0.0f;
     int my_idx = 0;
-    float lmax = 0.0f;
     for (int j = 0; j < k; ++j) {
-        float best = -INFINITY;
-        int bidx = 0x7fffffff;
+        uint32_t best = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int e = lane + 32 * i;
-            const bool live = (e < E) && !((removed >> i) & 1u);
-            if (live && (v[i] > best || (v[i] == best && e < bidx))) { best = v[i]; bidx = e; }
-        }
+        for (int i = 0; i < 32; ++i)
+            if ((live >> i) & 1u) best = max(best, key[i]);
+        const uint32_t top = __reduce_max_sync(0xffffffffu, best);
+        uint32_t mine = 0xffffffffu;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
-        }
-        if ((bidx & 31) == lane) removed |= 1u << (bidx >> 5);
-        if (j == 0) lmax = best;
-        if (lane == j) { my_val = best; my_idx = bidx; }
+        for (int i = 31; i >= 0; --i)
+            if (((live >> i) & 1u) && key[i] == top) mine = (uint32_t)(lane + 32 * i);
+        const uint32_t e = __reduce_min_sync(0xffffffffu, mine);
+        if ((int)(e & 31u) == lane) live &= ~(1u << (e >> 5));
+        const float v = __uint_as_float((top & 0x80000000u) ? (top & 0x7fffffffu) : ~top);   // key -> value
+        if (j == 0) lmax = v;
+        if (lane == j) { my_val = v; my_idx = (int)e; }
     }
     const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
     const float sum = warp_sum(ex);
@@ -60,86 +66,7 @@ MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __r
     }
 }
 
-// Top-k of one token by the 4 warps of a CTA: each warp selects the k best
-// of its quarter of the experts, then warp 0 selects the k best of those
-// 4k candidates.  Same order and weights as warp_topk.
-MOE_DEV void cta4_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                       float* __restrict__ wout, float* cand_v, int* cand_i) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = (E + 3) / 4, e0 = warp * q, e1 = min(E, e0 + q);
-    float v[8];
-    int vi[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = e0 + lane + 32 * i;
-        vi[i] = e;
-        v[i] = (e < e1) ? __ldcg(row + e) : -INFINITY;
-    }
-    uint32_t removed = 0;
-    for (int j = 0; j < k; ++j) {
-        float best = -INFINITY;
-        int bidx = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const bool live = (vi[i] < e1) && !((removed >> i) & 1u);
-            if (live && (v[i] > best || (v[i] == best && vi[i] < bidx))) { best = v[i]; bidx = vi[i]; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-            if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
-        }
-        if (bidx != 0x7fffffff && ((bidx - e0) & 31) == lane) removed |= 1u << ((bidx - e0) >> 5);
-        if (lane == 0) { cand_v[warp * kMaxK + j] = best; cand_i[warp * kMaxK + j] = bidx; }
-    }
-    __syncthreads();
-    if (warp == 0) {
-        // 4k <= 128 candidates, 4 per lane
-        float cv[4];
-        int ci[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int c = lane + 32 * i, w = c / kMaxK, jj = c % kMaxK;
-            const bool ok = jj < k;
-            cv[i] = ok ? cand_v[w * kMaxK + jj] : -INFINITY;
-            ci[i] = ok ? cand_i[w * kMaxK + jj] : 0x7fffffff;
-        }
-        uint32_t rem = 0;
-        float my_val = 0.0f, lmax = 0.0f;
-        int my_idx = 0;
-        for (int j = 0; j < k; ++j) {
-            float best = -INFINITY;
-            int bidx = 0x7fffffff, bslot = -1;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const bool live = !((rem >> i) & 1u) && ci[i] != 0x7fffffff;
-                if (live && (cv[i] > best || (cv[i] == best && ci[i] < bidx))) { best = cv[i]; bidx = ci[i]; bslot = i; }
-            }
-            int owner = (bslot >= 0) ? lane : 32;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-                const int oo = __shfl_xor_sync(0xffffffffu, owner, o);
-                const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
-                if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; owner = oo; bslot = os; }
-            }
-            if (owner == lane) rem |= 1u << bslot;
-            if (j == 0) lmax = best;
-            if (lane == j) { my_val = best; my_idx = bidx; }
-        }
-        const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
-        const float sum = warp_sum(ex);
-        if (lane < k) {
-            ids[lane] = my_idx;
-            wout[lane] = __fdiv_rn(ex, sum);
-        }
-    }
-    __syncthreads();
-}
-
-// Decode router (T <= 16): one warp per expert row, a grid-wide ticket lets
+// Decode router (T <= 8): one warp per expert row, a grid-wide ticket lets
 // the last CTA to finish run the top-k of every token (no waiting).
 __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     extern __shared__ float xs[];          // [T][H] fp32
@@ -216,19 +143,17 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
             }
         }
     }
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
+    if (threadIdx.x == 0) {
+        __threadfence();                      // this CTA's logits before its ticket
+        s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
+        if (s_last) __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    __shared__ float cand_v[4 * kMaxK];
-    __shared__ int cand_i[4 * kMaxK];
-    if (a.E <= 1024) {
-        for (int t = 0; t < T; ++t)
-            cta4_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k,
-                      cand_v, cand_i);
-    }
+    for (int t = warp; t < T; t += 4)
+        warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
+    __syncthreads();
     if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
 }
 

@@ -68,6 +68,7 @@ def lib():
             "moe_debug_unpack_matrix": [vp, i32, i32, vp, vp, vp, vp, vp],
             "moe_set_profile_events": [vp, ctypes.POINTER(vp), i32],
             "moe_sync_status": [vp, vp],
+            "moe_permute_noalloc": [vp, i32, i32, i32, vp, vp, vp, vp, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -219,4 +220,17 @@ def permute(ids, num_experts, stream=None):
     inv = torch.empty(T * k, dtype=torch.int32, device=dev)
     _check(lib().moe_permute(_ptr(ids), T, k, num_experts, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
                              _stream(stream)))
+    return counts, offsets, perm, inv
+
+
+def permute_noalloc(ids, num_experts, stream=None):
+    """moe_permute without device allocation (scratch in a static device array)."""
+    T, k = ids.shape
+    dev = ids.device
+    counts = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _check(lib().moe_permute_noalloc(_ptr(ids), T, k, num_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
+                                     _ptr(inv), _stream(stream)))
     return counts, offsets, perm, inv

@@ -187,6 +187,25 @@ moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                        moe_stream_t stream);
 
+/* moe_permute without any device allocation.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory at
+ * call time - runtimes that reserve their whole budget at start-up, hosts
+ * whose caching allocator already owns the device memory, or latency-critical
+ * paths that must not risk the implicit synchronisation of cudaMalloc and
+ * cudaFree.  Same arguments, outputs and determinism as moe_permute; the
+ * per-chunk histogram scratch lives in a file-scope device array of 1 MiB that
+ * every GPU loading the library keeps until the process exits.
+ * Limits: T*k <= 262144 and E <= 1024, else MOE_ERR_INVALID_ARG (message in
+ * moe_last_error(NULL)) before any device work.  The first call on a device
+ * looks up the array's device address (with that device current); make that
+ * first call before any stream capture.  All calls on a device share the one
+ * array: calls whose kernels overlap in time on the GPU (different streams
+ * without ordering) race and give wrong results.  Nothing in the array has to
+ * start at zero: each call writes every entry it reads. */
+moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                               moe_stream_t stream);
+
 /* ---------------------------------------------------------------- debug */
 
 /* Write loaded matrix `which` (0 gate, 1 up, 2 down) of `expert` back in
