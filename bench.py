@@ -238,15 +238,13 @@ def run_decode(args, wl, dev, rank, world):
     with torch.cuda.stream(stream):
         for i in range(nsteps):       # eager pass first (also a warm-up of every path)
             xi = xs[i * T:(i + 1) * T]
-            layer.route(xi, ids, w)
-            layer.forward(xi, ids, w, y)
+            layer.route_forward(xi, ids, w, y)
     stream.synchronize()
     for i in range(nsteps):
         g = torch.cuda.CUDAGraph()
         xi = xs[i * T:(i + 1) * T]
         with torch.cuda.graph(g, stream=stream):
-            layer.route(xi, ids, w)
-            layer.forward(xi, ids, w, y)
+            layer.route_forward(xi, ids, w, y)
         graphs.append(g)
     torch.cuda.synchronize(dev)
 
@@ -280,10 +278,9 @@ def run_decode(args, wl, dev, rank, world):
     total_ms_max = allreduce_max(total_ms, dev, world)
 
     # ---- per-kernel breakdown (events between the library's kernels)
-    # Per-kernel breakdown: eager launches with the library's profiling
-    # events between its kernels (events inside graphs cannot be timed).  The
-    # 512 MB flush before each step keeps the host ahead of the GPU, so the
-    # intervals hold the kernels and their launch latency, not host gaps.
+    # Kernel time: eager launches with the library's profiling events around
+    # its one kernel (events inside graphs cannot be timed).  The 512 MB flush
+    # before each step keeps the host ahead of the GPU.
     pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for evs in pev:            # torch creates the CUDA event on first record
@@ -293,18 +290,13 @@ def run_decode(args, wl, dev, rank, world):
     with torch.cuda.stream(stream):
         for s in range(args.steps):
             i = step_index(s)
-            xi = xs[i * T:(i + 1) * T]
             flush.zero_()
             layer.set_profile_events(pev[s])
-            layer.route(xi, ids, w)
-            layer.forward(xi, ids, w, y)
+            layer.route_forward(xs[i * T:(i + 1) * T], ids, w, y)
     layer.set_profile_events(None)
     stream.synchronize()
-    k_route = [p[0].elapsed_time(p[1]) for p in pev]
-    k_gu = [p[2].elapsed_time(p[3]) for p in pev]
-    k_dn = [p[3].elapsed_time(p[4]) for p in pev]
+    k_fused = [p[0].elapsed_time(p[4]) for p in pev]
     uniq_per_step = []
-    # distinct experts per step (from the seeded routing, recomputed on device)
     with torch.cuda.stream(stream):
         for s in range(args.steps):
             i = step_index(s)
@@ -318,8 +310,7 @@ def run_decode(args, wl, dev, rank, world):
     x_stage = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
     g_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_e2e, stream=stream):
-        layer.route(x_stage, ids, w)
-        layer.forward(x_stage, ids, w, y)
+        layer.route_forward(x_stage, ids, w, y)
     e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
@@ -336,35 +327,29 @@ def run_decode(args, wl, dev, rank, world):
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
     e2e_ms_max = allreduce_max(e2e_ms, dev, world)
 
-    # ---- roofline of the dominant kernel (gate/up GEMV over the experts)
+    # ---- roofline of the (single) fused decode kernel: algorithmic bytes of
+    # the whole step (router, distinct experts, shared expert, activations,
+    # intermediates and partials) over its event-measured duration
     gu_b, dn_b = expert_bytes(wl)
     H, I = wl.H, wl.I
-    sh_gu = 2 * I * H * 2 if wl.shared else 0
-    sh_dn = H * I * 2 if wl.shared else 0
-    kern = {"route": float(np.mean(k_route)), "gateup": float(np.mean(k_gu)), "down": float(np.mean(k_dn))}
+    sh = 3 * I * H * 2 if wl.shared else 0
     mean_uniq = float(np.mean(uniq_per_step))
-    bytes_gu = mean_uniq * gu_b + sh_gu + T * H * 2 + (T * k + T) * I * 4
-    bytes_dn = mean_uniq * dn_b + sh_dn + (T * k + T) * I * 4 + T * H * 2 + (T * k + T) * H * 4 * 2
-    bytes_rt = wl.E * H * 2 + T * H * 2 + T * wl.E * 4
-    per_kernel = {"route": bytes_rt, "gateup": bytes_gu, "down": bytes_dn}
-    dom = max(kern, key=kern.get)
+    step_bytes = (wl.E * H * 2 + T * H * 2 + T * wl.E * 4 + mean_uniq * (gu_b + dn_b) + sh
+                  + (T * k + T) * I * 4 * 2 + (T * k + T) * H * 4 * 2 + T * H * 2)
+    kern = {"decode_fused": float(np.mean(k_fused))}
     peaks, peak_kind = measured_peaks()
-    achieved = per_kernel[dom] / (kern[dom] * 1e-3) / 1e9
-    traffic = load_traffic(dom, wl.name)
-    step_bytes = bytes_rt + bytes_gu + bytes_dn
+    achieved = step_bytes / (kern["decode_fused"] * 1e-3) / 1e9
+    traffic = load_traffic("k_decode_fused", wl.name)
     layer.close()
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
-        "clocks": clocks.summary(), "kernels_ms": kern, "dominant": dom,
-        "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved, "peak": peaks["hbm_gbs"],
+        "clocks": clocks.summary(), "kernels_ms": kern, "dominant": "decode_fused",
+        "roofline": {"bound": "hbm", "kernel": "k_decode_fused", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": per_kernel[dom], "peak_source": peak_kind},
+                     "algorithmic_bytes_per_launch": step_bytes, "peak_source": peak_kind},
         "layer_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
-        "launches_per_step": 3, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
+        "launches_per_step": 1, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
     }
-
-
-KERNEL_NAMES = {"route": "k_router_small", "gateup": "k_dec_gateup", "down": "k_dec_down"}
 
 
 def load_traffic(kernel, workload):

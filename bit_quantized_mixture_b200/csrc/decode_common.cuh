@@ -1,0 +1,347 @@
+// Building blocks shared by the decode kernels (few tokens, tensor-core GEMV):
+// the per-launch plan of distinct experts, exact dequantization into MMA
+// fragments, the m16n8k16 row-block products and activation staging.
+// See decode.cu for the design.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kDecMaxT = 8;           // tokens per launch = MMA N
+constexpr int kDecMaxSlots = 256;
+constexpr int kXPad = 32;             // bf16 row padding of staged activations (bank spread)
+
+struct Plan {
+    int n_unique;
+    int ids[kDecMaxSlots];
+    int first[kDecMaxSlots];
+    unsigned char is_first[kDecMaxSlots];
+};
+
+MOE_DEV void build_plan(const int32_t* __restrict__ ids, int n, Plan& p) {
+    for (int s = threadIdx.x; s < n; s += blockDim.x) p.ids[s] = __ldcg(ids + s);
+    __syncthreads();
+    for (int s = threadIdx.x; s < n; s += blockDim.x) {
+        const int e = p.ids[s];
+        bool f = true;
+        for (int q = 0; q < s; ++q) f = f && (p.ids[q] != e);
+        p.is_first[s] = f;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int base = 0;
+        for (int s0 = 0; s0 < n; s0 += 32) {
+            const int s = s0 + lane;
+            const bool f = (s < n) && p.is_first[s];
+            const unsigned m = __ballot_sync(0xffffffffu, f);
+            if (f) p.first[base + __popc(m & ((1u << lane) - 1u))] = s;
+            base += __popc(m);
+        }
+        if (lane == 0) p.n_unique = base;
+    }
+    __syncthreads();
+}
+
+// Tokens of the item whose first slot is s0, in slot order.  With valid
+// input (distinct ids per token) there are at most T <= kDecMaxT; repeated
+// ids within a token are invalid input and the extra slots are dropped, so
+// no buffer is overrun.
+MOE_DEV int item_tokens(const int* __restrict__ ids, int n, int k, int s0, int* tok, int* slot) {
+    const int e0 = ids[s0];
+    int c = 0;
+    for (int s = s0; s < n && c < kDecMaxT; ++s) {
+        if (ids[s] == e0) {
+            if (threadIdx.x == 0) { tok[c] = s / k; slot[c] = s; }
+            ++c;
+        }
+    }
+    return c;
+}
+
+// ------------------------------------------------------------ MMA helpers
+MOE_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+MOE_DEV uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t bf16x2_splat(float v) {
+    const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+    return h | (h << 16);
+}
+// INT4 pair j of a word: bf16x2 (u - 8), exact
+MOE_DEV uint32_t int4_pair(uint32_t w, int j) {
+    return hsub2_bits(((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u, 0x43084308u);   // (128+u) - 136
+}
+// INT2 pair j of a word: bf16x2 (u - z), exact; off = bf16x2(128 + z)
+MOE_DEV uint32_t int2_pair(uint32_t w, int j, uint32_t off) {
+    return hsub2_bits(((w >> (2 * j)) & 0x00030003u) | 0x43004300u, off);
+}
+// E2M1 pair j of a word times the block scale (bf16x2 splat), exact:
+// the codes placed at bf16 bits [8:6] (magnitude) and 15 (sign) read as
+// e2m1 * 2^-126; one multiply by 2^126 and one by the scale.
+MOE_DEV uint32_t fp4_pair(uint32_t w, int j, uint32_t sb2) {
+    const uint32_t t = w >> (4 * j);
+    const uint32_t b = ((t & 0x00070007u) << 6) | ((t & 0x00080008u) << 12);
+    return hmul2_bits(hmul2_bits(b, 0x7E807E80u), sb2);       // 0x7E80 = 2^126
+}
+
+// ------------------------------------------------------------ format traits
+template <int Q> struct Fmt;
+template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 4; };
+template <> struct Fmt<Q_NVFP4> { static constexpr int KPW = 4; };
+template <> struct Fmt<Q_INT2>  { static constexpr int KPW = 4; };
+template <> struct Fmt<Q_BF16>  { static constexpr int KPW = 2; };
+
+struct MatPtr {
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const uint8_t* zeros;
+};
+
+// Operands of rows (rl, rl+8) of one 128x64 block for lane (g, c)
+template <int Q>
+struct Blk {
+    uint32_t w[2][2];        // INT4 / NVFP4: [chunk][row g, g+8]; INT2: w[0][row]
+    uint4 v[2][2];           // bf16: [32-column half][row g, g+8]
+    float s0, s1;            // INT4/INT2 scales of the two rows
+    uint32_t z0, z1;         // INT2: bf16x2(128 + z) of the two rows
+    uint32_t sb0, sb1;       // NVFP4: four E4M3 block scales of each row
+};
+
+template <int Q>
+MOE_DEV void load_blk(Blk<Q>& o, const MatPtr& m, int nb, int kb, int KB, int G, int rl, int c) {
+    if constexpr (Q == Q_BF16) {
+        const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * 16384;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = rl + 8 * rr;
+                const int c8 = 4 * h + c;
+                o.v[h][rr] = ldg_stream_v4(blk + (r >> 3) * 1024 + (r & 7) * 128 + ((c8 ^ (r & 7)) << 4));
+            }
+    } else if constexpr (Q == Q_INT2) {
+        const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 16);
+        o.w[0][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + rl * 16 + c * 4));
+        o.w[0][1] = __ldg(reinterpret_cast<const uint32_t*>(blk + (rl + 8) * 16 + c * 4));
+        const size_t gi = ((size_t)nb * G + kb / 2) * kBlkN + rl;
+        o.s0 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi));
+        o.s1 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi + 8));
+        o.z0 = bf16x2_splat(128.0f + (float)__ldg(m.zeros + gi));
+        o.z1 = bf16x2_splat(128.0f + (float)__ldg(m.zeros + gi + 8));
+    } else {
+        const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 32);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            o.w[ch][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + (ch * kBlkN + rl) * 16 + c * 4));
+            o.w[ch][1] = __ldg(reinterpret_cast<const uint32_t*>(blk + (ch * kBlkN + rl + 8) * 16 + c * 4));
+        }
+        if constexpr (Q == Q_INT4) {
+            const size_t gi = ((size_t)nb * G + kb / 2) * kBlkN + rl;
+            o.s0 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi));
+            o.s1 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi + 8));
+        } else {
+            const size_t si = (((size_t)nb * KB + kb) * kBlkN + rl) * 4;
+            o.sb0 = __ldg(reinterpret_cast<const uint32_t*>(m.scales + si));
+            o.sb1 = __ldg(reinterpret_cast<const uint32_t*>(m.scales + si + 32));
+        }
+    }
+}
+
+// acc[0..3] (rows g, g+8 x tokens 2c, 2c+1) += block . x; xrow points at
+// the lane's token row g of the staged activations at the block's column 0.
+template <int Q>
+MOE_DEV void mma_blk(float (&acc)[4], const Blk<Q>& o, const __nv_bfloat16* xrow, int c) {
+    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if constexpr (Q == Q_INT2) {
+        const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + 16 * c);
+        const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + 16 * c + 8);
+        const uint32_t xb[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+            mma16816(d, int2_pair(o.w[0][0], 2 * mi, o.z0), int2_pair(o.w[0][1], 2 * mi, o.z1),
+                     int2_pair(o.w[0][0], 2 * mi + 1, o.z0), int2_pair(o.w[0][1], 2 * mi + 1, o.z1), xb[2 * mi],
+                     xb[2 * mi + 1]);
+    } else {
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(xrow + 32 * ch + 8 * c);
+            if constexpr (Q == Q_BF16) {
+                const uint4 r0 = o.v[ch][0], r1 = o.v[ch][1];
+                mma16816(acc, r0.x, r1.x, r0.y, r1.y, xv.x, xv.y);
+                mma16816(acc, r0.z, r1.z, r0.w, r1.w, xv.z, xv.w);
+            } else if constexpr (Q == Q_INT4) {
+                const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
+                mma16816(d, int4_pair(w0, 0), int4_pair(w1, 0), int4_pair(w0, 1), int4_pair(w1, 1), xv.x, xv.y);
+                mma16816(d, int4_pair(w0, 2), int4_pair(w1, 2), int4_pair(w0, 3), int4_pair(w1, 3), xv.z, xv.w);
+            } else {  // NVFP4: word c of chunk ch lies in 16-column block 2ch + c/2
+                const int b = 2 * ch + (c >> 1);
+                const uint32_t s0 = bf16x2_splat(e4m3_to_f32((o.sb0 >> (8 * b)) & 0xffu));
+                const uint32_t s1 = bf16x2_splat(e4m3_to_f32((o.sb1 >> (8 * b)) & 0xffu));
+                const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
+                mma16816(d, fp4_pair(w0, 0, s0), fp4_pair(w1, 0, s1), fp4_pair(w0, 1, s0), fp4_pair(w1, 1, s1), xv.x,
+                         xv.y);
+                mma16816(d, fp4_pair(w0, 2, s0), fp4_pair(w1, 2, s1), fp4_pair(w0, 3, s0), fp4_pair(w1, 3, s1), xv.z,
+                         xv.w);
+            }
+        }
+    }
+    if constexpr (Q == Q_INT4 || Q == Q_INT2) {
+        acc[0] = fmaf(o.s0, d[0], acc[0]);
+        acc[1] = fmaf(o.s0, d[1], acc[1]);
+        acc[2] = fmaf(o.s1, d[2], acc[2]);
+        acc[3] = fmaf(o.s1, d[3], acc[3]);
+    } else if constexpr (Q == Q_NVFP4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += d[i];
+    }
+}
+
+// One warp: 16 rows (rl, rl+8 per lane) of NM matrices over k-blocks
+// warp, warp + nwarps, ...
+template <int Q, int NM>
+MOE_DEV void warp_rows(float (&acc)[NM][4], const MatPtr (&mats)[NM], int nb, int rl, int KB, int G, int warp,
+                       int nwarps, const __nv_bfloat16* xrow, int c) {
+    constexpr int KPW = Fmt<Q>::KPW;
+    for (int kb0 = warp; kb0 < KB; kb0 += nwarps * KPW) {
+        Blk<Q> blk[NM][KPW];
+#pragma unroll
+        for (int i = 0; i < KPW; ++i) {
+            const int kb = kb0 + i * nwarps;
+            if (kb < KB) {
+#pragma unroll
+                for (int q = 0; q < NM; ++q) load_blk<Q>(blk[q][i], mats[q], nb, kb, KB, G, rl, c);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < KPW; ++i) {
+            const int kb = kb0 + i * nwarps;
+            if (kb < KB) {
+#pragma unroll
+                for (int q = 0; q < NM; ++q) mma_blk<Q>(acc[q], blk[q][i], xrow + kb * kBlkK, c);
+            }
+        }
+    }
+}
+
+// W4A4: the value q * s_b of a 16-element block (the global scale g is left
+// to the epilogue), with the recipe of the activation quantization kernel.
+MOE_DEV void fp4_block_values(float (&v)[16], float g) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+    float sbv = 0.0f, r = 0.0f;
+    if (g != 0.0f) {
+        sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g))));
+        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
+    }
+#pragma unroll
+    for (int q = 0; q < 16; q += 2) {
+        const uint32_t cc = f32x2_to_e2m1(__fmul_rn(v[q], r), __fmul_rn(v[q + 1], r));
+        v[q] = e2m1_to_f32(cc & 0xFu) * sbv;
+        v[q + 1] = e2m1_to_f32(cc >> 4) * sbv;
+    }
+}
+
+// Stage rows (row_of[t], t < m) of a bf16 matrix [*, K] into smem rows of
+// ldx elements; rows m..7 are zero.  16-byte accesses, loads issued first.
+MOE_DEV void stage_rows_bf16(__nv_bfloat16* dst, int ldx, const __nv_bfloat16* src, int K, const int* row_of, int m,
+                             int tid, int nthreads) {
+    const int per_row = K / 8;
+    const int total = kDecMaxT * per_row;
+    for (int i0 = tid; i0 < total; i0 += 4 * nthreads) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * nthreads;
+            const int t = i / per_row, c = i % per_row;
+            v[u] = (i < total && t < m) ? *reinterpret_cast<const uint4*>(src + (size_t)row_of[t] * K + c * 8)
+                                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * nthreads;
+            if (i < total) *reinterpret_cast<uint4*>(dst + (i / per_row) * ldx + (i % per_row) * 8) = v[u];
+        }
+    }
+}
+
+// Stage rows of bf16 activations [*, K] as W4A4 values (q * s_b).
+MOE_DEV void stage_rows_fp4_from_bf16(__nv_bfloat16* dst, int ldx, const __nv_bfloat16* src, int K,
+                                      const int* row_of, int m, float g, int tid, int nthreads) {
+    const int per_row = K / 16;
+    const int total = kDecMaxT * per_row;
+    for (int i = tid; i < total; i += nthreads) {
+        const int t = i / per_row, b = i % per_row;
+        float v[16];
+        if (t < m) {
+            const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row_of[t] * K + b * 16);
+            const uint4 q0 = s[0], q1 = s[1];
+            const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) { v[2 * q] = bf16_lo(wv[q]); v[2 * q + 1] = bf16_hi(wv[q]); }
+            fp4_block_values(v, g);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = 0.0f;
+        }
+        uint32_t p[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) p[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+        uint4* d = reinterpret_cast<uint4*>(dst + t * ldx + b * 16);
+        d[0] = make_uint4(p[0], p[1], p[2], p[3]);
+        d[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    }
+}
+
+// Stage rows of fp32 intermediates [*, K] as bf16 (W4A4: as q * s_b).
+MOE_DEV void stage_rows_f32(__nv_bfloat16* dst, int ldx, const float* src, int K, const int* row_of, int m, bool fp4,
+                            float g, int tid, int nthreads) {
+    const int per_row = K / 16;
+    const int total = kDecMaxT * per_row;
+    for (int i = tid; i < total; i += nthreads) {
+        const int t = i / per_row, b = i % per_row;
+        float v[16];
+        if (t < m) {
+            const float4* s = reinterpret_cast<const float4*>(src + (size_t)row_of[t] * K + b * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 f = __ldcg(s + q);
+                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+            }
+            if (fp4) fp4_block_values(v, g);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = 0.0f;
+        }
+        uint32_t p[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) p[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+        uint4* d = reinterpret_cast<uint4*>(dst + t * ldx + b * 16);
+        d[0] = make_uint4(p[0], p[1], p[2], p[3]);
+        d[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    }
+}
+
+MOE_DEV MatPtr expert_mat(const MatView& v, int e) {
+    MatPtr p;
+    p.codes = v.codes + (size_t)e * v.stride;
+    p.scales = v.scales ? v.scales + (size_t)e * v.stride : nullptr;
+    p.zeros = v.zeros ? v.zeros + (size_t)e * v.stride : nullptr;
+    return p;
+}
+
+
+}  // namespace moe

@@ -72,6 +72,19 @@ struct DecodeArgs {
 bool decode_supported(int T, int k);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
+// decode_fused.cu: the whole decode step in one cooperative kernel
+struct FusedArgs {
+    DecodeArgs d;                  // ids / w are inputs when wr is null
+    const void* wr;                // bf16 [E, H] router, or null
+    float* logits;                 // workspace [T, E]
+    int32_t* ids_out;              // [T, k] (when wr is set)
+    float* w_out;                  // [T, k]
+    unsigned int* bar;             // workspace {arrivals, generation}, zero-initialised
+    int* err;                      // device error word
+};
+size_t fused_smem_bytes(int H, int I);
+cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st);
+
 // grouped_gemm.cu (prefill path)
 struct GemmTile {
     int expert;   // routed expert, or -1 for the shared expert

@@ -36,6 +36,7 @@ struct moe_layer {
     float* dec_part = nullptr;     // [8*k, H]
     float* dec_part_sh = nullptr;  // [8, H]
     unsigned int* dec_counters = nullptr;   // [H/16]
+    unsigned int* fused_bar = nullptr;      // {arrivals, generation} of the fused decode kernel
     uint8_t* staging = nullptr;    // interchange copy of one matrix
     size_t staging_bytes = 0;
     // prefill path
@@ -170,6 +171,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_part = carve(sizeof(float) * (size_t)MT * k * H);
     const size_t o_psh = carve(sizeof(float) * (size_t)MT * H);
     const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 16));
+    const size_t o_fbar = carve(sizeof(unsigned int) * 2);
     h->staging_bytes = (size_t)2 * H * I + 65536;
     const size_t o_stage = carve(h->staging_bytes);
     const size_t Tm = (size_t)c.max_tokens, slots = Tm * k;
@@ -201,6 +203,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->dec_part = reinterpret_cast<float*>(h->ws + o_part);
     h->dec_part_sh = reinterpret_cast<float*>(h->ws + o_psh);
     h->dec_counters = reinterpret_cast<unsigned int*>(h->ws + o_cnt);
+    h->fused_bar = reinterpret_cast<unsigned int*>(h->ws + o_fbar);
     h->staging = h->ws + o_stage;
     h->counts = reinterpret_cast<int32_t*>(h->ws + o_counts);
     h->offsets = reinterpret_cast<int32_t*>(h->ws + o_offsets);
@@ -416,6 +419,17 @@ static ExpertArgs expert_args(moe_layer* h) {
     return ex;
 }
 
+static DecodeArgs decode_args(moe_layer* h) {
+    DecodeArgs a{};
+    a.ex = expert_args(h);
+    a.a = h->dec_a;
+    a.a_sh = h->dec_a_sh;
+    a.part = h->dec_part;
+    a.part_sh = h->dec_part_sh;
+    a.counters = h->dec_counters;
+    return a;
+}
+
 moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* topk_ids, const float* topk_w, void* y,
                        moe_stream_t stream) {
     if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_forward: null handle");
@@ -447,7 +461,24 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         if (h->prof[4]) cudaEventRecord(h->prof[4], st);
         return MOE_OK;
     }
-    DecodeArgs a{};
+    DecodeArgs a = decode_args(h);
+    if (T <= 8) {
+        FusedArgs f{};
+        f.d = a;
+        f.d.x = x; f.d.ids = topk_ids; f.d.w = topk_w; f.d.y = y; f.d.T = T;
+        f.wr = nullptr;
+        f.bar = h->fused_bar;
+        f.err = h->dev_err;
+        if (h->prof[2]) cudaEventRecord(h->prof[2], st);
+        cudaError_t e = launch_decode_fused(f, st);
+        if (e == cudaSuccess) {
+            if (h->prof[4]) cudaEventRecord(h->prof[4], st);
+            return MOE_OK;
+        }
+        // a refused cooperative launch falls back to the two-kernel decode path
+        if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorNotSupported) return cuda_fail(h, e, "moe_forward");
+        cudaGetLastError();
+    }
     a.ex = expert_args(h);
     a.a = h->dec_a;
     a.a_sh = h->dec_a_sh;
@@ -472,6 +503,51 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
     return MOE_OK;
 }
 
+moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* topk_ids, float* topk_w, void* y,
+                             moe_stream_t stream) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_route_forward: null handle");
+    moe_status s = check_tokens(h, "moe_route_forward", T);
+    if (s != MOE_OK) return s;
+    if (!x || !topk_ids || !topk_w || !y) return fail(h, MOE_ERR_INVALID_ARG, "moe_route_forward: null pointer");
+    if (!aligned16(x) || !aligned16(y))
+        return fail(h, MOE_ERR_INVALID_ARG, "moe_route_forward: x and y must be 16-byte aligned");
+    const moe_config& c = h->cfg;
+    if (!h->router_loaded) return fail(h, MOE_ERR_STATE, "moe_route_forward: router not loaded");
+    if (h->experts_loaded != c.num_experts)
+        return fail(h, MOE_ERR_STATE, "moe_route_forward: %d of %d experts loaded", h->experts_loaded, c.num_experts);
+    if (c.has_shared && !h->shared_loaded) return fail(h, MOE_ERR_STATE, "moe_route_forward: shared expert not loaded");
+    if (c.quant == MOE_Q_NVFP4 && !h->act_scales_set)
+        return fail(h, MOE_ERR_STATE, "moe_route_forward: NVFP4 activation global scales not set");
+    if (T > 8 || !decode_supported(T, c.top_k)) {
+        s = moe_route(h, x, T, topk_ids, topk_w, nullptr, stream);
+        if (s != MOE_OK) return s;
+        return moe_forward(h, x, T, topk_ids, topk_w, y, stream);
+    }
+    DeviceGuard dg(c.device);
+    cudaStream_t st = (cudaStream_t)stream;
+    FusedArgs f{};
+    f.d = decode_args(h);
+    f.d.x = x; f.d.ids = topk_ids; f.d.w = topk_w; f.d.y = y; f.d.T = T;
+    f.wr = h->router;
+    f.logits = h->logits;
+    f.ids_out = topk_ids;
+    f.w_out = topk_w;
+    f.bar = h->fused_bar;
+    f.err = h->dev_err;
+    if (h->prof[0]) cudaEventRecord(h->prof[0], st);
+    cudaError_t e = launch_decode_fused(f, st);
+    if (e == cudaSuccess) {
+        if (h->prof[4]) cudaEventRecord(h->prof[4], st);
+        return MOE_OK;
+    }
+    if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorNotSupported)
+        return cuda_fail(h, e, "moe_route_forward");
+    cudaGetLastError();
+    s = moe_route(h, x, T, topk_ids, topk_w, nullptr, stream);
+    if (s != MOE_OK) return s;
+    return moe_forward(h, x, T, topk_ids, topk_w, y, stream);
+}
+
 moe_status moe_sync_status(moe_handle h, moe_stream_t stream) {
     if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_sync_status: null handle");
     DeviceGuard dg(h->cfg.device);
@@ -481,8 +557,11 @@ moe_status moe_sync_status(moe_handle h, moe_stream_t stream) {
     e = cudaMemcpy(&code, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_sync_status");
     if (code) {
+        // a stopped kernel may leave tickets and the grid barrier half-counted
         const int zero = 0;
         cudaMemcpy(h->dev_err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        cudaMemset(h->dec_counters, 0, sizeof(unsigned int) * (size_t)(h->cfg.hidden / 16));
+        cudaMemset(h->fused_bar, 0, sizeof(unsigned int));
         return fail(h, MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (site %d); outputs are invalid", code);
     }
     return MOE_OK;

@@ -61,6 +61,7 @@ def lib():
             "moe_route": [vp, vp, i32, vp, vp, vp, vp],
             "moe_route_from_logits": [vp, vp, i32, vp, vp, vp],
             "moe_forward": [vp, vp, i32, vp, vp, vp, vp],
+            "moe_route_forward": [vp, vp, i32, vp, vp, vp, vp],
             "moe_quantize": [i32, vp, i32, i32, f32, vp, vp, vp, vp],
             "moe_absmax": [vp, i64, vp, vp],
             "moe_quantize_act_nvfp4": [vp, i32, i32, f32, vp, vp, vp],
@@ -164,6 +165,11 @@ class MoeLayer:
     def sync_status(self, stream=None):
         """Synchronize the stream; raise on a device-side timeout or CUDA error."""
         _check(lib().moe_sync_status(self.h, _stream(stream)), self.h)
+
+    def route_forward(self, x, ids, w, y, stream=None):
+        """The whole layer (route + forward) in one call."""
+        _check(lib().moe_route_forward(self.h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(y), _stream(stream)),
+               self.h)
 
     def set_profile_events(self, events):
         """events: 5 torch.cuda.Event(enable_timing=True) or None."""

@@ -159,6 +159,14 @@ moe_status moe_route_from_logits(moe_handle h, const float* logits, int32_t T,
 moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* topk_ids,
                        const float* topk_w, void* y, moe_stream_t stream);
 
+/* The whole layer, moe_route followed by moe_forward, as one call: writes
+ * topk_ids / topk_w (as moe_route) and y (as moe_forward).  For T <= 8 it
+ * runs as one cooperative kernel (router, top-k, experts, shared expert and
+ * combine, separated by bounded grid-wide barriers); larger T, or a refused
+ * cooperative launch, runs moe_route then moe_forward.  Errors as those two. */
+moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* topk_ids,
+                             float* topk_w, void* y, moe_stream_t stream);
+
 /* ------------------------------------------------- format kernels (no handle) */
 
 /* Quantize W fp32 [N, K] (device) into interchange layout (device outputs).

@@ -302,3 +302,61 @@ def test_prefill_zipf_int4_full_size_sampled_tokens():
 
 def test_prefill_nvfp4_full_size_sampled_tokens():
     _full_size_sampled("prefill-nvfp4", 8)
+
+
+# --------------------------------------------- whole layer in one call (fused)
+@pytest.mark.parametrize("quant", ["int4", "int2", "nvfp4"])
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_route_forward_matches_route_then_oracle(quant, T):
+    """moe_route_forward (one cooperative kernel for T <= 8): ids/weights equal
+    moe_route's, output matches the oracle on those ids/weights."""
+    wl = SMALL[quant]
+    layer = get_layer(wl, 8)
+    ox = OracleExperts(wl)
+    x = synth.activations_bf16(wl, steps=2)[:T]
+    xd = bf16_tensor(x, DEV)
+    act = None
+    if quant == "nvfp4":
+        xf = O.bf16_bits_to_f32(x)
+        g_x = O.nvfp4_global_scale(np.abs(xf).max())
+        rid, _ = O.route_topk(O.router_logits(x, synth.router_bf16(wl)), wl.k)
+        g_a = O.nvfp4_global_scale(O.intermediate_amax(x, rid, "nvfp4", ox, g_x))
+        act = (g_x, g_a)
+        layer.set_act_global_scales(g_x, g_a)
+    ids_r = torch.empty((T, wl.k), dtype=torch.int32, device=DEV)
+    w_r = torch.empty((T, wl.k), dtype=torch.float32, device=DEV)
+    layer.route(xd, ids_r, w_r)
+    ids = torch.full((T, wl.k), -1, dtype=torch.int32, device=DEV)
+    w = torch.zeros((T, wl.k), dtype=torch.float32, device=DEV)
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+    layer.route_forward(xd, ids, w, y)
+    layer.sync_status()
+    assert torch.equal(ids, ids_r)
+    assert torch.allclose(w, w_r, rtol=2e-6, atol=1e-7)
+    ids_h, w_h = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    y_ref = O.moe_forward(x, ids_h, w_h, quant, ox, shared=ox.shared(), act_scales=act)
+    assert_close_output(to_bits(y), y_ref)
+    # twice in a row: tickets and the grid barrier are reusable, results identical
+    y2 = torch.empty_like(y)
+    layer.route_forward(xd, ids, w, y2)
+    layer.sync_status()
+    assert torch.equal(y, y2)
+
+
+def test_route_forward_decode_b1_full_size():
+    wl = synth.workload("decode-b1-int4")
+    layer = get_layer(wl, 4)
+    ox = OracleExperts(wl)
+    xs = synth.activations_bf16(wl)
+    for i in (3, 64):
+        x = xs[i:i + 1]
+        ids = torch.empty((1, wl.k), dtype=torch.int32, device=DEV)
+        w = torch.empty((1, wl.k), dtype=torch.float32, device=DEV)
+        y = torch.empty((1, wl.H), dtype=torch.bfloat16, device=DEV)
+        layer.route_forward(bf16_tensor(x, DEV), ids, w, y)
+        layer.sync_status()
+        ids_h, w_h = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+        rid, _ = O.route_topk(O.router_logits(x, synth.router_bf16(wl)), wl.k)
+        assert np.array_equal(ids_h, rid)
+        y_ref = O.moe_forward(x, ids_h, w_h, wl.quant, ox, shared=ox.shared())
+        assert_close_output(to_bits(y), y_ref)
