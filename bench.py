@@ -120,55 +120,91 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------- oracle arm
-def oracle_tokens_per_s(wl, seconds, rank_offset=0):
-    """Time the CPU oracle (as it stands) on a bounded sample of the workload:
-    whole decode steps (router, top-k, expert SwiGLU from the packed weights,
-    combine) until `seconds` of work are done.  Quantization of the weights
-    is set-up, as on the GPU, and is not timed."""
-    from threadpoolctl import threadpool_info
+NVFP4_INTER_AMAX = 8.0   # calibration bound of the W4A4 intermediate (see prefill_act_scales)
 
-    from bit_quantized_mixture_b200 import synth
-    from oracle import moe_oracle as O
 
-    xs = synth.activations_bf16(wl)
-    wr = synth.router_bf16(wl)
-    shared = tuple(O.bf16_bits_to_f64(m) for m in synth.shared_bf16(wl)) if wl.shared else None
-    q = {}
+class OracleSampler:
+    """Times the CPU oracle (as it stands) on bounded samples of a workload.
 
-    def quantized(e):
-        if e not in q:
-            mats = synth.expert_fp32(wl, e)
+    Decode workloads: whole decode steps (router, top-k, expert SwiGLU from
+    the packed weights, combine).  Prefill workloads: chunks of 4 consecutive
+    tokens of the batch (top-k of the workload's routing logits, expert
+    SwiGLU, combine).  Quantization of the weights is set-up, as on the GPU:
+    it is not timed, is kept across samples, and stops a sample early once it
+    has taken `setup_cap_s` in total."""
+
+    def __init__(self, wl, setup_cap_s=90.0):
+        from bit_quantized_mixture_b200 import synth
+        from oracle import moe_oracle as O
+        self.O, self.synth, self.wl = O, synth, wl
+        self.setup_cap_s = setup_cap_s
+        self.xs = synth.activations_bf16(wl)
+        self.prefill = wl.routing != "router"
+        self.wr = None if self.prefill else synth.router_bf16(wl)
+        self.logits = synth.routing_logits(wl) if self.prefill else None
+        self.shared = tuple(O.bf16_bits_to_f64(m) for m in synth.shared_bf16(wl)) if wl.shared else None
+        self.act = None
+        if wl.quant == "nvfp4":
+            g_x = O.nvfp4_global_scale(np.abs(O.bf16_bits_to_f32(self.xs)).max())
+            self.act = (g_x, O.nvfp4_global_scale(NVFP4_INTER_AMAX))
+        self.q = {}
+        self.setup = 0.0
+        self.chunk = 4 if self.prefill else wl.T
+        self.n_chunks = wl.T // self.chunk if self.prefill else wl.steps
+
+    def quantized(self, e):
+        O, wl = self.O, self.wl
+        if e not in self.q:
+            t0 = time.perf_counter()
+            g, u, d = self.synth.expert_fp32(wl, e)
             ew = {}
-            for name, m in zip(("gate", "up", "down"), mats):
+            if wl.quant == "nvfp4":
+                g_gu = O.nvfp4_global_scale(max(np.abs(g).max(), np.abs(u).max()))
+                g_d = O.nvfp4_global_scale(np.abs(d).max())
+            for name, m in zip(("gate", "up", "down"), (g, u, d)):
                 if wl.quant == "int4":
-                    c, s = O.quantize_int4(m)
-                    ew[name] = {"codes": c, "scales": s}
+                    c, sc = O.quantize_int4(m)
+                    ew[name] = {"codes": c, "scales": sc}
                 elif wl.quant == "int2":
-                    c, s, z = O.quantize_int2(m)
-                    ew[name] = {"codes": c, "scales": s, "zeros": z}
+                    c, sc, z = O.quantize_int2(m)
+                    ew[name] = {"codes": c, "scales": sc, "zeros": z}
                 else:
-                    raise ValueError("oracle timing covers the W4A16/W2A16 decode workloads")
-            q[e] = ew
-        return q[e]
+                    gg = g_d if name == "down" else g_gu
+                    c, sc = O.quantize_nvfp4(m, gg)
+                    ew[name] = {"codes": c, "scales": sc, "g": gg}
+            self.q[e] = ew
+            self.setup += time.perf_counter() - t0
+        return self.q[e]
 
-    # prepare (untimed) the experts of the first steps, then time whole steps
-    n_steps = wl.steps
-    spent, tokens, steps_done = 0.0, 0, 0
-    while spent < seconds and steps_done < n_steps:
-        i = (rank_offset + steps_done) % n_steps
-        x = xs[i * wl.T:(i + 1) * wl.T]
-        ids_probe, _ = O.route_topk(O.router_logits(x, wr), wl.k)
-        for e in np.unique(ids_probe):
-            quantized(int(e))
-        t0 = time.perf_counter()
-        ids, w = O.route_topk(O.router_logits(x, wr), wl.k)
-        O.moe_forward(x, ids, w, wl.quant, lambda e: O.dequantize_expert(wl.quant, quantized(e)), shared=shared)
-        spent += time.perf_counter() - t0
-        tokens += wl.T
-        steps_done += 1
-    threads = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
-    return tokens / spent, {"cores": int(threads), "sample": f"{steps_done} steps x {wl.T} tokens of {wl.name}",
-                            "seconds": spent}
+    def _route(self, i, x):
+        lg = self.logits[i * self.chunk:(i + 1) * self.chunk] if self.prefill else self.O.router_logits(x, self.wr)
+        return self.O.route_topk(lg, self.wl.k)
+
+    def sample(self, seconds, offset=0):
+        """(tokens/s, info) over chunks starting at chunk `offset`."""
+        from threadpoolctl import threadpool_info
+        O, wl = self.O, self.wl
+        spent, tokens, done = 0.0, 0, 0
+        while spent < seconds and done < self.n_chunks and (done == 0 or self.setup < self.setup_cap_s):
+            i = (offset + done) % self.n_chunks
+            x = self.xs[i * self.chunk:(i + 1) * self.chunk]
+            ids_probe, _ = self._route(i, x)
+            for e in np.unique(ids_probe):
+                self.quantized(int(e))
+            t0 = time.perf_counter()
+            ids, w = self._route(i, x)
+            O.moe_forward(x, ids, w, wl.quant, lambda e: O.dequantize_expert(wl.quant, self.quantized(e)),
+                          shared=self.shared, act_scales=self.act)
+            spent += time.perf_counter() - t0
+            tokens += self.chunk
+            done += 1
+        threads = max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+        what = f"{done} chunks x {self.chunk} tokens" if self.prefill else f"{done} steps x {wl.T} tokens"
+        return tokens / spent, {"cores": int(threads), "sample": f"{what} of {wl.name}", "seconds": spent}
+
+
+def oracle_tokens_per_s(wl, seconds, rank_offset=0):
+    return OracleSampler(wl).sample(seconds, rank_offset)
 
 
 def run_reference(args):
@@ -178,12 +214,13 @@ def run_reference(args):
     from bit_quantized_mixture_b200 import synth
     wl = synth.workload(args.workload)
     per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
+    sampler = OracleSampler(wl)
     vals = []
     for _ in range(args.warmup):
-        oracle_tokens_per_s(wl, per_step / 4)
+        sampler.sample(per_step / 4)
     info = None
     for s in range(args.steps):
-        v, info = oracle_tokens_per_s(wl, per_step, rank_offset=s)
+        v, info = sampler.sample(per_step, offset=s)
         vals.append(v)
     value = float(np.mean(vals))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -352,6 +389,141 @@ def run_decode(args, wl, dev, rank, world):
     }
 
 
+def prefill_flops(wl, slots):
+    """Algorithmic FLOPs of the grouped GEMMs of one prefill step: gate/up
+    2*m*H*2I and down 2*m*I*H over the routed slots and the shared rows."""
+    m = slots + (wl.T if wl.shared else 0)
+    return 2.0 * m * wl.H * 2 * wl.I, 2.0 * m * wl.I * wl.H
+
+
+def run_prefill(args, wl, dev, rank, world):
+    """A prefill step: router GEMM on x (logits kept), top-k of the
+    workload's synthetic routing logits (the skewed / uniform routing the
+    workload prescribes), permutation, gate/up and down grouped GEMMs,
+    combine.  Eager launches; per-kernel events in a separate pass."""
+    import torch
+
+    from bit_quantized_mixture_b200 import moe, synth
+    from bit_quantized_mixture_b200.layer import build_layer
+
+    layer, _ = build_layer(wl, dev.index, max_tokens=wl.T)
+    T, k, H, E = wl.T, wl.k, wl.H, wl.E
+    x_host = synth.activations_bf16(wl)
+    lg_host = synth.routing_logits(wl).astype(np.float32)
+    x = torch.from_numpy(x_host.view(np.int16)).to(dev).view(torch.bfloat16)
+    lg = torch.from_numpy(lg_host).to(dev)
+    if wl.quant == "nvfp4":
+        # static W4A4 activation scales (set-up, not timed): g_x from the
+        # batch's |x| max, g_a from a fixed calibration bound (values of the
+        # intermediate above it saturate to the largest code)
+        amax = torch.zeros(1, dtype=torch.float32, device=dev)
+        moe.absmax(x.float(), amax)
+        layer.set_act_global_scales(moe.nvfp4_global_scale(float(amax.item())),
+                                    moe.nvfp4_global_scale(NVFP4_INTER_AMAX))
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(args.flush_mb * (1 << 20) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(xin, lgin):
+        layer.route(xin, ids, w, logits=logits)       # router GEMM (logits) + its top-k
+        layer.route_from_logits(lgin, ids, w)         # the workload's routing
+        layer.forward(xin, ids, w, y)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            step(x, lg)
+    layer.sync_status(stream)
+
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    with clocks:
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                flush.zero_()
+                ev0[s].record(stream)
+                step(x, lg)
+                ev1[s].record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    layer.sync_status(stream)
+    total_ms = float(sum(a.elapsed_time(b) for a, b in zip(ev0, ev1)))
+    total_ms_max = allreduce_max(total_ms, dev, world)
+
+    # ---- per-kernel breakdown: the library's profiling events
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for evs in pev:
+            for ev in evs:
+                ev.record(stream)
+    stream.synchronize()
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            flush.zero_()
+            layer.set_profile_events(pev[s])
+            step(x, lg)
+    layer.set_profile_events(None)
+    stream.synchronize()
+
+    def mean_ms(i, j):
+        return float(np.mean([p[i].elapsed_time(p[j]) for p in pev]))
+
+    kern = {"route_router_gemm": mean_ms(0, 1), "forward": mean_ms(2, 4), "grouped_gemm_gate_up": mean_ms(5, 3),
+            "grouped_gemm_down": mean_ms(6, 7), "combine": mean_ms(7, 4)}
+
+    # ---- end to end through the public API: x and the routing logits from
+    # pinned host memory, y back to pinned host memory
+    x_pin = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_pin = torch.from_numpy(lg_host).pin_memory()
+    y_pin = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    x_st = torch.empty_like(x)
+    lg_st = torch.empty_like(lg)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for s in range(args.steps):
+            flush.zero_()
+            e0[s].record(stream)
+            x_st.copy_(x_pin, non_blocking=True)
+            lg_st.copy_(lg_pin, non_blocking=True)
+            step(x_st, lg_st)
+            y_pin.copy_(y, non_blocking=True)
+            e1[s].record(stream)
+    stream.synchronize()
+    layer.sync_status(stream)
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
+    e2e_ms_max = allreduce_max(e2e_ms, dev, world)
+
+    fl_gu, fl_dn = prefill_flops(wl, T * k)
+    peaks, peak_kind = measured_peaks()
+    peak = peaks["bf16_tflops"]
+    achieved = fl_gu / (kern["grouped_gemm_gate_up"] * 1e-3) / 1e12
+    traffic = load_traffic("k_grouped_gemm<0>", wl.name)
+    layer.close()
+    roof = {"bound": "tensor", "kernel": "k_grouped_gemm<0> (gate/up)", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "algorithmic_flops_per_launch": fl_gu,
+            "peak_source": f"{peak_kind} dense bf16 burst (the MMA runs kind::f16 on "
+                           f"{'bf16' if wl.quant == 'nvfp4' else 'fp16'} operands)",
+            "down_kernel_tflops": fl_dn / (kern["grouped_gemm_down"] * 1e-3) / 1e12}
+    if wl.quant == "nvfp4":
+        roof["frac_of_fp4_peak"] = achieved / (4.0 * peak)   # nominal fp4 : bf16 dense ratio 9 : 2.25
+    return {
+        "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
+        "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
+        "launches_per_step": 12, "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
+        "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
+        "dtype": "bf16" if wl.quant == "nvfp4" else "f16",
+    }
+
+
 def load_traffic(kernel, workload):
     """Per-launch DRAM bytes of `kernel` from a committed ncu summary, only if
     the kernel source has not changed since the counters were taken."""
@@ -400,27 +572,29 @@ def run_ours(args):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = synth.workload(args.workload)
-    if wl.T > 4:
-        raise SystemExit("this bench times the decode workloads (T <= 4)")
-    r = run_decode(args, wl, dev, rank, world)
+    prefill = wl.routing != "router"
+    r = run_prefill(args, wl, dev, rank, world) if prefill else run_decode(args, wl, dev, rank, world)
     tokens_all = r["steps_tokens"] * world
     value = tokens_all / (r["total_ms"] * 1e-3)
     e2e = tokens_all / (r["e2e_ms"] * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
+        "dtype": r.get("dtype", "bf16"), "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "quant": wl.quant,
-                   "shared": wl.shared, "parallelism": f"replicas x{world}",
+                   "shared": wl.shared, "routing": wl.routing, "parallelism": f"replicas x{world}",
                    "l2": f"flushed ({args.flush_mb} MB write) between timed steps",
-                   "cuda_graph": True},
+                   "cuda_graph": not prefill},
         "roofline": r["roofline"],
         "kernels_ms": r["kernels_ms"],
-        "layer_hbm_gbs": r["layer_gbs"],
         "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
+    if "layer_gbs" in r:
+        line["layer_hbm_gbs"] = r["layer_gbs"]
+    if "layer_tflops" in r:
+        line["layer_tflops"] = r["layer_tflops"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_tokens_per_s(wl, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",

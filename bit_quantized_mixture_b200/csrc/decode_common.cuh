@@ -99,10 +99,10 @@ MOE_DEV uint32_t fp4_pair(uint32_t w, int j, uint32_t sb2) {
 
 // ------------------------------------------------------------ format traits
 template <int Q> struct Fmt;
-template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 4; };
-template <> struct Fmt<Q_NVFP4> { static constexpr int KPW = 4; };
-template <> struct Fmt<Q_INT2>  { static constexpr int KPW = 4; };
-template <> struct Fmt<Q_BF16>  { static constexpr int KPW = 2; };
+template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_NVFP4> { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_INT2>  { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_BF16>  { static constexpr int KPW = 1; };
 
 struct MatPtr {
     const uint8_t* codes;

@@ -28,30 +28,36 @@ constexpr int kFWarps = 16;
 constexpr int kFThreads = kFWarps * 32;
 constexpr long long kBarrierLimitCycles = 4000000000LL;   // about 2 s
 
-// Grid-wide barrier on {arrivals, generation}: the last CTA to arrive resets
-// the count and advances the generation; the others spin on it (bounded).
-MOE_DEV bool grid_barrier(unsigned int* bar, int* err, volatile int* abort_s) {
+// Grid-wide barrier on one monotonically increasing 64-bit arrival count:
+// arrival i belongs to barrier episode i / gridDim.x, and a CTA leaves once
+// the count reaches the end of its episode.  One atomic per CTA, no reset;
+// release on arrival and acquire on the polls order the writes before the
+// barrier against the reads after it.  Bounded: on timeout the CTA records
+// an error code and stops.
+MOE_DEV unsigned long long ld_acquire64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+MOE_DEV unsigned long long atom_add_release64(unsigned long long* p, unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+    return old;
+}
+MOE_DEV bool grid_barrier(unsigned long long* bar, int* err, volatile int* abort_s) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        volatile unsigned int* gen = bar + 1;
-        const unsigned int g0 = *gen;
-        __threadfence();
-        if (atomicAdd(bar, 1u) == gridDim.x - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
-        } else {
-            const long long t0 = clock64();
-            while (*gen == g0) {
-                if (clock64() - t0 > kBarrierLimitCycles) {
-                    *abort_s = 1;
-                    if (err) atomicCAS(err, 0, 20);
-                    break;
-                }
-                __nanosleep(32);
+        const unsigned long long n = gridDim.x;
+        const unsigned long long ticket = atom_add_release64(bar, 1ull);
+        const unsigned long long target = (ticket / n + 1) * n;
+        const long long t0 = clock64();
+        while (ld_acquire64(bar) < target) {
+            if (clock64() - t0 > kBarrierLimitCycles) {
+                *abort_s = 1;
+                if (err) atomicCAS(err, 0, 20);
+                break;
             }
         }
-        __threadfence();
     }
     __syncthreads();
     return *abort_s == 0;
@@ -101,39 +107,46 @@ MOE_DEV void router_row(const uint8_t* __restrict__ wr, int e, int H, int T, con
     }
 }
 
-// Top-k of one token by one warp (same rule as route.cu), results in smem.
+// Top-k of one token by one warp (rule of route.cu: logit descending, expert
+// index ascending; weights = softmax over the selected).  Lane l holds the
+// experts l, l+32, ...; each lane caches its best remaining (key, expert), so
+// a round is two warp reductions plus a rescan by the winning lane only.
 MOE_DEV uint32_t fkey(float v) {
     const uint32_t b = __float_as_uint(v);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+MOE_DEV float fkey_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
 MOE_DEV void warp_topk_smem(const float* __restrict__ row, int E, int k, int* ids, float* wts) {
     const int lane = threadIdx.x & 31;
     uint32_t key[32];
+    uint32_t live = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int e = lane + 32 * i;
         key[i] = (e < E) ? fkey(__ldcg(row + e)) : 0u;
+        live |= (e < E ? 1u : 0u) << i;
     }
-    uint32_t live = 0;
+    uint32_t bk = 0, bi = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
+    for (int i = 0; i < 32; ++i)
+        if (((live >> i) & 1u) && key[i] > bk) { bk = key[i]; bi = (uint32_t)(lane + 32 * i); }
     float my_val = 0.0f, lmax = 0.0f;
     int my_idx = 0;
     for (int j = 0; j < k; ++j) {
-        uint32_t best = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if ((live >> i) & 1u) best = max(best, key[i]);
-        const uint32_t top = __reduce_max_sync(0xffffffffu, best);
-        uint32_t mine = 0xffffffffu;
-#pragma unroll
-        for (int i = 31; i >= 0; --i)
-            if (((live >> i) & 1u) && key[i] == top) mine = (uint32_t)(lane + 32 * i);
-        const uint32_t e = __reduce_min_sync(0xffffffffu, mine);
-        if ((int)(e & 31u) == lane) live &= ~(1u << (e >> 5));
-        const float v = __uint_as_float((top & 0x80000000u) ? (top & 0x7fffffffu) : ~top);
+        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t e = __reduce_min_sync(0xffffffffu, (bk == top) ? bi : 0xffffffffu);
+        const float v = fkey_value(top);
         if (j == 0) lmax = v;
         if (lane == j) { my_val = v; my_idx = (int)e; }
+        if (bi == e) {                                   // the owner drops it and rescans
+            live &= ~(1u << (e >> 5));
+            bk = 0; bi = 0xffffffffu;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (((live >> i) & 1u) && key[i] > bk) { bk = key[i]; bi = (uint32_t)(lane + 32 * i); }
+        }
     }
     const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
     const float sum = warp_sum(ex);
@@ -143,31 +156,24 @@ MOE_DEV void warp_topk_smem(const float* __restrict__ row, int E, int k, int* id
     }
 }
 
-// Rows of one unit: RB row blocks of 16 rows starting at r0; the 16 warps are
-// (row block rbi = warp % RB) x (K split ks = warp / RB of 16/RB); partials
-// of each warp go to red[warp][NM][16][8].
-template <int Q, int NM, int RB>
-MOE_DEV void unit_gemv(const MatPtr (&mats)[NM], int r0, int K, const __nv_bfloat16* xrow, float* red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, c = lane & 3;
-    const int rbi = warp % RB, ks = warp / RB;
-    const int r = r0 + rbi * 16;
-    const int nb = r / kBlkN, rl = r % kBlkN + g;
-    float acc[NM][4];
-#pragma unroll
-    for (int q = 0; q < NM; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[q][i] = 0.0f;
-    warp_rows<Q, NM>(acc, mats, nb, rl, K / kBlkK, K / kGroup, ks, kFWarps / RB, xrow, c);
-#pragma unroll
-    for (int q = 0; q < NM; ++q) {
-        float* rr = red + ((warp * NM + q) * 16) * 8;
-        rr[g * 8 + 2 * c] = acc[q][0];
-        rr[g * 8 + 2 * c + 1] = acc[q][1];
-        rr[(g + 8) * 8 + 2 * c] = acc[q][2];
-        rr[(g + 8) * 8 + 2 * c + 1] = acc[q][3];
+// Named barrier of one 4-warp group (ids 1..4; 0 is __syncthreads).
+MOE_DEV void group_sync(int group) { asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory"); }
+
+// Tokens of the item whose first slot is s0 (slot order), written by the
+// group's first thread; see item_tokens.
+MOE_DEV int group_item_tokens(const int* __restrict__ ids, int n, int k, int s0, int* tok, int* slot, bool writer) {
+    const int e0 = ids[s0];
+    int c = 0;
+    for (int s = s0; s < n && c < kDecMaxT; ++s) {
+        if (ids[s] == e0) {
+            if (writer) { tok[c] = s / k; slot[c] = s; }
+            ++c;
+        }
     }
+    return c;
 }
+
+constexpr int kGroups = kFWarps / 4;
 
 template <int Q>
 __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
@@ -175,8 +181,9 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
     __shared__ Plan plan;
     __shared__ int ids_s[kDecMaxSlots];
     __shared__ float w_s[kDecMaxSlots];
-    __shared__ int tok[kDecMaxT], slot_of[kDecMaxT], ident[kDecMaxT];
-    __shared__ int s_last;
+    __shared__ int ident[kDecMaxT];
+    __shared__ int g_tok[kGroups][kDecMaxT], g_slot[kGroups][kDecMaxT];
+    __shared__ int g_last[kGroups];
     __shared__ volatile int abort_s;
     const DecodeArgs& a = f.d;
     const ExpertArgs& ex = a.ex;
@@ -184,15 +191,23 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
     const int n = T * k;
     const int ldx = H + kXPad, lda = I + kXPad;
     const bool fp4 = (Q == Q_NVFP4);
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem_raw);                          // [9][ldx] raw x
-    __nv_bfloat16* xq = xs + (size_t)(kDecMaxT + 1) * ldx;                                   // [9][ldx] W4A4 x
-    __nv_bfloat16* as = xq + (size_t)(kDecMaxT + 1) * ldx;                                   // [9][lda]
-    float* red = reinterpret_cast<float*>(as + (size_t)(kDecMaxT + 1) * lda);                 // [16][2][16][8]
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem_raw);                 // [9][ldx] raw x
+    __nv_bfloat16* xq = xs + (size_t)(kDecMaxT + 1) * ldx;                          // [9][ldx] W4A4 x
+    __nv_bfloat16* as0 = xq + (size_t)(kDecMaxT + 1) * ldx;                         // [4][9][lda]
+    float* red0 = reinterpret_cast<float*>(as0 + (size_t)kGroups * (kDecMaxT + 1) * lda);   // [4][4][2][16][8]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int group = warp >> 2, wg = warp & 3;                  // 4-warp group, warp within it
+    const int gtid = threadIdx.x & 127;
+    __nv_bfloat16* as = as0 + (size_t)group * (kDecMaxT + 1) * lda;
+    float* red = red0 + (size_t)group * 4 * 2 * 16 * 8;
+    int* tok = g_tok[group];
+    int* slot_of = g_slot[group];
     if (threadIdx.x == 0) abort_s = 0;
     if (threadIdx.x < kDecMaxT) ident[threadIdx.x] = threadIdx.x;
     __syncthreads();
 
-    // ---- stage activations (rows t < T, rows T..8 zero)
+    // ---- stage activations (rows t < T; rows T..8 zero)
     const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
     stage_rows_bf16(xs, ldx, x, H, ident, T, threadIdx.x, blockDim.x);
     if (fp4) stage_rows_fp4_from_bf16(xq, ldx, x, H, ident, T, ex.g_x, threadIdx.x, blockDim.x);
@@ -201,41 +216,17 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
         reinterpret_cast<uint4*>(xq + kDecMaxT * ldx)[i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2;
 
-    // ---- phase 0: router rows + shared gate/up rows
-    {
-        const int router_units = f.wr ? (E + kFWarps - 1) / kFWarps : 0;
-        const int shared_units = ex.sh_gate ? I / 16 : 0;
-        for (int u = blockIdx.x; u < router_units + shared_units; u += gridDim.x) {
-            if (u < router_units) {
-                const int e = u * kFWarps + warp;
-                if (e < E) router_row(reinterpret_cast<const uint8_t*>(f.wr), e, H, T, xs, ldx, f.logits, E);
-            } else {
-                const int r0 = (u - router_units) * 16;
-                const MatPtr mats[2] = {{ex.sh_gate, nullptr, nullptr}, {ex.sh_up, nullptr, nullptr}};
-                const __nv_bfloat16* xrow = xs + (g < T ? g : kDecMaxT) * ldx;
-                unit_gemv<Q_BF16, 2, 1>(mats, r0, H, xrow, red);
-                __syncthreads();
-                if (threadIdx.x < 16 * kDecMaxT) {
-                    const int row = threadIdx.x / kDecMaxT, t = threadIdx.x % kDecMaxT;
-                    if (t < T) {
-                        float gg = 0.0f, uu = 0.0f;
-                        for (int w = 0; w < kFWarps; ++w) {
-                            gg += red[((w * 2 + 0) * 16 + row) * 8 + t];
-                            uu += red[((w * 2 + 1) * 16 + row) * 8 + t];
-                        }
-                        a.a_sh[(size_t)t * I + r0 + row] = gg / (1.0f + expf(-gg)) * uu;
-                    }
-                }
-                __syncthreads();
-            }
-        }
+    // ---- phase 0: router rows, one per warp, spread over all SMs
+    if (f.wr) {
+        for (int e = warp * gridDim.x + blockIdx.x; e < E; e += kFWarps * gridDim.x)
+            router_row(reinterpret_cast<const uint8_t*>(f.wr), e, H, T, xs, ldx, f.logits, E);
+        if (!grid_barrier(f.bar, f.err, &abort_s)) return;
     }
-    if (f.wr && !grid_barrier(f.bar, f.err, &abort_s)) return;
 
-    // ---- phase 1: top-k (every CTA), plan, routed gate/up rows
+    // ---- phase 1: top-k (every CTA), plan, gate/up of the selected experts
+    //      and of the shared expert; a unit = (expert, 16 rows) on one 4-warp
+    //      group whose warps split K
     if (f.wr) {
         for (int t = warp; t < T; t += kFWarps)
             warp_topk_smem(f.logits + (size_t)t * E, E, k, ids_s + t * k, w_s + t * k);
@@ -268,111 +259,136 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
     }
     __syncthreads();
     const int nu = plan.n_unique;
+    const int nslots = kGroups * gridDim.x;                      // concurrent units in the grid
+    const int my_slot = group * gridDim.x + blockIdx.x;          // spread groups over SMs
     {
-        const int units = nu * (I / 16);
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int ui = u / (I / 16), r0 = (u % (I / 16)) * 16;
-            const int m = item_tokens(plan.ids, n, k, plan.first[ui], tok, slot_of);
-            __syncthreads();
-            const int e = plan.ids[plan.first[ui]];
-            const bool valid = e >= 0 && e < E;
-            const __nv_bfloat16* xb = fp4 ? xq : xs;
-            const __nv_bfloat16* xrow = xb + (g < m ? tok[g] : kDecMaxT) * ldx;
-            if (valid) {
-                const MatPtr mats[2] = {expert_mat(ex.gate, e), expert_mat(ex.up, e)};
-                unit_gemv<Q, 2, 1>(mats, r0, H, xrow, red);
-            }
-            __syncthreads();
-            if (threadIdx.x < 16 * kDecMaxT) {
-                const int row = threadIdx.x / kDecMaxT, t = threadIdx.x % kDecMaxT;
-                if (t < m) {
-                    float gg = 0.0f, uu = 0.0f;
-                    if (valid)
-                        for (int w = 0; w < kFWarps; ++w) {
-                            gg += red[((w * 2 + 0) * 16 + row) * 8 + t];
-                            uu += red[((w * 2 + 1) * 16 + row) * 8 + t];
-                        }
-                    const float sc = (fp4 && valid) ? ex.g_gate[e] * ex.g_x : 1.0f;
-                    gg *= sc;
-                    uu *= sc;
-                    a.a[(size_t)slot_of[t] * I + r0 + row] = gg / (1.0f + expf(-gg)) * uu;
-                }
-            }
-            __syncthreads();
-        }
-    }
-    if (!grid_barrier(f.bar, f.err, &abort_s)) return;
-
-    // ---- phase 2: down rows (128 per unit: 8 row blocks x 2 K halves) + combine
-    {
-        constexpr int RB = 8;
-        const int rb128 = H / 128;
-        const int items_per_rb = nu + (ex.sh_down ? 1 : 0);
-        const int units = items_per_rb * rb128;
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int ui = u / rb128, hb = u % rb128, h0 = hb * 128;
+        const int per = I / 16;
+        const int units = (nu + (ex.sh_gate ? 1 : 0)) * per;
+        for (int u = my_slot; u < units; u += nslots) {
+            const int ui = u / per, r0 = (u % per) * 16;
             const bool is_shared = (ui == nu);
             int m, e = 0;
             if (is_shared) {
                 m = T;
-                if (threadIdx.x < kDecMaxT) { tok[threadIdx.x] = threadIdx.x; slot_of[threadIdx.x] = threadIdx.x; }
+                if (gtid < kDecMaxT) { tok[gtid] = gtid; slot_of[gtid] = gtid; }
             } else {
-                m = item_tokens(plan.ids, n, k, plan.first[ui], tok, slot_of);
+                m = group_item_tokens(plan.ids, n, k, plan.first[ui], tok, slot_of, gtid == 0);
                 e = plan.ids[plan.first[ui]];
             }
-            __syncthreads();
+            group_sync(group);
             const bool valid = is_shared || (e >= 0 && e < E);
-            stage_rows_f32(as, lda, is_shared ? a.a_sh : a.a, I, slot_of, m, fp4 && !is_shared, ex.g_a, threadIdx.x,
-                           blockDim.x);
-            __syncthreads();
-            const __nv_bfloat16* xrow = as + (g < m ? g : kDecMaxT) * lda;
+            const __nv_bfloat16* xb = (fp4 && !is_shared) ? xq : xs;
+            const __nv_bfloat16* xrow = xb + (g < m ? tok[g] : kDecMaxT) * ldx;
+            const int nb = r0 / kBlkN, rl = r0 % kBlkN + g;
+            float acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
             if (is_shared) {
-                const MatPtr mats[1] = {{ex.sh_down, nullptr, nullptr}};
-                unit_gemv<Q_BF16, 1, RB>(mats, h0, I, xrow, red);
+                const MatPtr mats[2] = {{ex.sh_gate, nullptr, nullptr}, {ex.sh_up, nullptr, nullptr}};
+                warp_rows<Q_BF16, 2>(acc, mats, nb, rl, H / kBlkK, H / kGroup, wg, 4, xrow, c);
             } else if (valid) {
-                const MatPtr mats[1] = {expert_mat(ex.down, e)};
-                unit_gemv<Q, 1, RB>(mats, h0, I, xrow, red);
+                const MatPtr mats[2] = {expert_mat(ex.gate, e), expert_mat(ex.up, e)};
+                warp_rows<Q, 2>(acc, mats, nb, rl, H / kBlkK, H / kGroup, wg, 4, xrow, c);
             }
-            __syncthreads();
-            const float dscale = (fp4 && !is_shared && valid) ? ex.g_down[e] * ex.g_a : 1.0f;
-            for (int i = threadIdx.x; i < 128 * kDecMaxT; i += blockDim.x) {
-                const int row = i / kDecMaxT, t = i % kDecMaxT;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float* rr = red + ((wg * 2 + q) * 16) * 8;
+                rr[g * 8 + 2 * c] = acc[q][0];
+                rr[g * 8 + 2 * c + 1] = acc[q][1];
+                rr[(g + 8) * 8 + 2 * c] = acc[q][2];
+                rr[(g + 8) * 8 + 2 * c + 1] = acc[q][3];
+            }
+            group_sync(group);
+            {
+                const int row = gtid / kDecMaxT, t = gtid % kDecMaxT;   // 128 = 16 rows x 8 tokens
                 if (t < m) {
-                    const int rbi = row / 16, rr = row % 16;
-                    float o = 0.0f;
-                    if (valid)
-                        for (int ks = 0; ks < kFWarps / RB; ++ks) o += red[((ks * RB + rbi) * 16 + rr) * 8 + t];
-                    o *= dscale;
-                    const int h = h0 + row;
-                    if (is_shared) a.part_sh[(size_t)t * H + h] = o;
-                    else a.part[(size_t)slot_of[t] * H + h] = w_s[slot_of[t]] * o;
+                    float gg = 0.0f, uu = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        gg += red[((w * 2 + 0) * 16 + row) * 8 + t];
+                        uu += red[((w * 2 + 1) * 16 + row) * 8 + t];
+                    }
+                    const float sc = (fp4 && !is_shared && valid) ? ex.g_gate[e] * ex.g_x : 1.0f;
+                    gg *= sc;
+                    uu *= sc;
+                    const float act = valid ? gg / (1.0f + expf(-gg)) * uu : 0.0f;
+                    if (is_shared) a.a_sh[(size_t)t * I + r0 + row] = act;
+                    else a.a[(size_t)slot_of[t] * I + r0 + row] = act;
                 }
             }
-            // the last unit of this 128-row block to finish sums the slots
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                __threadfence();
-                s_last = (atomicAdd(a.counters + hb, 1u) == (unsigned)items_per_rb - 1u);
-                if (s_last) __threadfence();
+            group_sync(group);
+        }
+    }
+    if (!grid_barrier(f.bar, f.err, &abort_s)) return;
+
+    // ---- phase 2: down; a unit = (expert, 64 rows) on one group, each warp
+    //      16 rows over the whole K; the last unit of a 64-row block combines
+    {
+        const int per = H / 64;
+        const int items_per_rb = nu + (ex.sh_down ? 1 : 0);
+        const int units = items_per_rb * per;
+        for (int u = my_slot; u < units; u += nslots) {
+            const int ui = u / per, hb = u % per, h0 = hb * 64;
+            const bool is_shared = (ui == nu);
+            int m, e = 0;
+            if (is_shared) {
+                m = T;
+                if (gtid < kDecMaxT) { tok[gtid] = gtid; slot_of[gtid] = gtid; }
+            } else {
+                m = group_item_tokens(plan.ids, n, k, plan.first[ui], tok, slot_of, gtid == 0);
+                e = plan.ids[plan.first[ui]];
             }
-            __syncthreads();
-            if (s_last) {
+            group_sync(group);
+            const bool valid = is_shared || (e >= 0 && e < E);
+            stage_rows_f32(as, lda, is_shared ? a.a_sh : a.a, I, slot_of, m, fp4 && !is_shared, ex.g_a, gtid, 128);
+            group_sync(group);
+            const __nv_bfloat16* xrow = as + (g < m ? g : kDecMaxT) * lda;
+            const int r = h0 + wg * 16;
+            const int nb = r / kBlkN, rl = r % kBlkN + g;
+            float acc[1][4] = {{0, 0, 0, 0}};
+            if (is_shared) {
+                const MatPtr mats[1] = {{ex.sh_down, nullptr, nullptr}};
+                warp_rows<Q_BF16, 1>(acc, mats, nb, rl, I / kBlkK, I / kGroup, 0, 1, xrow, c);
+            } else if (valid) {
+                const MatPtr mats[1] = {expert_mat(ex.down, e)};
+                warp_rows<Q, 1>(acc, mats, nb, rl, I / kBlkK, I / kGroup, 0, 1, xrow, c);
+            }
+            // this warp owns rows r..r+15 completely: write the partials
+            const float dscale = (fp4 && !is_shared && valid) ? ex.g_down[e] * ex.g_a : 1.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = r + g + (i >= 2 ? 8 : 0), t = 2 * c + (i & 1);
+                if (t < m) {
+                    const float o = valid ? acc[0][i] * dscale : 0.0f;
+                    if (is_shared) a.part_sh[(size_t)t * H + row] = o;
+                    else a.part[(size_t)slot_of[t] * H + row] = w_s[slot_of[t]] * o;
+                }
+            }
+            group_sync(group);
+            if (gtid == 0) {
+                __threadfence();
+                g_last[group] = (atomicAdd(a.counters + hb, 1u) == (unsigned)items_per_rb - 1u);
+                if (g_last[group]) __threadfence();
+            }
+            group_sync(group);
+            if (g_last[group]) {
                 __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.y);
-                for (int i = threadIdx.x; i < T * 128; i += blockDim.x) {
-                    const int t = i / 128, hh = h0 + i % 128;
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = (j < k) ? __ldcg(a.part + (size_t)(t * k + j) * H + hh) : 0.0f;
+                for (int i = gtid; i < T * 64; i += 128) {
+                    const int t = i / 64, hh = h0 + i % 64;
                     float sum = 0.0f;
+                    for (int j0 = 0; j0 < k; j0 += 8) {                // fixed order j = 0 .. k-1
+                        float v[8];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) sum += v[j];          // fixed order j = 0 .. k-1
+                        for (int j = 0; j < 8; ++j)
+                            v[j] = (j0 + j < k) ? __ldcg(a.part + (size_t)(t * k + j0 + j) * H + hh) : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) sum += v[j];
+                    }
                     if (ex.sh_down) sum += __ldcg(a.part_sh + (size_t)t * H + hh);
                     y[(size_t)t * H + hh] = __float2bfloat16_rn(sum);
                 }
-                __syncthreads();
-                if (threadIdx.x == 0) a.counters[hb] = 0u;
+                group_sync(group);
+                if (gtid == 0) a.counters[hb] = 0u;
             }
-            __syncthreads();
+            group_sync(group);
         }
     }
 }
@@ -380,7 +396,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
 size_t fused_smem_bytes(int H, int I) {
     const size_t xbuf = (size_t)(kDecMaxT + 1) * (H + kXPad) * 2;
     const size_t abuf = (size_t)(kDecMaxT + 1) * (I + kXPad) * 2;
-    return 2 * xbuf + abuf + (size_t)kFWarps * 2 * 16 * 8 * sizeof(float);
+    return 2 * xbuf + kGroups * abuf + (size_t)kFWarps * 2 * 16 * 8 * sizeof(float);
 }
 
 template <int Q>

@@ -16,9 +16,10 @@
 //   * persistent CTAs (one per SM) walk a tile list built on the device from
 //     the permutation, grouped by (expert, row block) so consecutive CTAs
 //     reuse the same weight tile from L2;
+//   * the token operand is stored in permuted (expert-major) order before the
+//     GEMMs, so each k-block of a tile is one 2D TMA box of 128 rows;
 //   * warp roles: a producer warp issues bulk copies of the packed weights
-//     and TMA loads of the token rows (tile::gather4 from x for gate/up, 2D
-//     tiles of the permuted intermediate for down); four dequant warps turn
+//     and the TMA loads of the token rows; four dequant warps turn
 //     INT4 / INT2 / NVFP4 codes into bf16 A tiles in the 128-byte swizzle the
 //     MMA reads; one thread issues tcgen05.mma (kind::f16, fp32 accumulators
 //     in TMEM, double buffered); four epilogue warps read TMEM and apply
@@ -204,6 +205,9 @@ MOE_DEV void stage_bytes(int quant, int& codes, int& scales, int& zeros) {
     zeros = quant == Q_INT2 ? 128 : 0;
 }
 
+// named barrier of the four epilogue warps
+MOE_DEV void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 // ------------------------------------------------------------------ kernel
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -216,7 +220,9 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
     __shared__ uint64_t wfull[S], full[S], empty[S], acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
-    __shared__ int rows[kBN];                   // producer: B row of each tile column
+    __shared__ float ep_scale[kBN];             // epilogue: per token column of the current tile
+    __shared__ int ep_row[kBN];
+    __shared__ int ep_stop;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -246,15 +252,6 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
         for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x) {
             const GemmTile t = a.tiles[ti];
             const bool shared = t.expert < 0;
-            const int n_mma = (t.count + 15) & ~15;
-            __syncwarp();
-            if (MODE == 0) {
-                for (int i = lane; i < n_mma; i += 32) {
-                    const int c = min(i, t.count - 1);
-                    rows[i] = shared ? t.seg + c : __ldg(a.perm + t.seg + c) / a.k_top;
-                }
-            }
-            __syncwarp();
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
@@ -263,7 +260,7 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                     uint8_t* A = smem + L::A + s * NMAT * kATile;
                     uint8_t* B = smem + L::B + s * kBTile;
                     uint8_t* stg = smem + L::STG + s * NMAT * kStgMat;
-                    const uint32_t b_bytes = (MODE == 0 ? (uint32_t)n_mma : (uint32_t)kBN) * 128u;
+                    const uint32_t b_bytes = kBTile;   // a whole box; rows past the end read as zero
                     if (shared) {
                         mbar_arrive(&wfull[s]);                       // nothing to dequantize
                         mbar_arrive_expect_tx(&full[s], b_bytes + NMAT * kATile);
@@ -292,14 +289,9 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                         }
                         mbar_arrive_expect_tx(&full[s], b_bytes);
                     }
-                    if (MODE == 0) {
-                        const CUtensorMap* map = shared ? &map_shared : &map_routed;
-                        for (int i = 0; i < n_mma; i += 4)
-                            tma_gather4(B + i * 128, map, kb * kBlkK, rows[i], rows[i + 1], rows[i + 2], rows[i + 3],
-                                        &full[s]);
-                    } else {
-                        tma_load_2d(B, shared ? &map_shared : &map_routed, kb * kBlkK, t.seg, &full[s]);
-                    }
+                    // token rows t.seg .. t.seg + 127 of the permuted operand
+                    // (shared tiles: of x / the shared intermediate)
+                    tma_load_2d(B, shared ? &map_shared : &map_routed, kb * kBlkK, t.seg, &full[s]);
                 }
                 __syncwarp();
             }
@@ -371,17 +363,43 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
         // ----------------------------------------------------------- epilogue
         const int lane_base = (warp & 3) * 32;
         const int row = lane_base + lane;                    // weight row within the block
+        const int ej = threadIdx.x - kWarpEpi0 * 32;         // 0..127: token column this thread looks up
+        // The four warps leave the loop together (named barriers): the stop
+        // decision is taken by one thread between two barriers.
         int local = 0;
-        for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x, ++local) {
+        for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x, ++local) {
             const GemmTile t = a.tiles[ti];
             const bool shared = t.expert < 0;
             const int ab = local & 1;
-            if (!mbar_wait(&acc_full[ab], (uint32_t)(local >> 1) & 1u, &abort_flag, a.err, 5)) break;
+            float gsc = 1.0f;
+            if (!shared && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
+            // token columns of the tile: scale (mode 0) or routing weight
+            // (mode 1) and output row, looked up once per tile
+            epi_sync();                                      // the previous tile's readers are done
+            if (ej == 0) ep_stop = abort_flag;
+            if (ej < t.count) {
+                if (shared) {
+                    ep_scale[ej] = gsc;
+                    ep_row[ej] = t.seg + ej;
+                } else {
+                    const int slot = __ldg(a.perm + t.seg + ej);
+                    if (MODE == 0) {
+                        ep_scale[ej] = a.tok_scale ? __ldg(a.tok_scale + slot / a.k_top) : gsc;
+                        ep_row[ej] = t.seg + ej;
+                    } else {
+                        ep_scale[ej] = gsc * __ldg(a.topk_w + slot);
+                        ep_row[ej] = slot;
+                    }
+                }
+            }
+            epi_sync();
+            if (ep_stop) break;
+            // a failed wait sets abort_flag: this tile is skipped and all four
+            // warps stop at the next tile's decision
+            if (!mbar_wait(&acc_full[ab], (uint32_t)(local >> 1) & 1u, &abort_flag, a.err, 5)) continue;
             tc_fence_after();
             const int n_mma = (t.count + 15) & ~15;
             const int col_out = t.rb * kBlkN + row;
-            float gsc = 1.0f;
-            if (!shared && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
             for (int c0 = 0; c0 < n_mma; c0 += 16) {
                 const uint32_t taddr = tmem + ((uint32_t)lane_base << 16) + ab * 256 + c0;
                 float v0[16];
@@ -389,11 +407,11 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                 if (MODE == 0) {
                     float v1[16];
                     tmem_ld16(taddr + 128, v1);
+                    __nv_bfloat16* dst = shared ? a.out_sh : a.out;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        float tsc = gsc;
-                        if (!shared && a.tok_scale && c0 + i < t.count)
-                            tsc = __ldg(a.tok_scale + __ldg(a.perm + t.seg + c0 + i) / a.k_top);
+                        const int col = c0 + i;
+                        const float tsc = col < t.count ? ep_scale[col] : 0.0f;
                         const float gg = v0[i] * tsc, uu = v1[i] * tsc;
                         float act = gg / (1.0f + expf(-gg)) * uu;
                         if (!shared && a.quant == Q_NVFP4) {
@@ -409,28 +427,17 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
                             }
                             act = e2m1_to_f32(f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu) * sbv;
                         }
-                        const int col = c0 + i;
-                        if (col < t.count) {
-                            const size_t orow = (size_t)t.seg + col;
-                            __nv_bfloat16* dst = shared ? a.out_sh : a.out;
-                            dst[orow * a.out_ld + col_out] = __float2bfloat16_rn(act);
-                        }
+                        if (col < t.count) dst[(size_t)ep_row[col] * a.out_ld + col_out] = __float2bfloat16_rn(act);
                     }
                 } else {
                     // per-slot outputs are fp16 (saturating at +-65504): their
                     // rounding error stays well below the final bf16 one
+                    __half* dst = shared ? a.o16_sh : a.o16;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int col = c0 + i;
-                        if (col < t.count) {
-                            if (shared) {
-                                a.o16_sh[((size_t)t.seg + col) * a.out_ld + col_out] = f16_sat(v0[i]);
-                            } else {
-                                const int slot = __ldg(a.perm + t.seg + col);
-                                const float o = v0[i] * gsc * __ldg(a.topk_w + slot);
-                                a.o16[(size_t)slot * a.out_ld + col_out] = f16_sat(o);
-                            }
-                        }
+                        if (col < t.count)
+                            dst[(size_t)ep_row[col] * a.out_ld + col_out] = f16_sat(v0[i] * ep_scale[col]);
                     }
                 }
             }
@@ -557,6 +564,18 @@ __global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, int T, int H, __
     if (lane == 0) scale[t] = ldexpf(1.0f, p);
 }
 
+// Rows of the gate/up token operand in permuted order: xp[p] = xq[perm[p] / k]
+// (16-byte copies; one thread per 8 columns).
+__global__ void k_gather_rows(const __nv_bfloat16* __restrict__ xq, const int32_t* __restrict__ perm, int slots,
+                              int H, int k, __nv_bfloat16* __restrict__ xp) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_row = H / 8;
+    if (i >= (long long)slots * per_row) return;
+    const int p = (int)(i / per_row), c = (int)(i % per_row);
+    const int t = __ldg(perm + p) / k;
+    reinterpret_cast<uint4*>(xp + (size_t)p * H)[c] = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)t * H) + c);
+}
+
 // NVFP4 activations: x -> bf16 values q * s_b (the global scale is applied in
 // the GEMM epilogue); one thread per 16-element block.
 __global__ void k_act_fp4_values(const __nv_bfloat16* __restrict__ x, int T, int H, float g,
@@ -639,7 +658,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st);
     if (err != cudaSuccess) return err;
     const bool fp4 = ex.quant == Q_NVFP4;
-    const void* xin = p.x;
+    const __nv_bfloat16* xin = nullptr;
     CUtensorMapDataType xdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (fp4) {
         const long long nblk = (long long)T * (H / kFp4Blk);
@@ -652,11 +671,15 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
         xin = p.xq;
         xdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     }
+    {
+        const long long n8 = (long long)slots * (H / 8);
+        k_gather_rows<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xin, p.perm, slots, H, k, p.xp);
+    }
     const bool has_sh = ex.sh_gate != nullptr;
     CUtensorMap m_routed, m_shared;
     // ---- gate / up
-    if (!make_map(&m_routed, xin, (uint64_t)T, (uint64_t)H, 1, xdt) ||
-        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, 1))
+    if (!make_map(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, kBN, xdt) ||
+        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, kBN))
         return cudaErrorInvalidValue;
     k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
     GemmArgs g{};
@@ -681,9 +704,11 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const int grid = num_sms();
     err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<0>::ALLOC);
     if (err != cudaSuccess) return err;
+    if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
     k_grouped_gemm<0><<<grid, kGemmThreads, SmemLayout<0>::ALLOC, st>>>(m_routed, m_shared, g);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
+    if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
     if (!make_map(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I, kBN) ||
         !make_map(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I, kBN))
@@ -705,9 +730,11 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.tok_scale = nullptr;
     err = cudaFuncSetAttribute(k_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<1>::ALLOC);
     if (err != cudaSuccess) return err;
+    if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
     k_grouped_gemm<1><<<grid, kGemmThreads, SmemLayout<1>::ALLOC, st>>>(m_routed, m_shared, g);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
+    if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     // ---- combine
     const long long threads = (long long)T * (H / 8);
     k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, T, H, k,

@@ -79,7 +79,7 @@ struct FusedArgs {
     float* logits;                 // workspace [T, E]
     int32_t* ids_out;              // [T, k] (when wr is set)
     float* w_out;                  // [T, k]
-    unsigned int* bar;             // workspace {arrivals, generation}, zero-initialised
+    unsigned long long* bar;       // workspace: monotonically increasing arrival count, zero-initialised
     int* err;                      // device error word
 };
 size_t fused_smem_bytes(int H, int I);
@@ -104,11 +104,15 @@ struct PrefillArgs {
     int* num_tiles;
     __nv_bfloat16* xq;             // [T, H]: NVFP4 W4A4 activation values, else fp16 scaled x
     float* tok_scale;              // [T]: power of two of each token's fp16 activations
+    __nv_bfloat16* xp;             // [T*k, H]: rows of xq in permuted (expert-major) order
     __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order
     __nv_bfloat16* a_sh;           // [T, I] shared-expert intermediate
     __half* o;                     // [T*k, H] weighted expert outputs by slot (fp16)
     __half* o_sh;                  // [T, H] shared-expert output (fp16)
     int* err;                      // device error word (bounded waits)
+    // profiling events (may be null): before / after the gate-up grouped
+    // GEMM, before / after the down grouped GEMM
+    cudaEvent_t ev_gu0, ev_gu1, ev_dn0, ev_dn1;
 };
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I);
 cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st);

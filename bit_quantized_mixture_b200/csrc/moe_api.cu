@@ -13,6 +13,8 @@
 
 using namespace moe;
 
+constexpr int kProfEvents = 8;   // see moe_set_profile_events
+
 struct moe_layer {
     moe_config cfg;
     // arena
@@ -36,7 +38,7 @@ struct moe_layer {
     float* dec_part = nullptr;     // [8*k, H]
     float* dec_part_sh = nullptr;  // [8, H]
     unsigned int* dec_counters = nullptr;   // [H/16]
-    unsigned int* fused_bar = nullptr;      // {arrivals, generation} of the fused decode kernel
+    unsigned long long* fused_bar = nullptr;   // arrival count of the fused decode kernel's grid barrier
     uint8_t* staging = nullptr;    // interchange copy of one matrix
     size_t staging_bytes = 0;
     // prefill path
@@ -44,7 +46,7 @@ struct moe_layer {
     GemmTile* tiles = nullptr;
     int* num_tiles = nullptr;
     int* dev_err = nullptr;
-    __nv_bfloat16 *xq = nullptr, *a_perm = nullptr, *a_sh = nullptr;
+    __nv_bfloat16 *xq = nullptr, *xp = nullptr, *a_perm = nullptr, *a_sh = nullptr;
     __half *o = nullptr, *o_sh = nullptr;
     float* tok_scale = nullptr;
     // state
@@ -55,7 +57,7 @@ struct moe_layer {
     float* g_host = nullptr;          // host copies of the NVFP4 global scales, [2E]
     float g_x = 0.0f, g_a = 0.0f;
     bool act_scales_set = false;
-    cudaEvent_t prof[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    cudaEvent_t prof[kProfEvents] = {};
     char err[512] = {0};
 };
 
@@ -171,7 +173,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_part = carve(sizeof(float) * (size_t)MT * k * H);
     const size_t o_psh = carve(sizeof(float) * (size_t)MT * H);
     const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 16));
-    const size_t o_fbar = carve(sizeof(unsigned int) * 2);
+    const size_t o_fbar = carve(sizeof(unsigned long long));
     h->staging_bytes = (size_t)2 * H * I + 65536;
     const size_t o_stage = carve(h->staging_bytes);
     const size_t Tm = (size_t)c.max_tokens, slots = Tm * k;
@@ -185,6 +187,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_err = carve(sizeof(int));
     const size_t o_xq = carve(Tm * H * 2);
     const size_t o_tsc = carve(Tm * sizeof(float));
+    const size_t o_xp = carve(slots * H * 2);
     const size_t o_aperm = carve(slots * I * 2);
     const size_t o_ash16 = carve(c.has_shared ? Tm * I * 2 : 0);
     const size_t o_o = carve(slots * H * 2);
@@ -203,7 +206,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->dec_part = reinterpret_cast<float*>(h->ws + o_part);
     h->dec_part_sh = reinterpret_cast<float*>(h->ws + o_psh);
     h->dec_counters = reinterpret_cast<unsigned int*>(h->ws + o_cnt);
-    h->fused_bar = reinterpret_cast<unsigned int*>(h->ws + o_fbar);
+    h->fused_bar = reinterpret_cast<unsigned long long*>(h->ws + o_fbar);
     h->staging = h->ws + o_stage;
     h->counts = reinterpret_cast<int32_t*>(h->ws + o_counts);
     h->offsets = reinterpret_cast<int32_t*>(h->ws + o_offsets);
@@ -215,6 +218,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
     h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
     h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
+    h->xp = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xp);
     h->a_perm = reinterpret_cast<__nv_bfloat16*>(h->ws + o_aperm);
     h->a_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_ash16);
     h->o = reinterpret_cast<__half*>(h->ws + o_o);
@@ -452,9 +456,10 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
         p.perm_scratch = h->perm_scratch;
         p.tiles = h->tiles; p.num_tiles = h->num_tiles;
-        p.xq = h->xq; p.tok_scale = h->tok_scale;
+        p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
+        p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_prefill(p, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_forward (grouped GEMM path)");
@@ -561,7 +566,7 @@ moe_status moe_sync_status(moe_handle h, moe_stream_t stream) {
         const int zero = 0;
         cudaMemcpy(h->dev_err, &zero, sizeof(int), cudaMemcpyHostToDevice);
         cudaMemset(h->dec_counters, 0, sizeof(unsigned int) * (size_t)(h->cfg.hidden / 16));
-        cudaMemset(h->fused_bar, 0, sizeof(unsigned int));
+        cudaMemset(h->fused_bar, 0, sizeof(unsigned long long));
         return fail(h, MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (site %d); outputs are invalid", code);
     }
     return MOE_OK;
@@ -569,8 +574,8 @@ moe_status moe_sync_status(moe_handle h, moe_stream_t stream) {
 
 moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n) {
     if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_set_profile_events: null handle");
-    if (events && n < 5) return fail(h, MOE_ERR_INVALID_ARG, "moe_set_profile_events: need 5 events");
-    for (int i = 0; i < 5; ++i) h->prof[i] = events ? (cudaEvent_t)events[i] : nullptr;
+    if (events && n < 5) return fail(h, MOE_ERR_INVALID_ARG, "moe_set_profile_events: need at least 5 events");
+    for (int i = 0; i < kProfEvents; ++i) h->prof[i] = (events && i < n) ? (cudaEvent_t)events[i] : nullptr;
     return MOE_OK;
 }
 

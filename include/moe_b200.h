@@ -223,14 +223,20 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
                                    void* codes, void* scales, void* zeros,
                                    float* global_scale_out, moe_stream_t stream);
 
-/* Profiling aid: when events != NULL, every later moe_route records
- * events[0] before and events[1] after its kernels, and every later
- * moe_forward records events[2] before the expert kernels, events[3] between
- * the gate/up and the down kernel (decode path) and events[4] after the last
- * kernel, all on the call's stream.  events are cudaEvent_t handles created
- * by the caller (n >= 5); NULL turns recording off.  Recording an event
- * between two kernels removes their launch overlap, so time the layer itself
- * with recording off. */
+/* Profiling aid: when events != NULL, every later call records, on its
+ * stream, the events of the slots it has:
+ *   [0] before and [1] after the routing kernels of moe_route;
+ *   [2] before the expert kernels and [4] after the last kernel of
+ *       moe_forward and moe_route_forward (the fused decode kernel takes
+ *       [0] and [4] for moe_route_forward);
+ *   [3] decode, two-kernel path: between the gate/up and the down kernel;
+ *       grouped-GEMM path: after the gate/up grouped GEMM;
+ *   [5] / [6] / [7] grouped-GEMM path only: before the gate/up grouped GEMM,
+ *       before the down grouped GEMM, after the down grouped GEMM.
+ * events are cudaEvent_t handles created by the caller; n >= 5 of them are
+ * read (slots n..7 are not recorded); NULL turns recording off.  Recording
+ * an event between two kernels removes their launch overlap, so time the
+ * layer itself with recording off. */
 moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n);
 
 /* Synchronize `stream` and report device-side failures of earlier calls on
