@@ -518,7 +518,7 @@ def run_prefill(args, wl, dev, rank, world):
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
-        "launches_per_step": 12, "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
+        "launches_per_step": 13 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
         "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
         "dtype": "bf16" if wl.quant == "nvfp4" else "f16",
     }

@@ -91,4 +91,37 @@ MOE_DEV uint4 ldg_stream_v4(const void* p) {   // read once: do not keep in L1
 MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 MOE_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ------------------------------------------------ packed codes -> bf16x2
+// Exact conversions of two codes of a packed word into a bf16 pair (low
+// half = the first column), shared by the GEMV and the grouped GEMM.
+MOE_DEV uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t bf16x2_splat(float v) {
+    const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+    return h | (h << 16);
+}
+// INT4 pair j of a word: bf16x2 (u - 8), exact
+MOE_DEV uint32_t int4_pair(uint32_t w, int j) {
+    return hsub2_bits(((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u, 0x43084308u);   // (128+u) - 136
+}
+// INT2 pair j of a word: bf16x2 (u - z), exact; off = bf16x2(128 + z)
+MOE_DEV uint32_t int2_pair(uint32_t w, int j, uint32_t off) {
+    return hsub2_bits(((w >> (2 * j)) & 0x00030003u) | 0x43004300u, off);
+}
+// E2M1 pair j of a word times the block scale (bf16x2 splat), exact:
+// the codes placed at bf16 bits [8:6] (magnitude) and 15 (sign) read as
+// e2m1 * 2^-126; one multiply by 2^126 and one by the scale.
+MOE_DEV uint32_t fp4_pair(uint32_t w, int j, uint32_t sb2) {
+    const uint32_t t = w >> (4 * j);
+    const uint32_t b = ((t & 0x00070007u) << 6) | ((t & 0x00080008u) << 12);
+    return hmul2_bits(hmul2_bits(b, 0x7E807E80u), sb2);       // 0x7E80 = 2^126
+}
+
+
 }  // namespace moe

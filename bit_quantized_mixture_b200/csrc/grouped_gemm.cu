@@ -37,26 +37,62 @@ namespace moe {
 using namespace sm100;
 
 constexpr int kBN = 128;            // tokens per tile (MMA N <= 128)
-constexpr int kGemmThreads = 320;   // 10 warps
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpDeq0 = 2, kWarpEpi0 = 6;
+constexpr int kEpiWarps = 8;        // two warps per TMEM lane quarter, 64 token columns each
+constexpr int kWarpProducer = 0, kWarpMma = 1;   // gate/up: warps 1 and 2 issue the MMAs
 constexpr uint32_t kTmemCols = 512;
 
-template <int MODE> struct GemmCfg;
-template <> struct GemmCfg<0> { static constexpr int NMAT = 2, STAGES = 3; };   // gate + up
-template <> struct GemmCfg<1> { static constexpr int NMAT = 1, STAGES = 4; };   // down
+constexpr int kATile = kBlkN * 128;          // 16 KB: 128 rows x 64 16-bit
+constexpr int kBTile = kBN * 128;            // 16 KB: 128 tokens x 64 16-bit
+constexpr int kOutTile = kBN * kBlkN * 2;    // 32 KB: epilogue staging, [token][128] 16-bit
 
-constexpr int kATile = kBlkN * 128;          // 16 KB: 128 rows x 64 bf16
-constexpr int kBTile = kBN * 128;            // 16 KB: 128 tokens x 64 bf16
-constexpr int kStgMat = 4096 + 512 + 256;    // packed codes + scales + zeros of one matrix block
-
-template <int MODE>
-struct SmemLayout {
-    static constexpr int NMAT = GemmCfg<MODE>::NMAT, S = GemmCfg<MODE>::STAGES;
-    static constexpr int A = 0;                                  // [S][NMAT][16 KB]
-    static constexpr int B = A + S * NMAT * kATile;              // [S][16 KB]
-    static constexpr int STG = B + S * kBTile;                   // [S][NMAT][kStgMat]
-    static constexpr int BYTES = STG + S * NMAT * kStgMat;
-    static constexpr int ALLOC = BYTES + 1024;                   // slack for 1024-byte alignment
+// MODE 0: gate + up (two matrices, SwiGLU epilogue); MODE 1: down; MODE 2:
+// the router logits x . Wr^T (fp32 out, A = Wr rows by TMA, no tile list).
+// SH = false: routed tiles, packed weights dequantized into TMEM (the MMA
+// reads A from TMEM); SH = true: shared-expert tiles, bf16 weight images in
+// shared memory (the MMA reads A from shared memory).
+template <int MODE, bool SH>
+struct Cfg {
+    static constexpr int NMAT = MODE == 0 ? 2 : 1;
+    // k-blocks (64 columns) per pipeline stage: routed stages cover 128
+    // columns, which halves the barrier round trips, commits and dequant
+    // hand-offs per MMA (a single thread issues every MMA of a matrix, and
+    // its per-instruction cost, not the tensor pipe, bounds small tiles)
+    static constexpr int KSTEP = SH ? 1 : 2;
+    static constexpr int S = SH ? (MODE == 0 ? 3 : 4) : (MODE == 0 ? 2 : 4);
+    // one MMA-issuing warp per matrix: gate and up accumulate independently
+    static constexpr int MMA_WARPS = NMAT;
+    static constexpr int DEQ0 = kWarpMma + MMA_WARPS;                 // first dequant warp
+    // dequant warps: groups of 4 * NMAT (one warp per TMEM lane quarter and
+    // matrix, one thread per weight row) take turns over the stages, so that
+    // DEQ_GROUPS stages are converted at once and the fixed latency of a
+    // stage (staged codes in, TMEM stores out) overlaps; a stage always
+    // belongs to the same group (S % DEQ_GROUPS == 0), which keeps the
+    // mbarrier parities unambiguous
+    static constexpr int DEQ_WARPS = SH ? 0 : 8 * NMAT;
+    static constexpr int DEQ_GROUP_WARPS = 4 * NMAT;
+    static constexpr int DEQ_GROUPS = SH ? 1 : DEQ_WARPS / DEQ_GROUP_WARPS;
+    static constexpr int EPI0 = DEQ0 + DEQ_WARPS;                    // first epilogue warp
+    static constexpr int THREADS = (EPI0 + kEpiWarps) * 32;
+    // accumulators: NMAT x 128 columns per buffer; routed gate/up keeps one
+    // buffer so that its A stages fit in the 512 columns
+    static constexpr int ACC_BUFS = (SH || MODE == 1) ? 2 : 1;
+    static constexpr int ACC_COLS = NMAT * kBN;
+    static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;   // TMEM column of A stage 0 (routed)
+    static constexpr int A_STAGE_COLS = NMAT * KSTEP * 32;
+    static_assert(SH || A_COL0 + S * A_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
+    static_assert(SH || S % DEQ_GROUPS == 0, "a stage belongs to one dequant group");
+    // staged packed bytes of one matrix and stage: KSTEP blocks of codes,
+    // then the scales (INT4/INT2: the one 128-column group; NVFP4: KSTEP x
+    // 512), then the INT2 zero points
+    static constexpr int STG_MAT = KSTEP * 4096 + KSTEP * 512;
+    // shared memory
+    static constexpr int A = 0;                                           // SH: [S][NMAT][16 KB]
+    static constexpr int B = A + (SH ? S * NMAT * kATile : 0);            // [S][KSTEP][16 KB]
+    static constexpr int STG = B + S * KSTEP * kBTile;                    // routed: [S][NMAT][STG_MAT]
+    static constexpr int OUT = STG + (SH ? 0 : S * NMAT * STG_MAT);       // [128][128] 16-bit
+    static constexpr int BYTES = OUT + (MODE == 2 ? 0 : kOutTile);
+    static constexpr int ALLOC = BYTES + 1024;                            // slack for 1024-byte alignment
+    static_assert(ALLOC <= 227 * 1024 - 2048, "shared memory budget");
 };
 
 struct GemmArgs {
@@ -66,7 +102,7 @@ struct GemmArgs {
     const uint8_t* sh1;
     const int32_t* perm;      // slot at each permuted position
     const GemmTile* tiles;
-    const int* num_tiles;
+    const int* num_tiles;     // [0]: routed tiles, [1]: all tiles (shared ones last)
     int K;                    // reduction length (H or I)
     int k_top;
     int out_ld;               // row length of the outputs (I or H)
@@ -79,142 +115,142 @@ struct GemmArgs {
     float g_act;              // NVFP4 activation global scale of the B operand
     float g_req;              // NVFP4: global scale of the requantized intermediate (mode 0)
     const float* tok_scale;   // mode 0, INT4/INT2: power of two of each token's fp16 activations
+    float* logits;            // mode 2: [n_tok, n_rows] fp32
+    int n_tok, n_rows;        // mode 2: tokens, router rows (experts)
+    int n_tiles;              // mode 2: (row blocks) x (token blocks)
     int* err;
 };
 
 // ------------------------------------------------------------------ dequant
-// Row r of one 128x64 block: codes at stg (device layout of layout.cuh),
-// written as 64 bf16 into the swizzled A tile.
-MOE_DEV void store_chunk(uint8_t* a_tile, int r, int c8, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
-    uint8_t* p = a_tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c8 ^ (r & 7)) << 4);
-    *reinterpret_cast<uint4*>(p) = make_uint4(w0, w1, w2, w3);
-}
-
 MOE_DEV uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 MOE_DEV uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 MOE_DEV __half f16_sat(float v) { return __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f)); }
 
-// INT4 / INT2 codes -> fp16 (u - 8) * s or (u - z) * s: the integer is exact
-// in fp16 and so is the fp16 scale, so each weight is rounded once (2^-12).
-MOE_DEV void dequant_row_f16(int quant, const uint8_t* stg, uint8_t* a_tile, int r) {
+// Dequantization of one half (32 columns, h = 0 / 1) of row r of a 128x64
+// block: codes of the block (device layout of layout.cuh), the block's
+// scales (INT4/INT2: fp16 per row of its 128-column group; NVFP4: four e4m3
+// per row) and INT2 zero points.  v[i] holds columns 32h + 2i and
+// 32h + 2i + 1 (low, high), the A-operand layout of one TMEM lane.
+//
+// INT4 / INT2 -> fp16 (u - 8) * s or (u - z) * s: the integer is exact in
+// fp16 and so is the fp16 scale, so each weight is rounded once (2^-12).
+MOE_DEV void dequant_half_f16(int quant, const uint8_t* codes, const uint8_t* scales, const uint8_t* zeros, int r,
+                              int h, uint32_t (&v)[16]) {
+    const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(scales)[r]);
     if (quant == Q_INT4) {
-        const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(stg + 4096)[r]);
         const __half2 off = __float2half2_rn(1032.0f);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(stg + (c * kBlkN + r) * 16);
-            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + u
-                    o[j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
-                }
-                store_chunk(a_tile, r, c * 4 + w, o[0], o[1], o[2], o[3]);
-            }
-        }
-    } else {
-        const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(stg + 2048)[r]);
-        const __half2 off = __float2half2_rn(1024.0f + (float)stg[2048 + 256 + r]);
-        const uint4 q = *reinterpret_cast<const uint4*>(stg + r * 16);
+        const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);   // chunk h
         const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            uint32_t o[8];
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + u
+                v[4 * w + j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
+            }
+    } else {
+        const __half2 off = __float2half2_rn(1024.0f + (float)zeros[r]);
+        const uint2 q = *reinterpret_cast<const uint2*>(codes + r * 16 + h * 8);          // words 2h, 2h+1
+        const uint32_t wv[2] = {q.x, q.y};
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t t = ((wv[w] >> (2 * j)) & 0x00030003u) | 0x64006400u;   // 1024 + u
-                o[j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
+                v[8 * w + j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
             }
-            store_chunk(a_tile, r, 2 * w, o[0], o[1], o[2], o[3]);
-            store_chunk(a_tile, r, 2 * w + 1, o[4], o[5], o[6], o[7]);
-        }
     }
 }
 
-MOE_DEV void dequant_row(int quant, const uint8_t* stg, uint8_t* a_tile, int r) {
+// bf16 variant (down projection, NVFP4): (u - 8) * s and (u - z) * s in
+// bf16; e2m1 * e4m3 block scale is exact in bf16 (the global scales are
+// applied in the epilogue).
+MOE_DEV void dequant_half(int quant, const uint8_t* codes, const uint8_t* scales, const uint8_t* zeros, int r, int h,
+                          uint32_t (&v)[16]) {
     if (quant == Q_INT4) {
-        const __half s16 = reinterpret_cast<const __half*>(stg + 4096)[r];
+        const __half s16 = reinterpret_cast<const __half*>(scales)[r];
         const __nv_bfloat162 s2 = __bfloat162bfloat162(__float2bfloat16_rn(__half2float(s16)));
         const __nv_bfloat162 off = __bfloat162bfloat162(__float2bfloat16_rn(136.0f));
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(stg + (c * kBlkN + r) * 16);
-            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // 128 + u
-                    __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&t);
-                    v = __hmul2(__hsub2(v, off), s2);                                   // (u - 8) * s
-                    o[j] = bf16x2_bits(v);
-                }
-                store_chunk(a_tile, r, c * 4 + w, o[0], o[1], o[2], o[3]);
-            }
-        }
-    } else if (quant == Q_INT2) {
-        const __half s16 = reinterpret_cast<const __half*>(stg + 2048)[r];
-        const __nv_bfloat162 s2 = __bfloat162bfloat162(__float2bfloat16_rn(__half2float(s16)));
-        const float z = (float)stg[2048 + 256 + r];
-        const __nv_bfloat162 off = __bfloat162bfloat162(__float2bfloat16_rn(128.0f + z));
-        const uint4 q = *reinterpret_cast<const uint4*>(stg + r * 16);
+        const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);
         const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            uint32_t o[8];
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // 128 + u
+                const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&t);
+                v[4 * w + j] = bf16x2_bits(__hmul2(__hsub2(b, off), s2));             // (u - 8) * s
+            }
+    } else if (quant == Q_INT2) {
+        const __half s16 = reinterpret_cast<const __half*>(scales)[r];
+        const __nv_bfloat162 s2 = __bfloat162bfloat162(__float2bfloat16_rn(__half2float(s16)));
+        const __nv_bfloat162 off = __bfloat162bfloat162(__float2bfloat16_rn(128.0f + (float)zeros[r]));
+        const uint2 q = *reinterpret_cast<const uint2*>(codes + r * 16 + h * 8);
+        const uint32_t wv[2] = {q.x, q.y};
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t t = ((wv[w] >> (2 * j)) & 0x00030003u) | 0x43004300u;   // 128 + u
-                __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&t);
-                v = __hmul2(__hsub2(v, off), s2);                                   // (u - z) * s
-                o[j] = bf16x2_bits(v);
+                const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&t);
+                v[8 * w + j] = bf16x2_bits(__hmul2(__hsub2(b, off), s2));             // (u - z) * s
             }
-            store_chunk(a_tile, r, 2 * w, o[0], o[1], o[2], o[3]);
-            store_chunk(a_tile, r, 2 * w + 1, o[4], o[5], o[6], o[7]);
-        }
-    } else {  // NVFP4: e2m1 * e4m3 block scale is exact in bf16 (global scale in the epilogue)
-        const uint32_t sb4 = *reinterpret_cast<const uint32_t*>(stg + 4096 + r * 4);
+    } else {  // NVFP4: two 16-column blocks per half, one e4m3 scale each
+        const uint32_t sb4 = reinterpret_cast<const uint32_t*>(scales)[r];
+        const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);
+        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+        const uint32_t sb2[2] = {bf16x2_splat(e4m3_to_f32((sb4 >> (16 * h)) & 0xffu)),
+                                 bf16x2_splat(e4m3_to_f32((sb4 >> (16 * h + 8)) & 0xffu))};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(stg + (c * kBlkN + r) * 16);
-            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+        for (int w = 0; w < 4; ++w)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float sb = e4m3_to_f32((sb4 >> (8 * ((c * 4 + w) >> 1))) & 0xffu);
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t t = wv[w] >> (4 * j);
-                    o[j] = pack_bf16x2(e2m1_to_f32(t & 0xFu) * sb, e2m1_to_f32((t >> 16) & 0xFu) * sb);
-                }
-                store_chunk(a_tile, r, c * 4 + w, o[0], o[1], o[2], o[3]);
-            }
-        }
+            for (int j = 0; j < 4; ++j) v[4 * w + j] = fp4_pair(wv[w], j, sb2[w >> 1]);
     }
 }
 
-// bytes of one matrix block in the staging area
-MOE_DEV void stage_bytes(int quant, int& codes, int& scales, int& zeros) {
-    codes = quant == Q_INT2 ? 2048 : 4096;
-    scales = quant == Q_NVFP4 ? 512 : 256;
-    zeros = quant == Q_INT2 ? 128 : 0;
+// bytes of the packed codes of one 128x64 block
+MOE_DEV int block_code_bytes(int quant) { return quant == Q_INT2 ? 2048 : 4096; }
+
+// Bounded mbarrier wait by a whole warp with a warp-uniform result (every
+// lane returns from mbar_wait, so every lane reaches the vote): a warp that
+// synchronises with __syncwarp never has lanes on both sides of a stop.
+MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int code) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, err, code);
+    return __all_sync(0xffffffffu, ok);
 }
 
-// named barrier of the four epilogue warps
-MOE_DEV void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barrier of the epilogue warps
+MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
+
+// SwiGLU of one accumulator pair: silu(g) * u with the fast exponential and
+// reciprocal (relative error ~1e-6, far below the bf16 / e2m1 rounding of
+// the stored intermediate)
+MOE_DEV float swiglu_fast(float g, float u) { return g * __frcp_rn(1.0f + __expf(-g)) * u; }
+
+// Tile ti: from the device-built list, or (router) row block ti % RB of
+// token block ti / RB.
+template <int MODE>
+MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti) {
+    if constexpr (MODE == 2) {
+        const int RB = (a.n_rows + kBlkN - 1) / kBlkN;
+        GemmTile t;
+        t.expert = -1;
+        t.rb = ti % RB;
+        t.seg = (ti / RB) * kBN;
+        t.count = min(kBN, a.n_tok - t.seg);
+        return t;
+    } else {
+        return a.tiles[ti];
+    }
+}
 
 // ------------------------------------------------------------------ kernel
-template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_constant__ CUtensorMap map_shared,
-               GemmArgs a) {
-    using L = SmemLayout<MODE>;
-    constexpr int NMAT = GemmCfg<MODE>::NMAT, S = GemmCfg<MODE>::STAGES;
+template <int MODE, bool SH>
+__global__ void __launch_bounds__(Cfg<MODE, SH>::THREADS, 1)
+k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a, GemmArgs a) {
+    using C = Cfg<MODE, SH>;
+    constexpr int NMAT = C::NMAT, S = C::S, KSTEP = C::KSTEP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t wfull[S], full[S], empty[S], acc_full[2], acc_empty[2];
@@ -228,12 +264,13 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&wfull[s], 1);
-            mbar_init(&full[s], 1 + 128);
-            mbar_init(&empty[s], 1);
+            // producer (bytes) [+ one arrival per warp of the stage's dequant group]
+            mbar_init(&full[s], SH ? 1 : 1 + C::DEQ_GROUP_WARPS);
+            mbar_init(&empty[s], C::MMA_WARPS);           // one commit per MMA warp
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 128);
+            mbar_init(&acc_full[b], C::MMA_WARPS);
+            mbar_init(&acc_empty[b], kEpiWarps);          // one arrival per epilogue warp
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -243,143 +280,182 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_slot;
-    const int num_tiles = __ldcg(a.num_tiles);
-    const int KB = a.K / kBlkK;
+    const int t_begin = (SH && MODE != 2) ? __ldcg(a.num_tiles) : 0;
+    const int t_end = MODE == 2 ? a.n_tiles : SH ? __ldcg(a.num_tiles + 1) : __ldcg(a.num_tiles);
+    const int NS = a.K / (kBlkK * KSTEP);                 // stages per tile
 
     if (warp == kWarpProducer) {
         // ---------------------------------------------------------- producer
         int g = 0;
-        for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = a.tiles[ti];
-            const bool shared = t.expert < 0;
-            for (int kb = 0; kb < KB; ++kb, ++g) {
+        for (int ti = t_begin + blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+            const GemmTile t = load_tile<MODE>(a, ti);
+            bool ok = true;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
-                if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 1)) break;
+                if (!warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 1)) { ok = false; break; }
                 if (lane == 0) {
-                    uint8_t* A = smem + L::A + s * NMAT * kATile;
-                    uint8_t* B = smem + L::B + s * kBTile;
-                    uint8_t* stg = smem + L::STG + s * NMAT * kStgMat;
-                    const uint32_t b_bytes = kBTile;   // a whole box; rows past the end read as zero
-                    if (shared) {
-                        mbar_arrive(&wfull[s]);                       // nothing to dequantize
-                        mbar_arrive_expect_tx(&full[s], b_bytes + NMAT * kATile);
+                    const int kb0 = ks * KSTEP;
+                    uint8_t* B = smem + C::B + s * KSTEP * kBTile;
+                    if constexpr (MODE == 2) {
+                        mbar_arrive_expect_tx(&full[s], kBTile + kATile);
+                        tma_load_2d(smem + C::A + s * kATile, &map_a, kb0 * kBlkK, t.rb * kBlkN, &full[s]);
+                    } else if constexpr (SH) {
+                        uint8_t* A = smem + C::A + s * NMAT * kATile;
+                        mbar_arrive_expect_tx(&full[s], kBTile + NMAT * kATile);
                         for (int m = 0; m < NMAT; ++m) {
-                            const uint8_t* img = (m == 0 ? a.sh0 : a.sh1) + ((size_t)t.rb * KB + kb) * kATile;
+                            const uint8_t* img = (m == 0 ? a.sh0 : a.sh1) + ((size_t)t.rb * (a.K / kBlkK) + kb0) * kATile;
                             bulk_g2s(A + m * kATile, img, kATile, &full[s]);
                         }
                     } else {
-                        int cb, sbb, zb;
-                        stage_bytes(a.quant, cb, sbb, zb);
-                        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(NMAT * (cb + sbb + zb)));
+                        // the codes of KSTEP consecutive blocks are contiguous,
+                        // and so are their NVFP4 scales
+                        uint8_t* stg = smem + C::STG + s * NMAT * C::STG_MAT;
+                        const int KB = a.K / kBlkK, G = a.K / kGroup;
+                        const int cb = block_code_bytes(a.quant) * KSTEP;
+                        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : 256;
+                        const int zb = a.quant == Q_INT2 ? 128 : 0;
+                        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(NMAT * (cb + sb + zb)));
                         for (int m = 0; m < NMAT; ++m) {
                             const MatView& v = m == 0 ? a.w0 : a.w1;
                             const size_t eo = (size_t)t.expert * v.stride;
-                            const size_t blk = ((size_t)t.rb * KB + kb) * (size_t)cb;
-                            uint8_t* d = stg + m * kStgMat;
-                            bulk_g2s(d, v.codes + eo + blk, cb, &wfull[s]);
+                            uint8_t* d = stg + m * C::STG_MAT;
+                            bulk_g2s(d, v.codes + eo + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
+                                     &wfull[s]);
                             if (a.quant == Q_NVFP4) {
-                                bulk_g2s(d + cb, v.scales + eo + ((size_t)t.rb * KB + kb) * 512, sbb, &wfull[s]);
+                                bulk_g2s(d + cb, v.scales + eo + ((size_t)t.rb * KB + kb0) * 512, sb, &wfull[s]);
                             } else {
-                                const int G = a.K / kGroup;
-                                const size_t go = ((size_t)t.rb * G + kb / 2) * 256;
-                                bulk_g2s(d + cb, v.scales + eo + go, sbb, &wfull[s]);
-                                if (zb) bulk_g2s(d + cb + sbb, v.zeros + eo + go / 2, zb, &wfull[s]);
+                                const size_t go = ((size_t)t.rb * G + kb0 / 2) * 256;   // kb0 even: one group
+                                bulk_g2s(d + cb, v.scales + eo + go, sb, &wfull[s]);
+                                if (zb) bulk_g2s(d + cb + sb, v.zeros + eo + go / 2, zb, &wfull[s]);
                             }
                         }
-                        mbar_arrive_expect_tx(&full[s], b_bytes);
+                        mbar_arrive_expect_tx(&full[s], KSTEP * kBTile);
                     }
-                    // token rows t.seg .. t.seg + 127 of the permuted operand
-                    // (shared tiles: of x / the shared intermediate)
-                    tma_load_2d(B, shared ? &map_shared : &map_routed, kb * kBlkK, t.seg, &full[s]);
+                    // token rows t.seg .. t.seg + 127 (a whole box; rows past
+                    // the end of the operand read as zero)
+                    for (int j = 0; j < KSTEP; ++j)
+                        tma_load_2d(B + j * kBTile, &map_b, (kb0 + j) * kBlkK, t.seg, &full[s]);
                 }
                 __syncwarp();
             }
+            if (!ok) break;
         }
-    } else if (warp == kWarpMma) {
+    } else if (warp >= kWarpMma && warp < C::DEQ0) {
         // --------------------------------------------------------- MMA issue
+        // warp kWarpMma + m issues the MMAs of matrix m (gate/up: two warps)
+        const int mi = warp - kWarpMma;
         int g = 0, local = 0;
-        for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x, ++local) {
-            const GemmTile t = a.tiles[ti];
+        for (int ti = t_begin + blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
+            const GemmTile t = load_tile<MODE>(a, ti);
             const int n_mma = (t.count + 15) & ~15;
-            const bool f16 = MODE == 0 && a.tok_scale != nullptr && t.expert >= 0;
+            const bool f16 = MODE == 0 && !SH && a.tok_scale != nullptr;
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
-            const int ab = local & 1;
-            if (!mbar_wait(&acc_empty[ab], ((uint32_t)(local >> 1) & 1u) ^ 1u, &abort_flag, a.err, 2)) break;
+            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
+            if (!warp_wait(&acc_empty[ab], (use & 1u) ^ 1u, &abort_flag, a.err, 2)) break;
             tc_fence_after();
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb, ++g) {
+            const uint32_t d = tmem + ab * C::ACC_COLS + mi * kBN;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
-                if (!mbar_wait(&full[s], r & 1u, &abort_flag, a.err, 3)) { ok = false; break; }
+                if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 3)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t A = smem_u32(smem + L::A + s * NMAT * kATile);
-                    const uint32_t B = smem_u32(smem + L::B + s * kBTile);
-                    const uint64_t bdesc = desc_kmajor_sw128(B);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
+                    for (int j = 0; j < KSTEP; ++j) {
+                        const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + (s * KSTEP + j) * kBTile));
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m) {
-                            const uint64_t adesc = desc_kmajor_sw128(A + m * kATile);
-                            mma_bf16(tmem + ab * 256 + m * 128, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                     (kb | kk) != 0);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (ks | j | kk) != 0;
+                            if constexpr (SH) {
+                                const uint64_t adesc = desc_kmajor_sw128(smem_u32(smem + C::A + (s * NMAT + mi) * kATile));
+                                mma_bf16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+                            } else {
+                                const uint32_t at = tmem + C::A_COL0 + s * C::A_STAGE_COLS + (mi * KSTEP + j) * 32 + kk * 8;
+                                mma_f16_tmem_a(d, at, bdesc + 2 * kk, idesc, acc);
+                            }
                         }
                     }
                     mma_commit(&empty[s]);
-                    if (kb == KB - 1) mma_commit(&acc_full[ab]);
+                    if (ks == NS - 1) mma_commit(&acc_full[ab]);
                 }
                 __syncwarp();
             }
             if (!ok) break;
         }
-    } else if (warp >= kWarpDeq0 && warp < kWarpDeq0 + 4) {
+    } else if (warp >= C::DEQ0 && warp < C::EPI0) {
         // ------------------------------------------------------------ dequant
-        const int r = threadIdx.x - kWarpDeq0 * 32;          // weight row 0..127
-        int g = 0;
-        for (int ti = blockIdx.x; ti < num_tiles && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = a.tiles[ti];
-            bool ok = true;
-            for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = g % S;
-                const uint32_t rr = (uint32_t)(g / S);
-                if (!mbar_wait(&wfull[s], rr & 1u, &abort_flag, a.err, 4)) { ok = false; break; }
-                if (t.expert >= 0) {
-                    uint8_t* A = smem + L::A + s * NMAT * kATile;
-                    const uint8_t* stg = smem + L::STG + s * NMAT * kStgMat;
-                    const bool f16 = MODE == 0 && a.tok_scale != nullptr;
+        // routed tiles only: thread (row r, matrix m) of its group writes
+        // TMEM lane r (its warp's lane quarter), all KSTEP blocks of a stage
+        if constexpr (!SH) {
+            const int quarter = warp & 3;
+            const int r = quarter * 32 + lane;                 // weight row = TMEM lane
+            const int wi = warp - C::DEQ0;
+            const int grp = wi / C::DEQ_GROUP_WARPS;
+            const int m = (wi % C::DEQ_GROUP_WARPS) >> 2;
+            const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+            const bool f16 = MODE == 0 && a.tok_scale != nullptr;
+            const int cb = block_code_bytes(a.quant);
+            int g = 0;
+            for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+                bool ok = true;
+                for (int ks = 0; ks < NS; ++ks, ++g) {
+                    if (g % C::DEQ_GROUPS != grp) continue;
+                    const int s = g % S;
+                    const uint32_t rr = (uint32_t)(g / S);
+                    // the stage's staging bytes arrived, so the MMAs that read
+                    // this stage's TMEM columns before have completed
+                    if (!warp_wait(&wfull[s], rr & 1u, &abort_flag, a.err, 4)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t* stg = smem + C::STG + (s * NMAT + m) * C::STG_MAT;
+                    const uint8_t* sc = stg + cb * KSTEP;
+                    const uint8_t* zr = sc + 256;
+                    uint32_t v[16];
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        if (f16) dequant_row_f16(a.quant, stg + m * kStgMat, A + m * kATile, r);
-                        else dequant_row(a.quant, stg + m * kStgMat, A + m * kATile, r);
-                    }
-                    fence_proxy_async_smem();
+                    for (int j = 0; j < KSTEP; ++j)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512 : sc;
+                            if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
+                            else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
+                            tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h,
+                                      v);
+                        }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[s]);
                 }
-                mbar_arrive(&full[s]);
+                if (!ok) break;
             }
-            if (!ok) break;
         }
-    } else if (warp >= kWarpEpi0) {
+    } else if (warp >= C::EPI0) {
         // ----------------------------------------------------------- epilogue
-        const int lane_base = (warp & 3) * 32;
-        const int row = lane_base + lane;                    // weight row within the block
-        const int ej = threadIdx.x - kWarpEpi0 * 32;         // 0..127: token column this thread looks up
-        // The four warps leave the loop together (named barriers): the stop
-        // decision is taken by one thread between two barriers.
+        // TMEM -> registers -> (SwiGLU / routing weight) -> 16-bit staging
+        // tile [token][128 outputs] in shared memory; the accumulator is
+        // released as soon as it is read, then the staged rows are written
+        // to global memory with 16-byte stores.
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;                 // weight row within the block = output column
+        const int ej = threadIdx.x - C::EPI0 * 32;           // 0 .. 32 * kEpiWarps - 1
+        const int cbeg = ((warp - C::EPI0) >> 2) * (kBN / 2);   // this warp's 64 token columns
+        uint16_t* out_s = reinterpret_cast<uint16_t*>(smem + C::OUT);
+        // The epilogue warps leave the loop together (named barriers): the
+        // stop decision is taken by one thread between two barriers.
         int local = 0;
-        for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x, ++local) {
-            const GemmTile t = a.tiles[ti];
-            const bool shared = t.expert < 0;
-            const int ab = local & 1;
+        for (int ti = t_begin + blockIdx.x; ti < t_end; ti += gridDim.x, ++local) {
+            const GemmTile t = load_tile<MODE>(a, ti);
+            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
             float gsc = 1.0f;
-            if (!shared && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
-            // token columns of the tile: scale (mode 0) or routing weight
-            // (mode 1) and output row, looked up once per tile
+            if (!SH && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
             epi_sync();                                      // the previous tile's readers are done
             if (ej == 0) ep_stop = abort_flag;
-            if (ej < t.count) {
-                if (shared) {
-                    ep_scale[ej] = gsc;
+            if (MODE != 2 && ej < t.count) {
+                if constexpr (SH) {
+                    ep_scale[ej] = 1.0f;
                     ep_row[ej] = t.seg + ej;
                 } else {
                     const int slot = __ldg(a.perm + t.seg + ej);
@@ -396,53 +472,77 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_routed, const __grid_cons
             if (ep_stop) break;
             // a failed wait sets abort_flag: this tile is skipped and all four
             // warps stop at the next tile's decision
-            if (!mbar_wait(&acc_full[ab], (uint32_t)(local >> 1) & 1u, &abort_flag, a.err, 5)) continue;
+            if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 5)) continue;
             tc_fence_after();
             const int n_mma = (t.count + 15) & ~15;
-            const int col_out = t.rb * kBlkN + row;
-            for (int c0 = 0; c0 < n_mma; c0 += 16) {
-                const uint32_t taddr = tmem + ((uint32_t)lane_base << 16) + ab * 256 + c0;
+            const int cend = min(n_mma, cbeg + kBN / 2);
+            if constexpr (MODE == 2) {
+                // logits: for each token, the 32 lanes store 32 consecutive
+                // experts (128 contiguous bytes)
+                const int e = t.rb * kBlkN + row;
+                for (int c0 = cbeg; c0 < cend; c0 += 16) {
+                    float v0[16];
+                    tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0, v0);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.count && e < a.n_rows) a.logits[(size_t)(t.seg + c0 + i) * a.n_rows + e] = v0[i];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                continue;
+            }
+            for (int c0 = cbeg; c0 < cend; c0 += 16) {
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0;
                 float v0[16];
                 tmem_ld16(taddr, v0);
-                if (MODE == 0) {
+                if constexpr (MODE == 0) {
                     float v1[16];
-                    tmem_ld16(taddr + 128, v1);
-                    __nv_bfloat16* dst = shared ? a.out_sh : a.out;
+                    tmem_ld16(taddr + kBN, v1);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int col = c0 + i;
                         const float tsc = col < t.count ? ep_scale[col] : 0.0f;
                         const float gg = v0[i] * tsc, uu = v1[i] * tsc;
-                        float act = gg / (1.0f + expf(-gg)) * uu;
-                        if (!shared && a.quant == Q_NVFP4) {
-                            // W4A4: requantize the intermediate per 16 consecutive rows
+                        float act = swiglu_fast(gg, uu);
+                        if (!SH && a.quant == Q_NVFP4) {
+                            // W4A4: requantize the intermediate per 16 consecutive outputs
                             float amax = fabsf(act);
 #pragma unroll
                             for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                            const float g = a.g_req;
+                            const float gq = a.g_req;
                             float sbv = 0.0f, rcp = 0.0f;
-                            if (g != 0.0f) {
-                                sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g))));
-                                rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
+                            if (gq != 0.0f) {
+                                sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, gq))));
+                                rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, gq));
                             }
                             act = e2m1_to_f32(f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu) * sbv;
                         }
-                        if (col < t.count) dst[(size_t)ep_row[col] * a.out_ld + col_out] = __float2bfloat16_rn(act);
+                        out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
                     }
                 } else {
                     // per-slot outputs are fp16 (saturating at +-65504): their
                     // rounding error stays well below the final bf16 one
-                    __half* dst = shared ? a.o16_sh : a.o16;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int col = c0 + i;
-                        if (col < t.count)
-                            dst[(size_t)ep_row[col] * a.out_ld + col_out] = f16_sat(v0[i] * ep_scale[col]);
+                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                        out_s[col * kBlkN + row] = __half_as_ushort(f16_sat(v0[i] * sc));
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[ab]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);      // the MMA may refill this accumulator
+            epi_sync();                                      // staging tile complete
+            uint16_t* dst = MODE == 0 ? reinterpret_cast<uint16_t*>(SH ? a.out_sh : a.out)
+                                      : reinterpret_cast<uint16_t*>(SH ? a.o16_sh : a.o16);
+            const int col0 = t.rb * kBlkN;
+            for (int i = ej; i < t.count * 16; i += kEpiWarps * 32) {
+                const int col = i >> 4, ch = i & 15;
+                const uint4 q = *reinterpret_cast<const uint4*>(out_s + col * kBlkN + ch * 8);
+                *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) = q;
+            }
         }
     }
     tc_fence_before();
@@ -495,7 +595,10 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
         g.count = min(kBN, T - tt * kBN);
         tiles[total + i] = g;
     }
-    if (e == 0) *num_tiles = total + nts * RB;
+    if (e == 0) {
+        num_tiles[0] = total;               // routed tiles
+        num_tiles[1] = total + nts * RB;    // + shared-expert tiles
+    }
 }
 
 // --------------------------------------------------------------- combine
@@ -651,6 +754,36 @@ static int num_sms() {
     return n;
 }
 
+// One persistent CTA per SM over the routed (SH = false) or the shared (SH =
+// true) tiles of the list.
+template <int MODE, bool SH>
+static cudaError_t launch_gemm(const CUtensorMap& map_b, const GemmArgs& g, cudaStream_t st,
+                               const CUtensorMap* map_a = nullptr, int grid = 0) {
+    constexpr int bytes = Cfg<MODE, SH>::ALLOC;
+    cudaError_t err = cudaFuncSetAttribute(k_grouped_gemm<MODE, SH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err != cudaSuccess) return err;
+    k_grouped_gemm<MODE, SH><<<grid > 0 ? grid : num_sms(), Cfg<MODE, SH>::THREADS, bytes, st>>>(
+        map_b, map_a ? *map_a : map_b, g);
+    return cudaGetLastError();
+}
+
+// Router logits on the tensor cores: logits[T, E] = x[T, H] . Wr[E, H]^T in
+// fp32 (bf16 products, fp32 accumulation); tiles of 128 experts x 128 tokens.
+cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E, float* logits, int* err,
+                             cudaStream_t st) {
+    CUtensorMap m_x, m_w;
+    if (!make_map(&m_x, x, (uint64_t)T, (uint64_t)H, kBN) || !make_map(&m_w, wr, (uint64_t)E, (uint64_t)H, kBlkN))
+        return cudaErrorInvalidValue;
+    GemmArgs g{};
+    g.K = H;
+    g.logits = logits;
+    g.n_tok = T;
+    g.n_rows = E;
+    g.n_tiles = ((E + kBlkN - 1) / kBlkN) * ((T + kBN - 1) / kBN);
+    g.err = err;
+    return launch_gemm<2, true>(m_x, g, st, &m_w, g.n_tiles < num_sms() ? g.n_tiles : num_sms());
+}
+
 cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const ExpertArgs& ex = p.ex;
     const int T = p.T, k = ex.k, H = ex.H, I = ex.I, E = ex.E;
@@ -701,12 +834,9 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.g_req = ex.g_a;
     g.tok_scale = fp4 ? nullptr : p.tok_scale;
     g.err = p.err;
-    const int grid = num_sms();
-    err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<0>::ALLOC);
-    if (err != cudaSuccess) return err;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
-    k_grouped_gemm<0><<<grid, kGemmThreads, SmemLayout<0>::ALLOC, st>>>(m_routed, m_shared, g);
-    err = cudaGetLastError();
+    err = launch_gemm<0, false>(m_routed, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
@@ -728,11 +858,9 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.g_w = fp4 ? ex.g_down : nullptr;
     g.g_act = fp4 ? ex.g_a : 1.0f;
     g.tok_scale = nullptr;
-    err = cudaFuncSetAttribute(k_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout<1>::ALLOC);
-    if (err != cudaSuccess) return err;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
-    k_grouped_gemm<1><<<grid, kGemmThreads, SmemLayout<1>::ALLOC, st>>>(m_routed, m_shared, g);
-    err = cudaGetLastError();
+    err = launch_gemm<1, false>(m_routed, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     // ---- combine

@@ -32,9 +32,13 @@ struct RouteArgs {
     int32_t* ids;           // [T, k]
     float* w;               // [T, k]
     unsigned int* counter;  // zero-initialised grid counter (decode router)
+    int* err;               // device error word (bounded waits of the tensor-core router)
     int T, H, E, k;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+// grouped_gemm.cu: router logits on the tensor cores (any T, E; H % 64 == 0)
+cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E, float* logits, int* err,
+                             cudaStream_t st);
 
 // moe_api.cu: text returned by moe_last_error(NULL) on this host thread
 void set_thread_error(const char* msg);

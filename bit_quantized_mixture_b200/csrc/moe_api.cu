@@ -183,7 +183,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_inv = carve(sizeof(int32_t) * slots);
     const size_t o_pscr = carve(sizeof(int32_t) * permute_scratch_ints((int)slots, E));
     const size_t o_tiles = carve(sizeof(GemmTile) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
-    const size_t o_ntiles = carve(sizeof(int));
+    const size_t o_ntiles = carve(2 * sizeof(int));   // routed tiles, all tiles
     const size_t o_err = carve(sizeof(int));
     const size_t o_xq = carve(Tm * H * 2);
     const size_t o_tsc = carve(Tm * sizeof(float));
@@ -372,6 +372,7 @@ moe_status moe_route(moe_handle h, const void* x, int32_t T, int32_t* topk_ids, 
     a.ids = topk_ids;
     a.w = topk_w;
     a.counter = h->route_counter;
+    a.err = h->dev_err;
     a.T = T; a.H = h->cfg.hidden; a.E = h->cfg.num_experts; a.k = h->cfg.top_k;
     cudaStream_t st = (cudaStream_t)stream;
     if (h->prof[0]) cudaEventRecord(h->prof[0], st);

@@ -157,44 +157,6 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
 }
 
-// Router GEMM for larger T on CUDA cores: 64 tokens x 64 experts per CTA.
-__global__ void __launch_bounds__(256) k_router_gemm(RouteArgs a) {
-    __shared__ float As[32][65];
-    __shared__ float Bs[32][65];
-    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
-    const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.wr);
-    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < a.H; k0 += 32) {
-        for (int i = threadIdx.x; i < 64 * 32; i += 256) {
-            const int r = i / 32, c = i % 32;
-            const int t = t0 + r, e = e0 + r;
-            As[c][r] = (t < a.T) ? __bfloat162float(x[(size_t)t * a.H + k0 + c]) : 0.0f;
-            Bs[c][r] = (e < a.E) ? __bfloat162float(wr[(size_t)e * a.H + k0 + c]) : 0.0f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int c = 0; c < 32; ++c) {
-            float av[4], bv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { av[i] = As[c][ty * 4 + i]; bv[i] = Bs[c][tx * 4 + i]; }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
-            if (t < a.T && e < a.E) a.logits[(size_t)t * a.E + e] = acc[i][j];
-        }
-}
-
 __global__ void __launch_bounds__(256) k_topk(RouteArgs a) {
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= a.T) return;
@@ -212,9 +174,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
             k_router_small<<<(a.E + 3) / 4, 128, smem, st>>>(a);
             return cudaGetLastError();
         }
-        dim3 grid((a.E + 63) / 64, (a.T + 63) / 64);
-        k_router_gemm<<<grid, 256, 0, st>>>(a);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_router_tc(a.x, a.wr, a.T, a.H, a.E, a.logits, a.err, st);
         if (e != cudaSuccess) return e;
     }
     k_topk<<<(a.T + 7) / 8, 256, 0, st>>>(a);

@@ -33,7 +33,7 @@ def _route_gpu(layer, x_bits, wl):
 
 
 # ------------------------------------------------------------------ route
-@pytest.mark.parametrize("T", [1, 3, 4, 16, 17, 100])
+@pytest.mark.parametrize("T", [1, 3, 4, 16, 17, 100, 300])
 def test_route_matches_oracle(T):
     wl = synth.custom("decode-b1-int4", T=T, E=512, k=10)
     layer = moe.MoeLayer(wl.H, wl.I, wl.E, wl.k, "int4", False, max(T, 1), 0)
