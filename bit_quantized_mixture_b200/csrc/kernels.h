@@ -84,10 +84,12 @@ struct FusedArgs {
     int32_t* ids_out;              // [T, k] (when wr is set)
     float* w_out;                  // [T, k]
     unsigned long long* bar;       // workspace: monotonically increasing arrival count, zero-initialised
+    float* gu_sh;                  // workspace [4][T][2 * I]: partial shared gate/up sums by K part
     int* err;                      // device error word
 };
 size_t fused_smem_bytes(int H, int I);
-cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st);
+cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st);   // cudaErrorNotSupported: shapes too large
+bool fused_supported(int T, int H, int I, int quant);
 
 // grouped_gemm.cu (prefill path)
 struct GemmTile {

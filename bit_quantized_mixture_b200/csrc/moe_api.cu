@@ -39,6 +39,7 @@ struct moe_layer {
     float* dec_part_sh = nullptr;  // [8, H]
     unsigned int* dec_counters = nullptr;   // [H/16]
     unsigned long long* fused_bar = nullptr;   // arrival count of the fused decode kernel's grid barrier
+    float* fused_gu_sh = nullptr;              // [4][8][2I] partial shared gate/up sums of the fused decode kernel
     uint8_t* staging = nullptr;    // interchange copy of one matrix
     size_t staging_bytes = 0;
     // prefill path
@@ -174,6 +175,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_psh = carve(sizeof(float) * (size_t)MT * H);
     const size_t o_cnt = carve(sizeof(unsigned int) * (size_t)(H / 16));
     const size_t o_fbar = carve(sizeof(unsigned long long));
+    const size_t o_gush = carve(sizeof(float) * 4 * (size_t)MT * 2 * I);
     h->staging_bytes = (size_t)2 * H * I + 65536;
     const size_t o_stage = carve(h->staging_bytes);
     const size_t Tm = (size_t)c.max_tokens, slots = Tm * k;
@@ -207,6 +209,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->dec_part_sh = reinterpret_cast<float*>(h->ws + o_psh);
     h->dec_counters = reinterpret_cast<unsigned int*>(h->ws + o_cnt);
     h->fused_bar = reinterpret_cast<unsigned long long*>(h->ws + o_fbar);
+    h->fused_gu_sh = reinterpret_cast<float*>(h->ws + o_gush);
     h->staging = h->ws + o_stage;
     h->counts = reinterpret_cast<int32_t*>(h->ws + o_counts);
     h->offsets = reinterpret_cast<int32_t*>(h->ws + o_offsets);
@@ -474,6 +477,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         f.d.x = x; f.d.ids = topk_ids; f.d.w = topk_w; f.d.y = y; f.d.T = T;
         f.wr = nullptr;
         f.bar = h->fused_bar;
+        f.gu_sh = h->fused_gu_sh;
         f.err = h->dev_err;
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_decode_fused(f, st);
@@ -539,6 +543,7 @@ moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* to
     f.ids_out = topk_ids;
     f.w_out = topk_w;
     f.bar = h->fused_bar;
+    f.gu_sh = h->fused_gu_sh;
     f.err = h->dev_err;
     if (h->prof[0]) cudaEventRecord(h->prof[0], st);
     cudaError_t e = launch_decode_fused(f, st);
