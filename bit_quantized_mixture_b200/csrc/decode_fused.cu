@@ -484,6 +484,75 @@ __host__ __device__ inline FusedSmem fused_layout(int T, int H, int I, bool fp4)
 }
 __host__ __device__ inline int stage_bytes(int I) { return (kDecMaxT + 1) * (I + kXPad) * 2; }
 
+// Slots of the item whose first slot is s0 (slot order), by one thread.
+__device__ __noinline__ int item_slots(const int* __restrict__ ids, int n, int s0, int* slot) {
+    const int e0 = ids[s0];
+    int c = 0;
+#pragma unroll 1
+    for (int s = s0; s < n && c < kDecMaxT; ++s)
+        if (ids[s] == e0) slot[c++] = s;
+    return c;
+}
+
+// Staging of the intermediate rows of several down units at once (one L2
+// round trip): unit j owns staging rows row0[j] .. row0[j] + m[j], the last
+// of them zero; rows of units with fp4_of[j] become NVFP4 values.
+__device__ __noinline__ void stage_units(__nv_bfloat16* dst, int ld, const float* src, int I, const int* m,
+                                         const int* row0, const int* slots, const unsigned char* fp4_of, int nu_,
+                                         int rows, float g, int gtid) {
+    const int per = I / 16;
+#pragma unroll 1
+    for (int i0 = gtid; i0 < rows * per; i0 += 2 * 128) {
+        float v[2][16];
+        int rr[2], bb[2], jj[2], tt[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int i = i0 + q * 128;
+            rr[q] = i / per;
+            bb[q] = i % per;
+            int j = 0;
+#pragma unroll 1
+            while (j + 1 < nu_ && row0[j + 1] <= rr[q]) ++j;
+            jj[q] = j;
+            tt[q] = rr[q] - row0[j];
+            const bool live = i < rows * per && tt[q] < m[j];
+            const float4* s = reinterpret_cast<const float4*>(src + (size_t)(live ? slots[j * kDecMaxT + tt[q]] : 0) * I + bb[q] * 16);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float4 f = live ? __ldcg(s + w) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                v[q][4 * w] = f.x; v[q][4 * w + 1] = f.y; v[q][4 * w + 2] = f.z; v[q][4 * w + 3] = f.w;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            if (i0 + q * 128 < rows * per) {
+                if (fp4_of[jj[q]]) fp4_block_values(v[q], g);
+                pack16(dst + (size_t)rr[q] * ld + bb[q] * 16, v[q]);
+            }
+        }
+    }
+}
+
+// y rows of block hb (16 columns of H, T tokens): sum of the k partials in
+// fixed slot order plus the shared expert's, by one group.
+__device__ __noinline__ void combine_block(const float* part, const float* part_sh, __nv_bfloat16* y, int H, int k,
+                                           int T, int hb, int gtid) {
+    if (gtid < 16 * T) {
+        const int t = gtid >> 4, hh = hb * 16 + (gtid & 15);
+        float sum = 0.0f;
+#pragma unroll 1
+        for (int j0 = 0; j0 < k; j0 += 8) {             // fixed order j = 0 .. k-1, 8 loads in flight
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = j0 + u < k ? __ldcg(part + (size_t)(t * k + j0 + u) * H + hh) : 0.0f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += v[u];
+        }
+        if (part_sh) sum += __ldcg(part_sh + (size_t)t * H + hh);
+        y[(size_t)t * H + hh] = __float2bfloat16_rn(sum);
+    }
+}
+
 // Ticket of a 16-row block of H: the last of its `items` units sums the
 // partials in fixed slot order, y_t = sum_j part[t*k+j] + shared_t, and
 // clears the counter.  Called by all threads of one group.
@@ -527,6 +596,11 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
     __shared__ int g_tok[kGroups][kDecMaxT], g_slot[kGroups][kDecMaxT];
     __shared__ volatile int g_last[kGroups];
     __shared__ volatile int abort_s;
+    constexpr int kMaxDn = 16;                   // down units per group handled as one batch
+    __shared__ int u_m[kGroups][kMaxDn], u_row0[kGroups][kMaxDn], u_slot[kGroups][kMaxDn * kDecMaxT];
+    __shared__ unsigned char u_fp4[kGroups][kMaxDn];
+    __shared__ int u_rows[kGroups];
+    __shared__ int u_last[kGroups][kMaxDn + 4];
     const DecodeArgs& a = f.d;
     const ExpertArgs& ex = a.ex;
     const int H = ex.H, I = ex.I, k = ex.k, E = ex.E, T = a.T;
@@ -825,6 +899,87 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
     __syncthreads();
     __nv_bfloat16* as = reinterpret_cast<__nv_bfloat16*>(gbase + sd_end);
     const int items = nu + (has_sh ? 1 : 0);
+    __nv_bfloat16* const y = reinterpret_cast<__nv_bfloat16*>(a.y);
+    // batched path: every down unit's rows staged at once, all units and the
+    // shared slices computed, then all tickets taken together
+    bool batch = dn_pre && n_dn <= kMaxDn && n_sd <= 4 && sd_pre;
+    if (batch) {
+        if (gtid < n_dn) {
+            const int u = dn_first + gtid * nslots, ui = u / RBH;
+            u_m[group][gtid] = item_slots(plan.ids, n, plan.first[ui], &u_slot[group][gtid * kDecMaxT]);
+            u_fp4[group][gtid] = fp4 && valid_expert(unit_expert(ui));
+        }
+        group_sync(group);
+        if (gtid == 0) {
+            int r = 0;
+#pragma unroll 1
+            for (int j = 0; j < n_dn; ++j) { u_row0[group][j] = r; r += u_m[group][j] + 1; }
+            u_rows[group] = r;
+        }
+        group_sync(group);
+        batch = u_rows[group] * lda * 2 <= dn_off - sd_end;
+    }
+    if (batch) {
+        stage_units(as, lda, a.a, I, u_m[group], u_row0[group], u_slot[group], u_fp4[group], n_dn, u_rows[group], ex.g_a,
+                    gtid);
+        group_sync(group);
+#pragma unroll 1
+        for (int j = 0; j < n_dn; ++j) {
+            const int u = dn_first + j * nslots;
+            const int ui = u / RBH, r0 = (u % RBH) * 16, e = unit_expert(ui);
+            const bool valid = valid_expert(e);
+            const int m = u_m[group][j];
+            float acc[1][4] = {{0, 0, 0, 0}};
+            if (valid) {
+                const uint8_t* const mats[1] = {gbase + dn_off + j * dn_bytes};
+                slice_mma<Q, 1>(acc, mats, s_dn, 0, KBI, wg, as + (u_row0[group][j] + (gl < m ? gl : m)) * lda, gl, c);
+            }
+            frag_store<1>(red, acc, wg, gl, c);
+            group_sync(group);
+            {
+                const int row = gtid >> 3, t = gtid & 7;
+                if (t < m) {
+                    const float dsc = (fp4 && valid) ? ex.g_down[e] * ex.g_a : 1.0f;
+                    const int s = u_slot[group][j * kDecMaxT + t];
+                    a.part[(size_t)s * H + r0 + row] = valid ? w_s[s] * frag_sum(red, 1, 0, row, t) * dsc : 0.0f;
+                }
+            }
+            group_sync(group);
+        }
+#pragma unroll 1
+        for (int j = 0; j < n_sd; ++j) {
+            const int r0 = (sd_first + j * nslots) * 16;
+            float acc[1][4] = {{0, 0, 0, 0}};
+            const uint8_t* const mats[1] = {gbase + j * sd_bytes};
+            slice_mma<Q_BF16, 1>(acc, mats, s_dn, 0, KBI, wg, ash + (gl < T ? gl : T) * lda, gl, c);
+            frag_store<1>(red, acc, wg, gl, c);
+            group_sync(group);
+            {
+                const int row = gtid >> 3, t = gtid & 7;
+                if (t < T) a.part_sh[(size_t)t * H + r0 + row] = frag_sum(red, 1, 0, row, t);
+            }
+            group_sync(group);
+        }
+        // tickets: one per unit, all in flight together
+        __threadfence();
+        group_sync(group);
+        if (gtid < n_dn + n_sd) {
+            const int hb = gtid < n_dn ? (dn_first + gtid * nslots) % RBH : sd_first + (gtid - n_dn) * nslots;
+            const bool last = atomicAdd(a.counters + hb, 1u) == (unsigned)items - 1u;
+            if (last) __threadfence();
+            u_last[group][gtid] = last ? hb : -1;
+        }
+        group_sync(group);
+#pragma unroll 1
+        for (int j = 0; j < n_dn + n_sd; ++j) {
+            const int hb = u_last[group][j];
+            if (hb >= 0) {
+                combine_block(a.part, has_sh ? a.part_sh : nullptr, y, H, k, T, hb, gtid);
+                if (gtid == 0) a.counters[hb] = 0u;
+            }
+        }
+        return;
+    }
 #pragma unroll 1
     for (int j = 0; j < n_dn; ++j) {
         const int u = dn_first + j * nslots;
