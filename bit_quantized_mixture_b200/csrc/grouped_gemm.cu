@@ -118,6 +118,8 @@ struct GemmArgs {
     float* logits;            // mode 2: [n_tok, n_rows] fp32
     int n_tok, n_rows;        // mode 2: tokens, router rows (experts)
     int n_tiles;              // mode 2: (row blocks) x (token blocks)
+    uint8_t* out4;            // NVFP4 gate/up: e2m1 intermediate [slots, I/2] (permuted rows)
+    uint8_t* out_sf;          // NVFP4 gate/up: its e4m3 block scales [slots, I/16]
     int* err;
 };
 
@@ -707,6 +709,312 @@ __global__ void k_act_fp4_values(const __nv_bfloat16* __restrict__ x, int T, int
     d[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// ------------------------------------------------------------ NVFP4 native
+// W4A4 routed tiles on the block-scaled tensor-core path.  A (weights, e2m1)
+// and B (tokens, e2m1) are TMA tiles of 128 rows x 256 values (128 bytes,
+// 128-byte swizzle) read from natural-layout images; their e4m3 block scales
+// (one per 16 values) are TMA tiles of 128 rows x 16 bytes that four warps
+// store into TMEM in the layout the MMA reads (for each K = 64 instruction,
+// four 32-bit columns: column c, lane l holds the four scales of row 32c + l,
+// replicated in every lane quarter), and
+// tcgen05.mma.kind::mxf4nvf4.block_scale.block16 multiplies 64 values of K
+// per instruction.  The fp32 global scales of weights and activations are
+// applied in the epilogue.  The gate/up epilogue requantizes the SwiGLU
+// intermediate to NVFP4 (codes and scales) for the down GEMM.
+constexpr int kFp4KS = 256;                  // K values per stage
+constexpr int kFp4Tile = 128 * 128;          // 16 KB: 128 rows x 128 bytes
+constexpr int kFp4SfTile = 128 * 16;         // 2 KB: 128 rows x 16 scale bytes
+
+template <int MODE>
+struct Fp4Cfg {
+    static constexpr int NMAT = MODE == 0 ? 2 : 1;
+    static constexpr int S = MODE == 0 ? 3 : 4;
+    static constexpr int SF0 = kWarpMma + NMAT;                       // four scale-factor warps
+    static constexpr int EPI0 = SF0 + 4;
+    static constexpr int THREADS = (EPI0 + kEpiWarps) * 32;
+    static constexpr int ACC_BUFS = MODE == 0 ? 1 : 2;
+    static constexpr int ACC_COLS = NMAT * kBN;
+    static constexpr int SF_COL0 = ACC_BUFS * ACC_COLS;
+    static constexpr int SF_STAGE_COLS = (NMAT + 1) * 16;             // A per matrix, then B; 4 MMAs x 4 columns
+    static_assert(SF_COL0 + S * SF_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
+    static constexpr int A = 0;                                       // [S][NMAT][16 KB]
+    static constexpr int B = A + S * NMAT * kFp4Tile;                 // [S][16 KB]
+    static constexpr int SFA = B + S * kFp4Tile;                      // [S][NMAT][2 KB]
+    static constexpr int SFB = SFA + S * NMAT * kFp4SfTile;           // [S][2 KB]
+    static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: [128][128] fp16
+    static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : kOutTile;
+    static constexpr int ALLOC = OUT + OUT_BYTES + 1024;
+    static_assert(ALLOC <= 227 * 1024 - 2048, "shared memory budget");
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(Fp4Cfg<MODE>::THREADS, 1)
+k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
+           const __grid_constant__ CUtensorMap map_sfa0, const __grid_constant__ CUtensorMap map_sfa1,
+           const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_sfb, GemmArgs a) {
+    using C = Fp4Cfg<MODE>;
+    constexpr int NMAT = C::NMAT, S = C::S;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[S], sfready[S], empty[S], acc_full[2], acc_empty[2];
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ volatile int abort_flag;
+    __shared__ float ep_scale[kBN];
+    __shared__ int ep_row[kBN];
+    __shared__ int ep_stop;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);                       // producer (bytes)
+            mbar_init(&sfready[s], 4);                    // the four scale-factor warps
+            mbar_init(&empty[s], NMAT);                   // one commit per MMA warp
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], NMAT);
+            mbar_init(&acc_empty[b], kEpiWarps);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) tmem_alloc(&tmem_base_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_slot;
+    const int t_end = __ldcg(a.num_tiles);                // routed tiles only
+    const int NS = a.K / kFp4KS;
+
+    if (warp == kWarpProducer) {
+        // ---------------------------------------------------------- producer
+        int g = 0;
+        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+            const GemmTile t = a.tiles[ti];
+            const int arow = t.expert * a.n_rows + t.rb * kBlkN;
+            bool ok = true;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
+                const int s = g % S;
+                const uint32_t r = (uint32_t)(g / S);
+                if (!warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 11)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)((NMAT + 1) * (kFp4Tile + kFp4SfTile)));
+                    for (int m = 0; m < NMAT; ++m) {
+                        tma_load_2d(smem + C::A + (s * NMAT + m) * kFp4Tile, m == 0 ? &map_a0 : &map_a1, ks * 128, arow,
+                                    &full[s]);
+                        tma_load_2d(smem + C::SFA + (s * NMAT + m) * kFp4SfTile, m == 0 ? &map_sfa0 : &map_sfa1,
+                                    ks * 16, arow, &full[s]);
+                    }
+                    tma_load_2d(smem + C::B + s * kFp4Tile, &map_b, ks * 128, t.seg, &full[s]);
+                    tma_load_2d(smem + C::SFB + s * kFp4SfTile, &map_sfb, ks * 16, t.seg, &full[s]);
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= kWarpMma && warp < C::SF0) {
+        // --------------------------------------------------------- MMA issue
+        const int mi = warp - kWarpMma;
+        int g = 0, local = 0;
+        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
+            const GemmTile t = a.tiles[ti];
+            const int n_mma = (t.count + 15) & ~15;
+            const uint32_t idesc = idesc_nvfp4(128, n_mma);
+            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
+            if (!warp_wait(&acc_empty[ab], (use & 1u) ^ 1u, &abort_flag, a.err, 12)) break;
+            tc_fence_after();
+            bool ok = true;
+            const uint32_t d = tmem + ab * C::ACC_COLS + mi * kBN;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
+                const int s = g % S;
+                const uint32_t r = (uint32_t)(g / S);
+                if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 13)) { ok = false; break; }
+                if (!warp_wait(&sfready[s], r & 1u, &abort_flag, a.err, 14)) { ok = false; break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t adesc = desc_kmajor_sw128(smem_u32(smem + C::A + (s * NMAT + mi) * kFp4Tile));
+                    const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + s * kFp4Tile));
+                    const uint32_t sf = tmem + C::SF_COL0 + s * C::SF_STAGE_COLS;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_fp4_block16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, sf + mi * 16 + kk * 4,
+                                        sf + NMAT * 16 + kk * 4, (ks | kk) != 0);
+                    mma_commit(&empty[s]);
+                    if (ks == NS - 1) mma_commit(&acc_full[ab]);
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= C::SF0 && warp < C::EPI0) {
+        // ---------------------------------------------- scale factors -> TMEM
+        const int quarter = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        int g = 0;
+        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+            bool ok = true;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
+                const int s = g % S;
+                const uint32_t r = (uint32_t)(g / S);
+                if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 15)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sf = tmem + lane_addr + C::SF_COL0 + s * C::SF_STAGE_COLS;
+#pragma unroll
+                for (int q = 0; q <= NMAT; ++q) {
+                    const uint8_t* tile = q < NMAT ? smem + C::SFA + (s * NMAT + q) * kFp4SfTile : smem + C::SFB + s * kFp4SfTile;
+                    uint32_t v[16];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(tile + (32 * cc + lane) * 16);
+                        v[0 * 4 + cc] = w.x;      // column 4 kk + cc: scales of K-blocks 4kk..4kk+3 of row 32cc + lane
+                        v[1 * 4 + cc] = w.y;
+                        v[2 * 4 + cc] = w.z;
+                        v[3 * 4 + cc] = w.w;
+                    }
+                    tmem_st16(sf + q * 16, v);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfready[s]);
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= C::EPI0) {
+        // ----------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int ej = threadIdx.x - C::EPI0 * 32;
+        const int cbeg = ((warp - C::EPI0) >> 2) * (kBN / 2);
+        uint8_t* out_s = smem + C::OUT;
+        int local = 0;
+        for (int ti = blockIdx.x; ti < t_end; ti += gridDim.x, ++local) {
+            const GemmTile t = a.tiles[ti];
+            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
+            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
+            const float gsc = a.g_w[t.expert] * a.g_act;
+            epi_sync();
+            if (ej == 0) ep_stop = abort_flag;
+            if (ej < t.count) {
+                const int slot = __ldg(a.perm + t.seg + ej);
+                ep_scale[ej] = MODE == 0 ? gsc : gsc * __ldg(a.topk_w + slot);
+                ep_row[ej] = MODE == 0 ? t.seg + ej : slot;
+            }
+            epi_sync();
+            if (ep_stop) break;
+            if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 16)) continue;
+            tc_fence_after();
+            const int n_mma = (t.count + 15) & ~15;
+            const int cend = min(n_mma, cbeg + kBN / 2);
+            for (int c0 = cbeg; c0 < cend; c0 += 16) {
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0;
+                float v0[16];
+                tmem_ld16(taddr, v0);
+                if constexpr (MODE == 0) {
+                    float v1[16];
+                    tmem_ld16(taddr + kBN, v1);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = c0 + i;
+                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                        const float act = swiglu_fast(v0[i] * sc, v1[i] * sc);
+                        // NVFP4 of 16 consecutive outputs (lanes) with the static global scale
+                        float amax = fabsf(act);
+#pragma unroll
+                        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                        const float gq = a.g_req;
+                        uint32_t sbc = 0;
+                        float rcp = 0.0f;
+                        if (gq != 0.0f) {
+                            sbc = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, gq)));
+                            const float sbv = e4m3_to_f32(sbc);
+                            rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, gq));
+                        }
+                        const uint32_t code = f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu;
+                        const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+                        if ((lane & 1) == 0) out_s[col * 80 + (row >> 1)] = (uint8_t)(code | (hi << 4));
+                        if ((lane & 15) == 0) out_s[col * 80 + 64 + (row >> 4)] = (uint8_t)sbc;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = c0 + i;
+                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                        reinterpret_cast<uint16_t*>(out_s)[col * kBlkN + row] = __half_as_ushort(f16_sat(v0[i] * sc));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            epi_sync();
+            if constexpr (MODE == 0) {
+                // per token: 64 code bytes and 8 scale bytes of this 128-row block
+                const int I2 = a.out_ld / 2, I16 = a.out_ld / 16;
+                for (int i = ej; i < t.count * 5; i += kEpiWarps * 32) {
+                    const int col = i / 5, part = i % 5;
+                    const size_t r = (size_t)ep_row[col];
+                    if (part < 4)
+                        *reinterpret_cast<uint4*>(a.out4 + r * I2 + t.rb * 64 + part * 16) =
+                            *reinterpret_cast<const uint4*>(out_s + col * 80 + part * 16);
+                    else
+                        *reinterpret_cast<uint2*>(a.out_sf + r * I16 + t.rb * 8) =
+                            *reinterpret_cast<const uint2*>(out_s + col * 80 + 64);
+                }
+            } else {
+                const uint16_t* o16 = reinterpret_cast<const uint16_t*>(out_s);
+                uint16_t* dst = reinterpret_cast<uint16_t*>(a.o16);
+                const int col0 = t.rb * kBlkN;
+                for (int i = ej; i < t.count * 16; i += kEpiWarps * 32) {
+                    const int col = i >> 4, ch = i & 15;
+                    *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) =
+                        *reinterpret_cast<const uint4*>(o16 + col * kBlkN + ch * 8);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+}
+
+// W4A4 activations of the gate/up GEMM in permuted order: row p of the
+// operand is token perm[p] / k, quantized per 16 values with the static
+// global scale g (codes [slots][H/2], low nibble = even column; scales
+// [slots][H/16]); one thread per 16-value block.
+__global__ void k_act_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int slots, int H,
+                               int k, float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per = H / 16;
+    if (i >= (long long)slots * per) return;
+    const int p = (int)(i / per), b = (int)(i % per);
+    const int t = __ldg(perm + p) / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + b * 16);
+    const uint4 q0 = src[0], q1 = src[1];
+    const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float v[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        v[2 * q] = bf16_lo(wv[q]);
+        v[2 * q + 1] = bf16_hi(wv[q]);
+        amax = fmaxf(amax, fmaxf(fabsf(v[2 * q]), fabsf(v[2 * q + 1])));
+    }
+    uint32_t sbc = 0;
+    float r = 0.0f;
+    if (g != 0.0f) {
+        sbc = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+        const float sbv = e4m3_to_f32(sbc);
+        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
+    }
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], r), __fmul_rn(v[2 * q + 1], r)) << (8 * (q & 3));
+    *reinterpret_cast<uint2*>(codes + (size_t)p * (H / 2) + b * 8) = make_uint2(w[0], w[1]);
+    sf[(size_t)p * (H / 16) + b] = (uint8_t)sbc;
+}
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -736,6 +1044,21 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
     return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D map over bytes [rows, row_bytes]: box box_bytes x box_rows, 128-byte
+// swizzle for operand tiles, none for scale tiles
+static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
+                        uint32_t box_rows, bool sw128) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_bytes, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I) {
@@ -784,6 +1107,100 @@ cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E,
     return launch_gemm<2, true>(m_x, g, st, &m_w, g.n_tiles < num_sms() ? g.n_tiles : num_sms());
 }
 
+// Block-scaled NVFP4 GEMM over the routed tiles; maps: A of gate (or down),
+// A of up, their scale tiles, B and its scale tiles.
+template <int MODE>
+static cudaError_t launch_fp4(const CUtensorMap (&m)[6], const GemmArgs& g, cudaStream_t st) {
+    constexpr int bytes = Fp4Cfg<MODE>::ALLOC;
+    cudaError_t err = cudaFuncSetAttribute(k_fp4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err != cudaSuccess) return err;
+    k_fp4_gemm<MODE><<<num_sms(), Fp4Cfg<MODE>::THREADS, bytes, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], g);
+    return cudaGetLastError();
+}
+
+// The prefill path of NVFP4 layers: activations quantized into permuted
+// rows, block-scaled gate/up (intermediate requantized to NVFP4), block-scaled
+// down; the bf16 shared expert and the combine as in the other formats.
+static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
+    const ExpertArgs& ex = p.ex;
+    const int T = p.T, k = ex.k, H = ex.H, I = ex.I, E = ex.E;
+    const int slots = T * k;
+    const bool has_sh = ex.sh_gate != nullptr;
+    uint8_t* xc = reinterpret_cast<uint8_t*>(p.xp);                  // [slots][H/2] e2m1
+    uint8_t* xs = xc + (size_t)slots * H / 2;                          // [slots][H/16] e4m3
+    uint8_t* a4 = reinterpret_cast<uint8_t*>(p.a_perm);               // [slots][I/2]
+    uint8_t* as = a4 + (size_t)slots * I / 2;                          // [slots][I/16]
+    {
+        const long long nb = (long long)slots * (H / 16);
+        k_act_fp4_perm<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)p.x, p.perm, slots, H, k,
+                                                                      ex.g_x, xc, xs);
+    }
+    // ---- gate / up
+    CUtensorMap m[6], m_shared;
+    if (!make_map_u8(&m[0], p.fp4_codes[0], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
+        !make_map_u8(&m[1], p.fp4_codes[1], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
+        !make_map_u8(&m[2], p.fp4_scales[0], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
+        !make_map_u8(&m[3], p.fp4_scales[1], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
+        !make_map_u8(&m[4], xc, (uint64_t)slots, H / 2, 128, kBN, true) ||
+        !make_map_u8(&m[5], xs, (uint64_t)slots, H / 16, 16, kBN, false) ||
+        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, kBN))
+        return cudaErrorInvalidValue;
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    GemmArgs g{};
+    g.quant = ex.quant;
+    g.sh0 = ex.sh_gate;
+    g.sh1 = ex.sh_up;
+    g.perm = p.perm;
+    g.tiles = p.tiles;
+    g.num_tiles = p.num_tiles;
+    g.K = H;
+    g.k_top = k;
+    g.n_rows = I;
+    g.out_ld = I;
+    g.out_sh = p.a_sh;
+    g.out4 = a4;
+    g.out_sf = as;
+    g.g_w = ex.g_gate;
+    g.g_act = ex.g_x;
+    g.g_req = ex.g_a;
+    g.err = p.err;
+    if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
+    cudaError_t err = launch_fp4<0>(m, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
+    if (err != cudaSuccess) return err;
+    if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
+    // ---- down
+    if (!make_map_u8(&m[0], p.fp4_codes[2], (uint64_t)E * H, I / 2, 128, kBlkN, true) ||
+        !make_map_u8(&m[2], p.fp4_scales[2], (uint64_t)E * H, I / 16, 16, kBlkN, false) ||
+        !make_map_u8(&m[4], a4, (uint64_t)slots, I / 2, 128, kBN, true) ||
+        !make_map_u8(&m[5], as, (uint64_t)slots, I / 16, 16, kBN, false) ||
+        !make_map(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I, kBN))
+        return cudaErrorInvalidValue;
+    m[1] = m[0];
+    m[3] = m[2];
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    g.sh0 = ex.sh_down;
+    g.sh1 = nullptr;
+    g.K = I;
+    g.n_rows = H;
+    g.out_ld = H;
+    g.out_sh = nullptr;
+    g.o16 = p.o;
+    g.o16_sh = p.o_sh;
+    g.topk_w = p.w;
+    g.g_w = ex.g_down;
+    g.g_act = ex.g_a;
+    if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
+    err = launch_fp4<1>(m, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
+    if (err != cudaSuccess) return err;
+    if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
+    const long long threads = (long long)T * (H / 8);
+    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, T, H, k,
+                                                               (__nv_bfloat16*)p.y);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const ExpertArgs& ex = p.ex;
     const int T = p.T, k = ex.k, H = ex.H, I = ex.I, E = ex.E;
@@ -791,6 +1208,10 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st);
     if (err != cudaSuccess) return err;
     const bool fp4 = ex.quant == Q_NVFP4;
+    // NVFP4 W4A4 on the block-scaled tensor cores when the shapes allow
+    // 256-value stages (else the exact bf16 dequantization path below)
+    const bool native = fp4 && p.fp4_codes[0] && H % kFp4KS == 0 && I % kFp4KS == 0;
+    if (native) return launch_prefill_fp4(p, st);
     const __nv_bfloat16* xin = nullptr;
     CUtensorMapDataType xdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (fp4) {

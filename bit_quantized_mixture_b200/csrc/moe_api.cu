@@ -26,6 +26,8 @@ struct moe_layer {
     uint8_t* experts = nullptr;    // expert e at experts + e * expert_stride
     uint8_t* router = nullptr;     // bf16 [E, H]
     uint8_t* shared[3] = {nullptr, nullptr, nullptr};   // bf16 device layout
+    uint8_t* fp4_codes[3] = {nullptr, nullptr, nullptr};    // NVFP4: natural-layout images [E][N][K/2]
+    uint8_t* fp4_scales[3] = {nullptr, nullptr, nullptr};   //        and their block scales [E][N][K/16]
     float* g_gate = nullptr;       // NVFP4 global scales [E]
     float* g_down = nullptr;
     // workspace
@@ -150,6 +152,15 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     if (c.has_shared)
         for (int m = 0; m < 3; ++m) { shared_off[m] = a; a = align_up(a + (size_t)H * I * 2, 256); }
     const size_t g_off = a; a = align_up(a + sizeof(float) * 2 * E, 256);
+    // NVFP4: the interchange codes and scales kept as natural-layout images,
+    // the operands of the block-scaled prefill GEMM (TMA tiles)
+    size_t img_off[3] = {0, 0, 0}, imgs_off[3] = {0, 0, 0};
+    if (c.quant == MOE_Q_NVFP4)
+        for (int m = 0; m < 3; ++m) {
+            const size_t nk = (size_t)h->geom[m].N * h->geom[m].K * E;
+            img_off[m] = a; a = align_up(a + nk / 2, 256);
+            imgs_off[m] = a; a = align_up(a + nk / 16, 256);
+        }
     h->arena_bytes = a;
     if (cudaMalloc(&h->arena, h->arena_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -157,6 +168,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
         return fail(nullptr, MOE_ERR_OOM, "moe_create: arena of %zu bytes", a);
     }
     h->experts = h->arena + experts_off;
+    if (c.quant == MOE_Q_NVFP4)
+        for (int m = 0; m < 3; ++m) { h->fp4_codes[m] = h->arena + img_off[m]; h->fp4_scales[m] = h->arena + imgs_off[m]; }
     h->router = h->arena + router_off;
     if (c.has_shared)
         for (int m = 0; m < 3; ++m) h->shared[m] = h->arena + shared_off[m];
@@ -272,7 +285,8 @@ moe_status moe_load_router(moe_handle h, const void* w_router_any, moe_stream_t 
 }
 
 static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix& q, uint8_t* dst_codes,
-                              uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st) {
+                              uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st, uint8_t* img_codes = nullptr,
+                              uint8_t* img_scales = nullptr) {
     const size_t codes_in = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K * 2
                                                : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : 2);
     const size_t scales_in = gm.scales_bytes();
@@ -285,6 +299,11 @@ static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: copy");
     e = launch_relayout(gm, h->staging, h->staging + o_s, h->staging + o_z, dst_codes, dst_scales, dst_zeros, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: relayout");
+    if (img_codes) {   // NVFP4: the interchange layout is the prefill GEMM's operand image
+        e = cudaMemcpyAsync(img_codes, h->staging, codes_in, cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(img_scales, h->staging + o_s, scales_in, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: NVFP4 image");
+    }
     return MOE_OK;
 }
 
@@ -321,7 +340,11 @@ moe_status moe_load_expert_weights(moe_handle h, int32_t expert, const moe_exper
             s = load_matrix(h, gm, *mats[m], h->shared[m], nullptr, nullptr, st);
         } else {
             uint8_t* base = h->experts + (size_t)expert * h->expert_stride;
-            s = load_matrix(h, gm, *mats[m], base + h->off_codes[m], base + h->off_scales[m], base + h->off_zeros[m], st);
+            const size_t nk = (size_t)gm.N * gm.K;
+            uint8_t* ic = h->fp4_codes[m] ? h->fp4_codes[m] + (size_t)expert * nk / 2 : nullptr;
+            uint8_t* is = h->fp4_scales[m] ? h->fp4_scales[m] + (size_t)expert * nk / 16 : nullptr;
+            s = load_matrix(h, gm, *mats[m], base + h->off_codes[m], base + h->off_scales[m], base + h->off_zeros[m], st,
+                            ic, is);
         }
         if (s != MOE_OK) return s;
     }
@@ -463,6 +486,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
+        for (int m = 0; m < 3; ++m) { p.fp4_codes[m] = h->fp4_codes[m]; p.fp4_scales[m] = h->fp4_scales[m]; }
         p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_prefill(p, st);

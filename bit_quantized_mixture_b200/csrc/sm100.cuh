@@ -100,6 +100,15 @@ MOE_DEV void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, u
                  "  tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
                  ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T with e2m1 operands (K = 64 per
+// instruction) and one e4m3 scale per 16 values of each row (A) and column
+// (B) read from TMEM (sfa, sfb: 4 columns each), fp32 accumulation
+MOE_DEV void mma_fp4_block16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t sfa,
+                             uint32_t sfb, uint32_t accumulate) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %6, 0;\n"
+                 "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p; }"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+}
 // arrive on bar once all previously issued MMAs of this thread completed
 MOE_DEV void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -151,6 +160,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 7)                      // A format bf16
          | (1u << 10)                     // B format bf16
          | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+// Block-scaled instruction descriptor: e2m1 A and B (K-major), e4m3 scale
+// factors (scale-factor ids 0), dense K = 64, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+    return (1u << 7)                      // A format E2M1
+         | (1u << 10)                     // B format E2M1
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | (0u << 23)                     // scale format UE4M3
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 // Same with fp16 A/B.

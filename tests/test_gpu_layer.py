@@ -244,6 +244,18 @@ def test_prefill_matches_oracle(quant, T):
     assert_close_output(y, y_ref)
 
 
+# H and I multiples of 256: NVFP4 runs the block-scaled (e2m1 x e2m1, e4m3
+# scales in TMEM) tensor-core GEMMs instead of the bf16 dequantization path
+NATIVE_FP4 = synth.custom("tiny-int4", quant="nvfp4", H=512, I=256, E=24, k=6, shared=True)
+
+
+@pytest.mark.parametrize("T", [5, 37, 300])
+def test_prefill_nvfp4_block_scaled_matches_oracle(T):
+    y, y_ref, layer, _ = _forward_case(NATIVE_FP4, T)
+    layer.sync_status()
+    assert_close_output(y, y_ref)
+
+
 def test_prefill_one_expert_takes_many_tokens():
     """All tokens on the same experts: segments of several 128-token tiles."""
     wl = MID["int4"]
