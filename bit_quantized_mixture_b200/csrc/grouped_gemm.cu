@@ -54,33 +54,36 @@ template <int MODE, bool SH>
 struct Cfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
     // k-blocks (64 columns) per pipeline stage: routed stages cover 128
-    // columns, which halves the barrier round trips, commits and dequant
-    // hand-offs per MMA (a single thread issues every MMA of a matrix, and
-    // its per-instruction cost, not the tensor pipe, bounds small tiles)
+    // columns, which halves the barrier round trips and commits per MMA
     static constexpr int KSTEP = SH ? 1 : 2;
+    // S: stages of the token operand ring, which for routed tiles are also
+    // the TMEM slots of the dequantized weights (a slot and its token tile
+    // are released by the same MMA commit)
     static constexpr int S = SH ? (MODE == 0 ? 3 : 4) : (MODE == 0 ? 2 : 4);
-    // one MMA-issuing warp per matrix: gate and up accumulate independently
-    static constexpr int MMA_WARPS = NMAT;
-    static constexpr int DEQ0 = kWarpMma + MMA_WARPS;                 // first dequant warp
-    // dequant warps: groups of 4 * NMAT (one warp per TMEM lane quarter and
-    // matrix, one thread per weight row) take turns over the stages, so that
-    // DEQ_GROUPS stages are converted at once and the fixed latency of a
-    // stage (staged codes in, TMEM stores out) overlaps; a stage always
-    // belongs to the same group (S % DEQ_GROUPS == 0), which keeps the
-    // mbarrier parities unambiguous
-    static constexpr int DEQ_WARPS = SH ? 0 : 8 * NMAT;
-    static constexpr int DEQ_GROUP_WARPS = 4 * NMAT;
-    static constexpr int DEQ_GROUPS = SH ? 1 : DEQ_WARPS / DEQ_GROUP_WARPS;
+    // SC: stages of the packed-weight ring (routed), decoupled from the TMEM
+    // slots so that the HBM reads of the codes run several stages ahead
+    static constexpr int SC = SH ? 0 : 6;
+    // MMA-issuing warps: gate/up, one per matrix (each stage gets NMAT
+    // commits); routed down, two that take alternate tiles (accumulator
+    // buffer j & 1), so that a second issuer works while the first waits
+    static constexpr int MMA_WARPS = (MODE == 1 && !SH) ? 2 : NMAT;
+    static constexpr bool TILE_SPLIT = MMA_WARPS > NMAT;
+    // routed: a second producer warp loads the token operand, the first the
+    // packed weights
+    static constexpr int BPROD = kWarpMma + MMA_WARPS;
+    static constexpr int DEQ0 = BPROD + (SH ? 0 : 1);                  // first dequant warp
+    // dequant warps: one per (TMEM lane quarter, matrix, k-block of the
+    // stage), one thread per weight row; all of them convert every stage
+    static constexpr int DEQ_WARPS = SH ? 0 : 4 * NMAT * KSTEP;
     static constexpr int EPI0 = DEQ0 + DEQ_WARPS;                    // first epilogue warp
     static constexpr int THREADS = (EPI0 + kEpiWarps) * 32;
     // accumulators: NMAT x 128 columns per buffer; routed gate/up keeps one
-    // buffer so that its A stages fit in the 512 columns
+    // buffer so that its A slots fit in the 512 columns
     static constexpr int ACC_BUFS = (SH || MODE == 1) ? 2 : 1;
     static constexpr int ACC_COLS = NMAT * kBN;
-    static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;   // TMEM column of A stage 0 (routed)
+    static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;   // TMEM column of A slot 0 (routed)
     static constexpr int A_STAGE_COLS = NMAT * KSTEP * 32;
     static_assert(SH || A_COL0 + S * A_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
-    static_assert(SH || S % DEQ_GROUPS == 0, "a stage belongs to one dequant group");
     // staged packed bytes of one matrix and stage: KSTEP blocks of codes,
     // then the scales (INT4/INT2: the one 128-column group; NVFP4: KSTEP x
     // 512), then the INT2 zero points
@@ -88,12 +91,34 @@ struct Cfg {
     // shared memory
     static constexpr int A = 0;                                           // SH: [S][NMAT][16 KB]
     static constexpr int B = A + (SH ? S * NMAT * kATile : 0);            // [S][KSTEP][16 KB]
-    static constexpr int STG = B + S * KSTEP * kBTile;                    // routed: [S][NMAT][STG_MAT]
-    static constexpr int OUT = STG + (SH ? 0 : S * NMAT * STG_MAT);       // [128][128] 16-bit
+    static constexpr int STG = B + S * KSTEP * kBTile;                    // routed: [SC][NMAT][STG_MAT]
+    static constexpr int OUT = STG + SC * NMAT * STG_MAT;                 // [128][128] 16-bit
     static constexpr int BYTES = OUT + (MODE == 2 ? 0 : kOutTile);
     static constexpr int ALLOC = BYTES + 1024;                            // slack for 1024-byte alignment
-    static_assert(ALLOC <= 227 * 1024 - 2048, "shared memory budget");
+    static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
+
+// Token-operand tensor maps with boxes of 128, 64, 32 and 16 rows: a tile
+// of n (a multiple of 16) tokens loads only its n rows, as at most three
+// boxes at 16-row (2 KB, swizzle-atom aligned) offsets.
+struct BMaps {
+    CUtensorMap m[4];
+};
+MOE_DEV uint32_t load_token_rows(uint8_t* dst, const BMaps& mb, int x, int y, int n, uint64_t* bar) {
+    const int n16 = n >> 4;
+    if (n16 >= 8) {
+        tma_load_2d(dst, &mb.m[0], x, y, bar);
+        return 128u * 128u;
+    }
+    int off = 0;
+#pragma unroll
+    for (int b = 2; b >= 0; --b)
+        if (n16 & (1 << b)) {
+            tma_load_2d(dst + off * 128, &mb.m[3 - b], x, y + off, bar);
+            off += 16 << b;
+        }
+    return (uint32_t)off * 128u;
+}
 
 struct GemmArgs {
     int quant;                // routed weight format
@@ -118,6 +143,8 @@ struct GemmArgs {
     float* logits;            // mode 2: [n_tok, n_rows] fp32
     int n_tok, n_rows;        // mode 2: tokens, router rows (experts)
     int n_tiles;              // mode 2: (row blocks) x (token blocks)
+    const float* w_perm;      // routing weight of each permuted position (down)
+    const float* ts_perm;     // INT4/INT2 gate/up: token scale of each permuted position
     uint8_t* out4;            // NVFP4 gate/up: e2m1 intermediate [slots, I/2] (permuted rows)
     uint8_t* out_sf;          // NVFP4 gate/up: its e4m3 block scales [slots, I/16]
     int* err;
@@ -226,14 +253,74 @@ MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
 
 // SwiGLU of one accumulator pair: silu(g) * u with the fast exponential and
-// reciprocal (relative error ~1e-6, far below the bf16 / e2m1 rounding of
+// division (relative error ~1e-6, far below the bf16 / e2m1 rounding of
 // the stored intermediate)
-MOE_DEV float swiglu_fast(float g, float u) { return g * __frcp_rn(1.0f + __expf(-g)) * u; }
+MOE_DEV float swiglu_fast(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
+
+// Accumulator placement. ACC_BUFS == 2: tile j takes buffer j & 1 (NMAT x
+// 128 columns each). Routed gate/up keeps one 256-column buffer: a tile of
+// at most 64 tokens takes one 128-column half (gate, then up 64 columns
+// further), so that two such tiles alternate and the epilogue of one
+// overlaps the MMAs of the next; a larger tile takes both halves (gate at
+// 0, up at 128). The MMA warps and the epilogue walk the same sequence.
+struct AccSeq {
+    uint32_t uses0 = 0, uses1 = 0;
+    int next = 0;
+};
+struct AccUse {
+    int mask;               // bit b: buffer (half) b
+    uint32_t col;           // first column of the matrix-0 accumulator
+    uint32_t mat_stride;    // columns from matrix 0 to matrix 1
+    uint32_t par0, par1;    // phase parity of this use of buffer 0 / 1
+};
+template <int ACC_BUFS, int ACC_COLS>
+MOE_DEV AccUse acc_next(AccSeq& q, int n_mma) {
+    AccUse u;
+    if (ACC_BUFS == 2) {
+        u.mask = 1 << q.next;
+        u.col = (uint32_t)(q.next * ACC_COLS);
+        u.mat_stride = kBN;
+    } else if (n_mma > 64) {
+        u.mask = 3;
+        u.col = 0;
+        u.mat_stride = kBN;
+    } else {
+        u.mask = 1 << q.next;
+        u.col = (uint32_t)(q.next * kBN);
+        u.mat_stride = 64;
+    }
+    u.par0 = q.uses0 & 1u;
+    u.par1 = q.uses1 & 1u;
+    q.uses0 += (uint32_t)(u.mask & 1);
+    q.uses1 += (uint32_t)(u.mask >> 1);
+    q.next = u.mask == 3 ? 0 : (q.next ^ 1);
+    return u;
+}
+
+struct PermMeta {
+    const float* topk_w;      // [T*k] routing weight of each slot
+    const float* tok_scale;   // [T] fp16 activation scale of each token, or null
+    float* w_perm;            // [T*k] out: routing weight of each permuted position
+    float* ts_perm;           // [T*k] out: token scale of each permuted position
+};
+
+// A CTA's tiles (ti = first + j * gridDim.x) are copied into shared memory
+// once, so that no role waits on a global load at the start of a tile.
+constexpr int kTileCache = 256;
+struct TileCache {
+    GemmTile t[kTileCache];
+};
+MOE_DEV void cache_tiles(TileCache& tc, const GemmTile* tiles, int first, int end) {
+    for (int j = threadIdx.x; j < kTileCache; j += blockDim.x) {
+        const int ti = first + j * gridDim.x;
+        if (ti < end) tc.t[j] = tiles[ti];
+    }
+}
 
 // Tile ti: from the device-built list, or (router) row block ti % RB of
 // token block ti / RB.
 template <int MODE>
-MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti) {
+MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = nullptr, int first = 0) {
     if constexpr (MODE == 2) {
         const int RB = (a.n_rows + kBlkN - 1) / kBlkN;
         GemmTile t;
@@ -243,35 +330,46 @@ MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti) {
         t.count = min(kBN, a.n_tok - t.seg);
         return t;
     } else {
-        return a.tiles[ti];
+        const int j = (ti - first) / (int)gridDim.x;
+        return (tc && j < kTileCache) ? tc->t[j] : a.tiles[ti];
     }
 }
 
 // ------------------------------------------------------------------ kernel
 template <int MODE, bool SH>
 __global__ void __launch_bounds__(Cfg<MODE, SH>::THREADS, 1)
-k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a, GemmArgs a) {
+k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUtensorMap map_a, GemmArgs a) {
     using C = Cfg<MODE, SH>;
     constexpr int NMAT = C::NMAT, S = C::S, KSTEP = C::KSTEP;
+    constexpr int SC = C::SC > 0 ? C::SC : 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t wfull[S], full[S], empty[S], acc_full[2], acc_empty[2];
+    __shared__ uint64_t cfull[SC], cempty[SC], full[S], empty[S], acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
     __shared__ float ep_scale[kBN];             // epilogue: per token column of the current tile
     __shared__ int ep_row[kBN];
     __shared__ int ep_stop;
+    __shared__ TileCache tcache;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    {
+        const int tb = (SH && MODE != 2) ? __ldcg(a.num_tiles) : 0;
+        const int te = MODE == 2 ? a.n_tiles : SH ? __ldcg(a.num_tiles + 1) : __ldcg(a.num_tiles);
+        if (MODE != 2) cache_tiles(tcache, a.tiles, tb + blockIdx.x, te);
+    }
     if (threadIdx.x == 0) {
+        for (int c = 0; c < SC; ++c) {
+            mbar_init(&cfull[c], 1);                      // codes producer (bytes)
+            mbar_init(&cempty[c], C::DEQ_WARPS);          // every dequant warp has read its part
+        }
         for (int s = 0; s < S; ++s) {
-            mbar_init(&wfull[s], 1);
-            // producer (bytes) [+ one arrival per warp of the stage's dequant group]
-            mbar_init(&full[s], SH ? 1 : 1 + C::DEQ_GROUP_WARPS);
-            mbar_init(&empty[s], C::MMA_WARPS);           // one commit per MMA warp
+            // token producer (bytes) [+ one arrival per dequant warp]
+            mbar_init(&full[s], 1 + C::DEQ_WARPS);
+            mbar_init(&empty[s], NMAT);                   // one commit per matrix
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], C::MMA_WARPS);
+            mbar_init(&acc_full[b], NMAT);
             mbar_init(&acc_empty[b], kEpiWarps);          // one arrival per epilogue warp
         }
         abort_flag = 0;
@@ -284,13 +382,54 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
     const uint32_t tmem = tmem_base_slot;
     const int t_begin = (SH && MODE != 2) ? __ldcg(a.num_tiles) : 0;
     const int t_end = MODE == 2 ? a.n_tiles : SH ? __ldcg(a.num_tiles + 1) : __ldcg(a.num_tiles);
+    const int t_first = t_begin + blockIdx.x;
     const int NS = a.K / (kBlkK * KSTEP);                 // stages per tile
 
-    if (warp == kWarpProducer) {
-        // ---------------------------------------------------------- producer
+    if (warp == kWarpProducer && !SH) {
+        // ------------------------------------------- producer: packed weights
+        // the codes of KSTEP consecutive blocks are contiguous, and so are
+        // their NVFP4 scales
+        const int KB = a.K / kBlkK, G = a.K / kGroup;
+        const int cb = block_code_bytes(a.quant) * KSTEP;
+        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : 256;
+        const int zb = a.quant == Q_INT2 ? 128 : 0;
         int g = 0;
-        for (int ti = t_begin + blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = load_tile<MODE>(a, ti);
+        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
+            bool ok = true;
+            for (int ks = 0; ks < NS; ++ks, ++g) {
+                const int c = g % SC;
+                if (!warp_wait(&cempty[c], ((uint32_t)(g / SC) & 1u) ^ 1u, &abort_flag, a.err, 1)) { ok = false; break; }
+                if (lane == 0) {
+                    const int kb0 = ks * KSTEP;
+                    uint8_t* stg = smem + C::STG + c * NMAT * C::STG_MAT;
+                    mbar_arrive_expect_tx(&cfull[c], (uint32_t)(NMAT * (cb + sb + zb)));
+                    for (int m = 0; m < NMAT; ++m) {
+                        const MatView& v = m == 0 ? a.w0 : a.w1;
+                        const size_t eo = (size_t)t.expert * v.stride;
+                        uint8_t* d = stg + m * C::STG_MAT;
+                        bulk_g2s(d, v.codes + eo + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
+                                 &cfull[c]);
+                        if (a.quant == Q_NVFP4) {
+                            bulk_g2s(d + cb, v.scales + eo + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
+                        } else {
+                            const size_t go = ((size_t)t.rb * G + kb0 / 2) * 256;   // kb0 even: one group
+                            bulk_g2s(d + cb, v.scales + eo + go, sb, &cfull[c]);
+                            if (zb) bulk_g2s(d + cb + sb, v.zeros + eo + go / 2, zb, &cfull[c]);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+        }
+    } else if ((SH && warp == kWarpProducer) || (!SH && warp == C::BPROD)) {
+        // ---------------------------------------- producer: token operand
+        // (+ the router / shared-expert weight tiles)
+        int g = 0;
+        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
+            const int n_mma = (t.count + 15) & ~15;
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
@@ -299,69 +438,57 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
                 if (lane == 0) {
                     const int kb0 = ks * KSTEP;
                     uint8_t* B = smem + C::B + s * KSTEP * kBTile;
+                    const uint32_t tb = (uint32_t)KSTEP * (uint32_t)n_mma * 128u;
                     if constexpr (MODE == 2) {
-                        mbar_arrive_expect_tx(&full[s], kBTile + kATile);
+                        mbar_arrive_expect_tx(&full[s], tb + kATile);
                         tma_load_2d(smem + C::A + s * kATile, &map_a, kb0 * kBlkK, t.rb * kBlkN, &full[s]);
                     } else if constexpr (SH) {
                         uint8_t* A = smem + C::A + s * NMAT * kATile;
-                        mbar_arrive_expect_tx(&full[s], kBTile + NMAT * kATile);
+                        mbar_arrive_expect_tx(&full[s], tb + NMAT * kATile);
                         for (int m = 0; m < NMAT; ++m) {
                             const uint8_t* img = (m == 0 ? a.sh0 : a.sh1) + ((size_t)t.rb * (a.K / kBlkK) + kb0) * kATile;
                             bulk_g2s(A + m * kATile, img, kATile, &full[s]);
                         }
                     } else {
-                        // the codes of KSTEP consecutive blocks are contiguous,
-                        // and so are their NVFP4 scales
-                        uint8_t* stg = smem + C::STG + s * NMAT * C::STG_MAT;
-                        const int KB = a.K / kBlkK, G = a.K / kGroup;
-                        const int cb = block_code_bytes(a.quant) * KSTEP;
-                        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : 256;
-                        const int zb = a.quant == Q_INT2 ? 128 : 0;
-                        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(NMAT * (cb + sb + zb)));
-                        for (int m = 0; m < NMAT; ++m) {
-                            const MatView& v = m == 0 ? a.w0 : a.w1;
-                            const size_t eo = (size_t)t.expert * v.stride;
-                            uint8_t* d = stg + m * C::STG_MAT;
-                            bulk_g2s(d, v.codes + eo + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
-                                     &wfull[s]);
-                            if (a.quant == Q_NVFP4) {
-                                bulk_g2s(d + cb, v.scales + eo + ((size_t)t.rb * KB + kb0) * 512, sb, &wfull[s]);
-                            } else {
-                                const size_t go = ((size_t)t.rb * G + kb0 / 2) * 256;   // kb0 even: one group
-                                bulk_g2s(d + cb, v.scales + eo + go, sb, &wfull[s]);
-                                if (zb) bulk_g2s(d + cb + sb, v.zeros + eo + go / 2, zb, &wfull[s]);
-                            }
-                        }
-                        mbar_arrive_expect_tx(&full[s], KSTEP * kBTile);
+                        mbar_arrive_expect_tx(&full[s], tb);
                     }
-                    // token rows t.seg .. t.seg + 127 (a whole box; rows past
-                    // the end of the operand read as zero)
+                    // token rows t.seg .. t.seg + n_mma - 1 (rows past the
+                    // end of the operand read as zero)
                     for (int j = 0; j < KSTEP; ++j)
-                        tma_load_2d(B + j * kBTile, &map_b, (kb0 + j) * kBlkK, t.seg, &full[s]);
+                        load_token_rows(B + j * kBTile, map_b, (kb0 + j) * kBlkK, t.seg, n_mma, &full[s]);
                 }
                 __syncwarp();
             }
             if (!ok) break;
         }
-    } else if (warp >= kWarpMma && warp < C::DEQ0) {
+    } else if (warp >= kWarpMma && warp < kWarpMma + C::MMA_WARPS) {
         // --------------------------------------------------------- MMA issue
         // warp kWarpMma + m issues the MMAs of matrix m (gate/up: two warps)
-        const int mi = warp - kWarpMma;
+        const int mi = C::TILE_SPLIT ? 0 : warp - kWarpMma;
         int g = 0, local = 0;
-        for (int ti = t_begin + blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
-            const GemmTile t = load_tile<MODE>(a, ti);
+        AccSeq aseq;
+        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
             const int n_mma = (t.count + 15) & ~15;
             const bool f16 = MODE == 0 && !SH && a.tok_scale != nullptr;
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
-            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
-            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
-            if (!warp_wait(&acc_empty[ab], (use & 1u) ^ 1u, &abort_flag, a.err, 2)) break;
+            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
+            if (C::TILE_SPLIT && (local & 1) != warp - kWarpMma) {   // the other warp's tile
+                g += NS;
+                continue;
+            }
+            if ((au.mask & 1) && !warp_wait(&acc_empty[0], au.par0 ^ 1u, &abort_flag, a.err, 2)) break;
+            if ((au.mask & 2) && !warp_wait(&acc_empty[1], au.par1 ^ 1u, &abort_flag, a.err, 2)) break;
             tc_fence_after();
             bool ok = true;
-            const uint32_t d = tmem + ab * C::ACC_COLS + mi * kBN;
+            const uint32_t d = tmem + au.col + mi * au.mat_stride;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
+                // with two issuers, one may reach stage g before the other has
+                // consumed stage g - S of the same slot: waiting for that
+                // commit first keeps the parity of full[s] unambiguous
+                if (C::TILE_SPLIT && !warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 7)) { ok = false; break; }
                 if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 3)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
@@ -381,7 +508,10 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
                         }
                     }
                     mma_commit(&empty[s]);
-                    if (ks == NS - 1) mma_commit(&acc_full[ab]);
+                    if (ks == NS - 1) {
+                        if (au.mask & 1) mma_commit(&acc_full[0]);
+                        if (au.mask & 2) mma_commit(&acc_full[1]);
+                    }
                 }
                 __syncwarp();
             }
@@ -389,42 +519,42 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
         }
     } else if (warp >= C::DEQ0 && warp < C::EPI0) {
         // ------------------------------------------------------------ dequant
-        // routed tiles only: thread (row r, matrix m) of its group writes
-        // TMEM lane r (its warp's lane quarter), all KSTEP blocks of a stage
+        // routed tiles only: thread (row r, matrix m, k-block j of the stage)
+        // writes TMEM lane r (its warp's lane quarter)
         if constexpr (!SH) {
             const int quarter = warp & 3;
             const int r = quarter * 32 + lane;                 // weight row = TMEM lane
-            const int wi = warp - C::DEQ0;
-            const int grp = wi / C::DEQ_GROUP_WARPS;
-            const int m = (wi % C::DEQ_GROUP_WARPS) >> 2;
+            const int wi = (warp - C::DEQ0) >> 2;
+            const int m = wi % NMAT, j = wi / NMAT;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool f16 = MODE == 0 && a.tok_scale != nullptr;
             const int cb = block_code_bytes(a.quant);
             int g = 0;
-            for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+            for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
                 bool ok = true;
                 for (int ks = 0; ks < NS; ++ks, ++g) {
-                    if (g % C::DEQ_GROUPS != grp) continue;
-                    const int s = g % S;
-                    const uint32_t rr = (uint32_t)(g / S);
-                    // the stage's staging bytes arrived, so the MMAs that read
-                    // this stage's TMEM columns before have completed
-                    if (!warp_wait(&wfull[s], rr & 1u, &abort_flag, a.err, 4)) { ok = false; break; }
+                    const int c = g % SC, s = g % S;
+                    // the packed codes arrived, and the MMAs that read this
+                    // TMEM slot before have completed
+                    if (!warp_wait(&cfull[c], (uint32_t)(g / SC) & 1u, &abort_flag, a.err, 4) ||
+                        !warp_wait(&empty[s], ((uint32_t)(g / S) & 1u) ^ 1u, &abort_flag, a.err, 6)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint8_t* stg = smem + C::STG + (s * NMAT + m) * C::STG_MAT;
+                    const uint8_t* stg = smem + C::STG + (c * NMAT + m) * C::STG_MAT;
                     const uint8_t* sc = stg + cb * KSTEP;
+                    const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512 : sc;
                     const uint8_t* zr = sc + 256;
                     uint32_t v[16];
 #pragma unroll
-                    for (int j = 0; j < KSTEP; ++j)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512 : sc;
-                            if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
-                            else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
-                            tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h,
-                                      v);
-                        }
+                    for (int h = 0; h < 2; ++h) {
+                        if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
+                        else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
+                        tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h, v);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&cempty[c]);       // this warp's staged bytes are consumed
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
@@ -442,65 +572,95 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;                 // weight row within the block = output column
         const int ej = threadIdx.x - C::EPI0 * 32;           // 0 .. 32 * kEpiWarps - 1
-        const int cbeg = ((warp - C::EPI0) >> 2) * (kBN / 2);   // this warp's 64 token columns
+        const int cset = (warp - C::EPI0) >> 2;              // this warp's half of the token columns
         uint16_t* out_s = reinterpret_cast<uint16_t*>(smem + C::OUT);
         // The epilogue warps leave the loop together (named barriers): the
         // stop decision is taken by one thread between two barriers.
-        int local = 0;
-        for (int ti = t_begin + blockIdx.x; ti < t_end; ti += gridDim.x, ++local) {
-            const GemmTile t = load_tile<MODE>(a, ti);
-            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
-            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
+        // token info of the next tile (scale factor, output row) is loaded
+        // while the current one is processed
+        float nx_sc = 1.0f;
+        int nx_row = 0;
+        auto fetch = [&](int tj) {
+            if (MODE == 2 || tj >= t_end) return;
+            const GemmTile tn = load_tile<MODE>(a, tj, &tcache, t_begin + blockIdx.x);
+            if (ej >= tn.count) return;
+            if constexpr (SH) {
+                nx_sc = 1.0f;
+                nx_row = tn.seg + ej;
+            } else if (MODE == 0) {
+                nx_sc = a.ts_perm ? __ldg(a.ts_perm + tn.seg + ej) : 1.0f;
+                nx_row = tn.seg + ej;
+            } else {
+                nx_sc = __ldg(a.w_perm + tn.seg + ej);
+                nx_row = __ldg(a.perm + tn.seg + ej);
+            }
+        };
+        fetch(t_begin + blockIdx.x);
+        AccSeq aseq;
+        for (int ti = t_begin + blockIdx.x; ti < t_end; ti += gridDim.x) {
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_begin + blockIdx.x);
+            const int n_mma = (t.count + 15) & ~15;
+            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
             float gsc = 1.0f;
             if (!SH && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
             epi_sync();                                      // the previous tile's readers are done
             if (ej == 0) ep_stop = abort_flag;
             if (MODE != 2 && ej < t.count) {
-                if constexpr (SH) {
-                    ep_scale[ej] = 1.0f;
-                    ep_row[ej] = t.seg + ej;
-                } else {
-                    const int slot = __ldg(a.perm + t.seg + ej);
-                    if (MODE == 0) {
-                        ep_scale[ej] = a.tok_scale ? __ldg(a.tok_scale + slot / a.k_top) : gsc;
-                        ep_row[ej] = t.seg + ej;
-                    } else {
-                        ep_scale[ej] = gsc * __ldg(a.topk_w + slot);
-                        ep_row[ej] = slot;
-                    }
-                }
+                ep_scale[ej] = nx_sc * gsc;
+                ep_row[ej] = nx_row;
             }
+            fetch(ti + gridDim.x);
             epi_sync();
             if (ep_stop) break;
             // a failed wait sets abort_flag: this tile is skipped and all four
             // warps stop at the next tile's decision
-            if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 5)) continue;
+            if ((au.mask & 1) && !warp_wait(&acc_full[0], au.par0, &abort_flag, a.err, 5)) continue;
+            if ((au.mask & 2) && !warp_wait(&acc_full[1], au.par1, &abort_flag, a.err, 5)) continue;
             tc_fence_after();
-            const int n_mma = (t.count + 15) & ~15;
-            const int cend = min(n_mma, cbeg + kBN / 2);
+            // the two warps of a lane quarter split the columns (16-aligned)
+            const int chalf = (((n_mma >> 4) + 1) >> 1) << 4;
+            const int cbeg = cset ? chalf : 0, cend = cset ? n_mma : chalf;
+            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + au.col;
             if constexpr (MODE == 2) {
                 // logits: for each token, the 32 lanes store 32 consecutive
                 // experts (128 contiguous bytes)
                 const int e = t.rb * kBlkN + row;
                 for (int c0 = cbeg; c0 < cend; c0 += 16) {
                     float v0[16];
-                    tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0, v0);
+                    tmem_ld16(lane_base + c0, v0);
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         if (c0 + i < t.count && e < a.n_rows) a.logits[(size_t)(t.seg + c0 + i) * a.n_rows + e] = v0[i];
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                if (lane == 0) mbar_arrive(&acc_empty[au.mask >> 1]);
                 continue;
             }
-            for (int c0 = cbeg; c0 < cend; c0 += 16) {
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0;
+            if constexpr (MODE == 1) {
+                // all of this warp's columns (at most 64) in one batch
+                uint32_t r[64];
+                const int nch = (cend - cbeg) >> 4;
+                tmem_ld_chunks(lane_base + cbeg, nch, r);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (q < nch) {
+                        // per-slot outputs are fp16 (saturating at +-65504):
+                        // their rounding error stays well below the final bf16 one
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = cbeg + 16 * q + i;
+                            const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                            out_s[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
+                        }
+                    }
+                }
+            }
+            for (int c0 = cbeg; MODE == 0 && c0 < cend; c0 += 16) {
                 float v0[16];
-                tmem_ld16(taddr, v0);
                 if constexpr (MODE == 0) {
                     float v1[16];
-                    tmem_ld16(taddr + kBN, v1);
+                    tmem_ld16x2(lane_base + c0, lane_base + au.mat_stride + c0, v0, v1);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int col = c0 + i;
@@ -522,20 +682,14 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
                         }
                         out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
                     }
-                } else {
-                    // per-slot outputs are fp16 (saturating at +-65504): their
-                    // rounding error stays well below the final bf16 one
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c0 + i;
-                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                        out_s[col * kBlkN + row] = __half_as_ushort(f16_sat(v0[i] * sc));
-                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);      // the MMA may refill this accumulator
+            if (lane == 0) {                                 // the MMA may refill this accumulator
+                if (au.mask & 1) mbar_arrive(&acc_empty[0]);
+                if (au.mask & 2) mbar_arrive(&acc_empty[1]);
+            }
             epi_sync();                                      // staging tile complete
             uint16_t* dst = MODE == 0 ? reinterpret_cast<uint16_t*>(SH ? a.out_sh : a.out)
                                       : reinterpret_cast<uint16_t*>(SH ? a.o16_sh : a.o16);
@@ -554,9 +708,9 @@ k_grouped_gemm(const __grid_constant__ CUtensorMap map_b, const __grid_constant_
 }
 
 // --------------------------------------------------------------- tile list
-// One CTA of 1024 threads: thread e emits the tiles of expert e, grouped by
-// (expert, row block) so that the token tiles of one weight block are
-// consecutive; the shared expert's tiles (all T tokens) come last.
+// One CTA of 1024 threads. Tile order: by expert, then row block, then
+// token tile, so that the token tiles of one weight block are consecutive;
+// the shared expert's tiles (all T tokens) come last.
 __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict__ counts,
                                                       const int32_t* __restrict__ offsets, int E, int T, int RB,
                                                       int has_shared, GemmTile* __restrict__ tiles,
@@ -564,8 +718,7 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
     __shared__ int sc[1024];
     const int e = threadIdx.x;
     const int cnt = (e < E) ? counts[e] : 0;
-    const int nt = (cnt + kBN - 1) / kBN;
-    const int mine = nt * RB;
+    const int mine = ((cnt + kBN - 1) / kBN) * RB;
     sc[e] = mine;
     __syncthreads();
     for (int o = 1; o < 1024; o <<= 1) {
@@ -574,18 +727,27 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
         sc[e] += v;
         __syncthreads();
     }
-    const int base = sc[e] - mine;
     const int total = sc[1023];
-    if (e < E) {
-        for (int rb = 0; rb < RB; ++rb)
-            for (int tt = 0; tt < nt; ++tt) {
-                GemmTile g;
-                g.expert = e;
-                g.rb = rb;
-                g.seg = offsets[e] + tt * kBN;
-                g.count = min(kBN, cnt - tt * kBN);
-                tiles[base + rb * nt + tt] = g;
-            }
+    // all threads emit the routed tiles: tile i belongs to the expert whose
+    // inclusive prefix is the first one above i (binary search)
+    for (int i = e; i < total; i += 1024) {
+        int lo = 0, hi = 1023;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sc[mid] > i) hi = mid;
+            else lo = mid + 1;
+        }
+        const int ex = lo;
+        const int c = counts[ex];
+        const int ntx = (c + kBN - 1) / kBN;
+        const int j = i - (sc[ex] - ntx * RB);          // index within the expert's tiles
+        const int rb = j / ntx, tt = j % ntx;
+        GemmTile g;
+        g.expert = ex;
+        g.rb = rb;
+        g.seg = offsets[ex] + tt * kBN;
+        g.count = min(kBN, c - tt * kBN);
+        tiles[i] = g;
     }
     const int nts = has_shared ? (T + kBN - 1) / kBN : 0;
     for (int i = e; i < nts * RB; i += 1024) {
@@ -669,15 +831,23 @@ __global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, int T, int H, __
     if (lane == 0) scale[t] = ldexpf(1.0f, p);
 }
 
+// Routing weight and token scale of permuted position p, read by the GEMM
+// epilogues as one independent load per token column.
+MOE_DEV void perm_meta(int p, int slot, int k, const PermMeta& m) {
+    m.w_perm[p] = __ldg(m.topk_w + slot);
+    if (m.tok_scale) m.ts_perm[p] = __ldg(m.tok_scale + slot / k);
+}
+
 // Rows of the gate/up token operand in permuted order: xp[p] = xq[perm[p] / k]
-// (16-byte copies; one thread per 8 columns).
+// (16-byte copies; one thread per 8 columns); also the per-position meta.
 __global__ void k_gather_rows(const __nv_bfloat16* __restrict__ xq, const int32_t* __restrict__ perm, int slots,
-                              int H, int k, __nv_bfloat16* __restrict__ xp) {
+                              int H, int k, __nv_bfloat16* __restrict__ xp, PermMeta meta) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int per_row = H / 8;
     if (i >= (long long)slots * per_row) return;
     const int p = (int)(i / per_row), c = (int)(i % per_row);
-    const int t = __ldg(perm + p) / k;
+    const int slot = __ldg(perm + p), t = slot / k;
+    if (c == 0) perm_meta(p, slot, k, meta);
     reinterpret_cast<uint4*>(xp + (size_t)p * H)[c] = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)t * H) + c);
 }
 
@@ -743,8 +913,10 @@ struct Fp4Cfg {
     static constexpr int SFB = SFA + S * NMAT * kFp4SfTile;           // [S][2 KB]
     static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: [128][128] fp16
     static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : kOutTile;
-    static constexpr int ALLOC = OUT + OUT_BYTES + 1024;
-    static_assert(ALLOC <= 227 * 1024 - 2048, "shared memory budget");
+    static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [16 tok][32] fp32
+    static constexpr int SCR_BYTES = MODE == 0 ? kEpiWarps * 16 * 32 * 4 : 0;
+    static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
+    static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
 
 template <int MODE>
@@ -762,8 +934,15 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     __shared__ float ep_scale[kBN];
     __shared__ int ep_row[kBN];
     __shared__ int ep_stop;
+    __shared__ float rcp_tab[256];              // gate/up: 1 / (e4m3(code) * g_req), IEEE division, 0 for zero
+    __shared__ TileCache tcache;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    cache_tiles(tcache, a.tiles, blockIdx.x, __ldcg(a.num_tiles));
+    if (MODE == 0 && threadIdx.x < 256) {
+        const float sbv = e4m3_to_f32((uint32_t)threadIdx.x);
+        rcp_tab[threadIdx.x] = (sbv == 0.0f || a.g_req == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, a.g_req));
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);                       // producer (bytes)
@@ -789,7 +968,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         // ---------------------------------------------------------- producer
         int g = 0;
         for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = a.tiles[ti];
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
             const int arow = t.expert * a.n_rows + t.rb * kBlkN;
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
@@ -816,7 +995,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int mi = warp - kWarpMma;
         int g = 0, local = 0;
         for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
-            const GemmTile t = a.tiles[ti];
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
             const int n_mma = (t.count + 15) & ~15;
             const uint32_t idesc = idesc_nvfp4(128, n_mma);
             const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
@@ -885,63 +1064,96 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int ej = threadIdx.x - C::EPI0 * 32;
-        const int cbeg = ((warp - C::EPI0) >> 2) * (kBN / 2);
+        const int cset = (warp - C::EPI0) >> 2;              // this warp's half of the token columns
         uint8_t* out_s = smem + C::OUT;
+        float nx_sc = 1.0f;                      // next tile's token info, loaded ahead
+        int nx_row = 0;
+        auto fetch = [&](int tj) {
+            if (tj >= t_end) return;
+            const GemmTile tn = load_tile<MODE>(a, tj, &tcache, blockIdx.x);
+            if (ej >= tn.count) return;
+            nx_sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
+            nx_row = MODE == 0 ? tn.seg + ej : __ldg(a.perm + tn.seg + ej);
+        };
+        fetch(blockIdx.x);
         int local = 0;
         for (int ti = blockIdx.x; ti < t_end; ti += gridDim.x, ++local) {
-            const GemmTile t = a.tiles[ti];
+            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
             const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
             const float gsc = a.g_w[t.expert] * a.g_act;
             epi_sync();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
-                const int slot = __ldg(a.perm + t.seg + ej);
-                ep_scale[ej] = MODE == 0 ? gsc : gsc * __ldg(a.topk_w + slot);
-                ep_row[ej] = MODE == 0 ? t.seg + ej : slot;
+                ep_scale[ej] = nx_sc * gsc;
+                ep_row[ej] = nx_row;
             }
+            fetch(ti + gridDim.x);
             epi_sync();
             if (ep_stop) break;
             if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 16)) continue;
             tc_fence_after();
             const int n_mma = (t.count + 15) & ~15;
-            const int cend = min(n_mma, cbeg + kBN / 2);
-            for (int c0 = cbeg; c0 < cend; c0 += 16) {
-                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS + c0;
+            // the two warps of a lane quarter split the columns (16-aligned)
+            const int chalf = (((n_mma >> 4) + 1) >> 1) << 4;
+            const int cbeg = cset ? chalf : 0, cend = cset ? n_mma : chalf;
+            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS;
+            if constexpr (MODE == 1) {
+                // all of this warp's columns (at most 64) in one batch
+                uint32_t r[64];
+                const int nch = (cend - cbeg) >> 4;
+                tmem_ld_chunks(lane_base + cbeg, nch, r);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (q < nch) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = cbeg + 16 * q + i;
+                            const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                            reinterpret_cast<uint16_t*>(out_s)[col * kBlkN + row] =
+                                __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
+                        }
+                    }
+                }
+            }
+            for (int c0 = cbeg; MODE == 0 && c0 < cend; c0 += 16) {
                 float v0[16];
-                tmem_ld16(taddr, v0);
                 if constexpr (MODE == 0) {
                     float v1[16];
-                    tmem_ld16(taddr + kBN, v1);
+                    tmem_ld16x2(lane_base + c0, lane_base + kBN + c0, v0, v1);
+                    // SwiGLU of 16 tokens x this warp's 32 outputs into the warp's scratch
+                    float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 16 * 32;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int col = c0 + i;
-                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                        const float act = swiglu_fast(v0[i] * sc, v1[i] * sc);
-                        // NVFP4 of 16 consecutive outputs (lanes) with the static global scale
-                        float amax = fabsf(act);
+                        const float sc = c0 + i < t.count ? ep_scale[c0 + i] : 0.0f;
+                        scr[i * 32 + lane] = swiglu_fast(v0[i] * sc, v1[i] * sc);
+                    }
+                    __syncwarp();
+                    // lane = (token i, 16-output block b): NVFP4 with the static global
+                    // scale; code decisions in fp32 as the format defines them
+                    {
+                        const int i = lane & 15, b = lane >> 4;
+                        const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
+                        float v[16];
 #pragma unroll
-                        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                        const float gq = a.g_req;
-                        uint32_t sbc = 0;
-                        float rcp = 0.0f;
-                        if (gq != 0.0f) {
-                            sbc = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, gq)));
-                            const float sbv = e4m3_to_f32(sbc);
-                            rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, gq));
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 f4 = src[q];
+                            v[4 * q] = f4.x; v[4 * q + 1] = f4.y; v[4 * q + 2] = f4.z; v[4 * q + 3] = f4.w;
                         }
-                        const uint32_t code = f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu;
-                        const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
-                        if ((lane & 1) == 0) out_s[col * 80 + (row >> 1)] = (uint8_t)(code | (hi << 4));
-                        if ((lane & 15) == 0) out_s[col * 80 + 64 + (row >> 4)] = (uint8_t)sbc;
-                    }
-                } else {
+                        float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c0 + i;
-                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                        reinterpret_cast<uint16_t*>(out_s)[col * kBlkN + row] = __half_as_ushort(f16_sat(v0[i] * sc));
+                        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+                        const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
+                        const float rcp = rcp_tab[sbc];
+                        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], rcp), __fmul_rn(v[2 * q + 1], rcp)) << (8 * (q & 3));
+                        const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
+                        *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
+                        out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -984,12 +1196,13 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
 // global scale g (codes [slots][H/2], low nibble = even column; scales
 // [slots][H/16]); one thread per 16-value block.
 __global__ void k_act_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int slots, int H,
-                               int k, float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                               int k, float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, PermMeta meta) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int per = H / 16;
     if (i >= (long long)slots * per) return;
     const int p = (int)(i / per), b = (int)(i % per);
-    const int t = __ldg(perm + p) / k;
+    const int slot = __ldg(perm + p), t = slot / k;
+    if (b == 0) perm_meta(p, slot, k, meta);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + b * 16);
     const uint4 q0 = src[0], q1 = src[1];
     const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
@@ -1046,6 +1259,14 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Token-operand maps with 128-, 64-, 32- and 16-row boxes
+static bool make_bmaps(BMaps* mb, const void* base, uint64_t rows, uint64_t cols,
+                       CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+    for (int i = 0; i < 4; ++i)
+        if (!make_map(&mb->m[i], base, rows, cols, (uint32_t)(kBN >> i), dt)) return false;
+    return true;
+}
+
 // 2D map over bytes [rows, row_bytes]: box box_bytes x box_rows, 128-byte
 // swizzle for operand tiles, none for scale tiles
 static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
@@ -1080,13 +1301,13 @@ static int num_sms() {
 // One persistent CTA per SM over the routed (SH = false) or the shared (SH =
 // true) tiles of the list.
 template <int MODE, bool SH>
-static cudaError_t launch_gemm(const CUtensorMap& map_b, const GemmArgs& g, cudaStream_t st,
+static cudaError_t launch_gemm(const BMaps& map_b, const GemmArgs& g, cudaStream_t st,
                                const CUtensorMap* map_a = nullptr, int grid = 0) {
     constexpr int bytes = Cfg<MODE, SH>::ALLOC;
     cudaError_t err = cudaFuncSetAttribute(k_grouped_gemm<MODE, SH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (err != cudaSuccess) return err;
     k_grouped_gemm<MODE, SH><<<grid > 0 ? grid : num_sms(), Cfg<MODE, SH>::THREADS, bytes, st>>>(
-        map_b, map_a ? *map_a : map_b, g);
+        map_b, map_a ? *map_a : map_b.m[0], g);
     return cudaGetLastError();
 }
 
@@ -1094,8 +1315,9 @@ static cudaError_t launch_gemm(const CUtensorMap& map_b, const GemmArgs& g, cuda
 // fp32 (bf16 products, fp32 accumulation); tiles of 128 experts x 128 tokens.
 cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E, float* logits, int* err,
                              cudaStream_t st) {
-    CUtensorMap m_x, m_w;
-    if (!make_map(&m_x, x, (uint64_t)T, (uint64_t)H, kBN) || !make_map(&m_w, wr, (uint64_t)E, (uint64_t)H, kBlkN))
+    BMaps m_x;
+    CUtensorMap m_w;
+    if (!make_bmaps(&m_x, x, (uint64_t)T, (uint64_t)H) || !make_map(&m_w, wr, (uint64_t)E, (uint64_t)H, kBlkN))
         return cudaErrorInvalidValue;
     GemmArgs g{};
     g.K = H;
@@ -1132,18 +1354,20 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     uint8_t* as = a4 + (size_t)slots * I / 2;                          // [slots][I/16]
     {
         const long long nb = (long long)slots * (H / 16);
+        const PermMeta meta{p.w, nullptr, p.w_perm, nullptr};
         k_act_fp4_perm<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)p.x, p.perm, slots, H, k,
-                                                                      ex.g_x, xc, xs);
+                                                                      ex.g_x, xc, xs, meta);
     }
     // ---- gate / up
-    CUtensorMap m[6], m_shared;
+    CUtensorMap m[6];
+    BMaps m_shared;
     if (!make_map_u8(&m[0], p.fp4_codes[0], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
         !make_map_u8(&m[1], p.fp4_codes[1], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
         !make_map_u8(&m[2], p.fp4_scales[0], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
         !make_map_u8(&m[3], p.fp4_scales[1], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
         !make_map_u8(&m[4], xc, (uint64_t)slots, H / 2, 128, kBN, true) ||
         !make_map_u8(&m[5], xs, (uint64_t)slots, H / 16, 16, kBN, false) ||
-        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, kBN))
+        !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
     k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
     GemmArgs g{};
@@ -1174,7 +1398,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         !make_map_u8(&m[2], p.fp4_scales[2], (uint64_t)E * H, I / 16, 16, kBlkN, false) ||
         !make_map_u8(&m[4], a4, (uint64_t)slots, I / 2, 128, kBN, true) ||
         !make_map_u8(&m[5], as, (uint64_t)slots, I / 16, 16, kBN, false) ||
-        !make_map(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I, kBN))
+        !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
     m[1] = m[0];
     m[3] = m[2];
@@ -1188,6 +1412,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.o16 = p.o;
     g.o16_sh = p.o_sh;
     g.topk_w = p.w;
+    g.w_perm = p.w_perm;
     g.g_w = ex.g_down;
     g.g_act = ex.g_a;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
@@ -1227,13 +1452,14 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     }
     {
         const long long n8 = (long long)slots * (H / 8);
-        k_gather_rows<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xin, p.perm, slots, H, k, p.xp);
+        const PermMeta meta{p.w, fp4 ? nullptr : p.tok_scale, p.w_perm, p.ts_perm};
+        k_gather_rows<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xin, p.perm, slots, H, k, p.xp, meta);
     }
     const bool has_sh = ex.sh_gate != nullptr;
-    CUtensorMap m_routed, m_shared;
+    BMaps m_routed, m_shared;
     // ---- gate / up
-    if (!make_map(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, kBN, xdt) ||
-        !make_map(&m_shared, p.x, (uint64_t)T, (uint64_t)H, kBN))
+    if (!make_bmaps(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, xdt) ||
+        !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
     k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
     GemmArgs g{};
@@ -1254,6 +1480,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.g_act = fp4 ? ex.g_x : 1.0f;
     g.g_req = ex.g_a;
     g.tok_scale = fp4 ? nullptr : p.tok_scale;
+    g.ts_perm = fp4 ? nullptr : p.ts_perm;
     g.err = p.err;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
     err = launch_gemm<0, false>(m_routed, g, st);
@@ -1261,8 +1488,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
-    if (!make_map(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I, kBN) ||
-        !make_map(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I, kBN))
+    if (!make_bmaps(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I) ||
+        !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
     k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
     g.w0 = ex.down;
@@ -1276,9 +1503,11 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.o16 = p.o;
     g.o16_sh = p.o_sh;
     g.topk_w = p.w;
+    g.w_perm = p.w_perm;
     g.g_w = fp4 ? ex.g_down : nullptr;
     g.g_act = fp4 ? ex.g_a : 1.0f;
     g.tok_scale = nullptr;
+    g.ts_perm = nullptr;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
     err = launch_gemm<1, false>(m_routed, g, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);

@@ -111,6 +111,8 @@ struct PrefillArgs {
     __nv_bfloat16* xq;             // [T, H]: NVFP4 W4A4 activation values, else fp16 scaled x
     float* tok_scale;              // [T]: power of two of each token's fp16 activations
     __nv_bfloat16* xp;             // [T*k, H]: rows of xq in permuted (expert-major) order
+    float* w_perm;                 // [T*k]: routing weight of each permuted position
+    float* ts_perm;                // [T*k]: token scale of each permuted position (INT4/INT2)
     const uint8_t* fp4_codes[3];   // NVFP4: natural-layout weight images (gate, up, down) or null
     const uint8_t* fp4_scales[3];
     __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order

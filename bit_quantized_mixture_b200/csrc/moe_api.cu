@@ -50,6 +50,7 @@ struct moe_layer {
     int* num_tiles = nullptr;
     int* dev_err = nullptr;
     __nv_bfloat16 *xq = nullptr, *xp = nullptr, *a_perm = nullptr, *a_sh = nullptr;
+    float *w_perm = nullptr, *ts_perm = nullptr;
     __half *o = nullptr, *o_sh = nullptr;
     float* tok_scale = nullptr;
     // state
@@ -203,6 +204,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_xq = carve(Tm * H * 2);
     const size_t o_tsc = carve(Tm * sizeof(float));
     const size_t o_xp = carve(slots * H * 2);
+    const size_t o_wperm = carve(slots * sizeof(float));
+    const size_t o_tsperm = carve(slots * sizeof(float));
     const size_t o_aperm = carve(slots * I * 2);
     const size_t o_ash16 = carve(c.has_shared ? Tm * I * 2 : 0);
     const size_t o_o = carve(slots * H * 2);
@@ -235,6 +238,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
     h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
     h->xp = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xp);
+    h->w_perm = reinterpret_cast<float*>(h->ws + o_wperm);
+    h->ts_perm = reinterpret_cast<float*>(h->ws + o_tsperm);
     h->a_perm = reinterpret_cast<__nv_bfloat16*>(h->ws + o_aperm);
     h->a_sh = reinterpret_cast<__nv_bfloat16*>(h->ws + o_ash16);
     h->o = reinterpret_cast<__half*>(h->ws + o_o);
@@ -483,7 +488,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
         p.perm_scratch = h->perm_scratch;
         p.tiles = h->tiles; p.num_tiles = h->num_tiles;
-        p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp;
+        p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp; p.w_perm = h->w_perm; p.ts_perm = h->ts_perm;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
         for (int m = 0; m < 3; ++m) { p.fp4_codes[m] = h->fp4_codes[m]; p.fp4_scales[m] = h->fp4_scales[m]; }

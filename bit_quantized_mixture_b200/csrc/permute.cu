@@ -41,10 +41,16 @@ __global__ void __launch_bounds__(kMaxE) k_perm_scan(int chunks, int E, int32_t*
     const int e = threadIdx.x;
     int total = 0;
     if (e < E) {
-        for (int c = 0; c < chunks; ++c) {
-            const int v = chunk_cnt[(size_t)c * E + e];
-            chunk_cnt[(size_t)c * E + e] = total;     // exclusive base within the expert
-            total += v;
+        // eight independent loads in flight per step
+        for (int c0 = 0; c0 < chunks; c0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (c0 + u < chunks) chunk_cnt[(size_t)(c0 + u) * E + e] = total;   // exclusive base within the expert
+                total += v[u];
+            }
         }
         counts[e] = total;
     }
@@ -60,7 +66,14 @@ __global__ void __launch_bounds__(kMaxE) k_perm_scan(int chunks, int E, int32_t*
     const int excl = s[e] - ((e < E) ? total : 0);
     if (e < E) {
         offsets[e] = excl;
-        for (int c = 0; c < chunks; ++c) chunk_cnt[(size_t)c * E + e] += excl;
+        for (int c0 = 0; c0 < chunks; c0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (c0 + u < chunks) chunk_cnt[(size_t)(c0 + u) * E + e] = v[u] + excl;
+        }
     }
     if (e == E - 1) offsets[E] = s[e];
 }
@@ -73,9 +86,16 @@ __global__ void __launch_bounds__(32) k_perm_scatter(const int32_t* __restrict__
     for (int e = lane; e < E; e += 32) cur[e] = chunk_base[(size_t)blockIdx.x * E + e];
     __syncwarp();
     const int base = blockIdx.x * kChunk;
+    int ev[kChunk / 32];                      // the chunk's expert ids, all loads in flight at once
+#pragma unroll
     for (int step = 0; step < kChunk / 32; ++step) {
         const int s = base + step * 32 + lane;
-        const int e_s = (s < n) ? ids[s] : -1;
+        ev[step] = (s < n) ? __ldg(ids + s) : -1;
+    }
+#pragma unroll
+    for (int step = 0; step < kChunk / 32; ++step) {
+        const int s = base + step * 32 + lane;
+        const int e_s = ev[step];
         const bool valid = (s < n) && e_s >= 0 && e_s < E;
         const unsigned active = __ballot_sync(0xffffffffu, valid);
         if (valid) {

@@ -26,8 +26,10 @@ MOE_DEV uint32_t order_key(float v) {
 
 // One warp selects the top-k of one token's logits (E <= 1024 values read
 // through L2, expert e held by lane e % 32) and writes ids / weights.  Each
-// round takes the largest remaining key with one warp max-reduction and,
-// among equal keys, the smallest expert index with one min-reduction.
+// lane keeps the best of its own live keys (largest key, smallest expert on
+// equal keys); a round takes the warp maximum of those with one
+// max-reduction and, among lanes holding it, the smallest expert with one
+// min-reduction; only the lane that lost its key rescans its slots.
 MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
                        float* __restrict__ wout) {
     const int lane = threadIdx.x & 31;
@@ -40,20 +42,30 @@ MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __r
     uint32_t live = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
+    // best live key of this lane and its slot (first slot on equal keys)
+    auto rescan = [&](uint32_t& best, int& slot) {
+        best = 0;
+        slot = -1;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (((live >> i) & 1u) && (slot < 0 || key[i] > best)) {
+                best = key[i];
+                slot = i;
+            }
+    };
+    uint32_t best;
+    int slot;
+    rescan(best, slot);
     float my_val = 0.0f, lmax = 0.0f;
     int my_idx = 0;
     for (int j = 0; j < k; ++j) {
-        uint32_t best = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if ((live >> i) & 1u) best = max(best, key[i]);
-        const uint32_t top = __reduce_max_sync(0xffffffffu, best);
-        uint32_t mine = 0xffffffffu;
-#pragma unroll
-        for (int i = 31; i >= 0; --i)
-            if (((live >> i) & 1u) && key[i] == top) mine = (uint32_t)(lane + 32 * i);
+        const uint32_t top = __reduce_max_sync(0xffffffffu, slot >= 0 ? best : 0u);
+        const uint32_t mine = (slot >= 0 && best == top) ? (uint32_t)(lane + 32 * slot) : 0xffffffffu;
         const uint32_t e = __reduce_min_sync(0xffffffffu, mine);
-        if ((int)(e & 31u) == lane) live &= ~(1u << (e >> 5));
+        if ((int)(e & 31u) == lane) {
+            live &= ~(1u << (e >> 5));
+            rescan(best, slot);
+        }
         const float v = __uint_as_float((top & 0x80000000u) ? (top & 0x7fffffffu) : ~top);   // key -> value
         if (j == 0) lmax = v;
         if (lane == j) { my_val = v; my_idx = (int)e; }
