@@ -396,6 +396,47 @@ def prefill_flops(wl, slots):
     return 2.0 * m * wl.H * 2 * wl.I, 2.0 * m * wl.I * wl.H
 
 
+def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
+    """Roofline of the routed gate/up grouped GEMM (one launch).  Algorithmic
+    work: FLOPs 2 * slots * H * 2I; bytes = the touched experts' packed gate
+    and up weights (codes + scales [+ zeros]) once, the token activations once
+    (bf16 x for INT4/INT2, e2m1 codes + e4m3 scales for NVFP4) and the
+    intermediate written once (bf16, or e2m1 + e4m3 for NVFP4).  The binding
+    bound is the larger of FLOPs / tensor peak and bytes / HBM bandwidth; the
+    tensor peak is the measured bf16 burst (fp16 operands run at the same
+    rate), times 4 for the block-scaled e2m1 MMA (nominal 9 : 2.25)."""
+    H, I, T = wl.H, wl.I, wl.T
+    n = 2 * I                                     # gate + up rows per expert
+    if wl.quant == "int4":
+        w_bytes = n * H // 2 + n * (H // 128) * 2
+        act, out = T * H * 2, slots * I * 2
+    elif wl.quant == "int2":
+        w_bytes = n * H // 4 + n * (H // 128) * 2 + (n // 4) * (H // 128)
+        act, out = T * H * 2, slots * I * 2
+    else:
+        w_bytes = n * H // 2 + n * (H // 16)
+        act, out = T * (H // 2 + H // 16), slots * (I // 2 + I // 16)
+    flops = 2.0 * slots * H * n
+    nbytes = float(experts_touched * w_bytes + act + out)
+    t = t_ms * 1e-3
+    tensor_peak = peaks["bf16_tflops"] * (4.0 if wl.quant == "nvfp4" else 1.0)
+    hbm = peaks["hbm_gbs"]
+    t_tensor, t_hbm = flops / (tensor_peak * 1e12), nbytes / (hbm * 1e9)
+    tfl, gbs = flops / t / 1e12, nbytes / t / 1e9
+    kname = "k_fp4_gemm<0> (routed gate/up)" if wl.quant == "nvfp4" else "k_grouped_gemm<0,false> (routed gate/up)"
+    common = {"kernel": kname, "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
+              "arithmetic_intensity": flops / nbytes, "ridge_flop_per_byte": tensor_peak * 1e3 / hbm,
+              "achieved_tflops": tfl, "tensor_peak_tflops": tensor_peak, "frac_of_tensor_peak": tfl / tensor_peak,
+              "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm, "ms_per_launch": t_ms,
+              "peak_source": (f"{peak_kind} dense bf16 burst" + (" x 4 (nominal e2m1 : bf16 dense ratio)"
+                                                                  if wl.quant == "nvfp4" else "") +
+                              f"; {peak_kind} HBM copy bandwidth")}
+    if t_hbm >= t_tensor:
+        return dict({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}, **common)
+    return dict({"bound": "tensor", "achieved": tfl, "peak": tensor_peak, "unit": "TFLOP/s", "frac": tfl / tensor_peak},
+                **common)
+
+
 def run_prefill(args, wl, dev, rank, world):
     """A prefill step: router GEMM on x (logits kept), top-k of the
     workload's synthetic routing logits (the skewed / uniform routing the
@@ -458,7 +499,7 @@ def run_prefill(args, wl, dev, rank, world):
     total_ms_max = allreduce_max(total_ms, dev, world)
 
     # ---- per-kernel breakdown: the library's profiling events
-    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for evs in pev:
             for ev in evs:
@@ -476,7 +517,9 @@ def run_prefill(args, wl, dev, rank, world):
         return float(np.mean([p[i].elapsed_time(p[j]) for p in pev]))
 
     kern = {"route_router_gemm": mean_ms(0, 1), "forward": mean_ms(2, 4), "grouped_gemm_gate_up": mean_ms(5, 3),
-            "grouped_gemm_down": mean_ms(6, 7), "combine": mean_ms(7, 4)}
+            "grouped_gemm_gate_up_routed": mean_ms(5, 8), "grouped_gemm_down": mean_ms(6, 7),
+            "grouped_gemm_down_routed": mean_ms(6, 9), "combine": mean_ms(7, 4)}
+    experts_touched = int(np.count_nonzero(np.bincount(ids.cpu().numpy().ravel(), minlength=E)))
 
     # ---- end to end through the public API: x and the routing logits from
     # pinned host memory, y back to pinned host memory
@@ -504,23 +547,18 @@ def run_prefill(args, wl, dev, rank, world):
 
     fl_gu, fl_dn = prefill_flops(wl, T * k)
     peaks, peak_kind = measured_peaks()
-    peak = peaks["bf16_tflops"]
-    achieved = fl_gu / (kern["grouped_gemm_gate_up"] * 1e-3) / 1e12
-    traffic = load_traffic("k_grouped_gemm<0>", wl.name)
     layer.close()
-    roof = {"bound": "tensor", "kernel": "k_grouped_gemm<0> (gate/up)", "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "algorithmic_flops_per_launch": fl_gu,
-            "peak_source": f"{peak_kind} dense bf16 burst (the MMA runs kind::f16 on "
-                           f"{'bf16' if wl.quant == 'nvfp4' else 'fp16'} operands)",
-            "down_kernel_tflops": fl_dn / (kern["grouped_gemm_down"] * 1e-3) / 1e12}
-    if wl.quant == "nvfp4":
-        roof["frac_of_fp4_peak"] = achieved / (4.0 * peak)   # nominal fp4 : bf16 dense ratio 9 : 2.25
+    roof = gateup_roofline(wl, T * k, experts_touched, kern["grouped_gemm_gate_up_routed"], peaks, peak_kind)
+    roof["traffic"] = load_traffic("k_fp4_gemm<0>" if wl.quant == "nvfp4" else "k_grouped_gemm<0,false>", wl.name)
+    roof["down_routed_tflops"] = 2.0 * T * k * wl.I * H / (kern["grouped_gemm_down_routed"] * 1e-3) / 1e12
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
-        "launches_per_step": 13 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
+        # router GEMM, 2 top-k, 3 permutation, activation pass(es), 2 tile
+        # lists, 2 routed GEMMs (+2 shared), combine
+        "launches_per_step": (12 if wl.quant == "nvfp4" else 13) + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
         "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
-        "dtype": "bf16" if wl.quant == "nvfp4" else "f16",
+        "dtype": "e2m1" if wl.quant == "nvfp4" else "f16",
     }
 
 

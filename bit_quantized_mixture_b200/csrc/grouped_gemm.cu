@@ -63,10 +63,12 @@ struct Cfg {
     // SC: stages of the packed-weight ring (routed), decoupled from the TMEM
     // slots so that the HBM reads of the codes run several stages ahead
     static constexpr int SC = SH ? 0 : 6;
-    // MMA-issuing warps: gate/up, one per matrix (each stage gets NMAT
-    // commits); routed down, two that take alternate tiles (accumulator
-    // buffer j & 1), so that a second issuer works while the first waits
-    static constexpr int MMA_WARPS = (MODE == 1 && !SH) ? 2 : NMAT;
+    // MMA-issuing warps: one per matrix (each stage gets NMAT commits). A
+    // split of the tiles over two issuers (TILE_SPLIT) is supported, but the
+    // down GEMM is bound by shared-memory bandwidth (the token operand read
+    // by the MMAs, the staged codes, the epilogue staging), where a second
+    // issuer only adds contention.
+    static constexpr int MMA_WARPS = NMAT;
     static constexpr bool TILE_SPLIT = MMA_WARPS > NMAT;
     // routed: a second producer warp loads the token operand, the first the
     // packed weights
@@ -1390,6 +1392,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.err = p.err;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
     cudaError_t err = launch_fp4<0>(m, g, st);
+    if (err == cudaSuccess && p.ev_gu_r) cudaEventRecord(p.ev_gu_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
@@ -1417,6 +1420,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.g_act = ex.g_a;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
     err = launch_fp4<1>(m, g, st);
+    if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
@@ -1484,6 +1488,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.err = p.err;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
     err = launch_gemm<0, false>(m_routed, g, st);
+    if (err == cudaSuccess && p.ev_gu_r) cudaEventRecord(p.ev_gu_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
@@ -1510,6 +1515,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.ts_perm = nullptr;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
     err = launch_gemm<1, false>(m_routed, g, st);
+    if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);

@@ -123,6 +123,9 @@ struct PrefillArgs {
     // profiling events (may be null): before / after the gate-up grouped
     // GEMM, before / after the down grouped GEMM
     cudaEvent_t ev_gu0, ev_gu1, ev_dn0, ev_dn1;
+    // after the routed gate/up and the routed down launch (before the
+    // shared-expert launch of each)
+    cudaEvent_t ev_gu_r, ev_dn_r;
 };
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I);
 cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st);

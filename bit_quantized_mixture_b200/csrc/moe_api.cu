@@ -13,7 +13,7 @@
 
 using namespace moe;
 
-constexpr int kProfEvents = 8;   // see moe_set_profile_events
+constexpr int kProfEvents = 10;  // see moe_set_profile_events
 
 struct moe_layer {
     moe_config cfg;
@@ -493,6 +493,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.err = h->dev_err;
         for (int m = 0; m < 3; ++m) { p.fp4_codes[m] = h->fp4_codes[m]; p.fp4_scales[m] = h->fp4_scales[m]; }
         p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
+        p.ev_gu_r = h->prof[8]; p.ev_dn_r = h->prof[9];
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_prefill(p, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_forward (grouped GEMM path)");

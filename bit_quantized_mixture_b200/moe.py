@@ -172,7 +172,7 @@ class MoeLayer:
                self.h)
 
     def set_profile_events(self, events):
-        """events: 5 to 8 torch.cuda.Event(enable_timing=True) (recorded once
+        """events: 5 to 10 torch.cuda.Event(enable_timing=True) (recorded once
         beforehand) or None; slot meanings as in moe_set_profile_events."""
         if events is None:
             _check(lib().moe_set_profile_events(self.h, None, 0), self.h)

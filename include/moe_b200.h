@@ -232,9 +232,12 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
  *   [3] decode, two-kernel path: between the gate/up and the down kernel;
  *       grouped-GEMM path: after the gate/up grouped GEMM;
  *   [5] / [6] / [7] grouped-GEMM path only: before the gate/up grouped GEMM,
- *       before the down grouped GEMM, after the down grouped GEMM.
+ *       before the down grouped GEMM, after the down grouped GEMM;
+ *   [8] / [9] grouped-GEMM path only: after the routed-expert gate/up and
+ *       after the routed-expert down launch (before the shared-expert
+ *       launch of each, which [3] and [7] close).
  * events are cudaEvent_t handles created by the caller; n >= 5 of them are
- * read (slots n..7 are not recorded); NULL turns recording off.  Recording
+ * read (slots n..9 are not recorded); NULL turns recording off.  Recording
  * an event between two kernels removes their launch overlap, so time the
  * layer itself with recording off. */
 moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n);
