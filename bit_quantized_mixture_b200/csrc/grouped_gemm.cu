@@ -129,7 +129,9 @@ struct GemmArgs {
     const uint8_t* sh1;
     const int32_t* perm;      // slot at each permuted position
     const GemmTile* tiles;
-    const int* num_tiles;     // [0]: routed tiles, [1]: all tiles (shared ones last)
+    const int* num_tiles;     // [0]: routed tiles, [1]: all tiles (shared ones last), [2]: routed
+                              // groups, [3]: 1 when routed launches take the group order
+    const int2* groups;       // routed groups: first tile, tiles
     int K;                    // reduction length (H or I)
     int k_top;
     int out_ld;               // row length of the outputs (I or H)
@@ -306,23 +308,65 @@ struct PermMeta {
     float* ts_perm;           // [T*k] out: token scale of each permuted position
 };
 
-// A CTA's tiles (ti = first + j * gridDim.x) are copied into shared memory
-// once, so that no role waits on a global load at the start of a tile.
+// A CTA's tile sequence is copied into shared memory once, so that no role
+// waits on a global load at the start of a tile.  The block-scaled NVFP4
+// launches take groups (up to kGroupTiles consecutive token tiles of one expert and weight
+// block, which read the same weights) in the order g = blockIdx.x + j *
+// gridDim.x, so that a CTA reads a weight block for its second token tile
+// while it is still in L2; otherwise (or when a CTA's tiles would not fit
+// the list) tiles go round robin, ti = first + j * gridDim.x.
 constexpr int kTileCache = 256;
+constexpr int kGroupTiles = 2;
 struct TileCache {
     GemmTile t[kTileCache];
+    int n;          // tiles of this CTA
+    int grouped;    // 1: group order (all n tiles in t), 0: round robin
 };
 MOE_DEV void cache_tiles(TileCache& tc, const GemmTile* tiles, int first, int end) {
     for (int j = threadIdx.x; j < kTileCache; j += blockDim.x) {
         const int ti = first + j * gridDim.x;
         if (ti < end) tc.t[j] = tiles[ti];
     }
+    if (threadIdx.x == 0) {
+        tc.n = first < end ? (end - first + gridDim.x - 1) / gridDim.x : 0;
+        tc.grouped = 0;
+    }
+}
+// Group order (needs blockDim.x >= kTileCache): thread i takes this CTA's
+// i-th group, an exclusive scan of the group sizes places its tiles.
+MOE_DEV void cache_groups(TileCache& tc, const GemmTile* tiles, const int2* groups, int ngroups, int* scan) {
+    const int i = threadIdx.x;
+    int2 gr = make_int2(0, 0);
+    if (i < kTileCache) {
+        const int g = blockIdx.x + i * gridDim.x;
+        if (g < ngroups) gr = groups[g];
+    }
+    // inclusive scan of gr.y over threads 0 .. kTileCache-1
+    const int lane = i & 31, w = i >> 5;
+    int v = gr.y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (i < kTileCache && lane == 31) scan[w] = v;
+    __syncthreads();
+    if (i < kTileCache) {
+        int base = 0;
+        for (int k = 0; k < w; ++k) base += scan[k];
+        const int pos = base + v - gr.y;
+        for (int k = 0; k < gr.y && pos + k < kTileCache; ++k) tc.t[pos + k] = tiles[gr.x + k];
+        if (i == kTileCache - 1) {
+            tc.n = min(base + v, kTileCache);
+            tc.grouped = 1;
+        }
+    }
 }
 
 // Tile ti: from the device-built list, or (router) row block ti % RB of
 // token block ti / RB.
 template <int MODE>
-MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = nullptr, int first = 0) {
+MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = nullptr, int first = 0, int j = -1) {
     if constexpr (MODE == 2) {
         const int RB = (a.n_rows + kBlkN - 1) / kBlkN;
         GemmTile t;
@@ -332,8 +376,9 @@ MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = null
         t.count = min(kBN, a.n_tok - t.seg);
         return t;
     } else {
-        const int j = (ti - first) / (int)gridDim.x;
-        return (tc && j < kTileCache) ? tc->t[j] : a.tiles[ti];
+        if (tc && tc->grouped) return tc->t[j];
+        const int jj = (ti - first) / (int)gridDim.x;
+        return (tc && jj < kTileCache) ? tc->t[jj] : a.tiles[ti];
     }
 }
 
@@ -358,6 +403,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
     {
         const int tb = (SH && MODE != 2) ? __ldcg(a.num_tiles) : 0;
         const int te = MODE == 2 ? a.n_tiles : SH ? __ldcg(a.num_tiles + 1) : __ldcg(a.num_tiles);
+        // round robin: with the dequantizing pipeline the skewed tile sizes
+        // of Zipf routing balance better than in the group order
         if (MODE != 2) cache_tiles(tcache, a.tiles, tb + blockIdx.x, te);
     }
     if (threadIdx.x == 0) {
@@ -386,6 +433,10 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
     const int t_end = MODE == 2 ? a.n_tiles : SH ? __ldcg(a.num_tiles + 1) : __ldcg(a.num_tiles);
     const int t_first = t_begin + blockIdx.x;
     const int NS = a.K / (kBlkK * KSTEP);                 // stages per tile
+    // this CTA's tile sequence
+    const int nseq = MODE == 2 ? (t_first < t_end ? (t_end - t_first + (int)gridDim.x - 1) / (int)gridDim.x : 0)
+                               : tcache.n;
+    auto tile_at = [&](int j) { return load_tile<MODE>(a, t_first + j * (int)gridDim.x, &tcache, t_first, j); };
 
     if (warp == kWarpProducer && !SH) {
         // ------------------------------------------- producer: packed weights
@@ -396,8 +447,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : 256;
         const int zb = a.quant == Q_INT2 ? 128 : 0;
         int g = 0;
-        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
+            const GemmTile t = tile_at(jt);
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int c = g % SC;
@@ -429,8 +480,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // ---------------------------------------- producer: token operand
         // (+ the router / shared-expert weight tiles)
         int g = 0;
-        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
+            const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
@@ -469,8 +520,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         const int mi = C::TILE_SPLIT ? 0 : warp - kWarpMma;
         int g = 0, local = 0;
         AccSeq aseq;
-        for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_first);
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt, ++local) {
+            const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const bool f16 = MODE == 0 && !SH && a.tok_scale != nullptr;
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
@@ -532,7 +583,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const bool f16 = MODE == 0 && a.tok_scale != nullptr;
             const int cb = block_code_bytes(a.quant);
             int g = 0;
-            for (int ti = t_first; ti < t_end && !abort_flag; ti += gridDim.x) {
+            for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
                 bool ok = true;
                 for (int ks = 0; ks < NS; ++ks, ++g) {
                     const int c = g % SC, s = g % S;
@@ -582,9 +633,9 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // while the current one is processed
         float nx_sc = 1.0f;
         int nx_row = 0;
-        auto fetch = [&](int tj) {
-            if (MODE == 2 || tj >= t_end) return;
-            const GemmTile tn = load_tile<MODE>(a, tj, &tcache, t_begin + blockIdx.x);
+        auto fetch = [&](int jn) {
+            if (MODE == 2 || jn >= nseq) return;
+            const GemmTile tn = tile_at(jn);
             if (ej >= tn.count) return;
             if constexpr (SH) {
                 nx_sc = 1.0f;
@@ -597,10 +648,10 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 nx_row = __ldg(a.perm + tn.seg + ej);
             }
         };
-        fetch(t_begin + blockIdx.x);
+        fetch(0);
         AccSeq aseq;
-        for (int ti = t_begin + blockIdx.x; ti < t_end; ti += gridDim.x) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, t_begin + blockIdx.x);
+        for (int jt = 0; jt < nseq; ++jt) {
+            const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
             float gsc = 1.0f;
@@ -611,7 +662,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 ep_scale[ej] = nx_sc * gsc;
                 ep_row[ej] = nx_row;
             }
-            fetch(ti + gridDim.x);
+            fetch(jt + 1);
             epi_sync();
             if (ep_stop) break;
             // a failed wait sets abort_flag: this tile is skipped and all four
@@ -715,21 +766,41 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
 // the shared expert's tiles (all T tokens) come last.
 __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict__ counts,
                                                       const int32_t* __restrict__ offsets, int E, int T, int RB,
-                                                      int has_shared, GemmTile* __restrict__ tiles,
-                                                      int* __restrict__ num_tiles) {
-    __shared__ int sc[1024];
+                                                      int has_shared, int grid, GemmTile* __restrict__ tiles,
+                                                      int2* __restrict__ groups, int* __restrict__ num_tiles) {
+    __shared__ int sc[1024], sg[1024];
     const int e = threadIdx.x;
     const int cnt = (e < E) ? counts[e] : 0;
-    const int mine = ((cnt + kBN - 1) / kBN) * RB;
+    const int nt = (cnt + kBN - 1) / kBN;
+    const int mine = nt * RB;
     sc[e] = mine;
+    sg[e] = ((nt + kGroupTiles - 1) / kGroupTiles) * RB;
     __syncthreads();
     for (int o = 1; o < 1024; o <<= 1) {
         const int v = (e >= o) ? sc[e - o] : 0;
+        const int w = (e >= o) ? sg[e - o] : 0;
         __syncthreads();
         sc[e] += v;
+        sg[e] += w;
         __syncthreads();
     }
-    const int total = sc[1023];
+    const int total = sc[1023], ngroups = sg[1023];
+    // groups: up to kGroupTiles consecutive token tiles of one (expert, row
+    // block), which read the same weight block
+    for (int i = e; i < ngroups; i += 1024) {
+        int lo = 0, hi = 1023;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sg[mid] > i) hi = mid;
+            else lo = mid + 1;
+        }
+        const int ex = lo;
+        const int ntx = (counts[ex] + kBN - 1) / kBN;
+        const int gpr = (ntx + kGroupTiles - 1) / kGroupTiles;     // groups per row block
+        const int j = i - (sg[ex] - gpr * RB);
+        const int rb = j / gpr, q = j % gpr;
+        groups[i] = make_int2(sc[ex] - ntx * RB + rb * ntx + q * kGroupTiles, min(kGroupTiles, ntx - q * kGroupTiles));
+    }
     // all threads emit the routed tiles: tile i belongs to the expert whose
     // inclusive prefix is the first one above i (binary search)
     for (int i = e; i < total; i += 1024) {
@@ -764,6 +835,9 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
     if (e == 0) {
         num_tiles[0] = total;               // routed tiles
         num_tiles[1] = total + nts * RB;    // + shared-expert tiles
+        num_tiles[2] = ngroups;
+        // group order when every CTA's tiles fit its shared-memory list
+        num_tiles[3] = ((ngroups + grid - 1) / grid) * kGroupTiles <= kTileCache ? 1 : 0;
     }
 }
 
@@ -802,12 +876,17 @@ __global__ void k_combine(const __half* __restrict__ O, const __half* __restrict
 // INT4 / INT2 gate/up operand: each token row of x scaled by a power of two
 // 2^-p (exact) so that its largest magnitude lies in [2^14, 2^15), stored as
 // fp16 (exact: bf16 has 8 significant bits); scale[t] = 2^p undoes it in the
-// GEMM epilogue.  One warp per token row.
-__global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, int T, int H, __half* __restrict__ x16,
-                           float* __restrict__ scale) {
+// GEMM epilogue.  The row is written straight into the permuted operand: the
+// warp of token t converts it once and stores it at the k positions
+// inv[t*k + j] of its slots (with each position's routing weight and token
+// scale for the GEMM epilogues).  Dropped slots (inv < 0) are skipped.
+__global__ void k_x_to_f16_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ inv, int T, int H,
+                                int k, __half* __restrict__ xp, float* __restrict__ scale, const float* __restrict__ topk_w,
+                                float* __restrict__ w_perm, float* __restrict__ ts_perm) {
     const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
+    const int mypos = lane < k ? __ldg(inv + (size_t)t * k + lane) : -1;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
     float amax = 0.0f;
     for (int c = lane; c < H / 8; c += 32) {
@@ -828,9 +907,18 @@ __global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, int T, int H, __
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             o[i] = h2_bits(__floats2half2_rn(bf16_lo(w[i]) * down, bf16_hi(w[i]) * down));
-        reinterpret_cast<uint4*>(x16 + (size_t)t * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < k; ++j) {
+            const int pos = __shfl_sync(0xffffffffu, mypos, j);
+            if (pos >= 0) reinterpret_cast<uint4*>(xp + (size_t)pos * H)[c] = ov;
+        }
     }
-    if (lane == 0) scale[t] = ldexpf(1.0f, p);
+    const float sc = ldexpf(1.0f, p);
+    if (lane < k && mypos >= 0) {
+        w_perm[mypos] = __ldg(topk_w + (size_t)t * k + lane);
+        ts_perm[mypos] = sc;
+    }
+    if (lane == 0) scale[t] = sc;
 }
 
 // Routing weight and token scale of permuted position p, read by the GEMM
@@ -938,9 +1026,11 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     __shared__ int ep_stop;
     __shared__ float rcp_tab[256];              // gate/up: 1 / (e4m3(code) * g_req), IEEE division, 0 for zero
     __shared__ TileCache tcache;
+    __shared__ int gscan[kTileCache / 32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    cache_tiles(tcache, a.tiles, blockIdx.x, __ldcg(a.num_tiles));
+    if (__ldcg(a.num_tiles + 3)) cache_groups(tcache, a.tiles, a.groups, __ldcg(a.num_tiles + 2), gscan);
+    else cache_tiles(tcache, a.tiles, blockIdx.x, __ldcg(a.num_tiles));
     if (MODE == 0 && threadIdx.x < 256) {
         const float sbv = e4m3_to_f32((uint32_t)threadIdx.x);
         rcp_tab[threadIdx.x] = (sbv == 0.0f || a.g_req == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, a.g_req));
@@ -964,13 +1054,15 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = tmem_base_slot;
     const int t_end = __ldcg(a.num_tiles);                // routed tiles only
+    const int nseq = tcache.n;                            // this CTA's tile sequence
+    auto tile_at = [&](int j) { return load_tile<MODE>(a, (int)blockIdx.x + j * (int)gridDim.x, &tcache, blockIdx.x, j); };
     const int NS = a.K / kFp4KS;
 
     if (warp == kWarpProducer) {
         // ---------------------------------------------------------- producer
         int g = 0;
-        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
+            const GemmTile t = tile_at(jt);
             const int arow = t.expert * a.n_rows + t.rb * kBlkN;
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
@@ -996,8 +1088,8 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         // --------------------------------------------------------- MMA issue
         const int mi = warp - kWarpMma;
         int g = 0, local = 0;
-        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x, ++local) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt, ++local) {
+            const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const uint32_t idesc = idesc_nvfp4(128, n_mma);
             const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
@@ -1032,7 +1124,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int quarter = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int g = 0;
-        for (int ti = blockIdx.x; ti < t_end && !abort_flag; ti += gridDim.x) {
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
@@ -1070,17 +1162,17 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         uint8_t* out_s = smem + C::OUT;
         float nx_sc = 1.0f;                      // next tile's token info, loaded ahead
         int nx_row = 0;
-        auto fetch = [&](int tj) {
-            if (tj >= t_end) return;
-            const GemmTile tn = load_tile<MODE>(a, tj, &tcache, blockIdx.x);
+        auto fetch = [&](int jn) {
+            if (jn >= nseq) return;
+            const GemmTile tn = tile_at(jn);
             if (ej >= tn.count) return;
             nx_sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
             nx_row = MODE == 0 ? tn.seg + ej : __ldg(a.perm + tn.seg + ej);
         };
-        fetch(blockIdx.x);
+        fetch(0);
         int local = 0;
-        for (int ti = blockIdx.x; ti < t_end; ti += gridDim.x, ++local) {
-            const GemmTile t = load_tile<MODE>(a, ti, &tcache, blockIdx.x);
+        for (int jt = 0; jt < nseq; ++jt, ++local) {
+            const GemmTile t = tile_at(jt);
             const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
             const float gsc = a.g_w[t.expert] * a.g_act;
@@ -1090,7 +1182,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 ep_scale[ej] = nx_sc * gsc;
                 ep_row[ej] = nx_row;
             }
-            fetch(ti + gridDim.x);
+            fetch(jt + 1);
             epi_sync();
             if (ep_stop) break;
             if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 16)) continue;
@@ -1193,29 +1285,14 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-// W4A4 activations of the gate/up GEMM in permuted order: row p of the
-// operand is token perm[p] / k, quantized per 16 values with the static
-// global scale g (codes [slots][H/2], low nibble = even column; scales
-// [slots][H/16]); one thread per 16-value block.
-__global__ void k_act_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int slots, int H,
-                               int k, float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, PermMeta meta) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const int per = H / 16;
-    if (i >= (long long)slots * per) return;
-    const int p = (int)(i / per), b = (int)(i % per);
-    const int slot = __ldg(perm + p), t = slot / k;
-    if (b == 0) perm_meta(p, slot, k, meta);
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + b * 16);
-    const uint4 q0 = src[0], q1 = src[1];
-    const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    float v[16];
+// One 16-value block of W4A4 activations: e4m3 scale code of amax / (6 g)
+// and the e2m1 codes of v / (s_b g), the decisions taken in fp32 with IEEE
+// division as the format defines them.  Returns the scale code; w[0..1]
+// hold the 16 codes (low nibble = even column).
+MOE_DEV uint32_t quant_block16(const float (&v)[16], float g, uint32_t (&w)[2]) {
     float amax = 0.0f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        v[2 * q] = bf16_lo(wv[q]);
-        v[2 * q + 1] = bf16_hi(wv[q]);
-        amax = fmaxf(amax, fmaxf(fabsf(v[2 * q]), fabsf(v[2 * q + 1])));
-    }
+    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
     uint32_t sbc = 0;
     float r = 0.0f;
     if (g != 0.0f) {
@@ -1223,11 +1300,44 @@ __global__ void k_act_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_
         const float sbv = e4m3_to_f32(sbc);
         r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
     }
-    uint32_t w[2] = {0u, 0u};
+    w[0] = w[1] = 0u;
 #pragma unroll
     for (int q = 0; q < 8; ++q) w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], r), __fmul_rn(v[2 * q + 1], r)) << (8 * (q & 3));
-    *reinterpret_cast<uint2*>(codes + (size_t)p * (H / 2) + b * 8) = make_uint2(w[0], w[1]);
-    sf[(size_t)p * (H / 16) + b] = (uint8_t)sbc;
+    return sbc;
+}
+
+// W4A4 activations of the gate/up GEMM in permuted order, quantized per 16
+// values with the static global scale g (codes [slots][H/2], scales
+// [slots][H/16]).  The warp of token t quantizes its row once and stores it
+// at the k positions inv[t*k + j] of its slots, with each position's
+// routing weight; dropped slots (inv < 0) are skipped.
+__global__ void k_x_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ inv, int T, int H, int k,
+                             float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                             const float* __restrict__ topk_w, float* __restrict__ w_perm) {
+    const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const int mypos = lane < k ? __ldg(inv + (size_t)t * k + lane) : -1;
+    for (int b = lane; b < H / 16; b += 32) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + b * 16);
+        const uint4 q0 = src[0], q1 = src[1];
+        const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            v[2 * q] = bf16_lo(wv[q]);
+            v[2 * q + 1] = bf16_hi(wv[q]);
+        }
+        uint32_t w[2];
+        const uint32_t sbc = quant_block16(v, g, w);
+        for (int j = 0; j < k; ++j) {
+            const int pos = __shfl_sync(0xffffffffu, mypos, j);
+            if (pos < 0) continue;
+            *reinterpret_cast<uint2*>(codes + (size_t)pos * (H / 2) + b * 8) = make_uint2(w[0], w[1]);
+            sf[(size_t)pos * (H / 16) + b] = (uint8_t)sbc;
+        }
+    }
+    if (lane < k && mypos >= 0) w_perm[mypos] = __ldg(topk_w + (size_t)t * k + lane);
 }
 
 // ----------------------------------------------------------------- host side
@@ -1355,10 +1465,8 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     uint8_t* a4 = reinterpret_cast<uint8_t*>(p.a_perm);               // [slots][I/2]
     uint8_t* as = a4 + (size_t)slots * I / 2;                          // [slots][I/16]
     {
-        const long long nb = (long long)slots * (H / 16);
-        const PermMeta meta{p.w, nullptr, p.w_perm, nullptr};
-        k_act_fp4_perm<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)p.x, p.perm, slots, H, k,
-                                                                      ex.g_x, xc, xs, meta);
+        k_x_fp4_perm<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, p.inv, T, H, k, ex.g_x, xc, xs, p.w,
+                                                   p.w_perm);
     }
     // ---- gate / up
     CUtensorMap m[6];
@@ -1371,7 +1479,8 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         !make_map_u8(&m[5], xs, (uint64_t)slots, H / 16, 16, kBN, false) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
+                                     p.groups, p.num_tiles);
     GemmArgs g{};
     g.quant = ex.quant;
     g.sh0 = ex.sh_gate;
@@ -1379,6 +1488,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.perm = p.perm;
     g.tiles = p.tiles;
     g.num_tiles = p.num_tiles;
+    g.groups = p.groups;
     g.K = H;
     g.k_top = k;
     g.n_rows = I;
@@ -1405,7 +1515,8 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     m[1] = m[0];
     m[3] = m[2];
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
+                                     p.groups, p.num_tiles);
     g.sh0 = ex.sh_down;
     g.sh1 = nullptr;
     g.K = I;
@@ -1448,16 +1559,15 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
         k_act_fp4_values<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)p.x, T, H, ex.g_x,
                                                                          p.xq);
         xin = p.xq;
-    } else {
-        k_x_to_f16<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, T, H, reinterpret_cast<__half*>(p.xq),
-                                                 p.tok_scale);
-        xin = p.xq;
-        xdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    }
-    {
         const long long n8 = (long long)slots * (H / 8);
-        const PermMeta meta{p.w, fp4 ? nullptr : p.tok_scale, p.w_perm, p.ts_perm};
+        const PermMeta meta{p.w, nullptr, p.w_perm, p.ts_perm};
         k_gather_rows<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xin, p.perm, slots, H, k, p.xp, meta);
+    } else {
+        // fp16 scaling and the permuted copy in one pass over x
+        k_x_to_f16_perm<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, p.inv, T, H, k,
+                                                      reinterpret_cast<__half*>(p.xp), p.tok_scale, p.w, p.w_perm,
+                                                      p.ts_perm);
+        xdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     }
     const bool has_sh = ex.sh_gate != nullptr;
     BMaps m_routed, m_shared;
@@ -1465,7 +1575,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (!make_bmaps(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, xdt) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
+                                     p.groups, p.num_tiles);
     GemmArgs g{};
     g.quant = ex.quant;
     g.w0 = ex.gate;
@@ -1475,6 +1586,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.perm = p.perm;
     g.tiles = p.tiles;
     g.num_tiles = p.num_tiles;
+    g.groups = p.groups;
     g.K = H;
     g.k_top = k;
     g.out_ld = I;
@@ -1496,7 +1608,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (!make_bmaps(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I) ||
         !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, p.tiles, p.num_tiles);
+    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
+                                     p.groups, p.num_tiles);
     g.w0 = ex.down;
     g.w1 = ex.down;
     g.sh0 = ex.sh_down;

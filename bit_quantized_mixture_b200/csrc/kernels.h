@@ -107,7 +107,8 @@ struct PrefillArgs {
     int T;
     int32_t *counts, *offsets, *perm, *inv, *perm_scratch;
     GemmTile* tiles;
-    int* num_tiles;
+    int2* groups;                  // routed tile groups (same capacity as tiles)
+    int* num_tiles;                // 4 ints
     __nv_bfloat16* xq;             // [T, H]: NVFP4 W4A4 activation values, else fp16 scaled x
     float* tok_scale;              // [T]: power of two of each token's fp16 activations
     __nv_bfloat16* xp;             // [T*k, H]: rows of xq in permuted (expert-major) order

@@ -48,6 +48,7 @@ struct moe_layer {
     int32_t *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr, *perm_scratch = nullptr;
     GemmTile* tiles = nullptr;
     int* num_tiles = nullptr;
+    int2* groups = nullptr;
     int* dev_err = nullptr;
     __nv_bfloat16 *xq = nullptr, *xp = nullptr, *a_perm = nullptr, *a_sh = nullptr;
     float *w_perm = nullptr, *ts_perm = nullptr;
@@ -199,7 +200,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_inv = carve(sizeof(int32_t) * slots);
     const size_t o_pscr = carve(sizeof(int32_t) * permute_scratch_ints((int)slots, E));
     const size_t o_tiles = carve(sizeof(GemmTile) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
-    const size_t o_ntiles = carve(2 * sizeof(int));   // routed tiles, all tiles
+    const size_t o_groups = carve(sizeof(int2) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
+    const size_t o_ntiles = carve(4 * sizeof(int));   // routed tiles, all tiles, routed groups, group order
     const size_t o_err = carve(sizeof(int));
     const size_t o_xq = carve(Tm * H * 2);
     const size_t o_tsc = carve(Tm * sizeof(float));
@@ -234,6 +236,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->perm_scratch = reinterpret_cast<int32_t*>(h->ws + o_pscr);
     h->tiles = reinterpret_cast<GemmTile*>(h->ws + o_tiles);
     h->num_tiles = reinterpret_cast<int*>(h->ws + o_ntiles);
+    h->groups = reinterpret_cast<int2*>(h->ws + o_groups);
     h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
     h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
     h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
@@ -487,7 +490,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.x = x; p.ids = topk_ids; p.w = topk_w; p.y = y; p.T = T;
         p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
         p.perm_scratch = h->perm_scratch;
-        p.tiles = h->tiles; p.num_tiles = h->num_tiles;
+        p.tiles = h->tiles; p.groups = h->groups; p.num_tiles = h->num_tiles;
         p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp; p.w_perm = h->w_perm; p.ts_perm = h->ts_perm;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;

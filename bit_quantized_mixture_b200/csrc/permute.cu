@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(32) k_perm_scatter(const int32_t* __restrict__
         const int e_s = ev[step];
         const bool valid = (s < n) && e_s >= 0 && e_s < E;
         const unsigned active = __ballot_sync(0xffffffffu, valid);
+        if (s < n && !valid) inv[s] = -1;          // dropped slot: no position
         if (valid) {
             const int e = e_s;
             const unsigned peers = __match_any_sync(active, e);
