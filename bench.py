@@ -438,10 +438,11 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
 
 
 def run_prefill(args, wl, dev, rank, world):
-    """A prefill step: router GEMM on x (logits kept), top-k of the
+    """A prefill step: router GEMM on x (logits only), softmax/top-k of the
     workload's synthetic routing logits (the skewed / uniform routing the
-    workload prescribes), permutation, gate/up and down grouped GEMMs,
-    combine.  Eager launches; per-kernel events in a separate pass."""
+    workload prescribes, standing in for the router's own), permutation,
+    gate/up and down grouped GEMMs, combine: the layer's work once.  Eager
+    launches; per-kernel events in a separate pass."""
     import torch
 
     from bit_quantized_mixture_b200 import moe, synth
@@ -469,7 +470,7 @@ def run_prefill(args, wl, dev, rank, world):
     stream = torch.cuda.Stream(device=dev)
 
     def step(xin, lgin):
-        layer.route(xin, ids, w, logits=logits)       # router GEMM (logits) + its top-k
+        layer.route(xin, None, None, logits=logits)   # router GEMM (logits only)
         layer.route_from_logits(lgin, ids, w)         # the workload's routing
         layer.forward(xin, ids, w, y)
 
@@ -554,9 +555,9 @@ def run_prefill(args, wl, dev, rank, world):
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
-        # router GEMM, 2 top-k, 3 permutation, 1 activation pass, 2 tile
+        # router GEMM, top-k, 3 permutation, 1 activation pass, 2 tile
         # lists, 2 routed GEMMs (+2 shared), combine
-        "launches_per_step": 12 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
+        "launches_per_step": 11 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
         "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
         "dtype": "e2m1" if wl.quant == "nvfp4" else "f16",
     }

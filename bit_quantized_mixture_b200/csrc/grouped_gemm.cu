@@ -768,9 +768,11 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
                                                       const int32_t* __restrict__ offsets, int E, int T, int RB,
                                                       int has_shared, int grid, GemmTile* __restrict__ tiles,
                                                       int2* __restrict__ groups, int* __restrict__ num_tiles) {
-    __shared__ int sc[1024], sg[1024];
+    __shared__ int sc[1024], sg[1024], s_cnt[1024], s_off[1024];
     const int e = threadIdx.x;
     const int cnt = (e < E) ? counts[e] : 0;
+    s_cnt[e] = cnt;
+    s_off[e] = (e < E) ? offsets[e] : 0;
     const int nt = (cnt + kBN - 1) / kBN;
     const int mine = nt * RB;
     sc[e] = mine;
@@ -795,7 +797,7 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
             else lo = mid + 1;
         }
         const int ex = lo;
-        const int ntx = (counts[ex] + kBN - 1) / kBN;
+        const int ntx = (s_cnt[ex] + kBN - 1) / kBN;
         const int gpr = (ntx + kGroupTiles - 1) / kGroupTiles;     // groups per row block
         const int j = i - (sg[ex] - gpr * RB);
         const int rb = j / gpr, q = j % gpr;
@@ -811,14 +813,14 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
             else lo = mid + 1;
         }
         const int ex = lo;
-        const int c = counts[ex];
+        const int c = s_cnt[ex];
         const int ntx = (c + kBN - 1) / kBN;
         const int j = i - (sc[ex] - ntx * RB);          // index within the expert's tiles
         const int rb = j / ntx, tt = j % ntx;
         GemmTile g;
         g.expert = ex;
         g.rb = rb;
-        g.seg = offsets[ex] + tt * kBN;
+        g.seg = s_off[ex] + tt * kBN;
         g.count = min(kBN, c - tt * kBN);
         tiles[i] = g;
     }

@@ -394,7 +394,8 @@ moe_status moe_route(moe_handle h, const void* x, int32_t T, int32_t* topk_ids, 
     if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_route: null handle");
     moe_status s = check_tokens(h, "moe_route", T);
     if (s != MOE_OK) return s;
-    if (!x || !topk_ids || !topk_w) return fail(h, MOE_ERR_INVALID_ARG, "moe_route: null pointer");
+    if (!x || (!topk_ids) != (!topk_w) || (!topk_ids && !logits_out))
+        return fail(h, MOE_ERR_INVALID_ARG, "moe_route: null pointer");
     if (!aligned16(x)) return fail(h, MOE_ERR_INVALID_ARG, "moe_route: x must be 16-byte aligned");
     if (!h->router_loaded) return fail(h, MOE_ERR_STATE, "moe_route: router not loaded");
     DeviceGuard dg(h->cfg.device);

@@ -41,13 +41,13 @@ __global__ void __launch_bounds__(kMaxE) k_perm_scan(int chunks, int E, int32_t*
     const int e = threadIdx.x;
     int total = 0;
     if (e < E) {
-        // eight independent loads in flight per step
-        for (int c0 = 0; c0 < chunks; c0 += 8) {
-            int v[8];
+        // sixteen independent loads in flight per step
+        for (int c0 = 0; c0 < chunks; c0 += 16) {
+            int v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
+            for (int u = 0; u < 16; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 16; ++u) {
                 if (c0 + u < chunks) chunk_cnt[(size_t)(c0 + u) * E + e] = total;   // exclusive base within the expert
                 total += v[u];
             }
@@ -66,12 +66,12 @@ __global__ void __launch_bounds__(kMaxE) k_perm_scan(int chunks, int E, int32_t*
     const int excl = s[e] - ((e < E) ? total : 0);
     if (e < E) {
         offsets[e] = excl;
-        for (int c0 = 0; c0 < chunks; c0 += 8) {
-            int v[8];
+        for (int c0 = 0; c0 < chunks; c0 += 16) {
+            int v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
+            for (int u = 0; u < 16; ++u) v[u] = (c0 + u < chunks) ? chunk_cnt[(size_t)(c0 + u) * E + e] : 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
+            for (int u = 0; u < 16; ++u)
                 if (c0 + u < chunks) chunk_cnt[(size_t)(c0 + u) * E + e] = v[u] + excl;
         }
     }

@@ -30,24 +30,25 @@ MOE_DEV uint32_t order_key(float v) {
 // equal keys); a round takes the warp maximum of those with one
 // max-reduction and, among lanes holding it, the smallest expert with one
 // min-reduction; only the lane that lost its key rescans its slots.
-MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                       float* __restrict__ wout) {
+template <int SLOTS>
+MOE_DEV void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                         float* __restrict__ wout) {
     const int lane = threadIdx.x & 31;
-    uint32_t key[32];
+    uint32_t key[SLOTS];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < SLOTS; ++i) {
         const int e = lane + 32 * i;
         key[i] = (e < E) ? order_key(__ldcg(row + e)) : 0u;
     }
     uint32_t live = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
+    for (int i = 0; i < SLOTS; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
     // best live key of this lane and its slot (first slot on equal keys)
     auto rescan = [&](uint32_t& best, int& slot) {
         best = 0;
         slot = -1;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < SLOTS; ++i)
             if (((live >> i) & 1u) && (slot < 0 || key[i] > best)) {
                 best = key[i];
                 slot = i;
@@ -76,6 +77,13 @@ MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __r
         ids[lane] = my_idx;
         wout[lane] = __fdiv_rn(ex, sum);
     }
+}
+
+// E <= 512: 16 slots per lane; E <= 1024: 32
+MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                       float* __restrict__ wout) {
+    if (E <= 512) warp_topk_n<16>(row, E, k, ids, wout);
+    else warp_topk_n<32>(row, E, k, ids, wout);
 }
 
 // Decode router (T <= 8): one warp per expert row, a grid-wide ticket lets
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     }
     __syncthreads();
     if (!s_last) return;
-    for (int t = warp; t < T; t += 4)
+    for (int t = warp; a.ids && t < T; t += 4)
         warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
     __syncthreads();
     if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
@@ -189,7 +197,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
         cudaError_t e = launch_router_tc(a.x, a.wr, a.T, a.H, a.E, a.logits, a.err, st);
         if (e != cudaSuccess) return e;
     }
-    k_topk<<<(a.T + 7) / 8, 256, 0, st>>>(a);
+    if (a.ids) k_topk<<<(a.T + 7) / 8, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -143,6 +143,8 @@ moe_status moe_set_act_global_scales(moe_handle h, float g_x, float g_a);
  * w_j = exp(l_j - l_max) / sum_selected exp(l - l_max).
  *   x          bf16 [T, H]           topk_ids int32 [T, k]
  *   topk_w     fp32 [T, k]           logits_out fp32 [T, E] or NULL
+ * topk_ids and topk_w may both be NULL when logits_out is given: only the
+ * logits are computed (e.g. when the routing itself comes from elsewhere).
  * 1 <= T <= max_tokens.  Errors: INVALID_ARG, STATE (router not loaded). */
 moe_status moe_route(moe_handle h, const void* x, int32_t T, int32_t* topk_ids,
                      float* topk_w, float* logits_out, moe_stream_t stream);

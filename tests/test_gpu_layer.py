@@ -58,6 +58,22 @@ def test_route_matches_oracle(T):
     layer.close()
 
 
+@pytest.mark.parametrize("T", [3, 300])
+def test_route_logits_only(T):
+    """moe_route with no ids / weights computes the same logits and nothing else."""
+    wl = synth.custom("decode-b1-int4", T=T, E=512, k=10)
+    layer = moe.MoeLayer(wl.H, wl.I, wl.E, wl.k, "int4", False, T, 0)
+    layer.load_router(bf16_tensor(synth.router_bf16(wl), DEV))
+    x = synth.activations_bf16(wl, steps=1)
+    ids, w, logits = _route_gpu(layer, x, wl)
+    xd = bf16_tensor(x, DEV)
+    lg2 = torch.full((T, wl.E), float("nan"), dtype=torch.float32, device=DEV)
+    layer.route(xd, None, None, logits=lg2)
+    layer.sync_status()
+    assert np.array_equal(lg2.cpu().numpy().view(np.uint32), logits.view(np.uint32))
+    layer.close()
+
+
 def test_route_from_logits_ties_and_order():
     wl = synth.custom("tiny-int4", T=64, E=40, k=7)
     layer = moe.MoeLayer(wl.H, wl.I, wl.E, wl.k, "int4", False, wl.T, 0)
