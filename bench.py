@@ -43,6 +43,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded oracle sample length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mb", type=int, default=512)
+    ap.add_argument("--expert-table", action="store_true",
+                    help="read the routed experts through the per-expert address table from a shuffled pool")
     return ap.parse_args(argv)
 
 
@@ -251,6 +253,23 @@ def expert_bytes(wl):
     return gu, dn
 
 
+def expert_pool(layer, wl, dev):
+    """Move the routed experts' blocks into a separate device pool in a
+    seeded shuffled order and point the layer's address table at them (the
+    kernels then read every expert through the table)."""
+    import torch
+    bb = layer.expert_block_bytes()
+    pool = torch.empty(wl.E * bb + 256, dtype=torch.uint8, device=dev)
+    base = (pool.data_ptr() + 255) // 256 * 256
+    slot = np.random.default_rng(1234).permutation(wl.E)
+    for e in range(wl.E):
+        off = base - pool.data_ptr() + int(slot[e]) * bb
+        layer.export_expert(e, pool[off:off + bb])
+    torch.cuda.synchronize(dev)
+    layer.set_expert_table([base + int(slot[e]) * bb for e in range(wl.E)])
+    return pool
+
+
 def run_decode(args, wl, dev, rank, world):
     import torch
 
@@ -258,6 +277,7 @@ def run_decode(args, wl, dev, rank, world):
     from bit_quantized_mixture_b200.layer import build_layer
 
     layer, _ = build_layer(wl, dev.index, max_tokens=wl.T)
+    pool = expert_pool(layer, wl, dev) if args.expert_table else None
     xs_host = synth.activations_bf16(wl)
     xs = torch.from_numpy(xs_host.view(np.int16)).to(dev).view(torch.bfloat16)
     T, k = wl.T, wl.k
@@ -449,6 +469,7 @@ def run_prefill(args, wl, dev, rank, world):
     from bit_quantized_mixture_b200.layer import build_layer
 
     layer, _ = build_layer(wl, dev.index, max_tokens=wl.T)
+    pool = expert_pool(layer, wl, dev) if args.expert_table else None
     T, k, H, E = wl.T, wl.k, wl.H, wl.E
     x_host = synth.activations_bf16(wl)
     lg_host = synth.routing_logits(wl).astype(np.float32)
@@ -623,7 +644,8 @@ def run_ours(args):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "quant": wl.quant,
                    "shared": wl.shared, "routing": wl.routing, "parallelism": f"replicas x{world}",
                    "l2": f"flushed ({args.flush_mb} MB write) between timed steps",
-                   "cuda_graph": not prefill},
+                   "cuda_graph": not prefill,
+                   "experts": "address table, shuffled pool" if args.expert_table else "arena"},
         "roofline": r["roofline"],
         "kernels_ms": r["kernels_ms"],
         "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},

@@ -307,10 +307,11 @@ MOE_DEV void stage_rows_f32(__nv_bfloat16* dst, int ldx, const float* src, int K
 }
 
 MOE_DEV MatPtr expert_mat(const MatView& v, int e) {
+    const ExpertMat m = expert_matrix(v, e);
     MatPtr p;
-    p.codes = v.codes + (size_t)e * v.stride;
-    p.scales = v.scales ? v.scales + (size_t)e * v.stride : nullptr;
-    p.zeros = v.zeros ? v.zeros + (size_t)e * v.stride : nullptr;
+    p.codes = m.codes;
+    p.scales = m.scales;
+    p.zeros = m.zeros;
     return p;
 }
 

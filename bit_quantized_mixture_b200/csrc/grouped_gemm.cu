@@ -458,17 +458,16 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     uint8_t* stg = smem + C::STG + c * NMAT * C::STG_MAT;
                     mbar_arrive_expect_tx(&cfull[c], (uint32_t)(NMAT * (cb + sb + zb)));
                     for (int m = 0; m < NMAT; ++m) {
-                        const MatView& v = m == 0 ? a.w0 : a.w1;
-                        const size_t eo = (size_t)t.expert * v.stride;
+                        const ExpertMat em = expert_matrix(m == 0 ? a.w0 : a.w1, t.expert);
                         uint8_t* d = stg + m * C::STG_MAT;
-                        bulk_g2s(d, v.codes + eo + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
+                        bulk_g2s(d, em.codes + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
                                  &cfull[c]);
                         if (a.quant == Q_NVFP4) {
-                            bulk_g2s(d + cb, v.scales + eo + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
+                            bulk_g2s(d + cb, em.scales + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
                         } else {
                             const size_t go = ((size_t)t.rb * G + kb0 / 2) * 256;   // kb0 even: one group
-                            bulk_g2s(d + cb, v.scales + eo + go, sb, &cfull[c]);
-                            if (zb) bulk_g2s(d + cb + sb, v.zeros + eo + go / 2, zb, &cfull[c]);
+                            bulk_g2s(d + cb, em.scales + go, sb, &cfull[c]);
+                            if (zb) bulk_g2s(d + cb + sb, em.zeros + go / 2, zb, &cfull[c]);
                         }
                     }
                 }

@@ -16,6 +16,8 @@ cudaError_t launch_quantize(int quant, const float* w, int N, int K, float g, vo
 cudaError_t launch_quantize_act_nvfp4(const void* x, int T, int K, float g, void* codes, void* scales,
                                       cudaStream_t st);
 cudaError_t launch_absmax(const float* x, long long n, float* out, cudaStream_t st);
+// g[e] = gate/up and g[E + e] = down global scale read from each table block at offset off
+cudaError_t launch_gather_global_scales(const uint8_t* const* table, size_t off, int E, float* g, cudaStream_t st);
 cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const uint8_t* src_scales,
                             const uint8_t* src_zeros, uint8_t* dst_codes, uint8_t* dst_scales,
                             uint8_t* dst_zeros, cudaStream_t st);

@@ -63,8 +63,34 @@ struct MatView {
     const uint8_t* scales;  // expert e at scales + e * stride
     const uint8_t* zeros;   // expert e at zeros + e * stride (INT2)
     size_t stride;          // bytes between consecutive experts
+    // per-expert address table: when set, expert e's block (all three
+    // matrices, the arena's per-expert layout) starts at table[e] and this
+    // matrix's codes / scales / zeros lie at the offsets below inside it
+    const uint8_t* const* table;
+    size_t off_codes, off_scales, off_zeros;
     int N, K;
 };
+
+// codes / scales / zeros (null when absent) of expert e
+struct ExpertMat {
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const uint8_t* zeros;
+};
+__host__ __device__ inline ExpertMat expert_matrix(const MatView& v, int e) {
+    ExpertMat m;
+    if (v.table) {
+        const uint8_t* b = v.table[e];
+        m.codes = b + v.off_codes;
+        m.scales = v.scales ? b + v.off_scales : nullptr;
+        m.zeros = v.zeros ? b + v.off_zeros : nullptr;
+    } else {
+        m.codes = v.codes + (size_t)e * v.stride;
+        m.scales = v.scales ? v.scales + (size_t)e * v.stride : nullptr;
+        m.zeros = v.zeros ? v.zeros + (size_t)e * v.stride : nullptr;
+    }
+    return m;
+}
 
 // byte offset of block (rb, kb) inside the codes of one matrix
 __host__ __device__ inline size_t block_offset(const MatGeom& g, int rb, int kb) {

@@ -22,6 +22,7 @@ struct moe_layer {
     size_t arena_bytes = 0;
     MatGeom geom[3];               // gate, up, down of a routed expert
     size_t off_codes[3], off_scales[3], off_zeros[3];
+    size_t off_gs = 0;             // NVFP4: the expert's two global scales inside its block
     size_t expert_stride = 0;      // bytes per routed expert
     uint8_t* experts = nullptr;    // expert e at experts + e * expert_stride
     uint8_t* router = nullptr;     // bf16 [E, H]
@@ -50,6 +51,10 @@ struct moe_layer {
     int* num_tiles = nullptr;
     int2* groups = nullptr;
     int* dev_err = nullptr;
+    // per-expert address table (moe_set_expert_table): device [E], in use when set
+    const uint8_t** table = nullptr;
+    bool table_set = false;
+    float* g_tab = nullptr;        // NVFP4: [2E] global scales gathered from the table's blocks
     __nv_bfloat16 *xq = nullptr, *xp = nullptr, *a_perm = nullptr, *a_sh = nullptr;
     float *w_perm = nullptr, *ts_perm = nullptr;
     __half *o = nullptr, *o_sh = nullptr;
@@ -146,6 +151,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     for (int m = 0; m < 3; ++m) { h->off_codes[m] = off; off = align_up(off + h->geom[m].codes_bytes(), 256); }
     for (int m = 0; m < 3; ++m) { h->off_scales[m] = off; off = align_up(off + h->geom[m].scales_bytes(), 256); }
     for (int m = 0; m < 3; ++m) { h->off_zeros[m] = off; off = align_up(off + h->geom[m].zeros_bytes(), 256); }
+    if (c.quant == MOE_Q_NVFP4) { h->off_gs = off; off = align_up(off + 2 * sizeof(float), 256); }
     h->expert_stride = off;
     size_t a = 0;
     const size_t experts_off = a; a = align_up(a + h->expert_stride * E, 4096);
@@ -203,6 +209,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_groups = carve(sizeof(int2) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
     const size_t o_ntiles = carve(4 * sizeof(int));   // routed tiles, all tiles, routed groups, group order
     const size_t o_err = carve(sizeof(int));
+    const size_t o_table = carve(sizeof(void*) * (size_t)E);
+    const size_t o_gtab = carve(sizeof(float) * 2 * (size_t)E);
     const size_t o_xq = carve(Tm * H * 2);
     const size_t o_tsc = carve(Tm * sizeof(float));
     const size_t o_xp = carve(slots * H * 2);
@@ -238,6 +246,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->num_tiles = reinterpret_cast<int*>(h->ws + o_ntiles);
     h->groups = reinterpret_cast<int2*>(h->ws + o_groups);
     h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
+    h->table = reinterpret_cast<const uint8_t**>(h->ws + o_table);
+    h->g_tab = reinterpret_cast<float*>(h->ws + o_gtab);
     h->xq = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xq);
     h->tok_scale = reinterpret_cast<float*>(h->ws + o_tsc);
     h->xp = reinterpret_cast<__nv_bfloat16*>(h->ws + o_xp);
@@ -366,6 +376,13 @@ moe_status moe_load_expert_weights(moe_handle h, int32_t expert, const moe_exper
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(h->g_down + expert, h->g_host + c.num_experts + expert, sizeof(float),
                                 cudaMemcpyHostToDevice, st);
+        // and inside the expert's block, which moe_export_expert copies
+        uint8_t* gb = h->experts + (size_t)expert * h->expert_stride + h->off_gs;
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(gb, h->g_host + expert, sizeof(float), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(gb + sizeof(float), h->g_host + c.num_experts + expert, sizeof(float),
+                                cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: global scales");
     }
     if (shared) h->shared_loaded = true;
@@ -444,14 +461,18 @@ static ExpertArgs expert_args(moe_layer* h) {
         v[m]->scales = h->experts + h->off_scales[m];
         v[m]->zeros = c.quant == MOE_Q_INT2 ? h->experts + h->off_zeros[m] : nullptr;
         v[m]->stride = h->expert_stride;
+        v[m]->table = h->table_set ? h->table : nullptr;
+        v[m]->off_codes = h->off_codes[m];
+        v[m]->off_scales = h->off_scales[m];
+        v[m]->off_zeros = h->off_zeros[m];
         v[m]->N = h->geom[m].N;
         v[m]->K = h->geom[m].K;
     }
     ex.sh_gate = c.has_shared ? h->shared[0] : nullptr;
     ex.sh_up = c.has_shared ? h->shared[1] : nullptr;
     ex.sh_down = c.has_shared ? h->shared[2] : nullptr;
-    ex.g_gate = h->g_gate;
-    ex.g_down = h->g_down;
+    ex.g_gate = h->table_set ? h->g_tab : h->g_gate;
+    ex.g_down = h->table_set ? h->g_tab + c.num_experts : h->g_down;
     ex.g_x = h->g_x;
     ex.g_a = h->g_a;
     ex.quant = c.quant;
@@ -495,7 +516,12 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp; p.w_perm = h->w_perm; p.ts_perm = h->ts_perm;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
-        for (int m = 0; m < 3; ++m) { p.fp4_codes[m] = h->fp4_codes[m]; p.fp4_scales[m] = h->fp4_scales[m]; }
+        // the block-scaled NVFP4 images live in the arena: with an address
+        // table the exact bf16-dequantization path reads the table's blocks
+        for (int m = 0; m < 3; ++m) {
+            p.fp4_codes[m] = h->table_set ? nullptr : h->fp4_codes[m];
+            p.fp4_scales[m] = h->table_set ? nullptr : h->fp4_scales[m];
+        }
         p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
         p.ev_gu_r = h->prof[8]; p.ev_dn_r = h->prof[9];
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
@@ -702,6 +728,47 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which, 
                                 cudaMemcpyDefault, st);
     }
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_unpack_matrix");
+    return MOE_OK;
+}
+
+moe_status moe_expert_block_bytes(moe_handle h, size_t* bytes) {
+    if (!h || !bytes) return fail(h, MOE_ERR_INVALID_ARG, "moe_expert_block_bytes: null pointer");
+    *bytes = h->expert_stride;
+    return MOE_OK;
+}
+
+moe_status moe_export_expert(moe_handle h, int32_t expert, void* dst, moe_stream_t stream) {
+    if (!h || !dst) return fail(h, MOE_ERR_INVALID_ARG, "moe_export_expert: null pointer");
+    if (expert < 0 || expert >= h->cfg.num_experts)
+        return fail(h, MOE_ERR_INVALID_ARG, "moe_export_expert: expert %d out of range", expert);
+    if ((reinterpret_cast<uintptr_t>(dst) & 255u) != 0)
+        return fail(h, MOE_ERR_INVALID_ARG, "moe_export_expert: dst must be 256-byte aligned");
+    DeviceGuard dg(h->cfg.device);
+    const cudaError_t e = cudaMemcpyAsync(dst, h->experts + (size_t)expert * h->expert_stride, h->expert_stride,
+                                          cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_export_expert");
+    return MOE_OK;
+}
+
+moe_status moe_set_expert_table(moe_handle h, const void* const* blocks, moe_stream_t stream) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_set_expert_table: null handle");
+    const int E = h->cfg.num_experts;
+    if (blocks)
+        for (int e = 0; e < E; ++e)
+            if (!blocks[e] || (reinterpret_cast<uintptr_t>(blocks[e]) & 255u) != 0)
+                return fail(h, MOE_ERR_INVALID_ARG, "moe_set_expert_table: block of expert %d is null or not "
+                                                    "256-byte aligned", e);
+    DeviceGuard dg(h->cfg.device);
+    // earlier work on the stream may still read the old table
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess && blocks)
+        e = cudaMemcpy(h->table, blocks, sizeof(void*) * (size_t)E, cudaMemcpyHostToDevice);
+    // NVFP4: the per-expert global scales travel in the blocks
+    if (e == cudaSuccess && blocks && h->cfg.quant == MOE_Q_NVFP4)
+        e = launch_gather_global_scales(h->table, h->off_gs, E, h->g_tab, (cudaStream_t)stream);
+    if (e == cudaSuccess && blocks) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_set_expert_table");
+    h->table_set = blocks != nullptr;
     return MOE_OK;
 }
 

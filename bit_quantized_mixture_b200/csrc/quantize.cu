@@ -333,6 +333,20 @@ cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const u
     return cudaGetLastError();
 }
 
+__global__ void k_gather_global_scales(const uint8_t* const* __restrict__ table, size_t off, int E,
+                                       float* __restrict__ g) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const float* src = reinterpret_cast<const float*>(table[e] + off);
+    g[e] = src[0];
+    g[E + e] = src[1];
+}
+
+cudaError_t launch_gather_global_scales(const uint8_t* const* table, size_t off, int E, float* g, cudaStream_t st) {
+    k_gather_global_scales<<<(E + 255) / 256, 256, 0, st>>>(table, off, E, g);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_unpack(const MatGeom& gm, const uint8_t* dev_codes, const uint8_t* dev_scales,
                           const uint8_t* dev_zeros, uint8_t* codes, uint8_t* scales, uint8_t* zeros,
                           cudaStream_t st) {

@@ -70,6 +70,9 @@ def lib():
             "moe_set_profile_events": [vp, ctypes.POINTER(vp), i32],
             "moe_sync_status": [vp, vp],
             "moe_permute_noalloc": [vp, i32, i32, i32, vp, vp, vp, vp, vp],
+            "moe_expert_block_bytes": [vp, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_export_expert": [vp, i32, vp, vp],
+            "moe_set_expert_table": [vp, ctypes.POINTER(vp), vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -179,6 +182,23 @@ class MoeLayer:
             return
         arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
         _check(lib().moe_set_profile_events(self.h, arr, len(events)), self.h)
+
+    def expert_block_bytes(self):
+        n = ctypes.c_size_t(0)
+        _check(lib().moe_expert_block_bytes(self.h, ctypes.byref(n)), self.h)
+        return int(n.value)
+
+    def export_expert(self, expert, dst, stream=None):
+        """Copy expert `expert`'s block (device layout) to the CUDA buffer dst."""
+        _check(lib().moe_export_expert(self.h, int(expert), _ptr(dst), _stream(stream)), self.h)
+
+    def set_expert_table(self, addresses, stream=None):
+        """addresses: E device addresses (ints) of expert blocks, or None for the arena."""
+        if addresses is None:
+            _check(lib().moe_set_expert_table(self.h, None, _stream(stream)), self.h)
+            return
+        arr = (ctypes.c_void_p * len(addresses))(*[int(a) for a in addresses])
+        _check(lib().moe_set_expert_table(self.h, arr, _stream(stream)), self.h)
 
     def debug_unpack(self, expert, which, codes, scales=None, zeros=None, global_scale=None, stream=None):
         _check(lib().moe_debug_unpack_matrix(self.h, int(expert), int(which), _ptr(codes), _ptr(scales),

@@ -216,6 +216,36 @@ moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, in
                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                                moe_stream_t stream);
 
+/* ------------------------------------------------- expert address table
+ *
+ * Experts read where they are: after moe_set_expert_table, the kernels read
+ * routed expert e's weights from blocks[e] instead of the handle's arena
+ * (the arena stays allocated; moe_load_expert_weights keeps writing it).
+ * A block holds one expert's three matrices in the library's device layout
+ * (NVFP4: and the expert's two fp32 global scales), moe_expert_block_bytes
+ * bytes, as moe_export_expert writes it; blocks may
+ * lie anywhere in device memory of the handle's device, in any order, and
+ * several entries may point at the same block.  Blocks must stay valid and
+ * unchanged while calls that read them are in flight. */
+
+/* Bytes of one expert block (a multiple of 256). */
+moe_status moe_expert_block_bytes(moe_handle h, size_t* bytes);
+
+/* Copy expert `expert`'s block from the arena to dst (device memory of the
+ * handle's device, 256-byte aligned), ordered on `stream`.
+ * Errors: INVALID_ARG (null or misaligned dst, expert out of range), CUDA. */
+moe_status moe_export_expert(moe_handle h, int32_t expert, void* dst, moe_stream_t stream);
+
+/* blocks: host array of E device addresses (each 256-byte aligned, not
+ * null), or NULL to read the arena again.  The call synchronizes `stream`
+ * (work already queued keeps the old table), copies the E addresses to the
+ * device (NVFP4: and reads each block's global scales on `stream`) and
+ * synchronizes again before it returns; the caller's array may be freed then.  With
+ * a table, NVFP4 layers run prefill on the exact bf16-dequantization path
+ * (their block-scaled weight images stay in the arena).
+ * Errors: INVALID_ARG (null or misaligned entry: nothing changes), CUDA. */
+moe_status moe_set_expert_table(moe_handle h, const void* const* blocks, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- debug */
 
 /* Write loaded matrix `which` (0 gate, 1 up, 2 down) of `expert` back in
