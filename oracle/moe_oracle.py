@@ -17,6 +17,10 @@ low-bit group quantization and whose routers stay 16-bit:
 * "Qwen3.8-Flash-Next on 2x RTX 3090", storage-format table, and
   "albucino/Qwen3.8-Flash-Next-W4A16-FP8PLE", section "Composition": routed
   experts are W4A16, symmetric INT4, group 128.
+* "Qwen3.8-Flash-Next on 2x RTX 3090", storage-format table, and
+  "albucino/Qwen3.8-Flash-Next-W4A16-FP8PLE", section "Composition": the
+  routed experts of the MTP draft are symmetric INT4 with group 32 (the same
+  recipe with one scale per 32 inputs).
 * "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", section "Format": routed
   experts are NVFP4 W4A4 (E2M1 values, one scale per 16 elements); the
   shared experts stay BF16.
@@ -51,6 +55,7 @@ from __future__ import annotations
 import numpy as np
 
 GROUP_INT = 128      # INT4 / INT2 group size along K
+GROUP_INT4_G32 = 32  # INT4 group size of the MTP-draft experts
 GROUP_FP4 = 16       # NVFP4 block size along K
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
@@ -145,7 +150,7 @@ def e2m1_rne_satfinite(v) -> np.ndarray:
 # Weight formats (interchange layout)
 #   A matrix W is [N, K] (output rows, input columns); groups run along K.
 #   INT4 : codes uint8 [N, K/2], element k=2j in the low nibble of byte j;
-#          scales fp16 [N, K/128].
+#          scales fp16 [N, K/128] (group 32: [N, K/32]).
 #   INT2 : codes uint8 [N, K/4], element k=4j+i at bits 2i..2i+1;
 #          scales fp16 [N, K/128]; zeros uint8 [N/4, K/128], the zero of
 #          row n at bits 2(n%4) of byte (n//4, group).
@@ -154,12 +159,12 @@ def e2m1_rne_satfinite(v) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 
-def quantize_int4(w):
-    """Symmetric INT4, group 128 (W4A16 experts)."""
+def quantize_int4(w, group=GROUP_INT):
+    """Symmetric INT4, group 128 (W4A16 experts) or 32 (MTP-draft experts)."""
     w = np.asarray(w, dtype=np.float32)
     N, K = w.shape
-    assert K % GROUP_INT == 0
-    g = w.reshape(N, K // GROUP_INT, GROUP_INT)
+    assert K % group == 0
+    g = w.reshape(N, K // group, group)
     amax = np.abs(g).max(axis=2)
     s16 = fp16_rne(amax / np.float32(7.0))
     s = s16.astype(np.float32)[..., None]
@@ -181,10 +186,12 @@ def unpack_int4(codes) -> np.ndarray:
 
 
 def dequantize_int4(codes, scales) -> np.ndarray:
+    """(u - 8) * s; the group size is K over the number of scales per row."""
     u = unpack_int4(codes).astype(np.float64)
     N, K = u.shape
     s = np.asarray(scales, dtype=np.float16).astype(np.float64)
-    return ((u - 8.0).reshape(N, K // GROUP_INT, GROUP_INT) * s[..., None]).reshape(N, K)
+    group = K // s.shape[1]
+    return ((u - 8.0).reshape(N, K // group, group) * s[..., None]).reshape(N, K)
 
 
 def quantize_int2(w):
@@ -342,12 +349,12 @@ def dequantize_expert(quant, ew):
     """Expert weights in interchange form -> fp64 (W_gate, W_up, W_down).
 
     ``ew`` maps 'gate'/'up'/'down' to dicts with keys codes, scales and,
-    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int2', 'nvfp4' or
+    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int4g32', 'int2', 'nvfp4' or
     'bf16' (codes are then bf16 bit patterns)."""
     out = []
     for name in ("gate", "up", "down"):
         m = ew[name]
-        if quant == "int4":
+        if quant in ("int4", "int4g32"):
             out.append(dequantize_int4(m["codes"], m["scales"]))
         elif quant == "int2":
             out.append(dequantize_int2(m["codes"], m["scales"], m["zeros"]))

@@ -65,6 +65,55 @@ def test_int4_zero_group_and_error_bound():
     assert q.min() >= -8 and q.max() <= 7
 
 
+def test_int4_group32_worked_example(golden):
+    g = golden["int4_g32"]
+    w = _group(g["row_values"], K=g["K"])
+    codes, s = O.quantize_int4(w, group=O.GROUP_INT4_G32)
+    assert s.shape == (1, 2)
+    for j, sc in enumerate(g["scales"]):
+        assert float(s[0, j]) == sc["value_num"] * 2.0 ** sc["value_exp"]
+    u = O.unpack_int4(codes)[0]
+    for k, c in g["codes"].items():
+        assert u[int(k)] == c
+    assert np.all(np.delete(u, [int(k) for k in g["codes"]]) == 8)
+    deq = O.dequantize_int4(codes, s)[0]
+    for k, v in g["dequant"].items():
+        assert deq[int(k)] == v
+    # the same row in one 64-column group quantizes column 0 differently
+    c2, s2 = O.quantize_int4(w, group=64)
+    h = g["group128_contrast"]
+    assert float(s2[0, 0]) == h["scale_value_num"] * 2.0 ** h["scale_value_exp"]
+    assert O.unpack_int4(c2)[0, 0] == h["code_0"]
+
+
+def test_int4_group32_dequant_by_element_loop():
+    """dequantize_int4 with 32-column groups against a plain per-element loop."""
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((5, 96)) * 0.03).astype(np.float32)
+    codes, s = O.quantize_int4(w, group=32)
+    assert s.shape == (5, 3)
+    deq = O.dequantize_int4(codes, s)
+    for n in range(5):
+        for k in range(96):
+            byte = int(codes[n, k // 2])
+            u = (byte >> 4) if k % 2 else (byte & 0xF)
+            assert deq[n, k] == (u - 8) * float(s[n, k // 32])
+
+
+def test_int4_group32_error_bound_and_finer_than_group128():
+    rng = np.random.default_rng(3)
+    w = (rng.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    w[:, ::37] *= 8.0                                   # outliers that widen a group's range
+    c32, s32 = O.quantize_int4(w, group=32)
+    deq32 = O.dequantize_int4(c32, s32)
+    sf = np.repeat(s32.astype(np.float64), 32, axis=1)
+    assert np.all(np.abs(w - deq32) <= sf * 0.5 * (1 + 2.0 ** -8) + 1e-30)
+    c128, s128 = O.quantize_int4(w)
+    err32 = np.sqrt(np.mean((w - deq32) ** 2))
+    err128 = np.sqrt(np.mean((w - O.dequantize_int4(c128, s128)) ** 2))
+    assert err32 < err128
+
+
 # ---------------------------------------------------------------- INT2 ----
 
 def test_int2_worked_example(golden):
