@@ -164,8 +164,8 @@ class OracleSampler:
                 g_gu = O.nvfp4_global_scale(max(np.abs(g).max(), np.abs(u).max()))
                 g_d = O.nvfp4_global_scale(np.abs(d).max())
             for name, m in zip(("gate", "up", "down"), (g, u, d)):
-                if wl.quant == "int4":
-                    c, sc = O.quantize_int4(m)
+                if wl.quant in ("int4", "int4g32"):
+                    c, sc = O.quantize_int4(m, group=32 if wl.quant == "int4g32" else 128)
                     ew[name] = {"codes": c, "scales": sc}
                 elif wl.quant == "int2":
                     c, sc, z = O.quantize_int2(m)
@@ -241,9 +241,10 @@ def run_reference(args):
 def expert_bytes(wl):
     """Packed bytes of one routed expert's gate+up and down matrices."""
     H, I = wl.H, wl.I
-    if wl.quant == "int4":
-        gu = 2 * (I * H // 2 + I * (H // 128) * 2)
-        dn = H * I // 2 + H * (I // 128) * 2
+    if wl.quant in ("int4", "int4g32"):
+        gs = 32 if wl.quant == "int4g32" else 128
+        gu = 2 * (I * H // 2 + I * (H // gs) * 2)
+        dn = H * I // 2 + H * (I // gs) * 2
     elif wl.quant == "int2":
         gu = 2 * (I * H // 4 + I * (H // 128) * 2 + I * (H // 128))
         dn = H * I // 4 + H * (I // 128) * 2 + H * (I // 128)
@@ -427,8 +428,8 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
     rate), times 4 for the block-scaled e2m1 MMA (nominal 9 : 2.25)."""
     H, I, T = wl.H, wl.I, wl.T
     n = 2 * I                                     # gate + up rows per expert
-    if wl.quant == "int4":
-        w_bytes = n * H // 2 + n * (H // 128) * 2
+    if wl.quant in ("int4", "int4g32"):
+        w_bytes = n * H // 2 + n * (H // (32 if wl.quant == "int4g32" else 128)) * 2
         act, out = T * H * 2, slots * I * 2
     elif wl.quant == "int2":
         w_bytes = n * H // 4 + n * (H // 128) * 2 + (n // 4) * (H // 128)

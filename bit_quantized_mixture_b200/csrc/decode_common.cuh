@@ -71,6 +71,7 @@ MOE_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
 // ------------------------------------------------------------ format traits
 template <int Q> struct Fmt;
 template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_INT4G32> { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_NVFP4> { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_INT2>  { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_BF16>  { static constexpr int KPW = 1; };
@@ -86,7 +87,8 @@ template <int Q>
 struct Blk {
     uint32_t w[2][2];        // INT4 / NVFP4: [chunk][row g, g+8]; INT2: w[0][row]
     uint4 v[2][2];           // bf16: [32-column half][row g, g+8]
-    float s0, s1;            // INT4/INT2 scales of the two rows
+    float s0, s1;            // INT4/INT2 scales of the two rows (INT4 group 32: of chunk 0)
+    float s2, s3;            // INT4 group 32: scales of the two rows for chunk 1
     uint32_t z0, z1;         // INT2: bf16x2(128 + z) of the two rows
     uint32_t sb0, sb1;       // NVFP4: four E4M3 block scales of each row
 };
@@ -123,6 +125,13 @@ MOE_DEV void load_blk(Blk<Q>& o, const MatPtr& m, int nb, int kb, int KB, int G,
             const size_t gi = ((size_t)nb * G + kb / 2) * kBlkN + rl;
             o.s0 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi));
             o.s1 = __half2float(__ldg(reinterpret_cast<const __half*>(m.scales) + gi + 8));
+        } else if constexpr (Q == Q_INT4G32) {      // chunk ch = group 2 kb + ch
+            const size_t gi = ((size_t)nb * G + 2 * kb) * kBlkN + rl;
+            const __half* sp = reinterpret_cast<const __half*>(m.scales);
+            o.s0 = __half2float(__ldg(sp + gi));
+            o.s1 = __half2float(__ldg(sp + gi + 8));
+            o.s2 = __half2float(__ldg(sp + gi + kBlkN));
+            o.s3 = __half2float(__ldg(sp + gi + kBlkN + 8));
         } else {
             const size_t si = (((size_t)nb * KB + kb) * kBlkN + rl) * 4;
             o.sb0 = __ldg(reinterpret_cast<const uint32_t*>(m.scales + si));
@@ -157,6 +166,16 @@ MOE_DEV void mma_blk(float (&acc)[4], const Blk<Q>& o, const __nv_bfloat16* xrow
                 const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
                 mma16816(d, int4_pair(w0, 0), int4_pair(w1, 0), int4_pair(w0, 1), int4_pair(w1, 1), xv.x, xv.y);
                 mma16816(d, int4_pair(w0, 2), int4_pair(w1, 2), int4_pair(w0, 3), int4_pair(w1, 3), xv.z, xv.w);
+            } else if constexpr (Q == Q_INT4G32) {   // one group per chunk: its own partial sum and scale
+                const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
+                float dc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma16816(dc, int4_pair(w0, 0), int4_pair(w1, 0), int4_pair(w0, 1), int4_pair(w1, 1), xv.x, xv.y);
+                mma16816(dc, int4_pair(w0, 2), int4_pair(w1, 2), int4_pair(w0, 3), int4_pair(w1, 3), xv.z, xv.w);
+                const float sa = ch ? o.s2 : o.s0, sb = ch ? o.s3 : o.s1;
+                acc[0] = fmaf(sa, dc[0], acc[0]);
+                acc[1] = fmaf(sa, dc[1], acc[1]);
+                acc[2] = fmaf(sb, dc[2], acc[2]);
+                acc[3] = fmaf(sb, dc[3], acc[3]);
             } else {  // NVFP4: word c of chunk ch lies in 16-column block 2ch + c/2
                 const int b = 2 * ch + (c >> 1);
                 const uint32_t s0 = bf16x2_splat(e4m3_to_f32((o.sb0 >> (8 * b)) & 0xffu));

@@ -99,7 +99,7 @@ struct Slice {
 __host__ __device__ inline Slice qslice(int quant, int K) {
     Slice s;
     s.KB = K / kBlkK;
-    s.G = K / kGroup;
+    s.G = K / group_size(quant);
     s.nch = quant == Q_INT2 ? 1 : 2;
     s.blk_bytes = kBlkN * 16 * s.nch;
     s.code_bytes = s.KB * s.nch * 256;
@@ -180,6 +180,12 @@ MOE_DEV void load_blk_s(Blk<Q>& o, const uint8_t* base, const Slice& s, int kb, 
         if constexpr (Q == Q_NVFP4) {
             o.sb0 = *reinterpret_cast<const uint32_t*>(sc + kb * 64 + gl * 4);
             o.sb1 = *reinterpret_cast<const uint32_t*>(sc + kb * 64 + (gl + 8) * 4);
+        } else if constexpr (Q == Q_INT4G32) {      // groups 2 kb, 2 kb + 1 (16 rows x fp16 each)
+            const __half* sh = reinterpret_cast<const __half*>(sc + kb * 64);
+            o.s0 = __half2float(sh[gl]);
+            o.s1 = __half2float(sh[gl + 8]);
+            o.s2 = __half2float(sh[16 + gl]);
+            o.s3 = __half2float(sh[16 + gl + 8]);
         } else {
             const __half* sh = reinterpret_cast<const __half*>(sc + (kb >> 1) * 32);
             o.s0 = __half2float(sh[gl]);
@@ -1096,6 +1102,7 @@ cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st) {
     if (sms <= 0) sms = 148;
     switch (f.d.ex.quant) {
         case Q_INT4: return launch_fused_q<Q_INT4>(f, st, sms);
+        case Q_INT4G32: return launch_fused_q<Q_INT4G32>(f, st, sms);
         case Q_INT2: return launch_fused_q<Q_INT2>(f, st, sms);
         case Q_NVFP4: return launch_fused_q<Q_NVFP4>(f, st, sms);
         default: return cudaErrorInvalidValue;

@@ -171,7 +171,7 @@ MOE_DEV __half f16_sat(float v) { return __float2half_rn(fminf(fmaxf(v, -65504.0
 MOE_DEV void dequant_half_f16(int quant, const uint8_t* codes, const uint8_t* scales, const uint8_t* zeros, int r,
                               int h, uint32_t (&v)[16]) {
     const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(scales)[r]);
-    if (quant == Q_INT4) {
+    if (is_int4(quant)) {
         const __half2 off = __float2half2_rn(1032.0f);
         const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);   // chunk h
         const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
@@ -201,7 +201,7 @@ MOE_DEV void dequant_half_f16(int quant, const uint8_t* codes, const uint8_t* sc
 // applied in the epilogue).
 MOE_DEV void dequant_half(int quant, const uint8_t* codes, const uint8_t* scales, const uint8_t* zeros, int r, int h,
                           uint32_t (&v)[16]) {
-    if (quant == Q_INT4) {
+    if (is_int4(quant)) {
         const __half s16 = reinterpret_cast<const __half*>(scales)[r];
         const __nv_bfloat162 s2 = __bfloat162bfloat162(__float2bfloat16_rn(__half2float(s16)));
         const __nv_bfloat162 off = __bfloat162bfloat162(__float2bfloat16_rn(136.0f));
@@ -442,9 +442,11 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // ------------------------------------------- producer: packed weights
         // the codes of KSTEP consecutive blocks are contiguous, and so are
         // their NVFP4 scales
-        const int KB = a.K / kBlkK, G = a.K / kGroup;
+        const int KB = a.K / kBlkK, G = a.K / group_size(a.quant);
         const int cb = block_code_bytes(a.quant) * KSTEP;
-        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : 256;
+        // scales of a stage: NVFP4 KSTEP x 512 bytes; INT4/INT2 group 128 one
+        // group (128 rows x fp16); INT4 group 32 the stage's 2 KSTEP groups
+        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : a.quant == Q_INT4G32 ? 256 * 2 * KSTEP : 256;
         const int zb = a.quant == Q_INT2 ? 128 : 0;
         int g = 0;
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
@@ -465,7 +467,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                         if (a.quant == Q_NVFP4) {
                             bulk_g2s(d + cb, em.scales + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
                         } else {
-                            const size_t go = ((size_t)t.rb * G + kb0 / 2) * 256;   // kb0 even: one group
+                            // first group of the stage (kb0 even: one group-128)
+                            const size_t go = ((size_t)t.rb * G + (a.quant == Q_INT4G32 ? 2 * kb0 : kb0 / 2)) * 256;
                             bulk_g2s(d + cb, em.scales + go, sb, &cfull[c]);
                             if (zb) bulk_g2s(d + cb + sb, em.zeros + go / 2, zb, &cfull[c]);
                         }
@@ -596,11 +599,14 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     tc_fence_after();
                     const uint8_t* stg = smem + C::STG + (c * NMAT + m) * C::STG_MAT;
                     const uint8_t* sc = stg + cb * KSTEP;
-                    const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512 : sc;
                     const uint8_t* zr = sc + 256;
                     uint32_t v[16];
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
+                        // chunk h of block j: NVFP4 scales of the block, INT4 group
+                        // 32 the chunk's own group, else the stage's one group
+                        const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512
+                                           : a.quant == Q_INT4G32 ? sc + (2 * j + h) * 256 : sc;
                         if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
                         else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
                         tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h, v);

@@ -19,8 +19,9 @@
 //       the tensor cores read: row r, 16-byte chunk c (columns 8c..8c+7) at
 //       byte (r/8)*1024 + (r%8)*128 + ((c ^ (r%8)) * 16).
 //
-// Scales (INT4/INT2): fp16 [nb][K/128][128 rows]; zeros (INT2): uint8, one
-// zero per byte, [nb][K/128][128]; NVFP4 block scales: E4M3 bytes
+// Scales (INT4/INT2): fp16 [nb][K/g][128 rows] with g the group size (128;
+// 32 for INT4 group 32); zeros (INT2): uint8, one zero per byte,
+// [nb][K/128][128]; NVFP4 block scales: E4M3 bytes
 // [nb][kb][128 rows][4] (the four 16-column blocks of the 64-column block).
 #pragma once
 
@@ -32,9 +33,15 @@ namespace moe {
 constexpr int kBlkN = 128;      // rows per block
 constexpr int kBlkK = 64;       // columns per block
 constexpr int kGroup = 128;     // INT4/INT2 quantization group
+constexpr int kGroup32 = 32;    // INT4 group-32 quantization group
 constexpr int kFp4Blk = 16;     // NVFP4 scale block
 
-enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3 };
+// Q_INT4G32: INT4 symmetric with one fp16 scale per 32 inputs; codes exactly
+// as Q_INT4 (one 32-column chunk of a block = one group)
+enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3, Q_INT4G32 = 4 };
+
+__host__ __device__ constexpr bool is_int4(int q) { return q == Q_INT4 || q == Q_INT4G32; }
+__host__ __device__ constexpr int group_size(int q) { return q == Q_INT4G32 ? kGroup32 : kGroup; }
 
 __host__ __device__ constexpr int row_bytes_per_kblock(int q) {
     return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : 32);
@@ -44,11 +51,11 @@ struct MatGeom {
     int N = 0, K = 0, quant = 0;
     __host__ __device__ int nb() const { return N / kBlkN; }
     __host__ __device__ int kbs() const { return K / kBlkK; }
-    __host__ __device__ int groups() const { return K / kGroup; }
+    __host__ __device__ int groups() const { return K / group_size(quant); }
     __host__ __device__ size_t block_bytes() const { return (size_t)kBlkN * row_bytes_per_kblock(quant); }
     __host__ __device__ size_t codes_bytes() const { return (size_t)nb() * kbs() * block_bytes(); }
     __host__ __device__ size_t scales_bytes() const {
-        if (quant == Q_INT4 || quant == Q_INT2) return (size_t)N * groups() * 2;
+        if (is_int4(quant) || quant == Q_INT2) return (size_t)N * groups() * 2;
         if (quant == Q_NVFP4) return (size_t)N * (K / kFp4Blk);
         return 0;
     }

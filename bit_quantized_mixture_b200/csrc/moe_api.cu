@@ -133,8 +133,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
         return fail(nullptr, MOE_ERR_UNSUPPORTED, "moe_create: hidden and inter must be multiples of 128");
     if (c.num_experts > 1024 || c.top_k > 32 || c.top_k > c.num_experts)
         return fail(nullptr, MOE_ERR_UNSUPPORTED, "moe_create: need E <= 1024 and k <= min(E, 32)");
-    if (c.quant != MOE_Q_INT4 && c.quant != MOE_Q_INT2 && c.quant != MOE_Q_NVFP4)
-        return fail(nullptr, MOE_ERR_UNSUPPORTED, "moe_create: routed quant must be INT4, INT2 or NVFP4");
+    if (c.quant != MOE_Q_INT4 && c.quant != MOE_Q_INT4_G32 && c.quant != MOE_Q_INT2 && c.quant != MOE_Q_NVFP4)
+        return fail(nullptr, MOE_ERR_UNSUPPORTED, "moe_create: routed quant must be INT4, INT4_G32, INT2 or NVFP4");
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device < 0 || c.device >= ndev)
         return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_create: no CUDA device %d", c.device);
@@ -649,7 +649,7 @@ moe_status moe_quantize(int32_t quant, const float* w, int32_t N, int32_t K, flo
                         void* scales, void* zeros, moe_stream_t stream) {
     if (!w || !codes || !scales) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: null pointer");
     if (N <= 0 || K <= 0) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: sizes must be positive");
-    if (quant == MOE_Q_INT4 || quant == MOE_Q_INT2) {
+    if (quant == MOE_Q_INT4 || quant == MOE_Q_INT4_G32 || quant == MOE_Q_INT2) {
         if (K % 128) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: K must be a multiple of 128");
         if (quant == MOE_Q_INT2 && (N % 4 || !zeros))
             return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: INT2 needs N %% 4 == 0 and zeros");

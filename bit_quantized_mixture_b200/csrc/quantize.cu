@@ -17,16 +17,19 @@
 namespace moe {
 
 // ------------------------------------------------------------------ INT4
-__global__ void k_quantize_int4(const float* __restrict__ w, int N, int K,
+// One warp per 128 consecutive values of a row (four per lane); a group of
+// `group` values (128 or 32) is held by group/4 consecutive lanes.
+__global__ void k_quantize_int4(const float* __restrict__ w, int N, int K, int group,
                                 uint8_t* __restrict__ codes, __half* __restrict__ scales) {
-    const int G = K / kGroup;
+    const int C = K / 128, G = K / group, lpg = group / 4;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (warp >= N * G) return;
-    const int n = warp / G, g = warp % G;
-    const float4 v = *reinterpret_cast<const float4*>(w + (size_t)n * K + g * kGroup + lane * 4);
+    if (warp >= N * C) return;
+    const int n = warp / C, ch = warp % C;
+    const int g = (ch * 128 + lane * 4) / group;
+    const float4 v = *reinterpret_cast<const float4*>(w + (size_t)n * K + ch * 128 + lane * 4);
     float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    amax = warp_max(amax);
+    for (int o = lpg >> 1; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const __half s = __float2half_rn(__fdiv_rn(amax, 7.0f));
     const float sf = __half2float(s);
     float e[4] = {v.x, v.y, v.z, v.w};
@@ -37,8 +40,8 @@ __global__ void k_quantize_int4(const float* __restrict__ w, int N, int K,
         u[i] = (uint32_t)((int)q + 8);
     }
     const uint16_t packed = (uint16_t)(u[0] | (u[1] << 4) | (u[2] << 8) | (u[3] << 12));
-    *reinterpret_cast<uint16_t*>(codes + (size_t)n * (K / 2) + g * 64 + lane * 2) = packed;
-    if (lane == 0) scales[(size_t)n * G + g] = s;
+    *reinterpret_cast<uint16_t*>(codes + (size_t)n * (K / 2) + ch * 64 + lane * 2) = packed;
+    if (lane % lpg == 0) scales[(size_t)n * G + g] = s;
 }
 
 // ------------------------------------------------------------------ INT2
@@ -291,9 +294,10 @@ static inline unsigned blocks_for(size_t n, int tpb) { return (unsigned)((n + tp
 
 cudaError_t launch_quantize(int quant, const float* w, int N, int K, float g, void* codes, void* scales,
                             void* zeros, cudaStream_t st) {
-    if (quant == Q_INT4) {
-        const size_t warps = (size_t)N * (K / kGroup);
-        k_quantize_int4<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (__half*)scales);
+    if (is_int4(quant)) {
+        const size_t warps = (size_t)N * (K / 128);
+        k_quantize_int4<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, group_size(quant), (uint8_t*)codes,
+                                                                     (__half*)scales);
     } else if (quant == Q_INT2) {
         const size_t warps = (size_t)(N / 4) * (K / kGroup);
         k_quantize_int2<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (__half*)scales,

@@ -53,6 +53,12 @@ WORKLOADS = [
              routing="zipf"),
     Workload(4, "prefill-nvfp4", T=8192, H=2048, I=512, E=512, k=10, quant="nvfp4", shared=True,
              routing="uniform"),
+    # the INT4 group-32 format of the MTP-draft experts on the decode-b1 and
+    # prefill-Zipf shapes
+    Workload(5, "decode-b1-int4g32", T=1, H=2048, I=512, E=512, k=10, quant="int4g32", shared=True,
+             routing="router", steps=100),
+    Workload(6, "prefill-int4g32-zipf", T=4096, H=2048, I=512, E=512, k=10, quant="int4g32", shared=False,
+             routing="zipf"),
 ]
 ZIPF_S = 1.1
 

@@ -24,7 +24,7 @@ def _weights(N, K, seed):
     return w
 
 
-@pytest.mark.parametrize("quant", ["int4", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
 @pytest.mark.parametrize("shape", [(128, 256), (512, 2048), (2048, 512), (132, 384)])
 def test_quantize_bit_exact(quant, shape):
     N, K = shape
@@ -38,8 +38,8 @@ def test_quantize_bit_exact(quant, shape):
         assert moe.nvfp4_global_scale(amax.item()) == g
     codes, scales, zeros = moe.quantize(quant, wd, g)
     torch.cuda.synchronize()
-    if quant == "int4":
-        rc, rs = O.quantize_int4(w)
+    if quant in ("int4", "int4g32"):
+        rc, rs = O.quantize_int4(w, group=32 if quant == "int4g32" else 128)
         assert np.array_equal(codes.cpu().numpy(), rc)
         assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
     elif quant == "int2":
@@ -92,7 +92,7 @@ def test_e2m1_conversion_around_every_midpoint():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
-@pytest.mark.parametrize("quant", ["int4", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
 def test_relayout_round_trip(quant):
     from bit_quantized_mixture_b200.layer import quantize_expert_gpu
     wl = synth.custom("tiny-int4", quant=quant, H=384, I=256, E=3, k=2, shared=True)
