@@ -21,6 +21,9 @@ low-bit group quantization and whose routers stay 16-bit:
   "albucino/Qwen3.8-Flash-Next-W4A16-FP8PLE", section "Composition": the
   routed experts of the MTP draft are symmetric INT4 with group 32 (the same
   recipe with one scale per 32 inputs).
+* "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", section "Format": the
+  MTP-draft routed experts are FP8 with 128x128 block scales (E4M3FN codes,
+  one fp32 scale per 128 rows x 128 inputs; reading: s = amax/448).
 * "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", section "Format": routed
   experts are NVFP4 W4A4 (E2M1 values, one scale per 16 elements); the
   shared experts stay BF16.
@@ -57,6 +60,7 @@ import numpy as np
 GROUP_INT = 128      # INT4 / INT2 group size along K
 GROUP_INT4_G32 = 32  # INT4 group size of the MTP-draft experts
 GROUP_FP4 = 16       # NVFP4 block size along K
+BLOCK_FP8 = 128      # FP8 experts: one scale per 128 x 128 block
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
 
@@ -156,6 +160,7 @@ def e2m1_rne_satfinite(v) -> np.ndarray:
 #          row n at bits 2(n%4) of byte (n//4, group).
 #   NVFP4: codes uint8 [N, K/2] (low nibble = even k); block scales E4M3
 #          bytes [N, K/16]; one fp32 global scale.
+#   FP8  : codes E4M3FN bytes [N, K]; scales fp32 [N/128, K/128].
 # --------------------------------------------------------------------------
 
 
@@ -266,6 +271,32 @@ def quantize_nvfp4(w, g):
     return codes, sb
 
 
+def quantize_fp8_block(w):
+    """FP8 E4M3FN with one fp32 scale per 128 x 128 block (MTP-draft experts):
+    s = amax_block / 448 and q = e4m3(w / s), both divisions IEEE fp32; an
+    all-zero block has s = 0 and codes of +-0."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    B = BLOCK_FP8
+    assert N % B == 0 and K % B == 0
+    b = w.reshape(N // B, B, K // B, B)
+    amax = np.abs(b).max(axis=(1, 3)).astype(np.float32)            # [N/B, K/B]
+    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    sb = s[:, None, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(sb == 0, b * np.float32(0.0), b / sb).astype(np.float32)
+    codes = e4m3_rne_satfinite(v).reshape(N, K)
+    return codes, s
+
+
+def dequantize_fp8_block(codes, scales) -> np.ndarray:
+    q = e4m3_decode(codes)
+    N, K = q.shape
+    B = BLOCK_FP8
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64)
+    return (q.reshape(N // B, B, K // B, B) * s[:, None, :, None]).reshape(N, K)
+
+
 def unpack_nvfp4(codes) -> np.ndarray:
     return unpack_int4(codes)            # same nibble order
 
@@ -349,7 +380,7 @@ def dequantize_expert(quant, ew):
     """Expert weights in interchange form -> fp64 (W_gate, W_up, W_down).
 
     ``ew`` maps 'gate'/'up'/'down' to dicts with keys codes, scales and,
-    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int4g32', 'int2', 'nvfp4' or
+    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int4g32', 'int2', 'nvfp4', 'fp8' or
     'bf16' (codes are then bf16 bit patterns)."""
     out = []
     for name in ("gate", "up", "down"):
@@ -360,6 +391,8 @@ def dequantize_expert(quant, ew):
             out.append(dequantize_int2(m["codes"], m["scales"], m["zeros"]))
         elif quant == "nvfp4":
             out.append(dequantize_nvfp4(m["codes"], m["scales"], m["g"]))
+        elif quant == "fp8":
+            out.append(dequantize_fp8_block(m["codes"], m["scales"]))
         elif quant == "bf16":
             out.append(bf16_bits_to_f64(m["codes"]))
         else:

@@ -114,6 +114,62 @@ def test_int4_group32_error_bound_and_finer_than_group128():
     assert err32 < err128
 
 
+# ----------------------------------------------------- FP8 128x128 blocks ----
+
+def test_fp8_block_worked_example(golden):
+    g = golden["fp8_block128"]
+    w = np.zeros((128, 128), np.float32)
+    for key, v in g["block_values"].items():
+        n, k = map(int, key.split(","))
+        w[n, k] = v
+    codes, s = O.quantize_fp8_block(w)
+    assert s.shape == (1, 1) and s.dtype == np.float32
+    assert float(s[0, 0]) == g["scale"]["value_num"] * 2.0 ** g["scale"]["value_exp"]
+    deq = O.dequantize_fp8_block(codes, s)
+    for key, c in g["codes"].items():
+        n, k = map(int, key.split(","))
+        assert codes[n, k] == c
+        assert deq[n, k] == g["dequant_e4m3"][key] * float(s[0, 0])
+    mask = np.ones_like(codes, bool)
+    for key in g["codes"]:
+        n, k = map(int, key.split(","))
+        mask[n, k] = False
+    assert np.all(codes[mask] == 0)
+
+
+def test_fp8_blocks_are_128_by_128():
+    """Each 128x128 block has its own scale: a block's codes depend only on
+    its own values."""
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((256, 384)) * 0.02).astype(np.float32)
+    w[128:, 256:] *= 50.0                                     # one block much larger
+    codes, s = O.quantize_fp8_block(w)
+    assert s.shape == (2, 3)
+    for bn in range(2):
+        for bk in range(3):
+            blk = w[bn * 128:(bn + 1) * 128, bk * 128:(bk + 1) * 128]
+            c1, s1 = O.quantize_fp8_block(blk)
+            assert s1[0, 0] == s[bn, bk]
+            assert np.array_equal(c1, codes[bn * 128:(bn + 1) * 128, bk * 128:(bk + 1) * 128])
+    assert s[1, 2] > 20 * s[0, 0]
+
+
+def test_fp8_block_error_bound_and_zero_block():
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((128, 256)) * 0.02).astype(np.float32)
+    w[:, 128:] = 0.0
+    codes, s = O.quantize_fp8_block(w)
+    assert s[0, 1] == 0 and np.all((codes[:, 128:] & 0x7F) == 0)
+    deq = O.dequantize_fp8_block(codes, s)
+    sc = float(s[0, 0])
+    r = np.abs(w[:, :128]).astype(np.float64)
+    err = np.abs(w[:, :128] - deq[:, :128])
+    # half a quantum: 2^-4 relative in the normal range (|w/s| >= 2^-6), 2^-10 s below
+    bound = np.where(r / sc >= 2.0 ** -6, r * 2.0 ** -4, sc * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    assert np.abs(codes[:, :128].astype(np.int64) & 0x7F).max() <= 0x7E   # finite, at most 448
+
+
 # ---------------------------------------------------------------- INT2 ----
 
 def test_int2_worked_example(golden):
