@@ -167,6 +167,9 @@ class OracleSampler:
                 if wl.quant in ("int4", "int4g32"):
                     c, sc = O.quantize_int4(m, group=32 if wl.quant == "int4g32" else 128)
                     ew[name] = {"codes": c, "scales": sc}
+                elif wl.quant == "fp8":
+                    c, sc = O.quantize_fp8_block(m)
+                    ew[name] = {"codes": c, "scales": sc}
                 elif wl.quant == "int2":
                     c, sc, z = O.quantize_int2(m)
                     ew[name] = {"codes": c, "scales": sc, "zeros": z}
@@ -245,6 +248,9 @@ def expert_bytes(wl):
         gs = 32 if wl.quant == "int4g32" else 128
         gu = 2 * (I * H // 2 + I * (H // gs) * 2)
         dn = H * I // 2 + H * (I // gs) * 2
+    elif wl.quant == "fp8":
+        gu = 2 * (I * H + (I // 128) * (H // 128) * 4)
+        dn = H * I + (H // 128) * (I // 128) * 4
     elif wl.quant == "int2":
         gu = 2 * (I * H // 4 + I * (H // 128) * 2 + I * (H // 128))
         dn = H * I // 4 + H * (I // 128) * 2 + H * (I // 128)
@@ -443,6 +449,9 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
     n = 2 * I                                     # gate + up rows per expert
     if wl.quant in ("int4", "int4g32"):
         w_bytes = n * H // 2 + n * (H // (32 if wl.quant == "int4g32" else 128)) * 2
+        act, out = T * H * 2, slots * I * 2
+    elif wl.quant == "fp8":
+        w_bytes = n * H + (n // 128) * (H // 128) * 4
         act, out = T * H * 2, slots * I * 2
     elif wl.quant == "int2":
         w_bytes = n * H // 4 + n * (H // 128) * 2 + (n // 4) * (H // 128)

@@ -55,6 +55,13 @@ MOE_DEV float e4m3_to_f32(uint32_t b) {
     asm("{ .reg .b16 t; mov.b16 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "h"(in));
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
+// Two E4M3FN bytes (the low one first) -> fp16x2 (exact)
+MOE_DEV uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    uint32_t h2;
+    const uint16_t in = (uint16_t)(two & 0xffffu);
+    asm("{ .reg .b16 t; mov.b16 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "h"(in));
+    return h2;
+}
 // Two fp32 -> two E2M1 nibbles (lo in bits 0-3), RNE, saturating to +-6.
 MOE_DEV uint32_t f32x2_to_e2m1(float lo, float hi) {
     uint32_t r;

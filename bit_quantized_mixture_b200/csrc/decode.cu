@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kGuThreads, 3) k_dec_gateup(DecodeArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int KB = H / kBlkK, G = H / group_size(Q);
+    const int KB = H / kBlkK, G = scale_stride(Q, H);
     const int r0 = rb16 * 16;
     const int nb = r0 / kBlkN, rl = r0 % kBlkN + g;
     const __nv_bfloat16* xrow = xs + (g < m ? tok[g] : kDecMaxT) * ldx;     // item column g = token tok[g]
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kDnThreads, 10) k_dec_down(DecodeArgs a) {
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int KB = I / kBlkK, G = I / group_size(Q);
+    const int KB = I / kBlkK, G = scale_stride(Q, I);
     const int h0 = hb * 16;
     const int nb = h0 / kBlkN, rl = h0 % kBlkN + g;
     const __nv_bfloat16* xrow = as + g * ldx;
@@ -276,6 +276,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     switch (a.ex.quant) {
         case Q_INT4: return launch_decode_q<Q_INT4>(a, st);
         case Q_INT4G32: return launch_decode_q<Q_INT4G32>(a, st);
+        case Q_FP8: return launch_decode_q<Q_FP8>(a, st);
         case Q_INT2: return launch_decode_q<Q_INT2>(a, st);
         case Q_NVFP4: return launch_decode_q<Q_NVFP4>(a, st);
         default: return cudaErrorInvalidValue;

@@ -72,6 +72,15 @@ MOE_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
 template <int Q> struct Fmt;
 template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_INT4G32> { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_FP8>   { static constexpr int KPW = 1; };
+
+// Two E4M3 codes (low byte first) -> bf16x2: exact, since every E4M3 value
+// is an fp16 and a bf16 value
+MOE_DEV uint32_t fp8_pair(uint32_t word, int half) {
+    const uint32_t h2 = e4m3x2_to_f16x2(word >> (16 * half));
+    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+    return pack_bf16x2(__low2float(h), __high2float(h));
+}
 template <> struct Fmt<Q_NVFP4> { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_INT2>  { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_BF16>  { static constexpr int KPW = 1; };
@@ -85,7 +94,7 @@ struct MatPtr {
 // Operands of rows (rl, rl+8) of one 128x64 block for lane (g, c)
 template <int Q>
 struct Blk {
-    uint32_t w[2][2];        // INT4 / NVFP4: [chunk][row g, g+8]; INT2: w[0][row]
+    uint32_t w[4][2];        // INT4 / NVFP4: [chunk][row g, g+8] (FP8: four chunks); INT2: w[0][row]
     uint4 v[2][2];           // bf16: [32-column half][row g, g+8]
     float s0, s1;            // INT4/INT2 scales of the two rows (INT4 group 32: of chunk 0)
     float s2, s3;            // INT4 group 32: scales of the two rows for chunk 1
@@ -105,6 +114,16 @@ MOE_DEV void load_blk(Blk<Q>& o, const MatPtr& m, int nb, int kb, int KB, int G,
                 const int c8 = 4 * h + c;
                 o.v[h][rr] = ldg_stream_v4(blk + (r >> 3) * 1024 + (r & 7) * 128 + ((c8 ^ (r & 7)) << 4));
             }
+    } else if constexpr (Q == Q_FP8) {
+        // four 16-column chunks; lane c takes columns 4c .. 4c+3 of each; the
+        // block scale of (row block, 128-column group) is G-strided (padded)
+        const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 64);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            o.w[q][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + (q * kBlkN + rl) * 16 + c * 4));
+            o.w[q][1] = __ldg(reinterpret_cast<const uint32_t*>(blk + (q * kBlkN + rl + 8) * 16 + c * 4));
+        }
+        o.s0 = __ldg(reinterpret_cast<const float*>(m.scales) + (size_t)nb * G + kb / 2);
     } else if constexpr (Q == Q_INT2) {
         const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 16);
         o.w[0][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + rl * 16 + c * 4));
@@ -145,7 +164,19 @@ MOE_DEV void load_blk(Blk<Q>& o, const MatPtr& m, int nb, int kb, int KB, int G,
 template <int Q>
 MOE_DEV void mma_blk(float (&acc)[4], const Blk<Q>& o, const __nv_bfloat16* xrow, int c) {
     float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if constexpr (Q == Q_INT2) {
+    if constexpr (Q == Q_FP8) {
+        // K16 step q: the lane's B pairs are columns (16q + 4c, +1) and
+        // (16q + 4c + 2, +3), so its A pairs are bytes 0-1 and 2-3 of word c
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint2 xv = *reinterpret_cast<const uint2*>(xrow + 16 * q + 4 * c);
+            mma16816(d, fp8_pair(o.w[q][0], 0), fp8_pair(o.w[q][1], 0), fp8_pair(o.w[q][0], 1),
+                     fp8_pair(o.w[q][1], 1), xv.x, xv.y);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = fmaf(o.s0, d[i], acc[i]);
+        return;
+    } else if constexpr (Q == Q_INT2) {
         const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + 16 * c);
         const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + 16 * c + 8);
         const uint32_t xb[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};

@@ -99,11 +99,13 @@ struct Slice {
 __host__ __device__ inline Slice qslice(int quant, int K) {
     Slice s;
     s.KB = K / kBlkK;
-    s.G = K / group_size(quant);
-    s.nch = quant == Q_INT2 ? 1 : 2;
+    s.G = scale_stride(quant, K);
+    s.nch = quant == Q_INT2 ? 1 : (quant == Q_FP8 ? 4 : 2);
     s.blk_bytes = kBlkN * 16 * s.nch;
     s.code_bytes = s.KB * s.nch * 256;
-    s.scale_bytes = quant == Q_NVFP4 ? s.KB * 64 : s.G * 32;
+    // NVFP4: 4 e4m3 per row and k-block; FP8: the row block's fp32 scales
+    // (G of them, a multiple of 4); else fp16 per row and group
+    s.scale_bytes = quant == Q_NVFP4 ? s.KB * 64 : (quant == Q_FP8 ? s.G * 4 : s.G * 32);
     s.zero_bytes = quant == Q_INT2 ? s.G * 16 : 0;
     s.bytes = s.code_bytes + s.scale_bytes + s.zero_bytes;
     return s;
@@ -116,7 +118,7 @@ __host__ __device__ inline Slice qslice(int quant, int K) {
 // destination advance by constants.
 template <int Q>
 __device__ __noinline__ void load_qslice(uint8_t* dst, MatPtr m, Slice s, int r0, int gtid) {
-    constexpr int NCH = Q == Q_INT2 ? 1 : 2;
+    constexpr int NCH = Q == Q_INT2 ? 1 : (Q == Q_FP8 ? 4 : 2);
     const int nb = r0 / kBlkN, rl0 = r0 % kBlkN;
     {
         const int p0 = gtid >> 4, c16 = gtid & 15;          // piece p0 + 8 j, chunk c16 of its 16
@@ -133,6 +135,9 @@ __device__ __noinline__ void load_qslice(uint8_t* dst, MatPtr m, Slice s, int r0
 #pragma unroll 1
         for (int j = gtid; j < s.KB * 4; j += 128)
             cp16(ds + j * 16, m.scales + (((size_t)nb * s.KB + (j >> 2)) * kBlkN + rl0) * 4 + (j & 3) * 16);
+    } else if constexpr (Q == Q_FP8) {
+#pragma unroll 1
+        for (int j = gtid; j < s.G / 4; j += 128) cp16(ds + j * 16, m.scales + ((size_t)nb * s.G + j * 4) * 4);
     } else {
 #pragma unroll 1
         for (int j = gtid; j < s.G * 2; j += 128)
@@ -169,7 +174,7 @@ MOE_DEV void load_blk_s(Blk<Q>& o, const uint8_t* base, const Slice& s, int kb, 
                 o.v[h][rr] = *reinterpret_cast<const uint4*>(blk + (r >> 3) * 1024 + (r & 7) * 128 + ((c8 ^ (r & 7)) << 4));
             }
     } else {
-        constexpr int NCH = Q == Q_INT2 ? 1 : 2;
+        constexpr int NCH = Q == Q_INT2 ? 1 : (Q == Q_FP8 ? 4 : 2);
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
             const uint8_t* p = base + (kb * NCH + ch) * 256 + c * 4;
@@ -177,7 +182,9 @@ MOE_DEV void load_blk_s(Blk<Q>& o, const uint8_t* base, const Slice& s, int kb, 
             o.w[ch][1] = *reinterpret_cast<const uint32_t*>(p + (gl + 8) * 16);
         }
         const uint8_t* sc = base + s.code_bytes;
-        if constexpr (Q == Q_NVFP4) {
+        if constexpr (Q == Q_FP8) {
+            o.s0 = reinterpret_cast<const float*>(sc)[kb >> 1];
+        } else if constexpr (Q == Q_NVFP4) {
             o.sb0 = *reinterpret_cast<const uint32_t*>(sc + kb * 64 + gl * 4);
             o.sb1 = *reinterpret_cast<const uint32_t*>(sc + kb * 64 + (gl + 8) * 4);
         } else if constexpr (Q == Q_INT4G32) {      // groups 2 kb, 2 kb + 1 (16 rows x fp16 each)
@@ -1103,6 +1110,7 @@ cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st) {
     switch (f.d.ex.quant) {
         case Q_INT4: return launch_fused_q<Q_INT4>(f, st, sms);
         case Q_INT4G32: return launch_fused_q<Q_INT4G32>(f, st, sms);
+        case Q_FP8: return launch_fused_q<Q_FP8>(f, st, sms);
         case Q_INT2: return launch_fused_q<Q_INT2>(f, st, sms);
         case Q_NVFP4: return launch_fused_q<Q_NVFP4>(f, st, sms);
         default: return cudaErrorInvalidValue;

@@ -243,7 +243,25 @@ MOE_DEV void dequant_half(int quant, const uint8_t* codes, const uint8_t* scales
 }
 
 // bytes of the packed codes of one 128x64 block
-MOE_DEV int block_code_bytes(int quant) { return quant == Q_INT2 ? 2048 : 4096; }
+MOE_DEV int block_code_bytes(int quant) { return quant == Q_INT2 ? 2048 : (quant == Q_FP8 ? 8192 : 4096); }
+
+// FP8 (E4M3, one fp32 scale per 128x128 block): chunk h (32 columns, two
+// 16-column chunks of the block's layout) of row r; the E4M3 values are
+// exact in fp16, w = e4m3 * s is rounded once to fp16 (f16) or bf16.
+MOE_DEV void dequant_half_fp8(const uint8_t* codes, float s, int r, int h, bool f16, uint32_t (&v)[16]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(codes + ((2 * h + q) * kBlkN + r) * 16);
+        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const uint32_t h2 = e4m3x2_to_f16x2(wd[p >> 1] >> (16 * (p & 1)));
+            const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
+            const float lo = __low2float(hv) * s, hi = __high2float(hv) * s;
+            v[q * 8 + p] = f16 ? h2_bits(__floats2half2_rn(lo, hi)) : pack_bf16x2(lo, hi);
+        }
+    }
+}
 
 // Bounded mbarrier wait by a whole warp with a warp-uniform result (every
 // lane returns from mbar_wait, so every lane reaches the vote): a warp that
@@ -442,31 +460,40 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // ------------------------------------------- producer: packed weights
         // the codes of KSTEP consecutive blocks are contiguous, and so are
         // their NVFP4 scales
-        const int KB = a.K / kBlkK, G = a.K / group_size(a.quant);
+        const int KB = a.K / kBlkK, G = scale_stride(a.quant, a.K);
+        const bool fp8 = a.quant == Q_FP8;
         const int cb = block_code_bytes(a.quant) * KSTEP;
         // scales of a stage: NVFP4 KSTEP x 512 bytes; INT4/INT2 group 128 one
-        // group (128 rows x fp16); INT4 group 32 the stage's 2 KSTEP groups
-        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : a.quant == Q_INT4G32 ? 256 * 2 * KSTEP : 256;
+        // group (128 rows x fp16); INT4 group 32 the stage's 2 KSTEP groups;
+        // FP8 the one block scale, stored by this thread
+        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : a.quant == Q_INT4G32 ? 256 * 2 * KSTEP : fp8 ? 0 : 256;
         const int zb = a.quant == Q_INT2 ? 128 : 0;
+        const int stg_mat = fp8 ? KSTEP * 8192 + 16 : C::STG_MAT;    // FP8 stages take more of the ring
+        const int SCr = fp8 ? (SC * C::STG_MAT) / stg_mat : SC;
         int g = 0;
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
-                const int c = g % SC;
-                if (!warp_wait(&cempty[c], ((uint32_t)(g / SC) & 1u) ^ 1u, &abort_flag, a.err, 1)) { ok = false; break; }
+                const int c = g % SCr;
+                if (!warp_wait(&cempty[c], ((uint32_t)(g / SCr) & 1u) ^ 1u, &abort_flag, a.err, 1)) { ok = false; break; }
                 if (lane == 0) {
                     const int kb0 = ks * KSTEP;
-                    uint8_t* stg = smem + C::STG + c * NMAT * C::STG_MAT;
+                    uint8_t* stg = smem + C::STG + c * NMAT * stg_mat;
+                    if (fp8)      // plain stores, released by the arrive below
+                        for (int m = 0; m < NMAT; ++m)
+                            *reinterpret_cast<float*>(stg + m * stg_mat + cb) =
+                                __ldg(reinterpret_cast<const float*>(expert_matrix(m == 0 ? a.w0 : a.w1, t.expert).scales) +
+                                      (size_t)t.rb * G + kb0 / 2);
                     mbar_arrive_expect_tx(&cfull[c], (uint32_t)(NMAT * (cb + sb + zb)));
                     for (int m = 0; m < NMAT; ++m) {
                         const ExpertMat em = expert_matrix(m == 0 ? a.w0 : a.w1, t.expert);
-                        uint8_t* d = stg + m * C::STG_MAT;
+                        uint8_t* d = stg + m * stg_mat;
                         bulk_g2s(d, em.codes + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
                                  &cfull[c]);
                         if (a.quant == Q_NVFP4) {
                             bulk_g2s(d + cb, em.scales + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
-                        } else {
+                        } else if (!fp8) {
                             // first group of the stage (kb0 even: one group-128)
                             const size_t go = ((size_t)t.rb * G + (a.quant == Q_INT4G32 ? 2 * kb0 : kb0 / 2)) * 256;
                             bulk_g2s(d + cb, em.scales + go, sb, &cfull[c]);
@@ -584,20 +611,23 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool f16 = MODE == 0 && a.tok_scale != nullptr;
             const int cb = block_code_bytes(a.quant);
+            const bool fp8 = a.quant == Q_FP8;
+            const int stg_mat = fp8 ? KSTEP * 8192 + 16 : C::STG_MAT;    // as the producer
+            const int SCr = fp8 ? (SC * C::STG_MAT) / stg_mat : SC;
             int g = 0;
             for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
                 bool ok = true;
                 for (int ks = 0; ks < NS; ++ks, ++g) {
-                    const int c = g % SC, s = g % S;
+                    const int c = g % SCr, s = g % S;
                     // the packed codes arrived, and the MMAs that read this
                     // TMEM slot before have completed
-                    if (!warp_wait(&cfull[c], (uint32_t)(g / SC) & 1u, &abort_flag, a.err, 4) ||
+                    if (!warp_wait(&cfull[c], (uint32_t)(g / SCr) & 1u, &abort_flag, a.err, 4) ||
                         !warp_wait(&empty[s], ((uint32_t)(g / S) & 1u) ^ 1u, &abort_flag, a.err, 6)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint8_t* stg = smem + C::STG + (c * NMAT + m) * C::STG_MAT;
+                    const uint8_t* stg = smem + C::STG + (c * NMAT + m) * stg_mat;
                     const uint8_t* sc = stg + cb * KSTEP;
                     const uint8_t* zr = sc + 256;
                     uint32_t v[16];
@@ -607,7 +637,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                         // 32 the chunk's own group, else the stage's one group
                         const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512
                                            : a.quant == Q_INT4G32 ? sc + (2 * j + h) * 256 : sc;
-                        if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
+                        if (fp8) dequant_half_fp8(stg + j * cb, *reinterpret_cast<const float*>(sc), r, h, f16, v);
+                        else if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
                         else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
                         tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h, v);
                     }

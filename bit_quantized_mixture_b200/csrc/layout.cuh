@@ -15,13 +15,16 @@
 //         INT2  crumb  p of the word holds column 2*(p%8) + p/8
 //       Chunk c of an INT4/NVFP4 row covers columns [32c, 32c+32); word w of
 //       a chunk covers [8w, 8w+8) (INT4) or [16w, 16w+16) (INT2, one chunk).
+//   FP8  : [16-byte chunk q (4)][row r (128)][16 bytes]: chunk q of a row
+//       holds the E4M3 codes of columns [16q, 16q+16) in natural order.
 //   bf16 : the 16 KB image of a 128x64 K-major tile in the 128-byte swizzle
 //       the tensor cores read: row r, 16-byte chunk c (columns 8c..8c+7) at
 //       byte (r/8)*1024 + (r%8)*128 + ((c ^ (r%8)) * 16).
 //
 // Scales (INT4/INT2): fp16 [nb][K/g][128 rows] with g the group size (128;
 // 32 for INT4 group 32); zeros (INT2): uint8, one zero per byte,
-// [nb][K/128][128]; NVFP4 block scales: E4M3 bytes
+// [nb][K/128][128]; FP8 block scales: fp32 [nb][align4(K/128)] (one per
+// 128x128 block, rows padded to 16 bytes); NVFP4 block scales: E4M3 bytes
 // [nb][kb][128 rows][4] (the four 16-column blocks of the 64-column block).
 #pragma once
 
@@ -38,13 +41,19 @@ constexpr int kFp4Blk = 16;     // NVFP4 scale block
 
 // Q_INT4G32: INT4 symmetric with one fp16 scale per 32 inputs; codes exactly
 // as Q_INT4 (one 32-column chunk of a block = one group)
-enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3, Q_INT4G32 = 4 };
+// Q_FP8: E4M3 codes with one fp32 scale per 128x128 block
+enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3, Q_INT4G32 = 4, Q_FP8 = 5 };
 
 __host__ __device__ constexpr bool is_int4(int q) { return q == Q_INT4 || q == Q_INT4G32; }
 __host__ __device__ constexpr int group_size(int q) { return q == Q_INT4G32 ? kGroup32 : kGroup; }
+// scale entries per row (INT4/INT2: per weight row; FP8: per 128-row block,
+// padded to a multiple of four) in the device layout
+__host__ __device__ constexpr int scale_stride(int q, int K) {
+    return q == Q_FP8 ? (((K / 128) + 3) & ~3) : K / group_size(q);
+}
 
 __host__ __device__ constexpr int row_bytes_per_kblock(int q) {
-    return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : 32);
+    return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : (q == Q_FP8 ? 64 : 32));
 }
 
 struct MatGeom {
@@ -57,8 +66,11 @@ struct MatGeom {
     __host__ __device__ size_t scales_bytes() const {
         if (is_int4(quant) || quant == Q_INT2) return (size_t)N * groups() * 2;
         if (quant == Q_NVFP4) return (size_t)N * (K / kFp4Blk);
+        if (quant == Q_FP8) return (size_t)nb() * fp8_scale_stride() * 4;
         return 0;
     }
+    // FP8: fp32 scales per row block, padded to a multiple of four
+    __host__ __device__ int fp8_scale_stride() const { return ((K / 128) + 3) & ~3; }
     __host__ __device__ size_t zeros_bytes() const { return quant == Q_INT2 ? (size_t)N * groups() : 0; }
 };
 

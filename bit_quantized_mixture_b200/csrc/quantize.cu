@@ -44,6 +44,43 @@ __global__ void k_quantize_int4(const float* __restrict__ w, int N, int K, int g
     if (lane % lpg == 0) scales[(size_t)n * G + g] = s;
 }
 
+// ------------------------------------------------------------------- FP8
+// One CTA of 256 threads per 128x128 block: s = amax / 448 and the E4M3 code
+// of w / s, both divisions IEEE fp32; an all-zero block has s = 0 and codes
+// of +-0 (w * 0 keeps the sign).  codes [N, K], scales fp32 [N/128, K/128].
+__global__ void __launch_bounds__(256) k_quantize_fp8(const float* __restrict__ w, int N, int K,
+                                                      uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    __shared__ float red[8];
+    const int KB = K / 128;
+    const int bn = blockIdx.x / KB, bk = blockIdx.x % KB;
+    const int c4 = threadIdx.x & 31, r0 = threadIdx.x >> 5;      // 4 columns, rows r0, r0 + 8, ...
+    const float* src = w + (size_t)(bn * 128) * K + bk * 128 + c4 * 4;
+    float amax = 0.0f;
+    for (int r = r0; r < 128; r += 8) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (size_t)r * K);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    float m = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+    const float s = __fdiv_rn(m, 448.0f);
+    for (int r = r0; r < 128; r += 8) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (size_t)r * K);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float q = (s == 0.0f) ? e[i] * 0.0f : __fdiv_rn(e[i], s);
+            packed |= f32_to_e4m3(q) << (8 * i);
+        }
+        *reinterpret_cast<uint32_t*>(codes + (size_t)(bn * 128 + r) * K + bk * 128 + c4 * 4) = packed;
+    }
+    if (threadIdx.x == 0) scales[blockIdx.x] = s;
+}
+
 // ------------------------------------------------------------------ INT2
 // One warp per (4 rows, 1 group): lanes 8r..8r+7 hold row r, 16 values each.
 __global__ void k_quantize_int2(const float* __restrict__ w, int N, int K, uint8_t* __restrict__ codes,
@@ -150,6 +187,9 @@ MOE_DEV void dev_code_pos(const MatGeom& gm, int n, int k, size_t& off, int& shi
         const int p = ki / 2 + (ki % 2) * 8;
         off = base + (size_t)r * 16 + w * 4 + p / 4;
         shift = (p % 4) * 2;
+    } else if (gm.quant == Q_FP8) {  // one byte per code, 16-column chunks
+        off = base + ((size_t)(kl / 16) * kBlkN + r) * 16 + kl % 16;
+        shift = 0;
     } else {  // INT4 / NVFP4 nibbles
         const int c = kl / 32, kc = kl % 32, w = kc / 8, ki = kc % 8;
         const int p = ki / 2 + (ki % 2) * 4;
@@ -159,6 +199,7 @@ MOE_DEV void dev_code_pos(const MatGeom& gm, int n, int k, size_t& off, int& shi
 }
 
 MOE_DEV uint32_t interchange_code(const MatGeom& gm, const uint8_t* src, int n, int k) {
+    if (gm.quant == Q_FP8) return src[(size_t)n * gm.K + k];
     if (gm.quant == Q_INT2) return (src[(size_t)n * (gm.K / 4) + k / 4] >> (2 * (k & 3))) & 3u;
     return (src[(size_t)n * (gm.K / 2) + k / 2] >> (4 * (k & 1))) & 15u;
 }
@@ -179,6 +220,14 @@ __global__ void k_relayout_codes(MatGeom gm, const uint8_t* __restrict__ src, ui
         const uint4 v = *reinterpret_cast<const uint4*>(src + ((size_t)n * gm.K + kb * kBlkK + c * 8) * 2);
         uint8_t* d = dst + blk * 16384 + (r / 8) * 1024 + (r % 8) * 128 + ((c ^ (r % 8)) * 16);
         *reinterpret_cast<uint4*>(d) = v;
+        return;
+    }
+    if (gm.quant == Q_FP8) {
+        const size_t blk = t / gm.block_bytes();
+        const int within = (int)(t % gm.block_bytes());
+        const int q = within / (kBlkN * 16), r = (within / 16) % kBlkN;
+        const int rb = (int)(blk / gm.kbs()), kb = (int)(blk % gm.kbs());
+        dst[t] = src[(size_t)(rb * kBlkN + r) * gm.K + kb * kBlkK + q * 16 + within % 16];
         return;
     }
     // invert dev_code_pos for this byte: locate block and row, then scan the
@@ -224,6 +273,13 @@ __global__ void k_relayout_scales(MatGeom gm, const uint8_t* __restrict__ src_sc
         dst_scales[(((size_t)rb * gm.kbs() + kb) * kBlkN + r) * 4 + sub] = src_scales[t];
         return;
     }
+    if (gm.quant == Q_FP8) {      // [N/128][K/128] -> rows padded to fp8_scale_stride
+        const int KB = gm.K / 128;
+        if (t >= (size_t)gm.nb() * KB) return;
+        reinterpret_cast<float*>(dst_scales)[(t / KB) * gm.fp8_scale_stride() + t % KB] =
+            reinterpret_cast<const float*>(src_scales)[t];
+        return;
+    }
     const int G = gm.groups();
     if (t >= (size_t)gm.N * G) return;
     const int n = (int)(t / G), g = (int)(t % G);
@@ -246,7 +302,7 @@ __global__ void k_unpack_codes(MatGeom gm, const uint8_t* __restrict__ dev, uint
         *reinterpret_cast<uint4*>(dst + t * 16) = *reinterpret_cast<const uint4*>(s);
         return;
     }
-    const int per_byte = gm.quant == Q_INT2 ? 4 : 2;
+    const int per_byte = gm.quant == Q_INT2 ? 4 : (gm.quant == Q_FP8 ? 1 : 2);
     const int bpr = gm.K / per_byte;
     if (t >= (size_t)gm.N * bpr) return;
     const int n = (int)(t / bpr), j = (int)(t % bpr);
@@ -256,7 +312,7 @@ __global__ void k_unpack_codes(MatGeom gm, const uint8_t* __restrict__ dev, uint
         size_t off;
         int shift;
         dev_code_pos(gm, n, k, off, shift);
-        const uint32_t v = (dev[off] >> shift) & (gm.quant == Q_INT2 ? 3u : 15u);
+        const uint32_t v = (dev[off] >> shift) & (gm.quant == Q_INT2 ? 3u : (gm.quant == Q_FP8 ? 255u : 15u));
         out |= v << ((8 / per_byte) * q);
     }
     dst[t] = (uint8_t)out;
@@ -272,6 +328,13 @@ __global__ void k_unpack_scales(MatGeom gm, const uint8_t* __restrict__ dev_scal
         const int n = (int)(t / nblk), b = (int)(t % nblk);
         const int rb = n / kBlkN, r = n % kBlkN;
         scales[t] = dev_scales[(((size_t)rb * gm.kbs() + b / 4) * kBlkN + r) * 4 + b % 4];
+        return;
+    }
+    if (gm.quant == Q_FP8) {
+        const int KB = gm.K / 128;
+        if (t >= (size_t)gm.nb() * KB) return;
+        reinterpret_cast<float*>(scales)[t] =
+            reinterpret_cast<const float*>(dev_scales)[(t / KB) * gm.fp8_scale_stride() + t % KB];
         return;
     }
     const int G = gm.groups();
@@ -302,6 +365,8 @@ cudaError_t launch_quantize(int quant, const float* w, int N, int K, float g, vo
         const size_t warps = (size_t)(N / 4) * (K / kGroup);
         k_quantize_int2<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (__half*)scales,
                                                                      (uint8_t*)zeros);
+    } else if (quant == Q_FP8) {
+        k_quantize_fp8<<<(unsigned)((N / 128) * (K / 128)), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (float*)scales);
     } else {
         const size_t blocks = (size_t)N * (K / kFp4Blk);
         k_quantize_nvfp4<float><<<blocks_for(blocks, 256), 256, 0, st>>>(w, N, K, g, (uint8_t*)codes,
@@ -331,7 +396,8 @@ cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const u
                             uint8_t* dst_zeros, cudaStream_t st) {
     k_relayout_codes<<<blocks_for(gm.codes_bytes(), 256), 256, 0, st>>>(gm, src_codes, dst_codes);
     if (gm.quant != Q_BF16) {
-        const size_t n = gm.quant == Q_NVFP4 ? (size_t)gm.N * (gm.K / kFp4Blk) : (size_t)gm.N * gm.groups();
+        const size_t n = gm.quant == Q_NVFP4 ? (size_t)gm.N * (gm.K / kFp4Blk)
+                         : gm.quant == Q_FP8 ? (size_t)gm.nb() * (gm.K / 128) : (size_t)gm.N * gm.groups();
         k_relayout_scales<<<blocks_for(n, 256), 256, 0, st>>>(gm, src_scales, src_zeros, dst_scales, dst_zeros);
     }
     return cudaGetLastError();
@@ -355,10 +421,11 @@ cudaError_t launch_unpack(const MatGeom& gm, const uint8_t* dev_codes, const uin
                           const uint8_t* dev_zeros, uint8_t* codes, uint8_t* scales, uint8_t* zeros,
                           cudaStream_t st) {
     const size_t nbytes = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K / 8
-                                             : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : 2);
+                                             : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : (gm.quant == Q_FP8 ? 1 : 2));
     k_unpack_codes<<<blocks_for(nbytes, 256), 256, 0, st>>>(gm, dev_codes, codes);
     if (gm.quant != Q_BF16) {
-        const size_t n = gm.quant == Q_NVFP4 ? (size_t)gm.N * (gm.K / kFp4Blk) : (size_t)gm.N * gm.groups();
+        const size_t n = gm.quant == Q_NVFP4 ? (size_t)gm.N * (gm.K / kFp4Blk)
+                         : gm.quant == Q_FP8 ? (size_t)gm.nb() * (gm.K / 128) : (size_t)gm.N * gm.groups();
         k_unpack_scales<<<blocks_for(n, 256), 256, 0, st>>>(gm, dev_scales, dev_zeros, scales, zeros);
     }
     return cudaGetLastError();

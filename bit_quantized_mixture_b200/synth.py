@@ -59,6 +59,12 @@ WORKLOADS = [
              routing="router", steps=100),
     Workload(6, "prefill-int4g32-zipf", T=4096, H=2048, I=512, E=512, k=10, quant="int4g32", shared=False,
              routing="zipf"),
+    # FP8 experts with 128x128 block scales (the MTP-draft format of the NVFP4
+    # card) on the same shapes
+    Workload(7, "decode-b1-fp8", T=1, H=2048, I=512, E=512, k=10, quant="fp8", shared=True,
+             routing="router", steps=100),
+    Workload(8, "prefill-fp8-zipf", T=4096, H=2048, I=512, E=512, k=10, quant="fp8", shared=False,
+             routing="zipf"),
 ]
 ZIPF_S = 1.1
 

@@ -41,6 +41,8 @@
  *                stored code u = q + 8 with q = clamp(rne(w/s), -8, 7)
  *         scales fp16  [N, K/128]; s = fp16(amax/7)
  *   INT4_G32  as INT4 with scales fp16 [N, K/32] (one scale per 32 inputs)
+ *   FP8_B128  codes uint8 [N, K] E4M3FN; scales fp32 [N/128, K/128];
+ *             s = amax_block / 448, q = e4m3(w / s); N and K multiples of 128
  *   INT2  codes  uint8 [N, K/4]; element k = 4j + i at bits 2i..2i+1;
  *                u = clamp(rne(w/s) + z, 0, 3)
  *         scales fp16  [N, K/128]; s = fp16((max - min)/3), min <= 0 <= max
@@ -80,8 +82,10 @@ typedef enum {
     MOE_Q_INT2 = 1,            /* INT2 asymmetric, group 128, fp16 scale + 2-bit zero (W2A16) */
     MOE_Q_NVFP4 = 2,           /* E2M1 + E4M3 per-16 scale + fp32 global (W4A4) */
     MOE_Q_BF16 = 3,            /* unquantized bf16 (shared expert) */
-    MOE_Q_INT4_G32 = 4         /* INT4 symmetric, group 32, fp16 scales (the MTP-draft experts of
+    MOE_Q_INT4_G32 = 4,        /* INT4 symmetric, group 32, fp16 scales (the MTP-draft experts of
                                   "Qwen3.8-Flash-Next on 2x RTX 3090", storage-format table) */
+    MOE_Q_FP8_B128 = 5         /* E4M3FN with one fp32 scale per 128x128 block (W8A16; the MTP-draft
+                                  experts of "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", Format) */
 } moe_quant;
 
 #define MOE_SHARED_EXPERT (-1)

@@ -24,10 +24,12 @@ def _weights(N, K, seed):
     return w
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
 @pytest.mark.parametrize("shape", [(128, 256), (512, 2048), (2048, 512), (132, 384)])
 def test_quantize_bit_exact(quant, shape):
     N, K = shape
+    if quant == "fp8" and N % 128:
+        pytest.skip("FP8 blocks are 128 x 128")
     w = _weights(N, K, seed=N + K)
     g = O.nvfp4_global_scale(np.abs(w).max()) if quant == "nvfp4" else 0.0
     wd = torch.from_numpy(w).to(DEV)
@@ -47,6 +49,10 @@ def test_quantize_bit_exact(quant, shape):
         assert np.array_equal(codes.cpu().numpy(), rc)
         assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
         assert np.array_equal(zeros.cpu().numpy(), rz)
+    elif quant == "fp8":
+        rc, rs = O.quantize_fp8_block(w)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     else:
         rc, rs = O.quantize_nvfp4(w, g)
         assert np.array_equal(scales.cpu().numpy(), rs)
@@ -92,7 +98,7 @@ def test_e2m1_conversion_around_every_midpoint():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
 def test_relayout_round_trip(quant):
     from bit_quantized_mixture_b200.layer import quantize_expert_gpu
     wl = synth.custom("tiny-int4", quant=quant, H=384, I=256, E=3, k=2, shared=True)

@@ -144,6 +144,7 @@ def _forward_case(wl, T, seed_tokens=None):
 SMALL = {
     "int4": synth.custom("tiny-int4", H=384, I=256, E=16, k=4, shared=True),
     "int4g32": synth.custom("tiny-int4", quant="int4g32", H=384, I=256, E=16, k=4, shared=True),
+    "fp8": synth.custom("tiny-int4", quant="fp8", H=384, I=256, E=16, k=4, shared=True),
     "int2": synth.custom("tiny-int4", quant="int2", H=384, I=256, E=16, k=4, shared=True),
     "nvfp4": synth.custom("tiny-int4", quant="nvfp4", H=384, I=256, E=16, k=4, shared=True),
 }
@@ -155,7 +156,7 @@ def test_forward_tiny_workload():
     assert_close_output(y, y_ref)
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
 @pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 9])
 def test_forward_small_layers(quant, T):
     y, y_ref, _, _ = _forward_case(SMALL[quant], T)
@@ -246,12 +247,13 @@ def test_errors_are_reported_without_device_work():
 MID = {
     "int4": synth.custom("tiny-int4", H=512, I=384, E=24, k=6, shared=True),
     "int4g32": synth.custom("tiny-int4", quant="int4g32", H=512, I=384, E=24, k=6, shared=True),
+    "fp8": synth.custom("tiny-int4", quant="fp8", H=512, I=384, E=24, k=6, shared=True),
     "int2": synth.custom("tiny-int4", quant="int2", H=512, I=384, E=24, k=6, shared=True),
     "nvfp4": synth.custom("tiny-int4", quant="nvfp4", H=512, I=384, E=24, k=6, shared=True),
 }
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
 @pytest.mark.parametrize("T", [5, 37, 300])
 def test_prefill_matches_oracle(quant, T):
     """T > 4 runs the permutation + tcgen05 grouped GEMMs: several 128-row
@@ -338,8 +340,12 @@ def test_prefill_zipf_int4g32_full_size_sampled_tokens():
     _full_size_sampled("prefill-int4g32-zipf", 8)
 
 
+def test_prefill_zipf_fp8_full_size_sampled_tokens():
+    _full_size_sampled("prefill-fp8-zipf", 8)
+
+
 # --------------------------------------------- whole layer in one call (fused)
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
 @pytest.mark.parametrize("T", [1, 3, 8])
 def test_route_forward_matches_route_then_oracle(quant, T):
     """moe_route_forward (one cooperative kernel for T <= 8): ids/weights equal
@@ -377,7 +383,7 @@ def test_route_forward_matches_route_then_oracle(quant, T):
     assert torch.equal(y, y2)
 
 
-@pytest.mark.parametrize("wl_name", ["decode-b1-int4", "decode-b1-int4g32"])
+@pytest.mark.parametrize("wl_name", ["decode-b1-int4", "decode-b1-int4g32", "decode-b1-fp8"])
 def test_route_forward_decode_b1_full_size(wl_name):
     wl = synth.workload(wl_name)
     layer = get_layer(wl, 4)
