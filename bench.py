@@ -285,6 +285,9 @@ def run_decode(args, wl, dev, rank, world):
 
     layer, _ = build_layer(wl, dev.index, max_tokens=wl.T)
     pool = expert_pool(layer, wl, dev) if args.expert_table else None
+    # the path moe_route_forward takes inside a CUDA graph (router kernel and
+    # the two GEMV kernels), also for the eager per-kernel breakdown below
+    layer.set_decode_path("kernels")
     xs_host = synth.activations_bf16(wl)
     xs = torch.from_numpy(xs_host.view(np.int16)).to(dev).view(torch.bfloat16)
     T, k = wl.T, wl.k
@@ -366,12 +369,18 @@ def run_decode(args, wl, dev, rank, world):
     with torch.cuda.stream(stream):
         for s in range(args.steps):
             i = step_index(s)
-            flush.zero_()
+            # several flushes: the GPU then takes longer than the host needs to
+            # queue the three kernels, so the events time the kernels, not
+            # the host's launch calls
+            for _ in range(4):
+                flush.zero_()
             layer.set_profile_events(pev[s])
             layer.route_forward(xs[i * T:(i + 1) * T], ids, w, y)
     layer.set_profile_events(None)
     stream.synchronize()
-    k_fused = [p[0].elapsed_time(p[4]) for p in pev]
+    k_router = [p[0].elapsed_time(p[1]) for p in pev]
+    k_gateup = [p[2].elapsed_time(p[3]) for p in pev]
+    k_down = [p[3].elapsed_time(p[4]) for p in pev]
     uniq_per_step = []
     with torch.cuda.stream(stream):
         for s in range(args.steps):
@@ -403,29 +412,39 @@ def run_decode(args, wl, dev, rank, world):
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
     e2e_ms_max = allreduce_max(e2e_ms, dev, world)
 
-    # ---- roofline of the (single) fused decode kernel: algorithmic bytes of
-    # the whole step (router, distinct experts, shared expert, activations,
-    # intermediates and partials) over its event-measured duration
+    # ---- roofline of the dominant decode kernel: its algorithmic bytes over
+    # its event-measured duration.  router: Wr, x, logits; gate/up: the
+    # distinct experts' gate and up weights, the shared gate/up, x and the fp32
+    # intermediates; down: the distinct experts' down weights, the shared down,
+    # the intermediates, the fp32 partials (written and read) and y.
     gu_b, dn_b = expert_bytes(wl)
     H, I = wl.H, wl.I
-    sh = 3 * I * H * 2 if wl.shared else 0
     mean_uniq = float(np.mean(uniq_per_step))
-    step_bytes = (wl.E * H * 2 + T * H * 2 + T * wl.E * 4 + mean_uniq * (gu_b + dn_b) + sh
-                  + (T * k + T) * I * 4 * 2 + (T * k + T) * H * 4 * 2 + T * H * 2)
-    kern = {"decode_fused": float(np.mean(k_fused))}
+    rows = T * k + T
+    by = {
+        "k_router_small": wl.E * H * 2 + T * H * 2 + T * wl.E * 4,
+        "k_dec_gateup": mean_uniq * gu_b + (2 * I * H * 2 if wl.shared else 0) + T * H * 2 + rows * I * 4,
+        "k_dec_down": mean_uniq * dn_b + (I * H * 2 if wl.shared else 0) + rows * I * 4 + rows * H * 4 * 2
+                      + T * H * 2,
+    }
+    step_bytes = float(sum(by.values()))
+    kern = {"k_router_small": float(np.mean(k_router)), "k_dec_gateup": float(np.mean(k_gateup)),
+            "k_dec_down": float(np.mean(k_down))}
+    dom = max(kern, key=kern.get)
     peaks, peak_kind = measured_peaks()
-    achieved = step_bytes / (kern["decode_fused"] * 1e-3) / 1e9
-    traffic = load_traffic("k_decode_fused", wl.name)
+    achieved = by[dom] / (kern[dom] * 1e-3) / 1e9
+    traffic = load_traffic(dom, wl.name)
     layer.close()
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
-        "clocks": clocks.summary(), "kernels_ms": kern, "dominant": "decode_fused",
-        "roofline": {"bound": "hbm", "kernel": "k_decode_fused", "achieved": achieved, "peak": peaks["hbm_gbs"],
+        "clocks": clocks.summary(), "kernels_ms": kern, "dominant": dom,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": step_bytes, "peak_source": peak_kind},
+                     "algorithmic_bytes_per_launch": by[dom], "peak_source": peak_kind,
+                     "decode_path": "router kernel + two GEMV kernels (CUDA graph)"},
         "layer_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
         "warm_ms_per_step": warm_ms / args.steps,
-        "launches_per_step": 1, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
+        "launches_per_step": 3, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
     }
 
 

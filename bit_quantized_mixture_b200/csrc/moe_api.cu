@@ -54,6 +54,7 @@ struct moe_layer {
     // per-expert address table (moe_set_expert_table): device [E], in use when set
     const uint8_t** table = nullptr;
     bool table_set = false;
+    int decode_path = 0;           // MOE_DECODE_AUTO / _FUSED / _KERNELS
     float* g_tab = nullptr;        // NVFP4: [2E] global scales gathered from the table's blocks
     __nv_bfloat16 *xq = nullptr, *xp = nullptr, *a_perm = nullptr, *a_sh = nullptr;
     float *w_perm = nullptr, *ts_perm = nullptr;
@@ -483,6 +484,18 @@ static ExpertArgs expert_args(moe_layer* h) {
     return ex;
 }
 
+// Decode (T <= 8) on the fused cooperative kernel?  It saves the launch gaps
+// of eager calls; inside a CUDA graph the GEMV kernels (programmatic launch
+// overlap, no grid barriers) are faster.  false with an error on failure.
+static bool use_fused_decode(moe_layer* h, cudaStream_t st, cudaError_t* err) {
+    *err = cudaSuccess;
+    if (h->decode_path == MOE_DECODE_FUSED) return true;
+    if (h->decode_path == MOE_DECODE_KERNELS) return false;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    *err = cudaStreamIsCapturing(st, &cs);
+    return *err == cudaSuccess && cs == cudaStreamCaptureStatusNone;
+}
+
 static DecodeArgs decode_args(moe_layer* h) {
     DecodeArgs a{};
     a.ex = expert_args(h);
@@ -534,7 +547,10 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         return MOE_OK;
     }
     DecodeArgs a = decode_args(h);
-    if (T <= 8) {
+    cudaError_t pe = cudaSuccess;
+    const bool fused = T <= 8 && use_fused_decode(h, st, &pe);
+    if (pe != cudaSuccess) return cuda_fail(h, pe, "moe_forward");
+    if (fused) {
         FusedArgs f{};
         f.d = a;
         f.d.x = x; f.d.ids = topk_ids; f.d.w = topk_w; f.d.y = y; f.d.T = T;
@@ -591,13 +607,16 @@ moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* to
     if (c.has_shared && !h->shared_loaded) return fail(h, MOE_ERR_STATE, "moe_route_forward: shared expert not loaded");
     if (c.quant == MOE_Q_NVFP4 && !h->act_scales_set)
         return fail(h, MOE_ERR_STATE, "moe_route_forward: NVFP4 activation global scales not set");
-    if (T > 8 || !decode_supported(T, c.top_k)) {
+    DeviceGuard dg(c.device);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t pe = cudaSuccess;
+    const bool fused = use_fused_decode(h, st, &pe);
+    if (pe != cudaSuccess) return cuda_fail(h, pe, "moe_route_forward");
+    if (!fused || T > 8 || !decode_supported(T, c.top_k)) {
         s = moe_route(h, x, T, topk_ids, topk_w, nullptr, stream);
         if (s != MOE_OK) return s;
         return moe_forward(h, x, T, topk_ids, topk_w, y, stream);
     }
-    DeviceGuard dg(c.device);
-    cudaStream_t st = (cudaStream_t)stream;
     FusedArgs f{};
     f.d = decode_args(h);
     f.d.x = x; f.d.ids = topk_ids; f.d.w = topk_w; f.d.y = y; f.d.T = T;
@@ -734,6 +753,14 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which, 
                                 cudaMemcpyDefault, st);
     }
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_unpack_matrix");
+    return MOE_OK;
+}
+
+moe_status moe_set_decode_path(moe_handle h, int32_t path) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_set_decode_path: null handle");
+    if (path != MOE_DECODE_AUTO && path != MOE_DECODE_FUSED && path != MOE_DECODE_KERNELS)
+        return fail(h, MOE_ERR_INVALID_ARG, "moe_set_decode_path: unknown path %d", path);
+    h->decode_path = path;
     return MOE_OK;
 }
 

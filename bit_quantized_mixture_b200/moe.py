@@ -71,6 +71,7 @@ def lib():
             "moe_sync_status": [vp, vp],
             "moe_permute_noalloc": [vp, i32, i32, i32, vp, vp, vp, vp, vp],
             "moe_expert_block_bytes": [vp, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_set_decode_path": [vp, i32],
             "moe_export_expert": [vp, i32, vp, vp],
             "moe_set_expert_table": [vp, ctypes.POINTER(vp), vp],
         }
@@ -182,6 +183,11 @@ class MoeLayer:
             return
         arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
         _check(lib().moe_set_profile_events(self.h, arr, len(events)), self.h)
+
+    def set_decode_path(self, path):
+        """'auto' (fused kernel eagerly, three kernels inside a CUDA graph),
+        'fused' or 'kernels'."""
+        _check(lib().moe_set_decode_path(self.h, {"auto": 0, "fused": 1, "kernels": 2}[path]), self.h)
 
     def expert_block_bytes(self):
         n = ctypes.c_size_t(0)

@@ -163,16 +163,21 @@ moe_status moe_route_from_logits(moe_handle h, const float* logits, int32_t T,
 /* Expert computation and combine:
  *   y_t = sum_{j<k} topk_w[t,j] * Expert_{topk_ids[t,j]}(x_t) + Shared(x_t)
  * x bf16 [T, H] in, y bf16 [T, H] out (single rounding of the fp32 sum).
+ * T <= 8 runs the fused decode kernel or the two GEMV kernels as
+ * moe_set_decode_path selects; larger T the grouped GEMMs.
  * Every id must lie in [0, E); ids of one token should be distinct.
  * Errors: INVALID_ARG, STATE (experts/shared/scales not loaded). */
 moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* topk_ids,
                        const float* topk_w, void* y, moe_stream_t stream);
 
 /* The whole layer, moe_route followed by moe_forward, as one call: writes
- * topk_ids / topk_w (as moe_route) and y (as moe_forward).  For T <= 8 it
- * runs as one cooperative kernel (router, top-k, experts, shared expert and
- * combine, separated by bounded grid-wide barriers); larger T, or a refused
- * cooperative launch, runs moe_route then moe_forward.  Errors as those two. */
+ * topk_ids / topk_w (as moe_route) and y (as moe_forward).  For T <= 8 an
+ * eager call runs one cooperative kernel (router, top-k, experts, shared
+ * expert and combine, separated by bounded grid-wide barriers) and a call
+ * under stream capture runs moe_route then moe_forward (see
+ * moe_set_decode_path); larger T, a format or shape the fused kernel does
+ * not take, or a refused cooperative launch, runs moe_route then
+ * moe_forward.  Errors as those two. */
 moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* topk_ids,
                              float* topk_w, void* y, moe_stream_t stream);
 
@@ -222,6 +227,20 @@ moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
 moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                                moe_stream_t stream);
+
+/* Path of moe_route_forward and moe_forward for T <= 8 (decode):
+ *   MOE_DECODE_AUTO     (default) the fused cooperative kernel for eager
+ *                       calls; inside a stream capture (CUDA graph) the
+ *                       router kernel and the two GEMV kernels, which overlap
+ *                       through programmatic launch and have no grid barriers
+ *   MOE_DECODE_FUSED    always the fused kernel (where the format fits it)
+ *   MOE_DECODE_KERNELS  always the router + two GEMV kernels
+ * Both paths compute the same layer; their fp32 sums may round differently.
+ * Errors: INVALID_ARG (unknown path). */
+#define MOE_DECODE_AUTO 0
+#define MOE_DECODE_FUSED 1
+#define MOE_DECODE_KERNELS 2
+moe_status moe_set_decode_path(moe_handle h, int32_t path);
 
 /* ------------------------------------------------- expert address table
  *

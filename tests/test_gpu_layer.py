@@ -383,6 +383,41 @@ def test_route_forward_matches_route_then_oracle(quant, T):
     assert torch.equal(y, y2)
 
 
+@pytest.mark.parametrize("quant", ["int4", "int2"])
+def test_route_forward_paths(quant):
+    """The fused kernel (eager default), the router + GEMV kernels (forced, and
+    chosen by default under stream capture) compute the same layer; the
+    captured graph equals moe_route followed by moe_forward bit for bit."""
+    wl = SMALL[quant]
+    T = 3
+    layer = get_layer(wl, 8)
+    ox = OracleExperts(wl)
+    x = synth.activations_bf16(wl, steps=2)[:T]
+    xd = bf16_tensor(x, DEV)
+    ids = torch.empty((T, wl.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, wl.k), dtype=torch.float32, device=DEV)
+    ys = {}
+    for path in ("fused", "kernels"):
+        layer.set_decode_path(path)
+        y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+        layer.route_forward(xd, ids, w, y)
+        layer.sync_status()
+        ys[path] = y
+        ids_h, w_h = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+        assert_close_output(to_bits(y), O.moe_forward(x, ids_h, w_h, quant, ox, shared=ox.shared()))
+    layer.set_decode_path("auto")
+    st = torch.cuda.Stream(device=DEV)
+    yg = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        layer.route_forward(xd, ids, w, yg)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(yg, ys["kernels"])
+    del g
+    layer.set_decode_path("auto")
+
+
 @pytest.mark.parametrize("wl_name", ["decode-b1-int4", "decode-b1-int4g32", "decode-b1-fp8"])
 def test_route_forward_decode_b1_full_size(wl_name):
     wl = synth.workload(wl_name)
