@@ -660,22 +660,10 @@ def allreduce_max(v, dev, world):
     return float(t.item())
 
 
-def run_ours(args):
-    import torch
-
-    from bit_quantized_mixture_b200 import synth
-    rank, local_rank, world = dist_env()
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    wl = synth.workload(args.workload)
-    prefill = wl.routing != "router"
-    r = run_prefill(args, wl, dev, rank, world) if prefill else run_decode(args, wl, dev, rank, world)
+def bench_line(args, wl, r, world, prefill):
+    """The JSON line of a run from the per-rank results r, whose times are
+    already the maximum over the ranks: value = all ranks' tokens over that
+    time (replicas, weak scaling)."""
     tokens_all = r["steps_tokens"] * world
     value = tokens_all / (r["total_ms"] * 1e-3)
     e2e = tokens_all / (r["e2e_ms"] * 1e-3)
@@ -700,6 +688,26 @@ def run_ours(args):
         line["warm_ms_per_step"] = r["warm_ms_per_step"]
     if "layer_tflops" in r:
         line["layer_tflops"] = r["layer_tflops"]
+    return line
+
+
+def run_ours(args):
+    import torch
+
+    from bit_quantized_mixture_b200 import synth
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.workload(args.workload)
+    prefill = wl.routing != "router"
+    r = run_prefill(args, wl, dev, rank, world) if prefill else run_decode(args, wl, dev, rank, world)
+    line = bench_line(args, wl, r, world, prefill)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_tokens_per_s(wl, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
