@@ -21,6 +21,12 @@ low-bit group quantization and whose routers stay 16-bit:
   "albucino/Qwen3.8-Flash-Next-W4A16-FP8PLE", section "Composition": the
   routed experts of the MTP draft are symmetric INT4 with group 32 (the same
   recipe with one scale per 32 inputs).
+* "Qwen3.8-Flash-Next-FP6-INT8", introduction and section "Quantization
+  quality": routed experts in fp6 e2m3 with fp16 scales.  Readings: the OCP
+  MX FP6 E2M3 element (1 sign, 2 exponent bits with bias 1, 3 mantissa bits;
+  magnitudes m/8 below 1, 2^(e-1) (1 + m/8) above, at most 7.5), one fp16
+  scale per 32 inputs (6.5 bits per weight, as the card's bit budget),
+  s = fp16(amax / 7.5) and q = e2m3(w / s) rounded half-to-even, saturating.
 * "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", section "Format": the
   MTP-draft routed experts are FP8 with 128x128 block scales (E4M3FN codes,
   one fp32 scale per 128 rows x 128 inputs; reading: s = amax/448).
@@ -61,6 +67,8 @@ GROUP_INT = 128      # INT4 / INT2 group size along K
 GROUP_INT4_G32 = 32  # INT4 group size of the MTP-draft experts
 GROUP_FP4 = 16       # NVFP4 block size along K
 BLOCK_FP8 = 128      # FP8 experts: one scale per 128 x 128 block
+GROUP_FP6 = 32       # FP6 e2m3 experts: one fp16 scale per 32 inputs
+E2M3_MAX = 7.5
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
 
@@ -161,6 +169,8 @@ def e2m1_rne_satfinite(v) -> np.ndarray:
 #   NVFP4: codes uint8 [N, K/2] (low nibble = even k); block scales E4M3
 #          bytes [N, K/16]; one fp32 global scale.
 #   FP8  : codes E4M3FN bytes [N, K]; scales fp32 [N/128, K/128].
+#   FP6  : codes e2m3 [N, K], one per byte (bits 0-5: sign at bit 5, exponent
+#          bits 3-4, mantissa bits 0-2); scales fp16 [N, K/32].
 # --------------------------------------------------------------------------
 
 
@@ -269,6 +279,54 @@ def quantize_nvfp4(w, g):
     q = e2m1_rne_satfinite(b * r[..., None]).reshape(N, K)
     codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
     return codes, sb
+
+
+def e2m3_decode(code) -> np.ndarray:
+    """FP6 E2M3 code (6 bits) -> float64: exponent 0 is m/8, else
+    2^(e-1) * (1 + m/8)."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    e = (c >> 3) & 3
+    m = c & 7
+    mag = np.where(e == 0, m / 8.0, np.exp2(e - 1.0) * (1.0 + m / 8.0))
+    return np.where(c & 0x20, -mag, mag)
+
+
+def e2m3_rne_satfinite(v) -> np.ndarray:
+    """fp32 -> FP6 E2M3 code, round-half-to-even, saturating to +-7.5.  The
+    grid spacing is 1/8 below 2 (subnormals and exponent 1), 1/4 in [2, 4)
+    and 1/2 in [4, 7.5].  Negative inputs keep their sign bit."""
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(v), E2M3_MAX)
+    quantum = np.where(a < 2.0, 0.125, np.where(a < 4.0, 0.25, 0.5))
+    q = np.minimum(_rne_to_grid(a, quantum), E2M3_MAX)
+    # encode the exactly representable magnitude q
+    e = np.where(q < 1.0, 0, np.where(q < 2.0, 1, np.where(q < 4.0, 2, 3)))
+    m = np.where(e == 0, q * 8.0, (q / np.exp2(e - 1.0) - 1.0) * 8.0)
+    code = (e << 3) | m.astype(np.int64)
+    return (code | (np.signbit(v).astype(np.int64) << 5)).astype(np.uint8)
+
+
+def quantize_fp6(w):
+    """FP6 E2M3 with one fp16 scale per 32 inputs: s = fp16(amax/7.5) and
+    q = e2m3(w / s) (IEEE fp32 division); an all-zero group has s = 0 and
+    codes of +-0."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    assert K % GROUP_FP6 == 0
+    g = w.reshape(N, K // GROUP_FP6, GROUP_FP6)
+    amax = np.abs(g).max(axis=2)
+    s16 = fp16_rne(amax / np.float32(E2M3_MAX))
+    s = s16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s == 0, g * np.float32(0.0), g / s).astype(np.float32)
+    return e2m3_rne_satfinite(v).reshape(N, K), s16
+
+
+def dequantize_fp6(codes, scales) -> np.ndarray:
+    q = e2m3_decode(codes)
+    N, K = q.shape
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)
+    return (q.reshape(N, K // GROUP_FP6, GROUP_FP6) * s[..., None]).reshape(N, K)
 
 
 def quantize_fp8_block(w):
@@ -380,7 +438,7 @@ def dequantize_expert(quant, ew):
     """Expert weights in interchange form -> fp64 (W_gate, W_up, W_down).
 
     ``ew`` maps 'gate'/'up'/'down' to dicts with keys codes, scales and,
-    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int4g32', 'int2', 'nvfp4', 'fp8' or
+    for INT2, zeros, for NVFP4, g.  quant is 'int4', 'int4g32', 'int2', 'nvfp4', 'fp8', 'fp6' or
     'bf16' (codes are then bf16 bit patterns)."""
     out = []
     for name in ("gate", "up", "down"):
@@ -393,6 +451,8 @@ def dequantize_expert(quant, ew):
             out.append(dequantize_nvfp4(m["codes"], m["scales"], m["g"]))
         elif quant == "fp8":
             out.append(dequantize_fp8_block(m["codes"], m["scales"]))
+        elif quant == "fp6":
+            out.append(dequantize_fp6(m["codes"], m["scales"]))
         elif quant == "bf16":
             out.append(bf16_bits_to_f64(m["codes"]))
         else:

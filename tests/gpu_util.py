@@ -21,6 +21,9 @@ def oracle_quantize_expert(quant, gate, up, down):
         if quant == "int4":
             c, s = O.quantize_int4(m)
             ew[name] = {"codes": c, "scales": s}
+        elif quant == "fp6":
+            c, s = O.quantize_fp6(m)
+            ew[name] = {"codes": c, "scales": s}
         elif quant == "fp8":
             c, s = O.quantize_fp8_block(m)
             ew[name] = {"codes": c, "scales": s}

@@ -114,6 +114,57 @@ def test_int4_group32_error_bound_and_finer_than_group128():
     assert err32 < err128
 
 
+# ---------------------------------------------------------- FP6 e2m3 ----
+
+def test_e2m3_table_all_codes(golden):
+    g = golden["fp6_e2m3"]
+    codes = np.arange(64, dtype=np.uint8)
+    vals = O.e2m3_decode(codes)
+    mags = np.array(g["magnitudes"])
+    assert np.array_equal(vals[:32], mags)
+    assert np.array_equal(vals[32:], -mags)
+    # every value encodes back to its own code (signed zeros included)
+    assert np.array_equal(O.e2m3_rne_satfinite(vals.astype(np.float32)), codes[:32].tolist() + [32 + i for i in range(32)])
+
+
+def test_e2m3_midpoints_round_half_even(golden):
+    for v, c in golden["fp6_e2m3"]["midpoints"].items():
+        assert int(O.e2m3_rne_satfinite(np.float32(float(v)))) == c, v
+    # every midpoint between neighbours goes to the even mantissa
+    mags = np.array(golden["fp6_e2m3"]["magnitudes"])
+    mids = (mags[1:] + mags[:-1]) / 2
+    got = O.e2m3_rne_satfinite(mids.astype(np.float32)).astype(int)
+    assert np.all(got % 2 == 0)
+
+
+def test_fp6_worked_group(golden):
+    g = golden["fp6_e2m3"]
+    w = _group(g["group_values"], K=32)
+    codes, s = O.quantize_fp6(w)
+    assert float(s[0, 0]) == g["scale"]["value_num"] * 2.0 ** g["scale"]["value_exp"]
+    for k, c in g["codes"].items():
+        assert codes[0, int(k)] == c
+    deq = O.dequantize_fp6(codes, s)[0]
+    for k, c in g["codes"].items():
+        assert deq[int(k)] == O.e2m3_decode(c) * float(s[0, 0])
+
+
+def test_fp6_error_bound_and_groups_of_32():
+    rng = np.random.default_rng(12)
+    w = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    w[:, 32:64] *= 20.0                                         # one wide group per row
+    codes, s = O.quantize_fp6(w)
+    assert s.shape == (16, 8)
+    deq = O.dequantize_fp6(codes, s)
+    sf = np.repeat(s.astype(np.float64), 32, axis=1)
+    r = np.abs(w) / np.where(sf == 0, 1, sf)
+    half_q = np.where(r < 2, 0.0625, np.where(r < 4, 0.125, 0.25)) * sf
+    assert np.all(np.abs(w - deq) <= half_q * (1 + 2.0 ** -8) + 1e-30)
+    # a group's codes depend only on its own 32 values
+    c2, s2 = O.quantize_fp6(w[:, 32:64])
+    assert np.array_equal(c2, codes[:, 32:64]) and np.array_equal(s2[:, 0], s[:, 1])
+
+
 # ----------------------------------------------------- FP8 128x128 blocks ----
 
 def test_fp8_block_worked_example(golden):
