@@ -170,6 +170,9 @@ class OracleSampler:
                 elif wl.quant == "fp8":
                     c, sc = O.quantize_fp8_block(m)
                     ew[name] = {"codes": c, "scales": sc}
+                elif wl.quant == "fp6":
+                    c, sc = O.quantize_fp6(m)
+                    ew[name] = {"codes": c, "scales": sc}
                 elif wl.quant == "int2":
                     c, sc, z = O.quantize_int2(m)
                     ew[name] = {"codes": c, "scales": sc, "zeros": z}
@@ -251,6 +254,9 @@ def expert_bytes(wl):
     elif wl.quant == "fp8":
         gu = 2 * (I * H + (I // 128) * (H // 128) * 4)
         dn = H * I + (H // 128) * (I // 128) * 4
+    elif wl.quant == "fp6":
+        gu = 2 * (I * H * 3 // 4 + I * (H // 32) * 2)
+        dn = H * I * 3 // 4 + H * (I // 32) * 2
     elif wl.quant == "int2":
         gu = 2 * (I * H // 4 + I * (H // 128) * 2 + I * (H // 128))
         dn = H * I // 4 + H * (I // 128) * 2 + H * (I // 128)
@@ -471,6 +477,9 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
         act, out = T * H * 2, slots * I * 2
     elif wl.quant == "fp8":
         w_bytes = n * H + (n // 128) * (H // 128) * 4
+        act, out = T * H * 2, slots * I * 2
+    elif wl.quant == "fp6":
+        w_bytes = n * H * 3 // 4 + n * (H // 32) * 2
         act, out = T * H * 2, slots * I * 2
     elif wl.quant == "int2":
         w_bytes = n * H // 4 + n * (H // 128) * 2 + (n // 4) * (H // 128)

@@ -55,6 +55,27 @@ MOE_DEV float e4m3_to_f32(uint32_t b) {
     asm("{ .reg .b16 t; mov.b16 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "h"(in));
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
+// fp32 -> FP6 E2M3 code (sign bit 5), round half to even, saturating to
+// +-7.5: rounded on the grid of its binade (1/8 below 2, 1/4 in [2, 4), 1/2
+// above); the scalings by powers of two are exact.
+MOE_DEV uint32_t f32_to_e2m3(float v) {
+    const float a = fminf(fabsf(v), 7.5f);
+    const float inv_q = a < 2.0f ? 8.0f : (a < 4.0f ? 4.0f : 2.0f);
+    const float q = fminf(rintf(a * inv_q) / inv_q, 7.5f);
+    uint32_t e, m;
+    if (q < 1.0f) { e = 0; m = (uint32_t)(q * 8.0f); }
+    else if (q < 2.0f) { e = 1; m = (uint32_t)((q - 1.0f) * 8.0f); }
+    else if (q < 4.0f) { e = 2; m = (uint32_t)((q * 0.5f - 1.0f) * 8.0f); }
+    else { e = 3; m = (uint32_t)((q * 0.25f - 1.0f) * 8.0f); }
+    return (signbit(v) ? 0x20u : 0u) | (e << 3) | m;
+}
+// Two e2m3 codes given as their low nibbles (bits 0-3 of each 16-bit half)
+// and high crumbs (bits 0-1 of each half) -> fp16x2 bits of e2m3 * 2^-14:
+// the mantissa and exponent bits land in the fp16 fields unchanged, so
+// exponent 0 becomes an fp16 subnormal with the same 2^-14 ratio (exact)
+MOE_DEV uint32_t e2m3x2_to_f16x2_scaled(uint32_t nib, uint32_t cr) {
+    return (nib << 7) | ((cr & 0x00010001u) << 11) | ((cr & 0x00020002u) << 14);
+}
 // Two E4M3FN bytes (the low one first) -> fp16x2 (exact)
 MOE_DEV uint32_t e4m3x2_to_f16x2(uint32_t two) {
     uint32_t h2;

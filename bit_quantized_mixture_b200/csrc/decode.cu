@@ -277,6 +277,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
         case Q_INT4: return launch_decode_q<Q_INT4>(a, st);
         case Q_INT4G32: return launch_decode_q<Q_INT4G32>(a, st);
         case Q_FP8: return launch_decode_q<Q_FP8>(a, st);
+        case Q_FP6: return launch_decode_q<Q_FP6>(a, st);
         case Q_INT2: return launch_decode_q<Q_INT2>(a, st);
         case Q_NVFP4: return launch_decode_q<Q_NVFP4>(a, st);
         default: return cudaErrorInvalidValue;

@@ -73,6 +73,18 @@ template <int Q> struct Fmt;
 template <> struct Fmt<Q_INT4>  { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_INT4G32> { static constexpr int KPW = 1; };
 template <> struct Fmt<Q_FP8>   { static constexpr int KPW = 1; };
+template <> struct Fmt<Q_FP6>   { static constexpr int KPW = 1; };
+
+// FP6: pair j (columns 2j, 2j+1 of INT4-style word w) -> bf16x2, exact:
+// low nibbles from w, high crumbs j and j+4 of the high-plane word hw
+MOE_DEV uint32_t fp6_pair(uint32_t w, uint32_t hw, int j) {
+    const uint32_t nib = (w >> (4 * j)) & 0x000F000Fu;
+    const uint32_t x = hw >> (2 * j);
+    const uint32_t cr = (x & 0x3u) | ((x & 0x300u) << 8);
+    const uint32_t h2 = e2m3x2_to_f16x2_scaled(nib, cr);
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h2), __float2half2_rn(16384.0f));   // exact
+    return pack_bf16x2(__low2float(v), __high2float(v));
+}
 
 // Two E4M3 codes (low byte first) -> bf16x2: exact, since every E4M3 value
 // is an fp16 and a bf16 value
@@ -97,7 +109,8 @@ struct Blk {
     uint32_t w[4][2];        // INT4 / NVFP4: [chunk][row g, g+8] (FP8: four chunks); INT2: w[0][row]
     uint4 v[2][2];           // bf16: [32-column half][row g, g+8]
     float s0, s1;            // INT4/INT2 scales of the two rows (INT4 group 32: of chunk 0)
-    float s2, s3;            // INT4 group 32: scales of the two rows for chunk 1
+    float s2, s3;            // INT4 group 32 / FP6: scales of the two rows for chunk 1
+    uint32_t hw[2][2];       // FP6: high-plane 16-bit word of [chunk][row g, g+8]
     uint32_t z0, z1;         // INT2: bf16x2(128 + z) of the two rows
     uint32_t sb0, sb1;       // NVFP4: four E4M3 block scales of each row
 };
@@ -124,6 +137,21 @@ MOE_DEV void load_blk(Blk<Q>& o, const MatPtr& m, int nb, int kb, int KB, int G,
             o.w[q][1] = __ldg(reinterpret_cast<const uint32_t*>(blk + (q * kBlkN + rl + 8) * 16 + c * 4));
         }
         o.s0 = __ldg(reinterpret_cast<const float*>(m.scales) + (size_t)nb * G + kb / 2);
+    } else if constexpr (Q == Q_FP6) {
+        const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 48);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            o.w[ch][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + (ch * kBlkN + rl) * 16 + c * 4));
+            o.w[ch][1] = __ldg(reinterpret_cast<const uint32_t*>(blk + (ch * kBlkN + rl + 8) * 16 + c * 4));
+            o.hw[ch][0] = __ldg(reinterpret_cast<const unsigned short*>(blk + 4096 + (ch * kBlkN + rl) * 8 + c * 2));
+            o.hw[ch][1] = __ldg(reinterpret_cast<const unsigned short*>(blk + 4096 + (ch * kBlkN + rl + 8) * 8 + c * 2));
+        }
+        const size_t gi = ((size_t)nb * G + 2 * kb) * kBlkN + rl;      // chunk ch = group 2 kb + ch
+        const __half* sp = reinterpret_cast<const __half*>(m.scales);
+        o.s0 = __half2float(__ldg(sp + gi));
+        o.s1 = __half2float(__ldg(sp + gi + 8));
+        o.s2 = __half2float(__ldg(sp + gi + kBlkN));
+        o.s3 = __half2float(__ldg(sp + gi + kBlkN + 8));
     } else if constexpr (Q == Q_INT2) {
         const uint8_t* blk = m.codes + ((size_t)nb * KB + kb) * (kBlkN * 16);
         o.w[0][0] = __ldg(reinterpret_cast<const uint32_t*>(blk + rl * 16 + c * 4));
@@ -197,6 +225,18 @@ MOE_DEV void mma_blk(float (&acc)[4], const Blk<Q>& o, const __nv_bfloat16* xrow
                 const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
                 mma16816(d, int4_pair(w0, 0), int4_pair(w1, 0), int4_pair(w0, 1), int4_pair(w1, 1), xv.x, xv.y);
                 mma16816(d, int4_pair(w0, 2), int4_pair(w1, 2), int4_pair(w0, 3), int4_pair(w1, 3), xv.z, xv.w);
+            } else if constexpr (Q == Q_FP6) {       // group 32 = one chunk, as INT4 group 32
+                const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1], h0 = o.hw[ch][0], h1 = o.hw[ch][1];
+                float dc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma16816(dc, fp6_pair(w0, h0, 0), fp6_pair(w1, h1, 0), fp6_pair(w0, h0, 1), fp6_pair(w1, h1, 1), xv.x,
+                         xv.y);
+                mma16816(dc, fp6_pair(w0, h0, 2), fp6_pair(w1, h1, 2), fp6_pair(w0, h0, 3), fp6_pair(w1, h1, 3), xv.z,
+                         xv.w);
+                const float sa = ch ? o.s2 : o.s0, sb = ch ? o.s3 : o.s1;
+                acc[0] = fmaf(sa, dc[0], acc[0]);
+                acc[1] = fmaf(sa, dc[1], acc[1]);
+                acc[2] = fmaf(sb, dc[2], acc[2]);
+                acc[3] = fmaf(sb, dc[3], acc[3]);
             } else if constexpr (Q == Q_INT4G32) {   // one group per chunk: its own partial sum and scale
                 const uint32_t w0 = o.w[ch][0], w1 = o.w[ch][1];
                 float dc[4] = {0.0f, 0.0f, 0.0f, 0.0f};

@@ -1062,6 +1062,7 @@ size_t fused_smem_bytes(int H, int I) {
 // otherwise the two-kernel decode path runs.
 bool fused_supported(int T, int H, int I, int quant) {
     if (T < 1 || T > kDecMaxT) return false;
+    if (quant == Q_FP6) return false;          // two-plane units: the two-kernel path
     const FusedSmem L = fused_layout(T, H, I, quant == Q_NVFP4);
     const Slice gu = qslice(quant, H), dn = qslice(quant, I);
     const int KBP = (H / kBlkK) / shared_kparts(H);

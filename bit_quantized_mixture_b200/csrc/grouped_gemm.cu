@@ -243,7 +243,33 @@ MOE_DEV void dequant_half(int quant, const uint8_t* codes, const uint8_t* scales
 }
 
 // bytes of the packed codes of one 128x64 block
-MOE_DEV int block_code_bytes(int quant) { return quant == Q_INT2 ? 2048 : (quant == Q_FP8 ? 8192 : 4096); }
+MOE_DEV int block_code_bytes(int quant) {
+    return quant == Q_INT2 ? 2048 : (quant == Q_FP8 ? 8192 : (quant == Q_FP6 ? 6144 : 4096));
+}
+
+// FP6 (e2m3, fp16 scale per 32 inputs): chunk h of row r from the two
+// planes of the block; e2m3 values are exact in fp16, w = e2m3 * s is
+// rounded once to fp16 (f16) or bf16.  v[4w + j] = columns 8w + 2j, +1.
+MOE_DEV void dequant_half_fp6(const uint8_t* codes, const uint8_t* scales, int r, int h, bool f16,
+                              uint32_t (&v)[16]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);
+    const uint2 hq = *reinterpret_cast<const uint2*>(codes + 4096 + (h * kBlkN + r) * 8);
+    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+    const uint32_t hv[4] = {hq.x & 0xffffu, hq.x >> 16, hq.y & 0xffffu, hq.y >> 16};
+    const __half s16 = reinterpret_cast<const __half*>(scales)[r];
+    const __half2 up = __float2half2_rn(16384.0f), s2 = __half2half2(s16);
+    const float sf = __half2float(s16);
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t nib = (wv[w] >> (4 * j)) & 0x000F000Fu;
+            const uint32_t x = hv[w] >> (2 * j);
+            const uint32_t h2 = e2m3x2_to_f16x2_scaled(nib, (x & 0x3u) | ((x & 0x300u) << 8));
+            const __half2 e = __hmul2(*reinterpret_cast<const __half2*>(&h2), up);      // exact e2m3 values
+            v[4 * w + j] = f16 ? h2_bits(__hmul2(e, s2)) : pack_bf16x2(__low2float(e) * sf, __high2float(e) * sf);
+        }
+}
 
 // FP8 (E4M3, one fp32 scale per 128x128 block): chunk h (32 columns, two
 // 16-column chunks of the block's layout) of row r; the E4M3 values are
@@ -466,10 +492,12 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // scales of a stage: NVFP4 KSTEP x 512 bytes; INT4/INT2 group 128 one
         // group (128 rows x fp16); INT4 group 32 the stage's 2 KSTEP groups;
         // FP8 the one block scale, stored by this thread
-        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : a.quant == Q_INT4G32 ? 256 * 2 * KSTEP : fp8 ? 0 : 256;
+        const bool g32 = a.quant == Q_INT4G32 || a.quant == Q_FP6;
+        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : g32 ? 256 * 2 * KSTEP : fp8 ? 0 : 256;
         const int zb = a.quant == Q_INT2 ? 128 : 0;
-        const int stg_mat = fp8 ? KSTEP * 8192 + 16 : C::STG_MAT;    // FP8 stages take more of the ring
-        const int SCr = fp8 ? (SC * C::STG_MAT) / stg_mat : SC;
+        // FP8 and FP6 stages take more of the ring
+        const int stg_mat = fp8 ? KSTEP * 8192 + 16 : a.quant == Q_FP6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
+        const int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
         int g = 0;
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
@@ -495,7 +523,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                             bulk_g2s(d + cb, em.scales + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
                         } else if (!fp8) {
                             // first group of the stage (kb0 even: one group-128)
-                            const size_t go = ((size_t)t.rb * G + (a.quant == Q_INT4G32 ? 2 * kb0 : kb0 / 2)) * 256;
+                            const size_t go = ((size_t)t.rb * G + (g32 ? 2 * kb0 : kb0 / 2)) * 256;
                             bulk_g2s(d + cb, em.scales + go, sb, &cfull[c]);
                             if (zb) bulk_g2s(d + cb + sb, em.zeros + go / 2, zb, &cfull[c]);
                         }
@@ -611,9 +639,10 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool f16 = MODE == 0 && a.tok_scale != nullptr;
             const int cb = block_code_bytes(a.quant);
-            const bool fp8 = a.quant == Q_FP8;
-            const int stg_mat = fp8 ? KSTEP * 8192 + 16 : C::STG_MAT;    // as the producer
-            const int SCr = fp8 ? (SC * C::STG_MAT) / stg_mat : SC;
+            const bool fp8 = a.quant == Q_FP8, fp6 = a.quant == Q_FP6;
+            // as the producer
+            const int stg_mat = fp8 ? KSTEP * 8192 + 16 : fp6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
+            const int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
             int g = 0;
             for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
                 bool ok = true;
@@ -636,8 +665,9 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                         // chunk h of block j: NVFP4 scales of the block, INT4 group
                         // 32 the chunk's own group, else the stage's one group
                         const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512
-                                           : a.quant == Q_INT4G32 ? sc + (2 * j + h) * 256 : sc;
+                                           : (a.quant == Q_INT4G32 || fp6) ? sc + (2 * j + h) * 256 : sc;
                         if (fp8) dequant_half_fp8(stg + j * cb, *reinterpret_cast<const float*>(sc), r, h, f16, v);
+                        else if (fp6) dequant_half_fp6(stg + j * cb, scj, r, h, f16, v);
                         else if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
                         else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
                         tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h, v);

@@ -17,6 +17,11 @@
 //       a chunk covers [8w, 8w+8) (INT4) or [16w, 16w+16) (INT2, one chunk).
 //   FP8  : [16-byte chunk q (4)][row r (128)][16 bytes]: chunk q of a row
 //       holds the E4M3 codes of columns [16q, 16q+16) in natural order.
+//   FP6  : two planes.  Low plane (4096 bytes): bits 0-3 of every e2m3 code
+//       exactly as the INT4 nibbles.  High plane (2048 bytes): bits 4-5 as
+//       [chunk c][row r][4 x 16 bits]: 16-bit word w of (c, r) holds, at
+//       bits 2p..2p+1, the high bits of the column whose low bits are
+//       nibble p of INT4 word w.
 //   bf16 : the 16 KB image of a 128x64 K-major tile in the 128-byte swizzle
 //       the tensor cores read: row r, 16-byte chunk c (columns 8c..8c+7) at
 //       byte (r/8)*1024 + (r%8)*128 + ((c ^ (r%8)) * 16).
@@ -41,11 +46,12 @@ constexpr int kFp4Blk = 16;     // NVFP4 scale block
 
 // Q_INT4G32: INT4 symmetric with one fp16 scale per 32 inputs; codes exactly
 // as Q_INT4 (one 32-column chunk of a block = one group)
-// Q_FP8: E4M3 codes with one fp32 scale per 128x128 block
-enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3, Q_INT4G32 = 4, Q_FP8 = 5 };
+// Q_FP8: E4M3 codes with one fp32 scale per 128x128 block; Q_FP6: e2m3
+// codes with one fp16 scale per 32 inputs (scales as Q_INT4G32)
+enum Quant : int { Q_INT4 = 0, Q_INT2 = 1, Q_NVFP4 = 2, Q_BF16 = 3, Q_INT4G32 = 4, Q_FP8 = 5, Q_FP6 = 6 };
 
 __host__ __device__ constexpr bool is_int4(int q) { return q == Q_INT4 || q == Q_INT4G32; }
-__host__ __device__ constexpr int group_size(int q) { return q == Q_INT4G32 ? kGroup32 : kGroup; }
+__host__ __device__ constexpr int group_size(int q) { return (q == Q_INT4G32 || q == Q_FP6) ? kGroup32 : kGroup; }
 // scale entries per row (INT4/INT2: per weight row; FP8: per 128-row block,
 // padded to a multiple of four) in the device layout
 __host__ __device__ constexpr int scale_stride(int q, int K) {
@@ -53,7 +59,7 @@ __host__ __device__ constexpr int scale_stride(int q, int K) {
 }
 
 __host__ __device__ constexpr int row_bytes_per_kblock(int q) {
-    return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : (q == Q_FP8 ? 64 : 32));
+    return q == Q_INT2 ? 16 : (q == Q_BF16 ? 128 : (q == Q_FP8 ? 64 : (q == Q_FP6 ? 48 : 32)));
 }
 
 struct MatGeom {
@@ -64,7 +70,7 @@ struct MatGeom {
     __host__ __device__ size_t block_bytes() const { return (size_t)kBlkN * row_bytes_per_kblock(quant); }
     __host__ __device__ size_t codes_bytes() const { return (size_t)nb() * kbs() * block_bytes(); }
     __host__ __device__ size_t scales_bytes() const {
-        if (is_int4(quant) || quant == Q_INT2) return (size_t)N * groups() * 2;
+        if (is_int4(quant) || quant == Q_INT2 || quant == Q_FP6) return (size_t)N * groups() * 2;
         if (quant == Q_NVFP4) return (size_t)N * (K / kFp4Blk);
         if (quant == Q_FP8) return (size_t)nb() * fp8_scale_stride() * 4;
         return 0;

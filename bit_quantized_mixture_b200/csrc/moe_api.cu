@@ -135,9 +135,9 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     if (c.num_experts > 1024 || c.top_k > 32 || c.top_k > c.num_experts)
         return fail(nullptr, MOE_ERR_UNSUPPORTED, "moe_create: need E <= 1024 and k <= min(E, 32)");
     if (c.quant != MOE_Q_INT4 && c.quant != MOE_Q_INT4_G32 && c.quant != MOE_Q_INT2 && c.quant != MOE_Q_NVFP4 &&
-        c.quant != MOE_Q_FP8_B128)
+        c.quant != MOE_Q_FP8_B128 && c.quant != MOE_Q_FP6_E2M3)
         return fail(nullptr, MOE_ERR_UNSUPPORTED,
-                    "moe_create: routed quant must be INT4, INT4_G32, INT2, NVFP4 or FP8_B128");
+                    "moe_create: routed quant must be INT4, INT4_G32, INT2, NVFP4, FP8_B128 or FP6_E2M3");
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device < 0 || c.device >= ndev)
         return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_create: no CUDA device %d", c.device);
@@ -309,7 +309,8 @@ static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix
                               uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st, uint8_t* img_codes = nullptr,
                               uint8_t* img_scales = nullptr) {
     const size_t codes_in = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K * 2
-                                               : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : (gm.quant == Q_FP8 ? 1 : 2));
+                                               : (size_t)gm.N * gm.K /
+                                                     (gm.quant == Q_INT2 ? 4 : ((gm.quant == Q_FP8 || gm.quant == Q_FP6) ? 1 : 2));
     // interchange scales (the device layout pads FP8 scale rows to 16 bytes)
     const size_t scales_in = gm.quant == Q_FP8 ? (size_t)gm.nb() * (gm.K / 128) * 4 : gm.scales_bytes();
     const size_t zeros_in = gm.quant == Q_INT2 ? (size_t)(gm.N / 4) * gm.groups() : 0;
@@ -674,7 +675,7 @@ moe_status moe_quantize(int32_t quant, const float* w, int32_t N, int32_t K, flo
     if (quant == MOE_Q_FP8_B128) {
         if (N % 128 || K % 128)
             return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: FP8 needs N and K multiples of 128");
-    } else if (quant == MOE_Q_INT4 || quant == MOE_Q_INT4_G32 || quant == MOE_Q_INT2) {
+    } else if (quant == MOE_Q_INT4 || quant == MOE_Q_INT4_G32 || quant == MOE_Q_INT2 || quant == MOE_Q_FP6_E2M3) {
         if (K % 128) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: K must be a multiple of 128");
         if (quant == MOE_Q_INT2 && (N % 4 || !zeros))
             return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_quantize: INT2 needs N %% 4 == 0 and zeros");

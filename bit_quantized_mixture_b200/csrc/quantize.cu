@@ -44,6 +44,33 @@ __global__ void k_quantize_int4(const float* __restrict__ w, int N, int K, int g
     if (lane % lpg == 0) scales[(size_t)n * G + g] = s;
 }
 
+// ------------------------------------------------------------------- FP6
+// One warp per 128 consecutive values of a row (four per lane), groups of 32
+// held by 8 lanes: s = fp16(amax / 7.5), code = e2m3(w / s) (IEEE fp32
+// division); an all-zero group has s = 0 and codes of +-0.  codes: one
+// e2m3 code per byte [N, K]; scales fp16 [N, K/32].
+__global__ void k_quantize_fp6(const float* __restrict__ w, int N, int K, uint8_t* __restrict__ codes,
+                               __half* __restrict__ scales) {
+    const int C = K / 128, G = K / 32;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= N * C) return;
+    const int n = warp / C, ch = warp % C;
+    const int g = (ch * 128 + lane * 4) / 32;
+    const float4 v = *reinterpret_cast<const float4*>(w + (size_t)n * K + ch * 128 + lane * 4);
+    float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half s = __float2half_rn(__fdiv_rn(amax, 7.5f));
+    const float sf = __half2float(s);
+    const float e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) packed |= f32_to_e2m3(sf == 0.0f ? e[i] * 0.0f : __fdiv_rn(e[i], sf)) << (8 * i);
+    *reinterpret_cast<uint32_t*>(codes + (size_t)n * K + ch * 128 + lane * 4) = packed;
+    if (lane % 8 == 0) scales[(size_t)n * G + g] = s;
+}
+
 // ------------------------------------------------------------------- FP8
 // One CTA of 256 threads per 128x128 block: s = amax / 448 and the E4M3 code
 // of w / s, both divisions IEEE fp32; an all-zero block has s = 0 and codes
@@ -200,6 +227,7 @@ MOE_DEV void dev_code_pos(const MatGeom& gm, int n, int k, size_t& off, int& shi
 
 MOE_DEV uint32_t interchange_code(const MatGeom& gm, const uint8_t* src, int n, int k) {
     if (gm.quant == Q_FP8) return src[(size_t)n * gm.K + k];
+    if (gm.quant == Q_FP6) return src[(size_t)n * gm.K + k] & 0xFu;      // low plane: bits 0-3
     if (gm.quant == Q_INT2) return (src[(size_t)n * (gm.K / 4) + k / 4] >> (2 * (k & 3))) & 3u;
     return (src[(size_t)n * (gm.K / 2) + k / 2] >> (4 * (k & 1))) & 15u;
 }
@@ -230,8 +258,23 @@ __global__ void k_relayout_codes(MatGeom gm, const uint8_t* __restrict__ src, ui
         dst[t] = src[(size_t)(rb * kBlkN + r) * gm.K + kb * kBlkK + q * 16 + within % 16];
         return;
     }
+    if (gm.quant == Q_FP6 && (int)(t % gm.block_bytes()) >= 4096) {   // high plane: 4 crumbs per byte
+        const size_t blk = t / gm.block_bytes();
+        const int hb = (int)(t % gm.block_bytes()) - 4096;
+        const int c = hb / (kBlkN * 8), r = (hb / 8) % kBlkN, w = (hb % 8) / 2, half = hb % 2;
+        const int rb = (int)(blk / gm.kbs()), kb = (int)(blk % gm.kbs());
+        const int n = rb * kBlkN + r;
+        uint32_t out = 0;
+        for (int q = 0; q < 4; ++q) {
+            const int p = half * 4 + q;                       // crumb p pairs with nibble p of word w
+            const int k = kb * kBlkK + c * 32 + w * 8 + (p % 4) * 2 + p / 4;
+            out |= ((uint32_t)(src[(size_t)n * gm.K + k] >> 4) & 3u) << (2 * q);
+        }
+        dst[t] = (uint8_t)out;
+        return;
+    }
     // invert dev_code_pos for this byte: locate block and row, then scan the
-    // elements of the 16-byte chunk word that owns the byte
+    // elements of the 16-byte chunk word that owns the byte (FP6: low plane)
     const size_t bb = gm.block_bytes();
     const size_t blk = t / bb;
     const int within = (int)(t % bb);
@@ -302,6 +345,18 @@ __global__ void k_unpack_codes(MatGeom gm, const uint8_t* __restrict__ dev, uint
         *reinterpret_cast<uint4*>(dst + t * 16) = *reinterpret_cast<const uint4*>(s);
         return;
     }
+    if (gm.quant == Q_FP6) {       // one code per byte: nibble of the low plane | crumb of the high plane
+        if (t >= (size_t)gm.N * gm.K) return;
+        const int n = (int)(t / gm.K), k = (int)(t % gm.K);
+        const int rb = n / kBlkN, r = n % kBlkN, kb = k / kBlkK, kl = k % kBlkK;
+        const int c = kl / 32, kc = kl % 32, w = kc / 8, ki = kc % 8;
+        const int p = ki / 2 + (ki % 2) * 4;
+        const uint8_t* base = dev + block_offset(gm, rb, kb);
+        const uint32_t lo = (base[((size_t)c * kBlkN + r) * 16 + w * 4 + p / 2] >> ((p % 2) * 4)) & 15u;
+        const uint32_t hi = (base[4096 + ((size_t)c * kBlkN + r) * 8 + w * 2 + p / 4] >> ((p % 4) * 2)) & 3u;
+        dst[t] = (uint8_t)(lo | (hi << 4));
+        return;
+    }
     const int per_byte = gm.quant == Q_INT2 ? 4 : (gm.quant == Q_FP8 ? 1 : 2);
     const int bpr = gm.K / per_byte;
     if (t >= (size_t)gm.N * bpr) return;
@@ -365,6 +420,9 @@ cudaError_t launch_quantize(int quant, const float* w, int N, int K, float g, vo
         const size_t warps = (size_t)(N / 4) * (K / kGroup);
         k_quantize_int2<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (__half*)scales,
                                                                      (uint8_t*)zeros);
+    } else if (quant == Q_FP6) {
+        const size_t warps = (size_t)N * (K / 128);
+        k_quantize_fp6<<<blocks_for(warps * 32, 256), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (__half*)scales);
     } else if (quant == Q_FP8) {
         k_quantize_fp8<<<(unsigned)((N / 128) * (K / 128)), 256, 0, st>>>(w, N, K, (uint8_t*)codes, (float*)scales);
     } else {
@@ -421,7 +479,7 @@ cudaError_t launch_unpack(const MatGeom& gm, const uint8_t* dev_codes, const uin
                           const uint8_t* dev_zeros, uint8_t* codes, uint8_t* scales, uint8_t* zeros,
                           cudaStream_t st) {
     const size_t nbytes = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K / 8
-                                             : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : (gm.quant == Q_FP8 ? 1 : 2));
+                                             : (size_t)gm.N * gm.K / (gm.quant == Q_INT2 ? 4 : ((gm.quant == Q_FP8 || gm.quant == Q_FP6) ? 1 : 2));
     k_unpack_codes<<<blocks_for(nbytes, 256), 256, 0, st>>>(gm, dev_codes, codes);
     if (gm.quant != Q_BF16) {
         const size_t n = gm.quant == Q_NVFP4 ? (size_t)gm.N * (gm.K / kFp4Blk)

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_STATE, MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(7)
-QUANT = {"int4": 0, "int2": 1, "nvfp4": 2, "bf16": 3, "int4g32": 4, "fp8": 5}
+QUANT = {"int4": 0, "int2": 1, "nvfp4": 2, "bf16": 3, "int4g32": 4, "fp8": 5, "fp6": 6}
 SHARED = -1
 
 
@@ -220,6 +220,9 @@ def quantize(quant, w, global_scale=0.0, stream=None):
     if quant in ("int4", "int4g32"):
         codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
         scales = torch.empty((N, K // (32 if quant == "int4g32" else 128)), dtype=torch.float16, device=dev)
+    elif quant == "fp6":
+        codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 32), dtype=torch.float16, device=dev)
     elif quant == "fp8":
         codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
         scales = torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev)

@@ -65,6 +65,12 @@ WORKLOADS = [
              routing="router", steps=100),
     Workload(8, "prefill-fp8-zipf", T=4096, H=2048, I=512, E=512, k=10, quant="fp8", shared=False,
              routing="zipf"),
+    # FP6 e2m3 experts with fp16 scales per 32 inputs (the FP6 card) on the
+    # same shapes
+    Workload(9, "decode-b1-fp6", T=1, H=2048, I=512, E=512, k=10, quant="fp6", shared=True,
+             routing="router", steps=100),
+    Workload(10, "prefill-fp6-zipf", T=4096, H=2048, I=512, E=512, k=10, quant="fp6", shared=False,
+             routing="zipf"),
 ]
 ZIPF_S = 1.1
 

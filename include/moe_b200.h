@@ -43,6 +43,9 @@
  *   INT4_G32  as INT4 with scales fp16 [N, K/32] (one scale per 32 inputs)
  *   FP8_B128  codes uint8 [N, K] E4M3FN; scales fp32 [N/128, K/128];
  *             s = amax_block / 448, q = e4m3(w / s); N and K multiples of 128
+ *   FP6_E2M3  codes uint8 [N, K], one e2m3 code per byte (bit 5 sign, bits
+ *             3-4 exponent with bias 1, bits 0-2 mantissa); scales fp16
+ *             [N, K/32]; s = fp16(amax/7.5), q = e2m3(w / s), saturating
  *   INT2  codes  uint8 [N, K/4]; element k = 4j + i at bits 2i..2i+1;
  *                u = clamp(rne(w/s) + z, 0, 3)
  *         scales fp16  [N, K/128]; s = fp16((max - min)/3), min <= 0 <= max
@@ -84,8 +87,10 @@ typedef enum {
     MOE_Q_BF16 = 3,            /* unquantized bf16 (shared expert) */
     MOE_Q_INT4_G32 = 4,        /* INT4 symmetric, group 32, fp16 scales (the MTP-draft experts of
                                   "Qwen3.8-Flash-Next on 2x RTX 3090", storage-format table) */
-    MOE_Q_FP8_B128 = 5         /* E4M3FN with one fp32 scale per 128x128 block (W8A16; the MTP-draft
+    MOE_Q_FP8_B128 = 5,        /* E4M3FN with one fp32 scale per 128x128 block (W8A16; the MTP-draft
                                   experts of "meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", Format) */
+    MOE_Q_FP6_E2M3 = 6         /* FP6 E2M3 with one fp16 scale per 32 inputs (W6A16; the routed experts
+                                  of "Qwen3.8-Flash-Next-FP6-INT8") */
 } moe_quant;
 
 #define MOE_SHARED_EXPERT (-1)

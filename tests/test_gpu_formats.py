@@ -24,7 +24,7 @@ def _weights(N, K, seed):
     return w
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
 @pytest.mark.parametrize("shape", [(128, 256), (512, 2048), (2048, 512), (132, 384)])
 def test_quantize_bit_exact(quant, shape):
     N, K = shape
@@ -49,6 +49,10 @@ def test_quantize_bit_exact(quant, shape):
         assert np.array_equal(codes.cpu().numpy(), rc)
         assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
         assert np.array_equal(zeros.cpu().numpy(), rz)
+    elif quant == "fp6":
+        rc, rs = O.quantize_fp6(w)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
     elif quant == "fp8":
         rc, rs = O.quantize_fp8_block(w)
         assert np.array_equal(codes.cpu().numpy(), rc)
@@ -98,7 +102,7 @@ def test_e2m1_conversion_around_every_midpoint():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
 def test_relayout_round_trip(quant):
     from bit_quantized_mixture_b200.layer import quantize_expert_gpu
     wl = synth.custom("tiny-int4", quant=quant, H=384, I=256, E=3, k=2, shared=True)

@@ -145,6 +145,7 @@ SMALL = {
     "int4": synth.custom("tiny-int4", H=384, I=256, E=16, k=4, shared=True),
     "int4g32": synth.custom("tiny-int4", quant="int4g32", H=384, I=256, E=16, k=4, shared=True),
     "fp8": synth.custom("tiny-int4", quant="fp8", H=384, I=256, E=16, k=4, shared=True),
+    "fp6": synth.custom("tiny-int4", quant="fp6", H=384, I=256, E=16, k=4, shared=True),
     "int2": synth.custom("tiny-int4", quant="int2", H=384, I=256, E=16, k=4, shared=True),
     "nvfp4": synth.custom("tiny-int4", quant="nvfp4", H=384, I=256, E=16, k=4, shared=True),
 }
@@ -156,7 +157,7 @@ def test_forward_tiny_workload():
     assert_close_output(y, y_ref)
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
 @pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 9])
 def test_forward_small_layers(quant, T):
     y, y_ref, _, _ = _forward_case(SMALL[quant], T)
@@ -248,12 +249,13 @@ MID = {
     "int4": synth.custom("tiny-int4", H=512, I=384, E=24, k=6, shared=True),
     "int4g32": synth.custom("tiny-int4", quant="int4g32", H=512, I=384, E=24, k=6, shared=True),
     "fp8": synth.custom("tiny-int4", quant="fp8", H=512, I=384, E=24, k=6, shared=True),
+    "fp6": synth.custom("tiny-int4", quant="fp6", H=512, I=384, E=24, k=6, shared=True),
     "int2": synth.custom("tiny-int4", quant="int2", H=512, I=384, E=24, k=6, shared=True),
     "nvfp4": synth.custom("tiny-int4", quant="nvfp4", H=512, I=384, E=24, k=6, shared=True),
 }
 
 
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
 @pytest.mark.parametrize("T", [5, 37, 300])
 def test_prefill_matches_oracle(quant, T):
     """T > 4 runs the permutation + tcgen05 grouped GEMMs: several 128-row
@@ -344,8 +346,12 @@ def test_prefill_zipf_fp8_full_size_sampled_tokens():
     _full_size_sampled("prefill-fp8-zipf", 8)
 
 
+def test_prefill_zipf_fp6_full_size_sampled_tokens():
+    _full_size_sampled("prefill-fp6-zipf", 8)
+
+
 # --------------------------------------------- whole layer in one call (fused)
-@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8"])
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
 @pytest.mark.parametrize("T", [1, 3, 8])
 def test_route_forward_matches_route_then_oracle(quant, T):
     """moe_route_forward (one cooperative kernel for T <= 8): ids/weights equal
@@ -418,7 +424,7 @@ def test_route_forward_paths(quant):
     layer.set_decode_path("auto")
 
 
-@pytest.mark.parametrize("wl_name", ["decode-b1-int4", "decode-b1-int4g32", "decode-b1-fp8"])
+@pytest.mark.parametrize("wl_name", ["decode-b1-int4", "decode-b1-int4g32", "decode-b1-fp8", "decode-b1-fp6"])
 def test_route_forward_decode_b1_full_size(wl_name):
     wl = synth.workload(wl_name)
     layer = get_layer(wl, 4)
