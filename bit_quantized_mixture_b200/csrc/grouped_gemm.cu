@@ -63,13 +63,11 @@ struct Cfg {
     // SC: stages of the packed-weight ring (routed), decoupled from the TMEM
     // slots so that the HBM reads of the codes run several stages ahead
     static constexpr int SC = SH ? 0 : 6;
-    // MMA-issuing warps: one per matrix (each stage gets NMAT commits). A
-    // split of the tiles over two issuers (TILE_SPLIT) is supported, but the
-    // down GEMM is bound by shared-memory bandwidth (the token operand read
-    // by the MMAs, the staged codes, the epilogue staging), where a second
-    // issuer only adds contention.
+    // MMA-issuing warps: one per matrix (each stage gets NMAT commits).  A
+    // second issuer taking alternate down tiles was measured slower: the
+    // down GEMM shares shared-memory bandwidth and issue slots between the
+    // MMA operand reads, the staged codes and the epilogue staging.
     static constexpr int MMA_WARPS = NMAT;
-    static constexpr bool TILE_SPLIT = MMA_WARPS > NMAT;
     // routed: a second producer warp loads the token operand, the first the
     // packed weights
     static constexpr int BPROD = kWarpMma + MMA_WARPS;
@@ -243,7 +241,7 @@ MOE_DEV void dequant_half(int quant, const uint8_t* codes, const uint8_t* scales
 }
 
 // bytes of the packed codes of one 128x64 block
-MOE_DEV int block_code_bytes(int quant) {
+__host__ __device__ constexpr int block_code_bytes(int quant) {
     return quant == Q_INT2 ? 2048 : (quant == Q_FP8 ? 8192 : (quant == Q_FP6 ? 6144 : 4096));
 }
 
@@ -299,6 +297,8 @@ MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 
 // named barrier of the epilogue warps
 MOE_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
+template <int NW>
+MOE_DEV void epi_sync_n() { asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory"); }
 
 // SwiGLU of one accumulator pair: silu(g) * u with the fast exponential and
 // division (relative error ~1e-6, far below the bf16 / e2m1 rounding of
@@ -427,7 +427,10 @@ MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = null
 }
 
 // ------------------------------------------------------------------ kernel
-template <int MODE, bool SH>
+// Q: the routed weights' format (a compile-time constant, so that each
+// instantiation holds only its own dequantization and ring geometry); the
+// shared-expert and router launches take Q_BF16.
+template <int MODE, bool SH, int Q>
 __global__ void __launch_bounds__(Cfg<MODE, SH>::THREADS, 1)
 k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUtensorMap map_a, GemmArgs a) {
     using C = Cfg<MODE, SH>;
@@ -486,18 +489,18 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // ------------------------------------------- producer: packed weights
         // the codes of KSTEP consecutive blocks are contiguous, and so are
         // their NVFP4 scales
-        const int KB = a.K / kBlkK, G = scale_stride(a.quant, a.K);
-        const bool fp8 = a.quant == Q_FP8;
-        const int cb = block_code_bytes(a.quant) * KSTEP;
+        const int KB = a.K / kBlkK, G = scale_stride(Q, a.K);
+        constexpr bool fp8 = Q == Q_FP8;
+        const int cb = block_code_bytes(Q) * KSTEP;
         // scales of a stage: NVFP4 KSTEP x 512 bytes; INT4/INT2 group 128 one
         // group (128 rows x fp16); INT4 group 32 the stage's 2 KSTEP groups;
         // FP8 the one block scale, stored by this thread
-        const bool g32 = a.quant == Q_INT4G32 || a.quant == Q_FP6;
-        const int sb = a.quant == Q_NVFP4 ? 512 * KSTEP : g32 ? 256 * 2 * KSTEP : fp8 ? 0 : 256;
-        const int zb = a.quant == Q_INT2 ? 128 : 0;
+        constexpr bool g32 = Q == Q_INT4G32 || Q == Q_FP6;
+        constexpr int sb = Q == Q_NVFP4 ? 512 * KSTEP : g32 ? 256 * 2 * KSTEP : fp8 ? 0 : 256;
+        constexpr int zb = Q == Q_INT2 ? 128 : 0;
         // FP8 and FP6 stages take more of the ring
-        const int stg_mat = fp8 ? KSTEP * 8192 + 16 : a.quant == Q_FP6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
-        const int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
+        constexpr int stg_mat = fp8 ? KSTEP * 8192 + 16 : Q == Q_FP6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
+        constexpr int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
         int g = 0;
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
@@ -517,9 +520,9 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     for (int m = 0; m < NMAT; ++m) {
                         const ExpertMat em = expert_matrix(m == 0 ? a.w0 : a.w1, t.expert);
                         uint8_t* d = stg + m * stg_mat;
-                        bulk_g2s(d, em.codes + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(a.quant), cb,
+                        bulk_g2s(d, em.codes + ((size_t)t.rb * KB + kb0) * (size_t)block_code_bytes(Q), cb,
                                  &cfull[c]);
-                        if (a.quant == Q_NVFP4) {
+                        if constexpr (Q == Q_NVFP4) {
                             bulk_g2s(d + cb, em.scales + ((size_t)t.rb * KB + kb0) * 512, sb, &cfull[c]);
                         } else if (!fp8) {
                             // first group of the stage (kb0 even: one group-128)
@@ -574,19 +577,15 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
     } else if (warp >= kWarpMma && warp < kWarpMma + C::MMA_WARPS) {
         // --------------------------------------------------------- MMA issue
         // warp kWarpMma + m issues the MMAs of matrix m (gate/up: two warps)
-        const int mi = C::TILE_SPLIT ? 0 : warp - kWarpMma;
-        int g = 0, local = 0;
+        const int mi = warp - kWarpMma;
+        int g = 0;
         AccSeq aseq;
-        for (int jt = 0; jt < nseq && !abort_flag; ++jt, ++local) {
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
-            const bool f16 = MODE == 0 && !SH && a.tok_scale != nullptr;
+            constexpr bool f16 = MODE == 0 && !SH && Q != Q_NVFP4;     // INT/FP8/FP6 gate/up: fp16 operands
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
             const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
-            if (C::TILE_SPLIT && (local & 1) != warp - kWarpMma) {   // the other warp's tile
-                g += NS;
-                continue;
-            }
             if ((au.mask & 1) && !warp_wait(&acc_empty[0], au.par0 ^ 1u, &abort_flag, a.err, 2)) break;
             if ((au.mask & 2) && !warp_wait(&acc_empty[1], au.par1 ^ 1u, &abort_flag, a.err, 2)) break;
             tc_fence_after();
@@ -595,10 +594,6 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
-                // with two issuers, one may reach stage g before the other has
-                // consumed stage g - S of the same slot: waiting for that
-                // commit first keeps the parity of full[s] unambiguous
-                if (C::TILE_SPLIT && !warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 7)) { ok = false; break; }
                 if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 3)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
@@ -637,12 +632,12 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const int wi = (warp - C::DEQ0) >> 2;
             const int m = wi % NMAT, j = wi / NMAT;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-            const bool f16 = MODE == 0 && a.tok_scale != nullptr;
-            const int cb = block_code_bytes(a.quant);
-            const bool fp8 = a.quant == Q_FP8, fp6 = a.quant == Q_FP6;
+            constexpr bool f16 = MODE == 0 && Q != Q_NVFP4;
+            constexpr int cb = block_code_bytes(Q);
+            constexpr bool fp8 = Q == Q_FP8, fp6 = Q == Q_FP6;
             // as the producer
-            const int stg_mat = fp8 ? KSTEP * 8192 + 16 : fp6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
-            const int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
+            constexpr int stg_mat = fp8 ? KSTEP * 8192 + 16 : fp6 ? KSTEP * 6144 + KSTEP * 512 : C::STG_MAT;
+            constexpr int SCr = stg_mat > C::STG_MAT ? (SC * C::STG_MAT) / stg_mat : SC;
             int g = 0;
             for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
                 bool ok = true;
@@ -664,12 +659,12 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     for (int h = 0; h < 2; ++h) {
                         // chunk h of block j: NVFP4 scales of the block, INT4 group
                         // 32 the chunk's own group, else the stage's one group
-                        const uint8_t* scj = a.quant == Q_NVFP4 ? sc + j * 512
-                                           : (a.quant == Q_INT4G32 || fp6) ? sc + (2 * j + h) * 256 : sc;
-                        if (fp8) dequant_half_fp8(stg + j * cb, *reinterpret_cast<const float*>(sc), r, h, f16, v);
-                        else if (fp6) dequant_half_fp6(stg + j * cb, scj, r, h, f16, v);
-                        else if (f16) dequant_half_f16(a.quant, stg + j * cb, scj, zr, r, h, v);
-                        else dequant_half(a.quant, stg + j * cb, scj, zr, r, h, v);
+                        const uint8_t* scj = Q == Q_NVFP4 ? sc + j * 512
+                                           : (Q == Q_INT4G32 || fp6) ? sc + (2 * j + h) * 256 : sc;
+                        if constexpr (fp8) dequant_half_fp8(stg + j * cb, *reinterpret_cast<const float*>(sc), r, h, f16, v);
+                        else if constexpr (fp6) dequant_half_fp6(stg + j * cb, scj, r, h, f16, v);
+                        else if constexpr (f16) dequant_half_f16(Q, stg + j * cb, scj, zr, r, h, v);
+                        else dequant_half(Q, stg + j * cb, scj, zr, r, h, v);
                         tmem_st16(tmem + lane_addr + C::A_COL0 + s * C::A_STAGE_COLS + (m * KSTEP + j) * 32 + 16 * h, v);
                     }
                     __syncwarp();
@@ -775,31 +770,33 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     }
                 }
             }
-            for (int c0 = cbeg; MODE == 0 && c0 < cend; c0 += 16) {
-                float v0[16];
-                if constexpr (MODE == 0) {
-                    float v1[16];
-                    tmem_ld16x2(lane_base + c0, lane_base + au.mat_stride + c0, v0, v1);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c0 + i;
-                        const float tsc = col < t.count ? ep_scale[col] : 0.0f;
-                        const float gg = v0[i] * tsc, uu = v1[i] * tsc;
-                        float act = swiglu_fast(gg, uu);
-                        if (!SH && a.quant == Q_NVFP4) {
-                            // W4A4: requantize the intermediate per 16 consecutive outputs
-                            float amax = fabsf(act);
-#pragma unroll
-                            for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                            const float gq = a.g_req;
-                            float sbv = 0.0f, rcp = 0.0f;
-                            if (gq != 0.0f) {
-                                sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, gq))));
-                                rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, gq));
+            if constexpr (MODE == 0) {
+                for (int c0 = cbeg; c0 < cend; c0 += 16) {
+                    float v0[16];
+                    if constexpr (MODE == 0) {
+                        float v1[16];
+                        tmem_ld16x2(lane_base + c0, lane_base + au.mat_stride + c0, v0, v1);
+    #pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = c0 + i;
+                            const float tsc = col < t.count ? ep_scale[col] : 0.0f;
+                            const float gg = v0[i] * tsc, uu = v1[i] * tsc;
+                            float act = swiglu_fast(gg, uu);
+                            if constexpr (!SH && Q == Q_NVFP4) {
+                                // W4A4: requantize the intermediate per 16 consecutive outputs
+                                float amax = fabsf(act);
+    #pragma unroll
+                                for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                                const float gq = a.g_req;
+                                float sbv = 0.0f, rcp = 0.0f;
+                                if (gq != 0.0f) {
+                                    sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, gq))));
+                                    rcp = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, gq));
+                                }
+                                act = e2m1_to_f32(f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu) * sbv;
                             }
-                            act = e2m1_to_f32(f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu) * sbv;
+                            out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
                         }
-                        out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
                     }
                 }
             }
@@ -1059,7 +1056,11 @@ struct Fp4Cfg {
     static constexpr int S = MODE == 0 ? 3 : 4;
     static constexpr int SF0 = kWarpMma + NMAT;                       // four scale-factor warps
     static constexpr int EPI0 = SF0 + 4;
-    static constexpr int THREADS = (EPI0 + kEpiWarps) * 32;
+    // epilogue warps: four (down: three) per TMEM lane quarter, each taking
+    // a part of the tile's token columns (the SwiGLU + requantization or the fp16
+    // staging of a tile is the longest step of these kernels)
+    static constexpr int EPI_WARPS = MODE == 0 ? 16 : 12;
+    static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
     static constexpr int ACC_BUFS = MODE == 0 ? 1 : 2;
     static constexpr int ACC_COLS = NMAT * kBN;
     static constexpr int SF_COL0 = ACC_BUFS * ACC_COLS;
@@ -1072,7 +1073,7 @@ struct Fp4Cfg {
     static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: [128][128] fp16
     static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : kOutTile;
     static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [16 tok][32] fp32
-    static constexpr int SCR_BYTES = MODE == 0 ? kEpiWarps * 16 * 32 * 4 : 0;
+    static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 16 * 32 * 4 : 0;
     static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
     static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
@@ -1111,7 +1112,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], NMAT);
-            mbar_init(&acc_empty[b], kEpiWarps);
+            mbar_init(&acc_empty[b], C::EPI_WARPS);
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -1226,7 +1227,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int ej = threadIdx.x - C::EPI0 * 32;
-        const int cset = (warp - C::EPI0) >> 2;              // this warp's half of the token columns
+        const int cset = (warp - C::EPI0) >> 2;              // this warp's quarter of the token columns
         uint8_t* out_s = smem + C::OUT;
         float nx_sc = 1.0f;                      // next tile's token info, loaded ahead
         int nx_row = 0;
@@ -1244,21 +1245,22 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
             const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
             const float gsc = a.g_w[t.expert] * a.g_act;
-            epi_sync();
+            epi_sync_n<C::EPI_WARPS>();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
                 ep_scale[ej] = nx_sc * gsc;
                 ep_row[ej] = nx_row;
             }
             fetch(jt + 1);
-            epi_sync();
+            epi_sync_n<C::EPI_WARPS>();
             if (ep_stop) break;
             if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 16)) continue;
             tc_fence_after();
             const int n_mma = (t.count + 15) & ~15;
-            // the two warps of a lane quarter split the columns (16-aligned)
-            const int chalf = (((n_mma >> 4) + 1) >> 1) << 4;
-            const int cbeg = cset ? chalf : 0, cend = cset ? n_mma : chalf;
+            // the warps of a lane quarter split the columns (16-aligned parts)
+            constexpr int NSET = C::EPI_WARPS / 4;
+            const int cpart = (((n_mma >> 4) + NSET - 1) / NSET) << 4;
+            const int cbeg = min(n_mma, cset * cpart), cend = min(n_mma, cbeg + cpart);
             const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS;
             if constexpr (MODE == 1) {
                 // all of this warp's columns (at most 64) in one batch
@@ -1321,11 +1323,11 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
-            epi_sync();
+            epi_sync_n<C::EPI_WARPS>();
             if constexpr (MODE == 0) {
                 // per token: 64 code bytes and 8 scale bytes of this 128-row block
                 const int I2 = a.out_ld / 2, I16 = a.out_ld / 16;
-                for (int i = ej; i < t.count * 5; i += kEpiWarps * 32) {
+                for (int i = ej; i < t.count * 5; i += C::EPI_WARPS * 32) {
                     const int col = i / 5, part = i % 5;
                     const size_t r = (size_t)ep_row[col];
                     if (part < 4)
@@ -1339,7 +1341,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 const uint16_t* o16 = reinterpret_cast<const uint16_t*>(out_s);
                 uint16_t* dst = reinterpret_cast<uint16_t*>(a.o16);
                 const int col0 = t.rb * kBlkN;
-                for (int i = ej; i < t.count * 16; i += kEpiWarps * 32) {
+                for (int i = ej; i < t.count * 16; i += C::EPI_WARPS * 32) {
                     const int col = i >> 4, ch = i & 15;
                     *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) =
                         *reinterpret_cast<const uint4*>(o16 + col * kBlkN + ch * 8);
@@ -1480,15 +1482,34 @@ static int num_sms() {
 
 // One persistent CTA per SM over the routed (SH = false) or the shared (SH =
 // true) tiles of the list.
+template <int MODE, bool SH, int Q>
+static cudaError_t launch_gemm_q(const BMaps& map_b, const GemmArgs& g, cudaStream_t st, const CUtensorMap* map_a,
+                                 int grid) {
+    constexpr int bytes = Cfg<MODE, SH>::ALLOC;
+    cudaError_t err =
+        cudaFuncSetAttribute(k_grouped_gemm<MODE, SH, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err != cudaSuccess) return err;
+    k_grouped_gemm<MODE, SH, Q><<<grid > 0 ? grid : num_sms(), Cfg<MODE, SH>::THREADS, bytes, st>>>(
+        map_b, map_a ? *map_a : map_b.m[0], g);
+    return cudaGetLastError();
+}
+
 template <int MODE, bool SH>
 static cudaError_t launch_gemm(const BMaps& map_b, const GemmArgs& g, cudaStream_t st,
                                const CUtensorMap* map_a = nullptr, int grid = 0) {
-    constexpr int bytes = Cfg<MODE, SH>::ALLOC;
-    cudaError_t err = cudaFuncSetAttribute(k_grouped_gemm<MODE, SH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (err != cudaSuccess) return err;
-    k_grouped_gemm<MODE, SH><<<grid > 0 ? grid : num_sms(), Cfg<MODE, SH>::THREADS, bytes, st>>>(
-        map_b, map_a ? *map_a : map_b.m[0], g);
-    return cudaGetLastError();
+    if constexpr (SH) {
+        return launch_gemm_q<MODE, true, Q_BF16>(map_b, g, st, map_a, grid);
+    } else {
+        switch (g.quant) {
+            case Q_INT4: return launch_gemm_q<MODE, false, Q_INT4>(map_b, g, st, map_a, grid);
+            case Q_INT4G32: return launch_gemm_q<MODE, false, Q_INT4G32>(map_b, g, st, map_a, grid);
+            case Q_INT2: return launch_gemm_q<MODE, false, Q_INT2>(map_b, g, st, map_a, grid);
+            case Q_NVFP4: return launch_gemm_q<MODE, false, Q_NVFP4>(map_b, g, st, map_a, grid);
+            case Q_FP8: return launch_gemm_q<MODE, false, Q_FP8>(map_b, g, st, map_a, grid);
+            case Q_FP6: return launch_gemm_q<MODE, false, Q_FP6>(map_b, g, st, map_a, grid);
+            default: return cudaErrorInvalidValue;
+        }
+    }
 }
 
 // Router logits on the tensor cores: logits[T, E] = x[T, H] . Wr[E, H]^T in

@@ -16,7 +16,6 @@ namespace moe {
 
 constexpr int kRouteMaxTSmall = 8;    // decode router: tokens staged in smem
 constexpr size_t kRouteMaxSmem = 160 * 1024;
-constexpr int kMaxK = 32;
 
 // Order-preserving key of an fp32 value (larger value -> larger key).
 MOE_DEV uint32_t order_key(float v) {
