@@ -86,7 +86,8 @@ MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __r
 }
 
 // Decode router (T <= 8): one warp per expert row, a grid-wide ticket lets
-// the last CTA to finish run the top-k of every token (no waiting).
+// the last CTA to finish run the top-k of every token (no waiting).  Asked
+// for logits only, the CTAs end after their logits.
 __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     extern __shared__ float xs[];          // [T][H] fp32
     __shared__ int s_last;
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
             }
         }
     }
+    if (!a.ids) return;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();                      // this CTA's logits before its ticket
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     }
     __syncthreads();
     if (!s_last) return;
-    for (int t = warp; a.ids && t < T; t += 4)
+    for (int t = warp; t < T; t += 4)
         warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, a.ids + (size_t)t * a.k, a.w + (size_t)t * a.k);
     __syncthreads();
     if (threadIdx.x == 0) *a.counter = 0u;      // ready for the next launch
