@@ -119,6 +119,17 @@ MOE_DEV uint4 ldg_stream_v4(const void* p) {   // read once: do not keep in L1
 MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 MOE_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Ticket of a grid-wide "last one finishes" pattern, taken by one thread
+// after a CTA barrier: the add releases this CTA's earlier writes (ordered
+// before it by the barrier) and acquires those released by the tickets
+// before it (visible to the CTA after the next barrier).  Returns the count
+// before the add.
+MOE_DEV unsigned ticket_acq_rel(unsigned* p) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
+
 // ------------------------------------------------ packed codes -> bf16x2
 // Exact conversions of two codes of a packed word into a bf16 pair (low
 // half = the first column), shared by the GEMV and the grouped GEMM.

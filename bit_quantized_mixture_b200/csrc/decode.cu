@@ -212,11 +212,7 @@ __global__ void __launch_bounds__(kDnThreads, 10) k_dec_down(DecodeArgs a) {
     }
     // the last item of this row block to finish combines
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();                      // this CTA's partials before its ticket
-        s_last = (atomicAdd(a.counters + hb, 1u) == (unsigned)items_per_rb - 1u);
-        if (s_last) __threadfence();
-    }
+    if (threadIdx.x == 0) s_last = (ticket_acq_rel(a.counters + hb) == (unsigned)items_per_rb - 1u);
     __syncthreads();
     if (!s_last) return;
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.y);

@@ -165,11 +165,7 @@ __global__ void __launch_bounds__(128) k_router_small(RouteArgs a) {
     }
     if (!a.ids) return;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();                      // this CTA's logits before its ticket
-        s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
-        if (s_last) __threadfence();
-    }
+    if (threadIdx.x == 0) s_last = (ticket_acq_rel(a.counter) == gridDim.x - 1);
     __syncthreads();
     if (!s_last) return;
     for (int t = warp; t < T; t += 4)
