@@ -573,11 +573,7 @@ __device__ __noinline__ void finish_block(unsigned int* counters, const float* p
                                           __nv_bfloat16* y, int H, int k, int T, int items, int hb, int group, int gtid,
                                           volatile int* last) {
     group_sync(group);
-    if (gtid == 0) {
-        __threadfence();
-        *last = (atomicAdd(counters + hb, 1u) == (unsigned)items - 1u);
-        if (*last) __threadfence();
-    }
+    if (gtid == 0) *last = (ticket_acq_rel(counters + hb) == (unsigned)items - 1u);
     group_sync(group);
     if (*last) {
         if (gtid < 16 * T) {
@@ -973,13 +969,12 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
             }
             group_sync(group);
         }
-        // tickets: one per unit, all in flight together
-        __threadfence();
+        // tickets: one per unit, all in flight together (each releases the
+        // group's partials, ordered before it by the barrier)
         group_sync(group);
         if (gtid < n_dn + n_sd) {
             const int hb = gtid < n_dn ? (dn_first + gtid * nslots) % RBH : sd_first + (gtid - n_dn) * nslots;
-            const bool last = atomicAdd(a.counters + hb, 1u) == (unsigned)items - 1u;
-            if (last) __threadfence();
+            const bool last = ticket_acq_rel(a.counters + hb) == (unsigned)items - 1u;
             u_last[group][gtid] = last ? hb : -1;
         }
         group_sync(group);
