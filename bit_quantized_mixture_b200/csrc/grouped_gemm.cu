@@ -170,16 +170,28 @@ MOE_DEV void dequant_half_f16(int quant, const uint8_t* codes, const uint8_t* sc
                               int h, uint32_t (&v)[16]) {
     const __half2 s2 = __half2half2(reinterpret_cast<const __half*>(scales)[r]);
     if (is_int4(quant)) {
+        // even nibbles j = 0, 2 at bits 0..3 give 1024 + u; odd ones j = 1, 3
+        // are masked in place at bits 4..7, giving 1024 + 16u, and take
+        // (1024 + 16u - 1152) * (s / 16): exact steps before the one rounding
+        // of (u - 8) * s, as for the even nibbles, while s / 16 is a normal
+        // fp16 (s >= 2^-10; below that s / 16 keeps one bit less)
         const __half2 off = __float2half2_rn(1032.0f);
+        const __half2 off16 = __float2half2_rn(1152.0f);
+        const __half2 s16 = __hmul2(s2, __float2half2_rn(0.0625f));                    // exact
         const uint4 q = *reinterpret_cast<const uint4*>(codes + (h * kBlkN + r) * 16);   // chunk h
         const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
+        for (int w = 0; w < 4; ++w) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t t = ((wv[w] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + u
-                v[4 * w + j] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&t), off), s2));
+            for (int jj = 0; jj < 2; ++jj) {
+                const uint32_t x = jj ? wv[w] >> 8 : wv[w];
+                const uint32_t te = (x & 0x000F000Fu) | 0x64006400u;                      // 1024 + u
+                const uint32_t to = (x & 0x00F000F0u) | 0x64006400u;                      // 1024 + 16u
+                v[4 * w + 2 * jj] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&te), off), s2));
+                v[4 * w + 2 * jj + 1] =
+                    h2_bits(__hmul2(__hsub2(*reinterpret_cast<const __half2*>(&to), off16), s16));
             }
+        }
     } else {
         const __half2 off = __float2half2_rn(1024.0f + (float)zeros[r]);
         const uint2 q = *reinterpret_cast<const uint2*>(codes + r * 16 + h * 8);          // words 2h, 2h+1
