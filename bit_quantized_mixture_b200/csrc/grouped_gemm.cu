@@ -840,9 +840,16 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
 // token tile, so that the token tiles of one weight block are consecutive;
 // the shared expert's tiles (all T tokens) come last.
 __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict__ counts,
-                                                      const int32_t* __restrict__ offsets, int E, int T, int RB,
-                                                      int has_shared, int grid, GemmTile* __restrict__ tiles,
-                                                      int2* __restrict__ groups, int* __restrict__ num_tiles) {
+                                                      const int32_t* __restrict__ offsets, int E, int T, int RB0,
+                                                      int RB1, int has_shared, int grid, GemmTile* __restrict__ tiles,
+                                                      int2* __restrict__ groups, int* __restrict__ num_tiles,
+                                                      size_t cap) {
+    // CTA b builds list b (row blocks RB0: gate/up, RB1: down) in its own
+    // part of the buffers, so both lists come from one launch
+    const int RB = blockIdx.x ? RB1 : RB0;
+    tiles += blockIdx.x * cap;
+    groups += blockIdx.x * cap;
+    num_tiles += 4 * blockIdx.x;
     __shared__ int sc[1024], sg[1024], s_cnt[1024], s_off[1024];
     const int e = threadIdx.x;
     const int cnt = (e < E) ? counts[e] : 0;
@@ -1580,8 +1587,8 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         !make_map_u8(&m[5], xs, (uint64_t)slots, H / 16, 16, kBN, false) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
-                                     p.groups, p.num_tiles);
+    k_build_tiles<<<2, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, H / kBlkN, has_sh ? 1 : 0, num_sms(),
+                                     p.tiles, p.groups, p.num_tiles, p.tile_cap);
     GemmArgs g{};
     g.quant = ex.quant;
     g.sh0 = ex.sh_gate;
@@ -1616,8 +1623,9 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     m[1] = m[0];
     m[3] = m[2];
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
-                                     p.groups, p.num_tiles);
+    g.tiles = p.tiles + p.tile_cap;          // the down list
+    g.groups = p.groups + p.tile_cap;
+    g.num_tiles = p.num_tiles + 4;
     g.sh0 = ex.sh_down;
     g.sh1 = nullptr;
     g.K = I;
@@ -1676,8 +1684,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (!make_bmaps(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, xdt) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
-                                     p.groups, p.num_tiles);
+    k_build_tiles<<<2, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, H / kBlkN, has_sh ? 1 : 0, num_sms(),
+                                     p.tiles, p.groups, p.num_tiles, p.tile_cap);
     GemmArgs g{};
     g.quant = ex.quant;
     g.w0 = ex.gate;
@@ -1709,8 +1717,9 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (!make_bmaps(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I) ||
         !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<1, 1024, 0, st>>>(p.counts, p.offsets, E, T, H / kBlkN, has_sh ? 1 : 0, num_sms(), p.tiles,
-                                     p.groups, p.num_tiles);
+    g.tiles = p.tiles + p.tile_cap;          // the down list
+    g.groups = p.groups + p.tile_cap;
+    g.num_tiles = p.num_tiles + 4;
     g.w0 = ex.down;
     g.w1 = ex.down;
     g.sh0 = ex.sh_down;

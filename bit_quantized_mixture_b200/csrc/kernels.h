@@ -108,9 +108,10 @@ struct PrefillArgs {
     void* y;                       // bf16 [T, H]
     int T;
     int32_t *counts, *offsets, *perm, *inv, *perm_scratch;
-    GemmTile* tiles;
-    int2* groups;                  // routed tile groups (same capacity as tiles)
-    int* num_tiles;                // 4 ints
+    GemmTile* tiles;               // two lists of tile_cap entries: gate/up, then down
+    int2* groups;                  // routed tile groups (same layout as tiles)
+    int* num_tiles;                // 4 ints per list
+    size_t tile_cap;               // entries per list (prefill_tile_capacity)
     __nv_bfloat16* xq;             // [T, H]: NVFP4 W4A4 activation values, else fp16 scaled x
     float* tok_scale;              // [T]: power of two of each token's fp16 activations
     __nv_bfloat16* xp;             // [T*k, H]: rows of xq in permuted (expert-major) order

@@ -50,6 +50,7 @@ struct moe_layer {
     GemmTile* tiles = nullptr;
     int* num_tiles = nullptr;
     int2* groups = nullptr;
+    size_t tile_cap = 0;
     int* dev_err = nullptr;
     // per-expert address table (moe_set_expert_table): device [E], in use when set
     const uint8_t** table = nullptr;
@@ -208,9 +209,12 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     const size_t o_perm = carve(sizeof(int32_t) * slots);
     const size_t o_inv = carve(sizeof(int32_t) * slots);
     const size_t o_pscr = carve(sizeof(int32_t) * permute_scratch_ints((int)slots, E));
-    const size_t o_tiles = carve(sizeof(GemmTile) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
-    const size_t o_groups = carve(sizeof(int2) * prefill_tile_capacity(c.max_tokens, k, E, H, I));
-    const size_t o_ntiles = carve(4 * sizeof(int));   // routed tiles, all tiles, routed groups, group order
+    // two tile lists (gate/up, down), each with its group list and four counts:
+    // routed tiles, all tiles, routed groups, group order
+    const size_t tile_cap = prefill_tile_capacity(c.max_tokens, k, E, H, I);
+    const size_t o_tiles = carve(sizeof(GemmTile) * 2 * tile_cap);
+    const size_t o_groups = carve(sizeof(int2) * 2 * tile_cap);
+    const size_t o_ntiles = carve(8 * sizeof(int));
     const size_t o_err = carve(sizeof(int));
     const size_t o_table = carve(sizeof(void*) * (size_t)E);
     const size_t o_gtab = carve(sizeof(float) * 2 * (size_t)E);
@@ -246,6 +250,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->inv = reinterpret_cast<int32_t*>(h->ws + o_inv);
     h->perm_scratch = reinterpret_cast<int32_t*>(h->ws + o_pscr);
     h->tiles = reinterpret_cast<GemmTile*>(h->ws + o_tiles);
+    h->tile_cap = tile_cap;
     h->num_tiles = reinterpret_cast<int*>(h->ws + o_ntiles);
     h->groups = reinterpret_cast<int2*>(h->ws + o_groups);
     h->dev_err = reinterpret_cast<int*>(h->ws + o_err);
@@ -529,7 +534,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.x = x; p.ids = topk_ids; p.w = topk_w; p.y = y; p.T = T;
         p.counts = h->counts; p.offsets = h->offsets; p.perm = h->perm; p.inv = h->inv;
         p.perm_scratch = h->perm_scratch;
-        p.tiles = h->tiles; p.groups = h->groups; p.num_tiles = h->num_tiles;
+        p.tiles = h->tiles; p.groups = h->groups; p.num_tiles = h->num_tiles; p.tile_cap = h->tile_cap;
         p.xq = h->xq; p.tok_scale = h->tok_scale; p.xp = h->xp; p.w_perm = h->w_perm; p.ts_perm = h->ts_perm;
         p.a_perm = h->a_perm; p.a_sh = h->a_sh; p.o = h->o; p.o_sh = h->o_sh;
         p.err = h->dev_err;
