@@ -524,6 +524,10 @@ def run_decode(args, wl, dev, rank, world):
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "dominant": dom,
+        "e2e_method": ("one CUDA graph per step, steps serial: " +
+                       ("a copy kernel reads x from mapped pinned host memory, the layer writes y into mapped "
+                        "pinned host memory" if e2e_method == "mapped" else
+                        "cudaMemcpyAsync of x from and of y to pinned host memory around the layer call")),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes_per_launch": by[dom], "peak_source": peak_kind,
@@ -739,6 +743,8 @@ def run_prefill(args, wl, dev, rank, world):
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
         "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
+        "e2e_method": ("chunks pipelined: inputs copied in and outputs copied out on two copy streams while the "
+                       "previous chunk computes; first input copy to last output copy"),
         # router GEMM, top-k, 3 permutation, 1 activation pass, 1 launch for
         # both tile lists, 2 routed GEMMs (+2 shared), combine
         "launches_per_step": 10 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
@@ -800,10 +806,7 @@ def bench_line(args, wl, r, world, prefill):
         "roofline": r["roofline"],
         "kernels_ms": r["kernels_ms"],
         "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "method": ("chunks pipelined: inputs copied in and outputs copied out on two copy streams while the "
-                           "previous chunk computes; first input copy to last output copy" if prefill else
-                           "one CUDA graph per step: copy of x from pinned host memory, the layer call, copy of y "
-                           "to pinned host memory; steps serial")},
+                "method": r.get("e2e_method", "")},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
