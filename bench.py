@@ -76,7 +76,9 @@ class ClockSampler:
         self.path = None
 
     def __enter__(self):
-        out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None
+        # samples go to a file named by BENCH_CLOCKS_DIR when set (to keep
+        # the raw record), else to a temporary file
+        out_dir = os.environ.get("BENCH_CLOCKS_DIR") or None
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv", dir=out_dir)
         os.close(fd)
         try:
