@@ -73,7 +73,7 @@ typedef struct CUstream_st* moe_stream_t;   /* same type as cudaStream_t */
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or index */
-    MOE_ERR_UNSUPPORTED = 2,   /* shape or format this build does not handle */
+    MOE_ERR_UNSUPPORTED = 2,   /* shape or format the library does not handle */
     MOE_ERR_STATE = 3,         /* e.g. forward before the weights are loaded */
     MOE_ERR_OOM = 4,           /* device allocation failed in moe_create     */
     MOE_ERR_CUDA = 5,          /* a CUDA call or launch failed               */
