@@ -63,3 +63,29 @@ def test_two_replicas_max_time_and_whole_job_value(tmp_path):
         assert int(n) == 2 and par == "replicas x2"
         assert scaling == "weak"
         assert float(ms) == pytest.approx(15.0 / 100)
+
+
+@pytest.mark.parametrize("name,prefill", [("decode-b1-int4", False), ("prefill-int4-zipf", True)])
+def test_bench_line_carries_the_contract_keys(name, prefill):
+    """One JSON line with every key the measurement contract names, the
+    roofline object's fields and the end-to-end object with its byte counts."""
+    wl = synth.workload(name)
+    args = types.SimpleNamespace(steps=20, warmup=3, flush_mb=512, expert_table=False)
+    roof = {"bound": "hbm", "achieved": 1000.0, "peak": 6538.6, "unit": "GB/s", "frac": 1000.0 / 6538.6,
+            "traffic": None}
+    r = {"steps_tokens": 20 * wl.T, "total_ms": 2.0, "e2e_ms": 3.0, "roofline": roof, "kernels_ms": {"k": 0.1},
+         "h2d": wl.T * wl.H * 2, "d2h": wl.T * wl.H * 2, "launches_per_step": 3,
+         "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, "e2e_method": "m"}
+    line = bench.bench_line(args, wl, r, 1, prefill=prefill)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["config"]["workload"] == name
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in line["roofline"], key
+    e2e = line["e2e"]
+    assert e2e["unit"] == line["unit"] and e2e["value"] == pytest.approx(20 * wl.T / 3.0e-3)
+    assert e2e["h2d_bytes_per_step"] == wl.T * wl.H * 2 and e2e["d2h_bytes_per_step"] == wl.T * wl.H * 2
+    assert line["value"] == pytest.approx(20 * wl.T / 2.0e-3)
+    assert line["gpu_launches"] == 3 * 20
+    assert line["higher_is_better"] is True and line["data"] == "synthetic"
