@@ -142,6 +142,25 @@ def test_tiny_layer_brute_force():
     assert rel < 1e-12
 
 
+_E2M1_GRID = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+
+def _brute_nvfp4(codes, sb, g):
+    """Python decode of packed E2M1 codes (low nibble first) with E4M3 scales
+    per 16 values and the fp32 global scale g, as lists of floats."""
+    N, Kh = codes.shape
+    out = []
+    for n in range(N):
+        row = []
+        for j in range(Kh):
+            for nib in (int(codes[n, j]) & 15, int(codes[n, j]) >> 4):
+                row.append(_E2M1_GRID[nib & 7] * (-1 if nib & 8 else 1))
+        sc = [((1 + (s & 7) / 8) * 2.0 ** (((s >> 3) & 15) - 7)) if (s >> 3) & 15 else (s & 7) / 8 * 2.0 ** -6
+              for s in (int(v) for v in sb[n])]
+        out.append([row[k] * sc[k // 16] * float(g) for k in range(len(row))])
+    return out
+
+
 def test_tiny_nvfp4_layer_brute_force():
     wl = synth.custom(TINY, quant="nvfp4", E=4, k=2, T=3)
     ews = _quantized_experts(wl, "nvfp4")
@@ -151,22 +170,7 @@ def test_tiny_nvfp4_layer_brute_force():
     ids, w = O.route_topk(O.router_logits(x_bits, synth.router_bf16(wl)), wl.k)
     fn = _expert_fn(ews, "nvfp4")
     g_a = O.nvfp4_global_scale(O.intermediate_amax(x_bits, ids, "nvfp4", fn, g_x))
-    grid = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
-
-    def dq(codes, sb, g):   # python decode of packed E2M1 + E4M3
-        N, Kh = codes.shape
-        out = []
-        for n in range(N):
-            row = []
-            for j in range(Kh):
-                for nib in (int(codes[n, j]) & 15, int(codes[n, j]) >> 4):
-                    v = grid[nib & 7] * (-1 if nib & 8 else 1)
-                    row.append(v)
-            b = [int(s) for s in sb[n]]
-            sc = [((1 + (s & 7) / 8) * 2.0 ** (((s >> 3) & 15) - 7)) if (s >> 3) & 15 else (s & 7) / 8 * 2.0 ** -6
-                  for s in b]
-            out.append([row[k] * sc[k // 16] * float(g) for k in range(len(row))])
-        return out
+    dq = _brute_nvfp4
 
     xc, xs = O.quantize_nvfp4(Xf, g_x)
     Xq = dq(xc, xs, g_x)
@@ -185,6 +189,42 @@ def test_tiny_nvfp4_layer_brute_force():
                 y_ref[t, h] += w[t, j] * _dot(aq, Wd[h])
     y = O.moe_forward(x_bits, ids, w, "nvfp4", fn, act_scales=(g_x, g_a))
     assert np.sqrt(np.mean((y - y_ref) ** 2) / np.mean(y_ref ** 2)) < 1e-9
+
+
+@pytest.mark.parametrize("quant", ["int4", "nvfp4"])
+def test_intermediate_amax_brute_force(quant):
+    """The calibration amax of the SwiGLU intermediate is the largest |a| over
+    every routed slot, here with experts repeated across tokens; a computed by
+    Python loops over the decoded weights (and, for NVFP4, the decoded
+    quantized activations)."""
+    wl = synth.custom(TINY, quant=quant, E=4, k=2, T=4)
+    ews = _quantized_experts(wl, quant)
+    x_bits = synth.activations_bf16(wl)
+    ids = np.array([[0, 1], [1, 2], [3, 0], [1, 3]], dtype=np.int32)
+    g_x = None
+    if quant == "nvfp4":
+        Xf = O.bf16_bits_to_f32(x_bits)
+        g_x = O.nvfp4_global_scale(np.abs(Xf).max())
+        xc, xs = O.quantize_nvfp4(Xf, g_x)
+        X = _brute_nvfp4(xc, xs, g_x)
+        W = {e: [_brute_nvfp4(ews[e][m]["codes"], ews[e][m]["scales"], ews[e][m]["g"]) for m in ("gate", "up")]
+             for e in range(wl.E)}
+    else:
+        X = _brute_bf16(x_bits)
+        W = {e: [_brute_unpack_int4(ews[e][m]["codes"], ews[e][m]["scales"]) for m in ("gate", "up")]
+             for e in range(wl.E)}
+    amax = 0.0
+    for t in range(wl.T):
+        for j in range(wl.k):
+            Wg, Wu = W[int(ids[t, j])]
+            for n in range(wl.I):
+                g = _dot(X[t], Wg[n])
+                amax = max(amax, abs(g / (1.0 + math.exp(-g)) * _dot(X[t], Wu[n])))
+    got = O.intermediate_amax(x_bits, ids, quant, _expert_fn(ews, quant), g_x)
+    assert got == pytest.approx(amax, rel=1e-12)
+    # fewer tokens cannot raise it (up to the summation order of a different batch)
+    got_sub = O.intermediate_amax(x_bits[:2], ids[:2], quant, _expert_fn(ews, quant), g_x)
+    assert got_sub <= got * (1 + 1e-12)
 
 
 # --------------------------------------------------- special cases ----
