@@ -23,7 +23,11 @@
  * Conventions for every entry point
  *   - Pointers named *_dev are device pointers of the handle's device.
  *     Pointers named *_any may be host or device memory (copied with
- *     cudaMemcpyDefault).  All other data pointers are device pointers.
+ *     cudaMemcpyDefault).  All other data pointers are device pointers; the
+ *     device address of mapped pinned host memory (cudaHostAllocMapped,
+ *     cudaHostGetDevicePointer) is one too, and the kernels then read or
+ *     write host memory across the bus (worth it for the few kilobytes of a
+ *     decode step's y, not for operands that many CTAs read).
  *   - All calls are asynchronous on the given stream unless stated.
  *     Argument and state errors are detected on the host before any work is
  *     enqueued and return without side effects.  A failed launch returns
