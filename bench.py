@@ -260,9 +260,9 @@ def expert_bytes(wl):
     elif wl.quant == "fp6":
         gu = 2 * (I * H * 3 // 4 + I * (H // 32) * 2)
         dn = H * I * 3 // 4 + H * (I // 32) * 2
-    elif wl.quant == "int2":
-        gu = 2 * (I * H // 4 + I * (H // 128) * 2 + I * (H // 128))
-        dn = H * I // 4 + H * (I // 128) * 2 + H * (I // 128)
+    elif wl.quant == "int2":      # 2-bit zeros, four per byte (the algorithmic minimum)
+        gu = 2 * (I * H // 4 + I * (H // 128) * 2 + (I // 4) * (H // 128))
+        dn = H * I // 4 + H * (I // 128) * 2 + (H // 4) * (I // 128)
     else:
         gu = 2 * (I * H // 2 + I * (H // 16))
         dn = H * I // 2 + H * (I // 16)
