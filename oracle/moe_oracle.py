@@ -406,18 +406,24 @@ def permute(ids, num_experts):
     """Expert-major order of the flat slots s = t*k + j, stable in s.
 
     Returns counts[E], offsets[E+1], perm[T*k] (slot id at each permuted
-    position) and inv[T*k] (permuted position of each slot)."""
+    position) and inv[T*k] (permuted position of each slot).  A slot whose
+    id lies outside [0, E) selects no expert: it is left out of the order
+    and its inv entry is -1; perm then has only offsets[E] meaningful
+    entries (the rest are -1)."""
     flat = np.asarray(ids, dtype=np.int64).reshape(-1)
-    counts = np.bincount(flat, minlength=num_experts).astype(np.int32)
+    valid = (flat >= 0) & (flat < num_experts)
+    counts = np.bincount(flat[valid], minlength=num_experts).astype(np.int32)
     offsets = np.zeros(num_experts + 1, dtype=np.int32)
     offsets[1:] = np.cumsum(counts)
     fill = offsets[:-1].astype(np.int64).copy()
-    perm = np.empty(flat.size, dtype=np.int32)
+    perm = np.full(flat.size, -1, dtype=np.int32)
+    inv = np.full(flat.size, -1, dtype=np.int32)
     for s, e in enumerate(flat):
+        if not valid[s]:
+            continue
         perm[fill[e]] = s
+        inv[s] = fill[e]
         fill[e] += 1
-    inv = np.empty_like(perm)
-    inv[perm] = np.arange(flat.size, dtype=np.int32)
     return counts, offsets, perm, inv
 
 
@@ -460,11 +466,13 @@ def dequantize_expert(quant, ew):
     return tuple(out)
 
 
-def moe_forward(x_bits, ids, w, quant, expert_fn, shared=None, act_scales=None):
+def moe_forward(x_bits, ids, w, quant, expert_fn, shared=None, act_scales=None, num_experts=None):
     """MoE layer output y [T, H] in fp64.
 
     x_bits     bf16 bit patterns [T, H]
-    ids, w     routing [T, k] (expert ids, weights)
+    ids, w     routing [T, k] (expert ids, weights); with num_experts given,
+               a slot whose id lies outside [0, num_experts) selects no
+               expert and contributes zero
     expert_fn  e -> fp64 (W_gate [I,H], W_up [I,H], W_down [H,I])
     shared     None or fp64 (W_gate, W_up, W_down) of the always-on expert
     act_scales (g_x, g_a) static global scales for NVFP4 activations and
@@ -480,6 +488,8 @@ def moe_forward(x_bits, ids, w, quant, expert_fn, shared=None, act_scales=None):
         Xq = X
     y = np.zeros((T, H), dtype=np.float64)
     for e in np.unique(ids):
+        if num_experts is not None and not 0 <= e < num_experts:
+            continue
         tok, slot = np.nonzero(ids == e)
         Wg, Wu, Wd = expert_fn(int(e))
         A = swiglu_intermediate(Xq[tok], Wg, Wu)

@@ -83,6 +83,29 @@ def test_permutation_matches_sorted():
     assert np.array_equal(perm[inv], np.arange(flat.size))
 
 
+def test_permutation_drops_out_of_range_ids():
+    """Slots whose id lies outside [0, E) take no position: brute force over
+    the valid slots, sorted by (expert, slot)."""
+    rng = np.random.default_rng(8)
+    E = 12
+    ids = np.stack([rng.choice(E, 4, replace=False) for _ in range(40)]).astype(np.int32)
+    flat = ids.reshape(-1).copy()
+    bad = rng.choice(flat.size, 23, replace=False)
+    flat[bad[:8]] = -1
+    flat[bad[8:16]] = E
+    flat[bad[16:]] = 1000
+    ids = flat.reshape(ids.shape)
+    counts, offsets, perm, inv = O.permute(ids, E)
+    good = [s for s in range(flat.size) if 0 <= flat[s] < E]
+    ref = sorted(good, key=lambda s: (flat[s], s))
+    n = len(ref)
+    assert n == flat.size - 23
+    assert list(perm[:n]) == ref and np.all(perm[n:] == -1)
+    assert offsets[-1] == n and list(counts) == [int((flat == e).sum()) for e in range(E)]
+    for s in range(flat.size):
+        assert inv[s] == (ref.index(s) if s in ref else -1)
+
+
 # ---------------------------------------------------- brute force tiny ----
 
 def _brute_unpack_int4(codes, scales):
@@ -322,3 +345,28 @@ def test_shared_expert_is_added_with_weight_one():
     X = torch.from_numpy(O.bf16_bits_to_f64(x_bits))
     ref = _torch_mlp(X, *(torch.from_numpy(m) for m in sh)).numpy()
     assert np.allclose(ys - y, ref, rtol=1e-10, atol=1e-13)
+
+
+def test_out_of_range_ids_contribute_zero():
+    """With num_experts given, a slot whose id lies outside [0, E) adds
+    nothing: the result equals the same routing with that slot's weight set
+    to zero (the slot then pointing at a valid expert), computed by the plain
+    Python-loop reference."""
+    wl = synth.custom(TINY, T=7)
+    ews = _quantized_experts(wl, "int4")
+    fn = _expert_fn(ews, "int4")
+    x_bits = synth.activations_bf16(wl)
+    ids, w = O.route_topk(O.router_logits(x_bits, synth.router_bf16(wl)), wl.k)
+    bad = ids.copy()
+    bad[0, 1], bad[3, 0], bad[6, 1] = -1, wl.E, 10 ** 6
+    y = O.moe_forward(x_bits, bad, w, "int4", fn, num_experts=wl.E)
+    w0 = w.copy()
+    w0[0, 1] = w0[3, 0] = w0[6, 1] = 0.0
+    X = O.bf16_bits_to_f64(x_bits)
+    ref = np.zeros_like(y)
+    for t in range(wl.T):
+        for j in range(wl.k):
+            Wg, Wu, Wd = fn(int(ids[t, j]))
+            ref[t] += w0[t, j] * (O.silu(X[t] @ Wg.T) * (X[t] @ Wu.T)) @ Wd.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+    assert not np.allclose(y[0], O.moe_forward(x_bits, ids, w, "int4", fn)[0])
