@@ -361,3 +361,21 @@ def test_nvfp4_error_bound_random():
     # the block scale maps the block amax near the top of the E2M1 range
     ratio = amax_b / (O.e4m3_decode(sb) * float(gs))
     assert np.all((ratio > 6 / 1.07) & (ratio < 6 * 1.07))
+
+
+def test_output_tolerance_discounts_only_the_bf16_rounding():
+    """The comparison helper of the GPU tests: the exact result rounded to
+    bf16 always passes, whatever its magnitude; one bf16 ulp more than that
+    at an output of 9 x RMS fails."""
+    import torch
+    from tests.gpu_util import assert_close_output, bf16_rounding_error
+    rng = np.random.default_rng(3)
+    y = rng.standard_normal((64, 256))
+    y[5, 7] = 9.0 * np.sqrt(np.mean(y ** 2)) * 1.0009765625        # a large output just above a bf16 binade start
+    bits = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert_close_output(bits, y)
+    assert bf16_rounding_error(y).max() > 0
+    bad = bits.copy()
+    bad[5, 7] += 4                                   # four ulps off at 9 x RMS: about 7 % of the RMS
+    with pytest.raises(AssertionError):
+        assert_close_output(bad, y)
