@@ -100,6 +100,40 @@ MOE_DEV float e2m1_to_f32(uint32_t c) {
     return (c & 8u) ? -m : m;
 }
 
+// ------------------------------------------------------ NVFP4 block of 16
+// The one NVFP4 quantizer of the library ("meshapplied/Qwen3.8-Flash-Next-
+// NVFP4-Latest", section "Format": E2M1 values with one E4M3 scale per 16):
+// with the fp32 global scale g, the scale code is e4m3(amax / (6 g)) and the
+// codes are e2m1(v * r) with r = 1 / (s_b g), every decision in fp32 with
+// IEEE division.  A block whose scale decodes to zero has r = 0, so its codes
+// are signed zeros (0x8 for negative inputs, as an IEEE conversion gives);
+// g == 0 gives scale code 0 and all-zero codes.  Returns the scale code;
+// w[0] holds elements 0..7 and w[1] elements 8..15, element 2i in the low
+// nibble of byte i.  The weight quantizer, the activation quantizers of the
+// prefill and decode paths and the W4A4 value staging all call this.
+MOE_DEV uint32_t nvfp4_quant_block16(const float (&v)[16], float g, uint32_t (&w)[2]) {
+    w[0] = w[1] = 0u;
+    if (g == 0.0f) return 0u;
+    float amax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+    const uint32_t sbc = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+    const float sbv = e4m3_to_f32(sbc);
+    const float r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], r), __fmul_rn(v[2 * q + 1], r)) << (8 * (q & 3));
+    return sbc;
+}
+// The values q * s_b of the block quantized as above (the global scale g is
+// left to the caller), in place.
+MOE_DEV void nvfp4_block16_values(float (&v)[16], float g) {
+    uint32_t w[2];
+    const float sbv = e4m3_to_f32(nvfp4_quant_block16(v, g, w));
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[q] = e2m1_to_f32((w[q >> 3] >> (4 * (q & 7))) & 0xFu) * sbv;
+}
+
 // ------------------------------------------------------------ memory access
 MOE_DEV uint4 ldg_nc_v4(const void* p) {
     uint4 r;

@@ -302,23 +302,8 @@ MOE_DEV void warp_rows(float (&acc)[NM][4], const MatPtr (&mats)[NM], int nb, in
 }
 
 // W4A4: the value q * s_b of a 16-element block (the global scale g is left
-// to the epilogue), with the recipe of the activation quantization kernel.
-MOE_DEV void fp4_block_values(float (&v)[16], float g) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-    float sbv = 0.0f, r = 0.0f;
-    if (g != 0.0f) {
-        sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g))));
-        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
-    }
-#pragma unroll
-    for (int q = 0; q < 16; q += 2) {
-        const uint32_t cc = f32x2_to_e2m1(__fmul_rn(v[q], r), __fmul_rn(v[q + 1], r));
-        v[q] = e2m1_to_f32(cc & 0xFu) * sbv;
-        v[q + 1] = e2m1_to_f32(cc >> 4) * sbv;
-    }
-}
+// to the epilogue), from the library's one NVFP4 block quantizer.
+MOE_DEV void fp4_block_values(float (&v)[16], float g) { nvfp4_block16_values(v, g); }
 
 // Stage rows (row_of[t], t < m) of a bf16 matrix [*, K] into smem rows of
 // ldx elements; rows m..7 are zero.  16-byte accesses, loads issued first.

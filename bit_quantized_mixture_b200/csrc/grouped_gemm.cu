@@ -595,7 +595,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
-            constexpr bool f16 = MODE == 0 && !SH && Q != Q_NVFP4;     // INT/FP8/FP6 gate/up: fp16 operands
+            // INT/FP8/FP6 routed tiles, gate/up and down: fp16 operands
+            constexpr bool f16 = MODE != 2 && !SH && Q != Q_NVFP4;
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
             const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
             if ((au.mask & 1) && !warp_wait(&acc_empty[0], au.par0 ^ 1u, &abort_flag, a.err, 2)) break;
@@ -644,7 +645,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const int wi = (warp - C::DEQ0) >> 2;
             const int m = wi % NMAT, j = wi / NMAT;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-            constexpr bool f16 = MODE == 0 && Q != Q_NVFP4;
+            constexpr bool f16 = Q != Q_NVFP4;
             constexpr int cb = block_code_bytes(Q);
             constexpr bool fp8 = Q == Q_FP8, fp6 = Q == Q_FP6;
             // as the producer
@@ -807,7 +808,13 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                                 }
                                 act = e2m1_to_f32(f32x2_to_e2m1(__fmul_rn(act, rcp), 0.0f) & 0xFu) * sbv;
                             }
-                            out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
+                            // the routed INT/FP8/FP6 intermediate is the fp16 B operand
+                            // of the down GEMM (saturating at +-65504); the shared expert's
+                            // and the W4A4 values stay bf16
+                            if constexpr (!SH && Q != Q_NVFP4)
+                                out_s[col * kBlkN + row] = __half_as_ushort(f16_sat(act));
+                            else
+                                out_s[col * kBlkN + row] = __bfloat16_as_ushort(__float2bfloat16_rn(act));
                         }
                     }
                 }
@@ -926,18 +933,21 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
 }
 
 // --------------------------------------------------------------- combine
-// y[t] = sum_{j<k} O[t*k + j] + S[t], fp32 sum in fixed j order, one bf16 rounding.
+// y[t] = sum_{j<k} O[t*k + j] + S[t], fp32 sum in fixed j order, one bf16
+// rounding.  A slot without a position (id outside [0, E): inv < 0) has no
+// expert output and contributes zero.
 MOE_DEV float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 MOE_DEV float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
-__global__ void k_combine(const __half* __restrict__ O, const __half* __restrict__ S, int T, int H, int k,
-                          __nv_bfloat16* __restrict__ y) {
+__global__ void k_combine(const __half* __restrict__ O, const __half* __restrict__ S, const int32_t* __restrict__ inv,
+                          int T, int H, int k, __nv_bfloat16* __restrict__ y) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one thread per 8 columns
     const int per_row = H / 8;
     if (i >= (long long)T * per_row) return;
     const int t = (int)(i / per_row), c = (int)(i % per_row) * 8;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
+        if (__ldg(inv + (size_t)t * k + j) < 0) continue;
         const uint4 q = *reinterpret_cast<const uint4*>(O + ((size_t)t * k + j) * H + c);
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -1034,20 +1044,12 @@ __global__ void k_act_fp4_values(const __nv_bfloat16* __restrict__ x, int T, int
     if (t >= (long long)T * nblk) return;
     const __nv_bfloat16* src = x + (size_t)t * kFp4Blk;
     float v[16];
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) { v[i] = __bfloat162float(src[i]); amax = fmaxf(amax, fabsf(v[i])); }
-    float sbv = 0.0f, r = 0.0f;
-    if (g != 0.0f) {
-        sbv = e4m3_to_f32(f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g))));
-        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __bfloat162float(src[i]);
+    nvfp4_block16_values(v, g);
     uint32_t o[8];
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const uint32_t c = f32x2_to_e2m1(__fmul_rn(v[i], r), __fmul_rn(v[i + 1], r));
-        o[i / 2] = pack_bf16x2(e2m1_to_f32(c & 0xFu) * sbv, e2m1_to_f32(c >> 4) * sbv);
-    }
+    for (int i = 0; i < 16; i += 2) o[i / 2] = pack_bf16x2(v[i], v[i + 1]);
     uint4* d = reinterpret_cast<uint4*>(xq + (size_t)t * kFp4Blk);
     d[0] = make_uint4(o[0], o[1], o[2], o[3]);
     d[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -1281,11 +1283,18 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             const int cpart = (((n_mma >> 4) + NSET - 1) / NSET) << 4;
             const int cbeg = min(n_mma, cset * cpart), cend = min(n_mma, cbeg + cpart);
             const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS;
+            const int nch = (cend - cbeg) >> 4;
+            // Every warp first copies its accumulator columns into registers
+            // and releases the accumulator, so that the MMAs of the next tile
+            // start while this tile's SwiGLU / requantization or fp16
+            // conversion runs.
             if constexpr (MODE == 1) {
-                // all of this warp's columns (at most 64) in one batch
+                static_assert(C::EPI_WARPS / 4 >= 2, "down: at most 64 columns per warp");
                 uint32_t r[64];
-                const int nch = (cend - cbeg) >> 4;
                 tmem_ld_chunks(lane_base + cbeg, nch, r);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (q < nch) {
@@ -1298,50 +1307,65 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                         }
                     }
                 }
-            }
-            for (int c0 = cbeg; MODE == 0 && c0 < cend; c0 += 16) {
-                float v0[16];
-                if constexpr (MODE == 0) {
-                    float v1[16];
-                    tmem_ld16x2(lane_base + c0, lane_base + kBN + c0, v0, v1);
-                    // SwiGLU of 16 tokens x this warp's 32 outputs into the warp's scratch
-                    float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 16 * 32;
+            } else {
+                static_assert(C::EPI_WARPS == 16, "gate/up: at most 32 columns per warp");
+                // SwiGLU as each 16-column chunk is read: only the 2 x 16
+                // results stay live across the release
+                float act[2][16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float sc = c0 + i < t.count ? ep_scale[c0 + i] : 0.0f;
-                        scr[i * 32 + lane] = swiglu_fast(v0[i] * sc, v1[i] * sc);
-                    }
-                    __syncwarp();
-                    // lane = (token i, 16-output block b): NVFP4 with the static global
-                    // scale; code decisions in fp32 as the format defines them
-                    {
-                        const int i = lane & 15, b = lane >> 4;
-                        const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
-                        float v[16];
+                for (int q = 0; q < 2; ++q) {
+                    if (q < nch) {
+                        const int c0 = cbeg + 16 * q;
+                        float vg[16], vu[16];
+                        tmem_ld16x2(lane_base + c0, lane_base + kBN + c0, vg, vu);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 f4 = src[q];
-                            v[4 * q] = f4.x; v[4 * q + 1] = f4.y; v[4 * q + 2] = f4.z; v[4 * q + 3] = f4.w;
+                        for (int i = 0; i < 16; ++i) {
+                            const float sc = c0 + i < t.count ? ep_scale[c0 + i] : 0.0f;
+                            act[q][i] = swiglu_fast(vg[i] * sc, vu[i] * sc);
                         }
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-                        const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
-                        const float rcp = rcp_tab[sbc];
-                        uint32_t w[2] = {0u, 0u};
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], rcp), __fmul_rn(v[2 * q + 1], rcp)) << (8 * (q & 3));
-                        const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
-                        *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
-                        out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
                     }
-                    __syncwarp();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                // the warp's scratch [16 tokens][32 outputs] turns the results
+                // into 16-output blocks per lane for the requantization
+                float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 16 * 32;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    if (q < nch) {
+                        const int c0 = cbeg + 16 * q;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) scr[i * 32 + lane] = act[q][i];
+                        __syncwarp();
+                        // lane = (token i, 16-output block b): NVFP4 with the static global
+                        // scale; code decisions in fp32 as the format defines them
+                        {
+                            const int i = lane & 15, b = lane >> 4;
+                            const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
+                            float v[16];
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const float4 f4 = src[qq];
+                                v[4 * qq] = f4.x; v[4 * qq + 1] = f4.y; v[4 * qq + 2] = f4.z; v[4 * qq + 3] = f4.w;
+                            }
+                            float amax = 0.0f;
+#pragma unroll
+                            for (int qq = 0; qq < 16; ++qq) amax = fmaxf(amax, fabsf(v[qq]));
+                            const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
+                            const float rcp = rcp_tab[sbc];
+                            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                            for (int qq = 0; qq < 8; ++qq)
+                                w[qq >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * qq], rcp), __fmul_rn(v[2 * qq + 1], rcp)) << (8 * (qq & 3));
+                            const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
+                            *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
+                            out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
+                        }
+                        __syncwarp();
+                    }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
             epi_sync_n<C::EPI_WARPS>();
             if constexpr (MODE == 0) {
                 // per token: 64 code bytes and 8 scale bytes of this 128-row block
@@ -1374,27 +1398,6 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-// One 16-value block of W4A4 activations: e4m3 scale code of amax / (6 g)
-// and the e2m1 codes of v / (s_b g), the decisions taken in fp32 with IEEE
-// division as the format defines them.  Returns the scale code; w[0..1]
-// hold the 16 codes (low nibble = even column).
-MOE_DEV uint32_t quant_block16(const float (&v)[16], float g, uint32_t (&w)[2]) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-    uint32_t sbc = 0;
-    float r = 0.0f;
-    if (g != 0.0f) {
-        sbc = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
-        const float sbv = e4m3_to_f32(sbc);
-        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
-    }
-    w[0] = w[1] = 0u;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) w[q >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * q], r), __fmul_rn(v[2 * q + 1], r)) << (8 * (q & 3));
-    return sbc;
-}
-
 // W4A4 activations of the gate/up GEMM in permuted order, quantized per 16
 // values with the static global scale g (codes [slots][H/2], scales
 // [slots][H/16]).  The warp of token t quantizes its row once and stores it
@@ -1418,7 +1421,7 @@ __global__ void k_x_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t*
             v[2 * q + 1] = bf16_hi(wv[q]);
         }
         uint32_t w[2];
-        const uint32_t sbc = quant_block16(v, g, w);
+        const uint32_t sbc = nvfp4_quant_block16(v, g, w);
         for (int j = 0; j < k; ++j) {
             const int pos = __shfl_sync(0xffffffffu, mypos, j);
             if (pos < 0) continue;
@@ -1482,6 +1485,8 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+bool prefill_native_fp4(int H, int I) { return H % kFp4KS == 0 && I % kFp4KS == 0; }
 
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I) {
     const int RB = (H > I ? H : I) / kBlkN;
@@ -1645,7 +1650,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     const long long threads = (long long)T * (H / 8);
-    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, T, H, k,
+    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
                                                                (__nv_bfloat16*)p.y);
     return cudaGetLastError();
 }
@@ -1659,7 +1664,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const bool fp4 = ex.quant == Q_NVFP4;
     // NVFP4 W4A4 on the block-scaled tensor cores when the shapes allow
     // 256-value stages (else the exact bf16 dequantization path below)
-    const bool native = fp4 && p.fp4_codes[0] && H % kFp4KS == 0 && I % kFp4KS == 0;
+    const bool native = fp4 && p.fp4_codes[0] && prefill_native_fp4(H, I);
     if (native) return launch_prefill_fp4(p, st);
     const __nv_bfloat16* xin = nullptr;
     CUtensorMapDataType xdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -1714,7 +1719,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
-    if (!make_bmaps(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I) ||
+    if (!make_bmaps(&m_routed, p.a_perm, (uint64_t)slots, (uint64_t)I, xdt) ||
         !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
     g.tiles = p.tiles + p.tile_cap;          // the down list
@@ -1744,7 +1749,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     // ---- combine
     const long long threads = (long long)T * (H / 8);
-    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, T, H, k,
+    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
                                                                (__nv_bfloat16*)p.y);
     return cudaGetLastError();
 }

@@ -88,6 +88,11 @@ struct FusedArgs {
     unsigned long long* bar;       // workspace: monotonically increasing arrival count, zero-initialised
     float* gu_sh;                  // workspace [4][T][2 * I]: partial shared gate/up sums by K part
     int* err;                      // device error word
+    // test hook of the bounded grid-barrier waits: CTA withhold_cta (>= 0)
+    // skips its arrival at the first grid barrier; wait_limit (> 0) replaces
+    // the default limit of the waits, in SM clock cycles
+    int withhold_cta = -1;
+    long long wait_limit = 0;
 };
 size_t fused_smem_bytes(int H, int I);
 cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st);   // cudaErrorNotSupported: shapes too large
@@ -132,6 +137,9 @@ struct PrefillArgs {
     cudaEvent_t ev_gu_r, ev_dn_r;
 };
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I);
+// NVFP4 prefill runs on the block-scaled tensor cores when H and I allow
+// 256-value stages (else the exact bf16 dequantization path)
+bool prefill_native_fp4(int H, int I);
 cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st);
 
 }  // namespace moe

@@ -70,6 +70,13 @@ struct moe_layer {
     float g_x = 0.0f, g_a = 0.0f;
     bool act_scales_set = false;
     cudaEvent_t prof[kProfEvents] = {};
+    // the last grouped-GEMM forward: its token count and whether it took the
+    // block-scaled NVFP4 path (read by the debug getters)
+    int last_prefill_T = 0;
+    bool last_prefill_fp4 = false;
+    // moe_debug_set_wait_test: one-shot test hook of the next fused decode launch
+    int dbg_withhold_cta = -1;
+    long long dbg_wait_limit = 0;
     char err[512] = {0};
 };
 
@@ -502,6 +509,14 @@ static bool use_fused_decode(moe_layer* h, cudaStream_t st, cudaError_t* err) {
     return *err == cudaSuccess && cs == cudaStreamCaptureStatusNone;
 }
 
+// the one-shot test hook of the bounded waits goes to this launch only
+static void take_wait_test(moe_layer* h, FusedArgs& f) {
+    f.withhold_cta = h->dbg_withhold_cta;
+    f.wait_limit = h->dbg_wait_limit;
+    h->dbg_withhold_cta = -1;
+    h->dbg_wait_limit = 0;
+}
+
 static DecodeArgs decode_args(moe_layer* h) {
     DecodeArgs a{};
     a.ex = expert_args(h);
@@ -546,6 +561,8 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         }
         p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
         p.ev_gu_r = h->prof[8]; p.ev_dn_r = h->prof[9];
+        h->last_prefill_T = T;
+        h->last_prefill_fp4 = c.quant == MOE_Q_NVFP4 && !h->table_set && prefill_native_fp4(c.hidden, c.inter);
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_prefill(p, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_forward (grouped GEMM path)");
@@ -564,6 +581,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         f.bar = h->fused_bar;
         f.gu_sh = h->fused_gu_sh;
         f.err = h->dev_err;
+        take_wait_test(h, f);
         if (h->prof[2]) cudaEventRecord(h->prof[2], st);
         cudaError_t e = launch_decode_fused(f, st);
         if (e == cudaSuccess) {
@@ -633,6 +651,7 @@ moe_status moe_route_forward(moe_handle h, const void* x, int32_t T, int32_t* to
     f.bar = h->fused_bar;
     f.gu_sh = h->fused_gu_sh;
     f.err = h->dev_err;
+    take_wait_test(h, f);
     if (h->prof[0]) cudaEventRecord(h->prof[0], st);
     cudaError_t e = launch_decode_fused(f, st);
     if (e == cudaSuccess) {
@@ -759,6 +778,46 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which, 
                                 cudaMemcpyDefault, st);
     }
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_unpack_matrix");
+    return MOE_OK;
+}
+
+moe_status moe_debug_get_permutation(moe_handle h, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                                     moe_stream_t stream) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_debug_get_permutation: null handle");
+    if (!counts || !offsets || !perm || !inv) return fail(h, MOE_ERR_INVALID_ARG, "moe_debug_get_permutation: null pointer");
+    if (h->last_prefill_T <= 0) return fail(h, MOE_ERR_STATE, "moe_debug_get_permutation: no grouped-GEMM forward yet");
+    DeviceGuard dg(h->cfg.device);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int E = h->cfg.num_experts;
+    const size_t slots = (size_t)h->last_prefill_T * h->cfg.top_k;
+    cudaError_t e = cudaMemcpyAsync(counts, h->counts, sizeof(int32_t) * E, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(offsets, h->offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(perm, h->perm, sizeof(int32_t) * slots, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(inv, h->inv, sizeof(int32_t) * slots, cudaMemcpyDefault, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_get_permutation");
+    return MOE_OK;
+}
+
+moe_status moe_debug_get_act_nvfp4(moe_handle h, void* codes, void* scales, moe_stream_t stream) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_debug_get_act_nvfp4: null handle");
+    if (!codes || !scales) return fail(h, MOE_ERR_INVALID_ARG, "moe_debug_get_act_nvfp4: null pointer");
+    if (h->last_prefill_T <= 0 || !h->last_prefill_fp4)
+        return fail(h, MOE_ERR_STATE, "moe_debug_get_act_nvfp4: no block-scaled NVFP4 grouped-GEMM forward yet");
+    DeviceGuard dg(h->cfg.device);
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t slots = (size_t)h->last_prefill_T * h->cfg.top_k, H = (size_t)h->cfg.hidden;
+    const uint8_t* xc = reinterpret_cast<const uint8_t*>(h->xp);    // [slots][H/2], then [slots][H/16]
+    cudaError_t e = cudaMemcpyAsync(codes, xc, slots * H / 2, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(scales, xc + slots * H / 2, slots * H / 16, cudaMemcpyDefault, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_get_act_nvfp4");
+    return MOE_OK;
+}
+
+moe_status moe_debug_set_wait_test(moe_handle h, int32_t withhold_cta, int64_t wait_limit_cycles) {
+    if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_debug_set_wait_test: null handle");
+    if (wait_limit_cycles < 0) return fail(h, MOE_ERR_INVALID_ARG, "moe_debug_set_wait_test: negative limit");
+    h->dbg_withhold_cta = withhold_cta < 0 ? -1 : withhold_cta;
+    h->dbg_wait_limit = wait_limit_cycles;
     return MOE_OK;
 }
 

@@ -172,24 +172,11 @@ __global__ void k_quantize_nvfp4(const SRC* __restrict__ w, int N, int K, float 
     const int n = (int)(t / nblk), b = (int)(t % nblk);
     const SRC* src = w + (size_t)n * K + b * kFp4Blk;
     float e[16];
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) { e[i] = load_elem<SRC>(src, i); amax = fmaxf(amax, fabsf(e[i])); }
-    uint32_t sb = 0;
-    float r = 0.0f;
-    if (g != 0.0f) {
-        sb = f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
-        const float sbv = e4m3_to_f32(sb);
-        r = (sbv == 0.0f) ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sbv, g));
-    }
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-        lo |= f32x2_to_e2m1(__fmul_rn(e[i], r), __fmul_rn(e[i + 1], r)) << (4 * i);
-        hi |= f32x2_to_e2m1(__fmul_rn(e[i + 8], r), __fmul_rn(e[i + 9], r)) << (4 * i);
-    }
-    if (g == 0.0f) { lo = 0; hi = 0; }
-    *reinterpret_cast<uint2*>(codes + (size_t)n * (K / 2) + b * 8) = make_uint2(lo, hi);
+    for (int i = 0; i < 16; ++i) e[i] = load_elem<SRC>(src, i);
+    uint32_t wc[2];
+    const uint32_t sb = nvfp4_quant_block16(e, g, wc);
+    *reinterpret_cast<uint2*>(codes + (size_t)n * (K / 2) + b * 8) = make_uint2(wc[0], wc[1]);
     scales[(size_t)n * nblk + b] = (uint8_t)sb;
 }
 

@@ -74,6 +74,10 @@ def lib():
             "moe_set_decode_path": [vp, i32],
             "moe_export_expert": [vp, i32, vp, vp],
             "moe_set_expert_table": [vp, ctypes.POINTER(vp), vp],
+            "moe_debug_get_permutation": [vp, vp, vp, vp, vp, vp],
+            "moe_debug_get_act_nvfp4": [vp, vp, vp, vp],
+            "moe_debug_set_wait_test": [vp, i32, i64],
+            "moe_mma_peak_loop": [i32, i32, i64, vp, ctypes.POINTER(ctypes.c_double), vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -206,6 +210,34 @@ class MoeLayer:
         arr = (ctypes.c_void_p * len(addresses))(*[int(a) for a in addresses])
         _check(lib().moe_set_expert_table(self.h, arr, _stream(stream)), self.h)
 
+    def debug_permutation(self, T, stream=None):
+        """(counts, offsets, perm, inv) of the last grouped-GEMM forward of T tokens."""
+        E, k = self.cfg.num_experts, self.cfg.top_k
+        dev = torch.device("cuda", self.cfg.device)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+        inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+        _check(lib().moe_debug_get_permutation(self.h, _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+                                               _stream(stream)), self.h)
+        return counts, offsets, perm, inv
+
+    def debug_act_nvfp4(self, T, stream=None):
+        """(codes [T*k, H/2], scales [T*k, H/16]) of the W4A4 operand of the last
+        block-scaled NVFP4 grouped-GEMM forward of T tokens, permuted order."""
+        slots, H = T * self.cfg.top_k, self.cfg.hidden
+        dev = torch.device("cuda", self.cfg.device)
+        codes = torch.empty((slots, H // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((slots, H // 16), dtype=torch.uint8, device=dev)
+        _check(lib().moe_debug_get_act_nvfp4(self.h, _ptr(codes), _ptr(scales), _stream(stream)), self.h)
+        return codes, scales
+
+    def debug_set_wait_test(self, withhold_cta, wait_limit_cycles=0):
+        """One-shot test hook: the next fused decode launch has CTA
+        withhold_cta skip a grid-barrier arrival, and its waits give up after
+        wait_limit_cycles (0: the default limit)."""
+        _check(lib().moe_debug_set_wait_test(self.h, int(withhold_cta), int(wait_limit_cycles)), self.h)
+
     def debug_unpack(self, expert, which, codes, scales=None, zeros=None, global_scale=None, stream=None):
         _check(lib().moe_debug_unpack_matrix(self.h, int(expert), int(which), _ptr(codes), _ptr(scales),
                                              _ptr(zeros), _ptr(global_scale), _stream(stream)), self.h)
@@ -273,3 +305,13 @@ def permute_noalloc(ids, num_experts, stream=None):
     _check(lib().moe_permute_noalloc(_ptr(ids), T, k, num_experts, _ptr(counts), _ptr(offsets), _ptr(perm),
                                      _ptr(inv), _stream(stream)))
     return counts, offsets, perm, inv
+
+
+def mma_peak_loop(kind, issuers, iters, err, stream=None):
+    """Launch the tensor-core throughput loop (kind 0: bf16 kind::f16, 1: e2m1
+    block-scaled) on every SM; returns the FLOPs of the launch.  err: a
+    zeroed int32 CUDA tensor that receives a code if a wait gave up."""
+    flops = ctypes.c_double(0.0)
+    _check(lib().moe_mma_peak_loop(int(kind), int(issuers), int(iters), _ptr(err), ctypes.byref(flops),
+                                   _stream(stream)))
+    return flops.value

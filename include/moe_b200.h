@@ -290,6 +290,42 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
                                    void* codes, void* scales, void* zeros,
                                    float* global_scale_out, moe_stream_t stream);
 
+/* Copy the token permutation of the last grouped-GEMM forward (T > 8) of this
+ * handle: counts [E], offsets [E+1], perm [T*k] (the flat slot s = t*k + j at
+ * each expert-major position, ascending s inside an expert) and inv [T*k]
+ * (the position of each slot; -1 for a slot whose id lies outside [0, E)).
+ * Only the first offsets[E] entries of perm are written by the forward.  The
+ * order is the expert-major gather of the selected experts of each token
+ * ("Qwen3.8-Flash-Next on one 24 GB GPU", section "What the patch does").
+ * Buffers may be host or device memory; the copies are asynchronous on
+ * `stream` (synchronize before reading host buffers).
+ * Errors: INVALID_ARG (null), STATE (no grouped-GEMM forward yet), CUDA. */
+moe_status moe_debug_get_permutation(moe_handle h, int32_t* counts, int32_t* offsets, int32_t* perm,
+                                     int32_t* inv, moe_stream_t stream);
+
+/* Copy the W4A4 activation operand of the last block-scaled NVFP4
+ * grouped-GEMM forward: in permuted order (position p holds the row of token
+ * perm[p] / k), codes [T*k][H/2] (E2M1, even column in the low nibble) and
+ * scales [T*k][H/16] (E4M3, one per 16 values), quantized with the static
+ * global scale g_x ("meshapplied/Qwen3.8-Flash-Next-NVFP4-Latest", section
+ * "Format").  Positions from offsets[E] on are not written by the forward.
+ * Buffers host or device, copies asynchronous on `stream`.
+ * Errors: INVALID_ARG (null), STATE (no such forward yet), CUDA. */
+moe_status moe_debug_get_act_nvfp4(moe_handle h, void* codes, void* scales, moe_stream_t stream);
+
+/* Test hook of the bounded device-side waits (no counterpart on the pages;
+ * it exists so that the timeout path can be exercised without a fault): the
+ * next launch of the fused decode kernel on this handle (moe_route_forward
+ * or moe_forward with T <= 8 outside stream capture) has CTA `withhold_cta`
+ * skip its arrival at its first grid barrier, and every grid-barrier wait of
+ * that launch gives up after `wait_limit_cycles` SM clock cycles (0: the
+ * default limit of about 2 s).  That launch then stops every CTA at the
+ * barrier and reports MOE_ERR_TIMEOUT through moe_sync_status, which also
+ * resets the barrier so that the next call is correct.  One-shot: the
+ * setting applies to one launch and then clears; withhold_cta < 0 clears it.
+ * Errors: INVALID_ARG (null handle, negative limit). */
+moe_status moe_debug_set_wait_test(moe_handle h, int32_t withhold_cta, int64_t wait_limit_cycles);
+
 /* Profiling aid: when events != NULL, every later call records, on its
  * stream, the events of the slots it has:
  *   [0] before and [1] after the routing kernels of moe_route;
@@ -308,6 +344,22 @@ moe_status moe_debug_unpack_matrix(moe_handle h, int32_t expert, int32_t which,
  * an event between two kernels removes their launch overlap, so time the
  * layer itself with recording off. */
 moe_status moe_set_profile_events(moe_handle h, void* const* events, int32_t n);
+
+/* Measurement aid (no counterpart on the pages): a tensor-core throughput
+ * loop on every SM of the current device, the denominator of the tensor-pipe
+ * fraction of the grouped GEMMs.  Each CTA (one per SM) has `issuers` warps
+ * issue `iters` MMAs each, back to back, from operand tiles resident in
+ * shared memory into their own TMEM accumulators:
+ *   kind 0: tcgen05.mma kind::f16, bf16 operands, M = 128, N = 256, K = 16
+ *           (issuers 1..2);
+ *   kind 1: tcgen05.mma kind::mxf4nvf4.block_scale.block16, E2M1 operands
+ *           with E4M3 scales, M = 128, N = 128, K = 64 (issuers 1..3).
+ * *flops_out (host) receives the FLOPs of the launch (2 M N K per MMA); time
+ * the launch on `stream` with events.  A wait that gives up writes a code to
+ * *err_dev (device int, zero on entry).  Asynchronous.
+ * Errors: INVALID_ARG (kind, issuers, iters, null), CUDA. */
+moe_status moe_mma_peak_loop(int32_t kind, int32_t issuers, int64_t iters, int32_t* err_dev,
+                             double* flops_out, moe_stream_t stream);
 
 /* Synchronize `stream` and report device-side failures of earlier calls on
  * this handle: MOE_ERR_TIMEOUT when a kernel gave up a bounded wait (the

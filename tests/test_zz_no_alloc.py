@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from bit_quantized_mixture_b200 import moe
+from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
@@ -29,6 +30,9 @@ def test_noalloc_permutation_equals_allocating_one_on_consecutive_calls():
         torch.cuda.synchronize()
         for r, g in zip(ref, got):
             assert torch.equal(r, g)          # integer outputs: bit-exact
+        # and directly against the oracle's permutation
+        for o, g in zip(O.permute(ids.cpu().numpy(), E), got):
+            assert np.array_equal(o, g.cpu().numpy())
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
