@@ -55,15 +55,18 @@ MOE_DEV unsigned long long atom_add_release64(unsigned long long* p, unsigned lo
     asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
     return old;
 }
-MOE_DEV bool grid_barrier(unsigned long long* bar, int* err, volatile int* abort_s) {
+// `withhold` (a test hook of the bounded wait) makes this CTA skip its
+// arrival, so the episode never completes and every CTA gives up after
+// `limit` cycles.
+MOE_DEV bool grid_barrier(unsigned long long* bar, int* err, volatile int* abort_s, bool withhold, long long limit) {
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned long long n = gridDim.x;
-        const unsigned long long ticket = atom_add_release64(bar, 1ull);
+        const unsigned long long ticket = withhold ? ld_acquire64(bar) : atom_add_release64(bar, 1ull);
         const unsigned long long target = (ticket / n + 1) * n;
         const long long t0 = clock64();
         while (ld_acquire64(bar) < target) {
-            if (clock64() - t0 > kBarrierLimitCycles) {
+            if (clock64() - t0 > limit) {
                 *abort_s = 1;
                 if (err) atomicCAS(err, 0, 20);
                 break;
@@ -775,7 +778,13 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
         }
     }
 
-    if (f.wr && !grid_barrier(f.bar, f.err, &abort_s)) return;
+    const long long wait_limit = f.wait_limit > 0 ? f.wait_limit : kBarrierLimitCycles;
+    bool withhold = f.withhold_cta == (int)blockIdx.x;
+    if (f.wr && !grid_barrier(f.bar, f.err, &abort_s, withhold, wait_limit)) {
+        cp_wait<0>();                    // no copy of this CTA outlives it
+        return;
+    }
+    if (f.wr) withhold = false;          // the test hook withholds one arrival only
 
     // ---- phase 1: top-k (every CTA), plan, routed gate/up units
     if (f.wr) {
@@ -900,7 +909,10 @@ __global__ void __launch_bounds__(kFThreads, 1) k_decode_fused(FusedArgs f) {
             group_sync(group);
         }
     }
-    if (!grid_barrier(f.bar, f.err, &abort_s)) return;
+    if (!grid_barrier(f.bar, f.err, &abort_s, withhold, wait_limit)) {
+        cp_wait<0>();
+        return;
+    }
 
     // ---- phase 2: down units and the shared down slices; tickets, combine
     cp_wait<0>();                                                        // every prefetch landed
