@@ -6,8 +6,12 @@
 
 A step is one pass of the whole layer (router, top-k, expert GEMVs/GEMMs,
 combine) over one batch of seeded synthetic tokens of the workload.  Default
-workload: decode batch 1, W4A16 INT4 experts (T=1, H=2048, I=512, E=512,
-top-10 plus one bf16 shared expert), 100 seeded tokens cycled over the steps.
+workload: the largest configuration, a prefill chunk of T=8192 tokens with
+NVFP4 W4A4 routed experts (H=2048, I=512, E=512, top-10, uniform routing,
+one bf16 shared expert).  The same run also measures the other workloads of
+the metric (decode batch 1 INT4, decode batch 4 INT2, prefill INT4 with Zipf
+routing) and reports each under "workloads", and it measures the tensor-core
+peaks it reports fractions against with its own tcgen05 throughput loops.
 Multi-GPU: one process per GPU (torchrun); every rank runs an independent
 replica on its own tokens (the layer is per-token, so there is no exchange),
 and the slowest rank's device time defines the whole-job throughput.
@@ -29,7 +33,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "decode-b1-int4"
+DEFAULT_WORKLOAD = "prefill-nvfp4"
+EXTRA_WORKLOADS = "decode-b1-int4,decode-b4-int2,prefill-int4-zipf"
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 roofline"
 UNIT = "tokens/s"
 
@@ -41,6 +46,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--extra-workloads", default=EXTRA_WORKLOADS,
+                    help="comma-separated workloads measured after the main one ('none': only the main one)")
+    ap.add_argument("--no-peak-loop", action="store_true", help="skip the tensor-core peak loops")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded oracle sample length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mb", type=int, default=512)
@@ -134,11 +142,13 @@ class OracleSampler:
     Decode workloads: whole decode steps (router, top-k, expert SwiGLU from
     the packed weights, combine).  Prefill workloads: chunks of 4 consecutive
     tokens of the batch (top-k of the workload's routing logits, expert
-    SwiGLU, combine).  Quantization of the weights is set-up, as on the GPU:
-    it is not timed, is kept across samples, and stops a sample early once it
-    has taken `setup_cap_s` in total."""
+    SwiGLU, combine).  Prefill samples cycle over the first `prefill_chunks`
+    chunks of the batch, so the set of experts to quantize stays bounded.
+    Quantization of the weights is set-up, as on the GPU: it is not timed,
+    runs in a thread pool, is kept across samples, and stops a sample early
+    once it has taken `setup_cap_s` in total."""
 
-    def __init__(self, wl, setup_cap_s=90.0):
+    def __init__(self, wl, setup_cap_s=90.0, prefill_chunks=4):
         from bit_quantized_mixture_b200 import synth
         from oracle import moe_oracle as O
         self.O, self.synth, self.wl = O, synth, wl
@@ -155,7 +165,7 @@ class OracleSampler:
         self.q = {}
         self.setup = 0.0
         self.chunk = 4 if self.prefill else wl.T
-        self.n_chunks = wl.T // self.chunk if self.prefill else wl.steps
+        self.n_chunks = min(wl.T // self.chunk, prefill_chunks) if self.prefill else wl.steps
 
     def quantized(self, e):
         O, wl = self.O, self.wl
@@ -200,8 +210,11 @@ class OracleSampler:
             i = (offset + done) % self.n_chunks
             x = self.xs[i * self.chunk:(i + 1) * self.chunk]
             ids_probe, _ = self._route(i, x)
-            for e in np.unique(ids_probe):
-                self.quantized(int(e))
+            new = [int(e) for e in np.unique(ids_probe) if int(e) not in self.q]
+            if new:
+                from concurrent.futures import ThreadPoolExecutor
+                with ThreadPoolExecutor(max(1, min(len(new), os.cpu_count() or 4))) as ex:
+                    list(ex.map(self.quantized, new))
             t0 = time.perf_counter()
             ids, w = self._route(i, x)
             O.moe_forward(x, ids, w, wl.quant, lambda e: O.dequantize_expert(wl.quant, self.quantized(e)),
@@ -313,6 +326,42 @@ def _mapped_host_pair(cudart, nbytes, dev):
         out.append((h, d))
     (hx, dx), (hy, dy) = out
     return hx, hy, torch.as_tensor(_DeviceView(dx, nbytes), device=dev), torch.as_tensor(_DeviceView(dy, nbytes), device=dev)
+
+
+def measure_tensor_peaks(dev):
+    """Burst throughput of the library's tcgen05 loops on this GPU (every SM;
+    operands resident in shared memory): bf16 kind::f16 (M128 N256 K16) and
+    the block-scaled e2m1 kind::mxf4nvf4 (M128 N128 K64), best of several
+    launches and issuing-warp counts, each launch a few milliseconds."""
+    import torch
+
+    from bit_quantized_mixture_b200 import moe
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+    for kind, name, issuers, iters in ((0, "bf16_tflops", (1, 2), 20000), (1, "e2m1_block16_tflops", (1, 2, 3), 40000)):
+        best, best_iss = 0.0, 0
+        for iss in issuers:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(6)]
+            flops = 0.0
+            with torch.cuda.stream(stream):
+                for e0, e1 in evs:
+                    e0.record(stream)
+                    flops = moe.mma_peak_loop(kind, iss, iters, err, stream)
+                    e1.record(stream)
+            stream.synchronize()
+            t = min(a.elapsed_time(b) for a, b in evs[1:])
+            tf = flops / (t * 1e-3) / 1e12
+            if tf > best:
+                best, best_iss = tf, iss
+        out[name] = best
+        out[name.replace("_tflops", "_issuers")] = best_iss
+    if int(err.item()) != 0:
+        raise RuntimeError(f"tensor peak loop: a bounded wait gave up (code {int(err.item())})")
+    out["method"] = ("tcgen05 throughput loops of the library (moe_mma_peak_loop): one CTA per SM, operands "
+                     "resident in shared memory, fp32 accumulators in TMEM; best of 5 timed launches (CUDA events) "
+                     "over 1..3 issuing warps")
+    return out
 
 
 def run_decode(args, wl, dev, rank, world):
@@ -535,6 +584,11 @@ def run_decode(args, wl, dev, rank, world):
                      "algorithmic_bytes_per_launch": by[dom], "peak_source": peak_kind,
                      "decode_path": "router kernel + two GEMV kernels (CUDA graph)"},
         "layer_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
+        "layer": {"bytes_per_step": step_bytes, "hbm_gbs": step_bytes / (total_ms / args.steps * 1e-3) / 1e9,
+                  "frac_of_hbm": step_bytes / (total_ms / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "ms_per_step": total_ms / args.steps,
+                  "note": "whole step (graph-timed, kernels overlapping through programmatic launch) against "
+                          "HBM; the roofline object is the dominant kernel timed alone with events"},
         "warm_ms_per_step": warm_ms / args.steps,
         "launches_per_step": 3, "h2d": T * H * 2, "d2h": T * H * 2, "mean_distinct_experts": mean_uniq,
     }
@@ -547,7 +601,7 @@ def prefill_flops(wl, slots):
     return 2.0 * m * wl.H * 2 * wl.I, 2.0 * m * wl.I * wl.H
 
 
-def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
+def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind, tensor_peaks=None):
     """Roofline of the routed gate/up grouped GEMM (one launch).  Algorithmic
     work: FLOPs 2 * slots * H * 2I; bytes = the touched experts' packed gate
     and up weights (codes + scales [+ zeros]) once, the token activations once
@@ -555,7 +609,9 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
     intermediate written once (bf16, or e2m1 + e4m3 for NVFP4).  The binding
     bound is the larger of FLOPs / tensor peak and bytes / HBM bandwidth; the
     tensor peak is the measured bf16 burst (fp16 operands run at the same
-    rate), times 4 for the block-scaled e2m1 MMA (nominal 9 : 2.25)."""
+    rate); for the block-scaled e2m1 MMA it is the e2m1 peak measured by this
+    run's tcgen05 loop when given (else 4 x the bf16 burst, the nominal
+    9 : 2.25 ratio, which is also reported)."""
     H, I, T = wl.H, wl.I, wl.T
     n = 2 * I                                     # gate + up rows per expert
     if wl.quant in ("int4", "int4g32"):
@@ -576,7 +632,10 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
     flops = 2.0 * slots * H * n
     nbytes = float(experts_touched * w_bytes + act + out)
     t = t_ms * 1e-3
-    tensor_peak = peaks["bf16_tflops"] * (4.0 if wl.quant == "nvfp4" else 1.0)
+    fp4 = wl.quant == "nvfp4"
+    nominal_fp4 = peaks["bf16_tflops"] * 4.0
+    fp4_measured = bool(fp4 and tensor_peaks and tensor_peaks.get("e2m1_block16_tflops"))
+    tensor_peak = (tensor_peaks["e2m1_block16_tflops"] if fp4_measured else nominal_fp4) if fp4 else peaks["bf16_tflops"]
     hbm = peaks["hbm_gbs"]
     t_tensor, t_hbm = flops / (tensor_peak * 1e12), nbytes / (hbm * 1e9)
     tfl, gbs = flops / t / 1e12, nbytes / t / 1e9
@@ -585,16 +644,18 @@ def gateup_roofline(wl, slots, experts_touched, t_ms, peaks, peak_kind):
               "arithmetic_intensity": flops / nbytes, "ridge_flop_per_byte": tensor_peak * 1e3 / hbm,
               "achieved_tflops": tfl, "tensor_peak_tflops": tensor_peak, "frac_of_tensor_peak": tfl / tensor_peak,
               "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm, "ms_per_launch": t_ms,
-              "peak_source": (f"{peak_kind} dense bf16 burst" + (" x 4 (nominal e2m1 : bf16 dense ratio)"
-                                                                  if wl.quant == "nvfp4" else "") +
-                              f"; {peak_kind} HBM copy bandwidth")}
+              "peak_source": ((("e2m1 block-scaled peak measured in this run by the library's tcgen05 loop"
+                                if fp4_measured else f"{peak_kind} dense bf16 burst x 4 (nominal e2m1 : bf16 ratio)")
+                               if fp4 else f"{peak_kind} dense bf16 burst") + f"; {peak_kind} HBM copy bandwidth")}
+    if fp4:
+        common["frac_of_tensor_peak_nominal_ratio"] = tfl / nominal_fp4
     if t_hbm >= t_tensor:
         return dict({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}, **common)
     return dict({"bound": "tensor", "achieved": tfl, "peak": tensor_peak, "unit": "TFLOP/s", "frac": tfl / tensor_peak},
                 **common)
 
 
-def run_prefill(args, wl, dev, rank, world):
+def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
     """A prefill step: router GEMM on x (logits only), softmax/top-k of the
     workload's synthetic routing logits (the skewed / uniform routing the
     workload prescribes, standing in for the router's own), permutation,
@@ -739,7 +800,8 @@ def run_prefill(args, wl, dev, rank, world):
     fl_gu, fl_dn = prefill_flops(wl, T * k)
     peaks, peak_kind = measured_peaks()
     layer.close()
-    roof = gateup_roofline(wl, T * k, experts_touched, kern["grouped_gemm_gate_up_routed"], peaks, peak_kind)
+    roof = gateup_roofline(wl, T * k, experts_touched, kern["grouped_gemm_gate_up_routed"], peaks, peak_kind,
+                           tensor_peaks)
     roof["traffic"] = load_traffic("k_fp4_gemm<0>" if wl.quant == "nvfp4" else "k_grouped_gemm<0,false>", wl.name)
     roof["down_routed_tflops"] = 2.0 * T * k * wl.I * H / (kern["grouped_gemm_down_routed"] * 1e-3) / 1e12
     return {
@@ -751,8 +813,26 @@ def run_prefill(args, wl, dev, rank, world):
         # both tile lists, 2 routed GEMMs (+2 shared), combine
         "launches_per_step": 10 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
         "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
+        "layer": prefill_layer_fractions(wl, experts_touched, total_ms / args.steps, peaks, roof["tensor_peak_tflops"]),
         "dtype": "e2m1" if wl.quant == "nvfp4" else "f16",
     }
+
+
+def prefill_layer_fractions(wl, experts_touched, ms_per_step, peaks, tensor_peak):
+    """The whole step against the roofline (beside the dominant kernel's
+    figure): FLOPs of the router GEMM and of the routed and shared expert
+    GEMMs over the step time, and the step's algorithmic bytes (the touched
+    experts' packed weights, the bf16 router and shared expert, x in and y
+    out) over the step time."""
+    T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
+    fl_gu, fl_dn = prefill_flops(wl, T * k)
+    flops = fl_gu + fl_dn + 2.0 * T * E * H
+    gu_b, dn_b = expert_bytes(wl)
+    nbytes = experts_touched * (gu_b + dn_b) + E * H * 2 + (3 * H * I * 2 if wl.shared else 0) + 2 * T * H * 2
+    t = ms_per_step * 1e-3
+    return {"flops_per_step": flops, "bytes_per_step": float(nbytes), "tflops": flops / t / 1e12,
+            "frac_of_tensor_peak": flops / t / 1e12 / tensor_peak, "hbm_gbs": nbytes / t / 1e9,
+            "frac_of_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"], "ms_per_step": ms_per_step}
 
 
 def load_traffic(kernel, workload):
@@ -818,7 +898,17 @@ def bench_line(args, wl, r, world, prefill):
         line["warm_ms_per_step"] = r["warm_ms_per_step"]
     if "layer_tflops" in r:
         line["layer_tflops"] = r["layer_tflops"]
+    if "layer" in r:
+        line["layer"] = r["layer"]
     return line
+
+
+def workload_entry(line):
+    """A workload measured after the main one: its own value, step time,
+    roofline, per-kernel times, end-to-end figure and clocks."""
+    keep = ("value", "unit", "ms_per_step", "dtype", "config", "roofline", "layer", "kernels_ms", "e2e",
+            "gpu_launches", "clocks", "layer_hbm_gbs", "layer_tflops", "warm_ms_per_step")
+    return {k: line[k] for k in keep if k in line}
 
 
 def run_ours(args):
@@ -834,10 +924,21 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = synth.workload(args.workload)
-    prefill = wl.routing != "router"
-    r = run_prefill(args, wl, dev, rank, world) if prefill else run_decode(args, wl, dev, rank, world)
-    line = bench_line(args, wl, r, world, prefill)
+    tensor_peaks = None if args.no_peak_loop else measure_tensor_peaks(dev)
+
+    def run_workload(name):
+        wl = synth.workload(name)
+        prefill = wl.routing != "router"
+        r = run_prefill(args, wl, dev, rank, world, tensor_peaks) if prefill else run_decode(args, wl, dev, rank, world)
+        torch.cuda.empty_cache()
+        return wl, bench_line(args, wl, r, world, prefill)
+
+    wl, line = run_workload(args.workload)
+    if tensor_peaks:
+        line["tensor_peaks_measured"] = tensor_peaks
+    extras = [n for n in (args.extra_workloads or "").split(",") if n and n != "none" and n != wl.name]
+    if extras:
+        line["workloads"] = {n: workload_entry(run_workload(n)[1]) for n in extras}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_tokens_per_s(wl, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",

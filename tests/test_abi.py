@@ -88,3 +88,13 @@ def test_format_kernels_reject_null_arguments():
     assert L.moe_sync_status(None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_forward(None, None, 1, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_route_forward(None, None, 1, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_peak_loop_arguments_are_checked_on_the_host():
+    from bit_quantized_mixture_b200 import moe
+    L = moe.lib()
+    flops = ctypes.c_double(0.0)
+    dummy = ctypes.c_void_p(16)      # never dereferenced: the checks come first
+    for kind, iss, iters in ((2, 1, 10), (0, 3, 10), (1, 4, 10), (1, 0, 10), (0, 1, 0)):
+        assert L.moe_mma_peak_loop(kind, iss, iters, dummy, ctypes.byref(flops), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_mma_peak_loop(0, 1, 10, None, ctypes.byref(flops), None) == moe.MOE_ERR_INVALID_ARG

@@ -60,3 +60,37 @@ def test_gateup_bound_follows_arithmetic_intensity():
     assert r4["bound"] == "hbm" and r4["unit"] == "GB/s"
     assert r4["tensor_peak_tflops"] == pytest.approx(4 * 1663.3)
     assert r4["arithmetic_intensity"] < r4["ridge_flop_per_byte"]
+
+
+def test_nvfp4_roofline_takes_the_measured_e2m1_peak():
+    wl4 = synth.workload("prefill-nvfp4")
+    tp = {"e2m1_block16_tflops": 7000.0, "bf16_tflops": 2000.0}
+    r = bench.gateup_roofline(wl4, wl4.T * wl4.k, wl4.E, 0.254, PEAKS, "measured", tp)
+    assert r["tensor_peak_tflops"] == 7000.0
+    assert r["frac_of_tensor_peak"] == pytest.approx(r["achieved_tflops"] / 7000.0)
+    assert r["frac_of_tensor_peak_nominal_ratio"] == pytest.approx(r["achieved_tflops"] / (4 * 1663.3))
+    assert "measured in this run" in r["peak_source"]
+    # the bf16 formats keep the measured bf16 burst
+    wl = synth.workload("prefill-int4-zipf")
+    assert bench.gateup_roofline(wl, wl.T * wl.k, wl.E, 0.335, PEAKS, "measured", tp)["tensor_peak_tflops"] == 1663.3
+
+
+def test_prefill_layer_fractions():
+    wl = synth.workload("prefill-nvfp4")
+    f = bench.prefill_layer_fractions(wl, 512, 0.5, PEAKS, 7000.0)
+    gu, dn = bench.prefill_flops(wl, wl.T * wl.k)
+    assert f["flops_per_step"] == pytest.approx(gu + dn + 2 * 8192 * 512 * 2048)
+    g, d = bench.expert_bytes(wl)
+    assert f["bytes_per_step"] == 512 * (g + d) + 512 * 2048 * 2 + 3 * 2048 * 512 * 2 + 2 * 8192 * 2048 * 2
+    assert f["frac_of_hbm"] == pytest.approx(f["bytes_per_step"] / 0.5e-3 / 1e9 / 6538.6)
+
+
+def test_default_line_is_the_largest_workload():
+    args = bench.parse_args([])
+    assert args.workload == "prefill-nvfp4"
+    extra = args.extra_workloads.split(",")
+    assert set(extra) == {"decode-b1-int4", "decode-b4-int2", "prefill-int4-zipf"}
+    line = {"value": 1.0, "unit": "tokens/s", "ms_per_step": 2.0, "config": {}, "roofline": {}, "metric": "m",
+            "n_gpus": 1, "e2e": {}, "clocks": {}, "kernels_ms": {}, "layer": {}}
+    e = bench.workload_entry(line)
+    assert "metric" not in e and "n_gpus" not in e and e["roofline"] == {} and e["layer"] == {}
