@@ -945,16 +945,30 @@ __global__ void k_combine(const __half* __restrict__ O, const __half* __restrict
     const int per_row = H / 8;
     if (i >= (long long)T * per_row) return;
     const int t = (int)(i / per_row), c = (int)(i % per_row) * 8;
+    // which of the token's slots have an expert output (k <= 32)
+    uint32_t valid = 0;
+    for (int j = 0; j < k; ++j) valid |= (__ldg(inv + (size_t)t * k + j) >= 0 ? 1u : 0u) << j;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-        if (__ldg(inv + (size_t)t * k + j) < 0) continue;
-        const uint4 q = *reinterpret_cast<const uint4*>(O + ((size_t)t * k + j) * H + c);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    // eight 16-byte rows in flight per thread, summed in the fixed j order
+    for (int j0 = 0; j0 < k; j0 += 8) {
+        uint4 q[8];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
+        for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u;
+            q[u] = (j < k && ((valid >> j) & 1u)) ? ldg_stream_v4(O + ((size_t)t * k + j) * H + c)
+                                                  : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (j0 + u < k && ((valid >> (j0 + u)) & 1u)) {
+                const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+                for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
+            }
+        }
     }
     if (S) {
-        const uint4 q = *reinterpret_cast<const uint4*>(S + (size_t)t * H + c);
+        const uint4 q = ldg_stream_v4(S + (size_t)t * H + c);
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
