@@ -148,7 +148,15 @@ struct GemmArgs {
     const float* w_perm;      // routing weight of each permuted position (down)
     const float* ts_perm;     // INT4/INT2 gate/up: token scale of each permuted position
     uint8_t* out4;            // NVFP4 gate/up: e2m1 intermediate [slots, I/2] (permuted rows)
-    uint8_t* out_sf;          // NVFP4 gate/up: its e4m3 block scales [slots, I/16]
+    uint8_t* out_sf;          // NVFP4 gate/up: its e4m3 block scales, stage-major [I/256][slots][16]
+    // NVFP4 block-scaled GEMMs: the e4m3 scales of the weights (per matrix)
+    // and of the token operand, stage-major [K/256][rows][16 B] with
+    // sfa_rows = E * N and sfb_rows = slots rows per stage
+    const uint8_t* sfa0;
+    const uint8_t* sfa1;
+    const uint8_t* sfb;
+    long long sfa_rows, sfb_rows;
+    long long sfb_rows_out;   // NVFP4 gate/up: rows per stage of out_sf (the slots)
     int* err;
 };
 
@@ -718,8 +726,10 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 nx_sc = a.ts_perm ? __ldg(a.ts_perm + tn.seg + ej) : 1.0f;
                 nx_row = tn.seg + ej;
             } else {
+                // per-slot outputs are stored by permuted position (the
+                // combine finds them through the inverse permutation)
                 nx_sc = __ldg(a.w_perm + tn.seg + ej);
-                nx_row = __ldg(a.perm + tn.seg + ej);
+                nx_row = tn.seg + ej;
             }
         };
         fetch(0);
@@ -933,9 +943,10 @@ __global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict_
 }
 
 // --------------------------------------------------------------- combine
-// y[t] = sum_{j<k} O[t*k + j] + S[t], fp32 sum in fixed j order, one bf16
-// rounding.  A slot without a position (id outside [0, E): inv < 0) has no
-// expert output and contributes zero.
+// y[t] = sum_{j<k} O[inv[t*k + j]] + S[t], fp32 sum in fixed j order, one
+// bf16 rounding; O holds the weighted expert outputs by permuted position.
+// A slot without a position (id outside [0, E): inv < 0) has no expert
+// output and contributes zero.
 MOE_DEV float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 MOE_DEV float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
@@ -945,22 +956,21 @@ __global__ void k_combine(const __half* __restrict__ O, const __half* __restrict
     const int per_row = H / 8;
     if (i >= (long long)T * per_row) return;
     const int t = (int)(i / per_row), c = (int)(i % per_row) * 8;
-    // which of the token's slots have an expert output (k <= 32)
-    uint32_t valid = 0;
-    for (int j = 0; j < k; ++j) valid |= (__ldg(inv + (size_t)t * k + j) >= 0 ? 1u : 0u) << j;
+    // the permuted position of each of the token's slots (-1: no expert
+    // output); eight 16-byte slot rows in flight per thread, summed in the
+    // fixed j order
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    // eight 16-byte rows in flight per thread, summed in the fixed j order
     for (int j0 = 0; j0 < k; j0 += 8) {
+        int pos[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pos[u] = j0 + u < k ? __ldg(inv + (size_t)t * k + j0 + u) : -1;
         uint4 q[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = j0 + u;
-            q[u] = (j < k && ((valid >> j) & 1u)) ? ldg_stream_v4(O + ((size_t)t * k + j) * H + c)
-                                                  : make_uint4(0, 0, 0, 0);
-        }
+        for (int u = 0; u < 8; ++u)
+            q[u] = pos[u] >= 0 ? ldg_stream_v4(O + (size_t)pos[u] * H + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            if (j0 + u < k && ((valid >> (j0 + u)) & 1u)) {
+            if (pos[u] >= 0) {
                 const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
@@ -1085,6 +1095,68 @@ constexpr int kFp4KS = 256;                  // K values per stage
 constexpr int kFp4Tile = 128 * 128;          // 16 KB: 128 rows x 128 bytes
 constexpr int kFp4SfTile = 128 * 16;         // 2 KB: 128 rows x 16 scale bytes
 
+// Token-operand maps of the block-scaled GEMM (e2m1 codes, 128-byte rows,
+// 128-byte swizzle) with boxes of 128, 64, 32 and 16 rows: a tile of n (a
+// multiple of 16) tokens loads only its rows.
+struct Fp4BMaps {
+    CUtensorMap codes[4];
+};
+MOE_DEV void load_fp4_token_rows(uint8_t* dst_codes, const Fp4BMaps& mb, int x_codes, int y, int n, uint64_t* bar) {
+    const int n16 = n >> 4;
+    if (n16 >= 8) {
+        tma_load_2d(dst_codes, &mb.codes[0], x_codes, y, bar);
+        return;
+    }
+    int off = 0;
+#pragma unroll
+    for (int b = 2; b >= 0; --b)
+        if (n16 & (1 << b)) {
+            tma_load_2d(dst_codes + off * 128, &mb.codes[3 - b], x_codes, y + off, bar);
+            off += 16 << b;
+        }
+}
+
+// Store maps of the per-slot output [slots][H] fp16 with boxes of 128 / 2^i
+// rows x 128 columns: a tile's n rows leave as at most eight TMA stores.
+struct OMaps {
+    CUtensorMap m[8];
+};
+
+constexpr int kFp4SmallN = 48;               // tokens of the gate/up small accumulator
+
+// The accumulator of the next tile, walked identically by the MMA warps and
+// the epilogue: buffer, first column, matrix stride and phase parity.
+struct Fp4Acc {
+    int buf;
+    uint32_t col, mat_stride, parity;
+};
+struct Fp4AccSeq {
+    uint32_t uses0 = 0u, uses1 = 0u;   // completed uses of buffer 0 / 1
+    int local = 0;
+};
+template <int MODE>
+MOE_DEV Fp4Acc fp4_acc_next(Fp4AccSeq& q, int n_mma) {
+    Fp4Acc a;
+    if (MODE == 1) {
+        a.buf = q.local & 1;
+        a.col = (uint32_t)(a.buf * kBN);
+        a.mat_stride = kBN;
+    } else if (n_mma <= kFp4SmallN) {
+        a.buf = 1;
+        a.col = 2 * kBN;
+        a.mat_stride = kFp4SmallN;
+    } else {
+        a.buf = 0;
+        a.col = 0;
+        a.mat_stride = kBN;
+    }
+    a.parity = (a.buf ? q.uses1 : q.uses0) & 1u;
+    q.uses0 += a.buf == 0 ? 1u : 0u;
+    q.uses1 += a.buf == 1 ? 1u : 0u;
+    ++q.local;
+    return a;
+}
+
 template <int MODE>
 struct Fp4Cfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
@@ -1096,17 +1168,20 @@ struct Fp4Cfg {
     // staging of a tile is the longest step of these kernels)
     static constexpr int EPI_WARPS = MODE == 0 ? 16 : 12;
     static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
-    static constexpr int ACC_BUFS = MODE == 0 ? 1 : 2;
+    // accumulators: gate/up keeps one of 2 x 128 columns and a small one of
+    // 2 x kFp4SmallN columns for tiles of at most kFp4SmallN tokens, so that
+    // such a tile and its neighbours take turns; down alternates two of 128
+    static constexpr int ACC_BUFS = 2;
     static constexpr int ACC_COLS = NMAT * kBN;
-    static constexpr int SF_COL0 = ACC_BUFS * ACC_COLS;
+    static constexpr int SF_COL0 = MODE == 0 ? ACC_COLS + 2 * kFp4SmallN : 2 * ACC_COLS;
     static constexpr int SF_STAGE_COLS = (NMAT + 1) * 16;             // A per matrix, then B; 4 MMAs x 4 columns
     static_assert(SF_COL0 + S * SF_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
     static constexpr int A = 0;                                       // [S][NMAT][16 KB]
     static constexpr int B = A + S * NMAT * kFp4Tile;                 // [S][16 KB]
     static constexpr int SFA = B + S * kFp4Tile;                      // [S][NMAT][2 KB]
     static constexpr int SFB = SFA + S * NMAT * kFp4SfTile;           // [S][2 KB]
-    static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: [128][128] fp16
-    static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : kOutTile;
+    static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: 2 x [128][128] fp16
+    static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : 2 * kOutTile;
     static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [16 tok][32] fp32
     static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 16 * 32 * 4 : 0;
     static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
@@ -1116,8 +1191,7 @@ struct Fp4Cfg {
 template <int MODE>
 __global__ void __launch_bounds__(Fp4Cfg<MODE>::THREADS, 1)
 k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
-           const __grid_constant__ CUtensorMap map_sfa0, const __grid_constant__ CUtensorMap map_sfa1,
-           const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_sfb, GemmArgs a) {
+           const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps map_o, GemmArgs a) {
     using C = Fp4Cfg<MODE>;
     constexpr int NMAT = C::NMAT, S = C::S;
     extern __shared__ uint8_t smem_raw[];
@@ -1174,15 +1248,21 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 const uint32_t r = (uint32_t)(g / S);
                 if (!warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 11)) { ok = false; break; }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)((NMAT + 1) * (kFp4Tile + kFp4SfTile)));
+                    // the weight tiles and their scales, then the tile's token rows
+                    const int n_mma = (t.count + 15) & ~15;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * (kFp4Tile + kFp4SfTile)) + (uint32_t)n_mma * 144u);
                     for (int m = 0; m < NMAT; ++m) {
                         tma_load_2d(smem + C::A + (s * NMAT + m) * kFp4Tile, m == 0 ? &map_a0 : &map_a1, ks * 128, arow,
                                     &full[s]);
-                        tma_load_2d(smem + C::SFA + (s * NMAT + m) * kFp4SfTile, m == 0 ? &map_sfa0 : &map_sfa1,
-                                    ks * 16, arow, &full[s]);
+                        // the stage's scale tile: 128 rows x 16 B, contiguous (stage-major)
+                        bulk_g2s(smem + C::SFA + (s * NMAT + m) * kFp4SfTile,
+                                 (m == 0 ? a.sfa0 : a.sfa1) + ((size_t)ks * a.sfa_rows + arow) * 16, kFp4SfTile, &full[s]);
                     }
-                    tma_load_2d(smem + C::B + s * kFp4Tile, &map_b, ks * 128, t.seg, &full[s]);
-                    tma_load_2d(smem + C::SFB + s * kFp4SfTile, &map_sfb, ks * 16, t.seg, &full[s]);
+                    // the token rows' scales: n_mma x 16 B, contiguous (rows past
+                    // the end of the slots read workspace slack, never used)
+                    bulk_g2s(smem + C::SFB + s * kFp4SfTile, a.sfb + ((size_t)ks * a.sfb_rows + t.seg) * 16,
+                             (uint32_t)n_mma * 16u, &full[s]);
+                    load_fp4_token_rows(smem + C::B + s * kFp4Tile, map_b, ks * 128, t.seg, n_mma, &full[s]);
                 }
                 __syncwarp();
             }
@@ -1191,17 +1271,18 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
     } else if (warp >= kWarpMma && warp < C::SF0) {
         // --------------------------------------------------------- MMA issue
         const int mi = warp - kWarpMma;
-        int g = 0, local = 0;
-        for (int jt = 0; jt < nseq && !abort_flag; ++jt, ++local) {
+        int g = 0;
+        Fp4AccSeq aseq;
+        for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const uint32_t idesc = idesc_nvfp4(128, n_mma);
-            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
-            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
-            if (!warp_wait(&acc_empty[ab], (use & 1u) ^ 1u, &abort_flag, a.err, 12)) break;
+            const Fp4Acc acc = fp4_acc_next<MODE>(aseq, n_mma);
+            const int ab = acc.buf;
+            if (!warp_wait(&acc_empty[ab], acc.parity ^ 1u, &abort_flag, a.err, 12)) break;
             tc_fence_after();
             bool ok = true;
-            const uint32_t d = tmem + ab * C::ACC_COLS + mi * kBN;
+            const uint32_t d = tmem + acc.col + mi * acc.mat_stride;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
@@ -1271,15 +1352,19 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             const GemmTile tn = tile_at(jn);
             if (ej >= tn.count) return;
             nx_sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
-            nx_row = MODE == 0 ? tn.seg + ej : __ldg(a.perm + tn.seg + ej);
+            nx_row = tn.seg + ej;
         };
         fetch(0);
         int local = 0;
+        Fp4AccSeq aseq;
         for (int jt = 0; jt < nseq; ++jt, ++local) {
             const GemmTile t = tile_at(jt);
-            const int ab = C::ACC_BUFS == 2 ? (local & 1) : 0;
-            const uint32_t use = C::ACC_BUFS == 2 ? (uint32_t)(local >> 1) : (uint32_t)local;
+            const Fp4Acc acc = fp4_acc_next<MODE>(aseq, (t.count + 15) & ~15);
+            const int ab = acc.buf;
             const float gsc = a.g_w[t.expert] * a.g_act;
+            // down: this tile's staging buffer was last read by the TMA store
+            // of the tile two back (one bulk group per tile)
+            if (MODE == 1 && ej == 0) bulk_wait_read<1>();
             epi_sync_n<C::EPI_WARPS>();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
@@ -1289,14 +1374,14 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             fetch(jt + 1);
             epi_sync_n<C::EPI_WARPS>();
             if (ep_stop) break;
-            if (!warp_wait(&acc_full[ab], use & 1u, &abort_flag, a.err, 16)) continue;
+            if (!warp_wait(&acc_full[ab], acc.parity, &abort_flag, a.err, 16)) continue;
             tc_fence_after();
             const int n_mma = (t.count + 15) & ~15;
             // the warps of a lane quarter split the columns (16-aligned parts)
             constexpr int NSET = C::EPI_WARPS / 4;
             const int cpart = (((n_mma >> 4) + NSET - 1) / NSET) << 4;
             const int cbeg = min(n_mma, cset * cpart), cend = min(n_mma, cbeg + cpart);
-            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + ab * C::ACC_COLS;
+            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + acc.col;
             const int nch = (cend - cbeg) >> 4;
             // Every warp first copies its accumulator columns into registers
             // and releases the accumulator, so that the MMAs of the next tile
@@ -1309,6 +1394,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * kOutTile);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (q < nch) {
@@ -1316,11 +1402,11 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                         for (int i = 0; i < 16; ++i) {
                             const int col = cbeg + 16 * q + i;
                             const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                            reinterpret_cast<uint16_t*>(out_s)[col * kBlkN + row] =
-                                __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
+                            ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
                         }
                     }
                 }
+                fence_proxy_async_smem();        // the TMA store reads what this thread wrote
             } else {
                 static_assert(C::EPI_WARPS == 16, "gate/up: at most 32 columns per warp");
                 // SwiGLU as each 16-column chunk is read: only the 2 x 16
@@ -1331,7 +1417,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                     if (q < nch) {
                         const int c0 = cbeg + 16 * q;
                         float vg[16], vu[16];
-                        tmem_ld16x2(lane_base + c0, lane_base + kBN + c0, vg, vu);
+                        tmem_ld16x2(lane_base + c0, lane_base + acc.mat_stride + c0, vg, vu);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float sc = c0 + i < t.count ? ep_scale[c0 + i] : 0.0f;
@@ -1383,28 +1469,36 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             epi_sync_n<C::EPI_WARPS>();
             if constexpr (MODE == 0) {
                 // per token: 64 code bytes and 8 scale bytes of this 128-row block
-                const int I2 = a.out_ld / 2, I16 = a.out_ld / 16;
+                const int I2 = a.out_ld / 2;
                 for (int i = ej; i < t.count * 5; i += C::EPI_WARPS * 32) {
                     const int col = i / 5, part = i % 5;
                     const size_t r = (size_t)ep_row[col];
                     if (part < 4)
                         *reinterpret_cast<uint4*>(a.out4 + r * I2 + t.rb * 64 + part * 16) =
                             *reinterpret_cast<const uint4*>(out_s + col * 80 + part * 16);
-                    else
-                        *reinterpret_cast<uint2*>(a.out_sf + r * I16 + t.rb * 8) =
+                    else   // stage-major scales: stage rb / 2, bytes 8 (rb % 2) .. +8
+                        *reinterpret_cast<uint2*>(a.out_sf + ((size_t)(t.rb >> 1) * a.sfb_rows_out + r) * 16 + (t.rb & 1) * 8) =
                             *reinterpret_cast<const uint2*>(out_s + col * 80 + 64);
                 }
-            } else {
-                const uint16_t* o16 = reinterpret_cast<const uint16_t*>(out_s);
-                uint16_t* dst = reinterpret_cast<uint16_t*>(a.o16);
-                const int col0 = t.rb * kBlkN;
-                for (int i = ej; i < t.count * 16; i += C::EPI_WARPS * 32) {
-                    const int col = i >> 4, ch = i & 15;
-                    *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) =
-                        *reinterpret_cast<const uint4*>(o16 + col * kBlkN + ch * 8);
+            } else if (ej == 0) {
+                // the tile's rows are the permuted positions seg .. seg+count-1:
+                // TMA stores of boxes of 128, 64, ..., 1 rows, one bulk group
+                const uint8_t* ob = out_s + (local & 1) * kOutTile;
+                if (t.count == kBN) {
+                    tma_store_2d(&map_o.m[0], t.rb * kBlkN, t.seg, ob);
+                } else {
+                    int off = 0;
+#pragma unroll
+                    for (int b = 6; b >= 0; --b)
+                        if ((t.count >> b) & 1) {
+                            tma_store_2d(&map_o.m[7 - b], t.rb * kBlkN, t.seg + off, ob + off * (kBlkN * 2));
+                            off += 1 << b;
+                        }
                 }
+                bulk_commit();
             }
         }
+        if (MODE == 1 && ej == 0) bulk_wait_all();     // every store done before the CTA leaves
     }
     tc_fence_before();
     __syncthreads();
@@ -1413,12 +1507,13 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
 }
 
 // W4A4 activations of the gate/up GEMM in permuted order, quantized per 16
-// values with the static global scale g (codes [slots][H/2], scales
-// [slots][H/16]).  The warp of token t quantizes its row once and stores it
+// values with the static global scale g (codes [slots][H/2]; scales
+// stage-major [H/256][slots][16 B], so that a GEMM stage's scale rows are
+// contiguous).  The warp of token t quantizes its row once and stores it
 // at the k positions inv[t*k + j] of its slots, with each position's
 // routing weight; dropped slots (inv < 0) are skipped.
 __global__ void k_x_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ inv, int T, int H, int k,
-                             float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                             float g, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, long long slots,
                              const float* __restrict__ topk_w, float* __restrict__ w_perm) {
     const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -1440,7 +1535,7 @@ __global__ void k_x_fp4_perm(const __nv_bfloat16* __restrict__ x, const int32_t*
             const int pos = __shfl_sync(0xffffffffu, mypos, j);
             if (pos < 0) continue;
             *reinterpret_cast<uint2*>(codes + (size_t)pos * (H / 2) + b * 8) = make_uint2(w[0], w[1]);
-            sf[(size_t)pos * (H / 16) + b] = (uint8_t)sbc;
+            sf[((size_t)(b >> 4) * slots + pos) * 16 + (b & 15)] = (uint8_t)sbc;
         }
     }
     if (lane < k && mypos >= 0) w_perm[mypos] = __ldg(topk_w + (size_t)t * k + lane);
@@ -1501,6 +1596,28 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 }
 
 bool prefill_native_fp4(int H, int I) { return H % kFp4KS == 0 && I % kFp4KS == 0; }
+
+// Token-operand maps of the block-scaled GEMM over codes [rows][K/2], boxes
+// of 128 / 64 / 32 / 16 rows
+static bool make_fp4_bmaps(Fp4BMaps* mb, const void* codes, uint64_t rows, int K) {
+    for (int i = 0; i < 4; ++i)
+        if (!make_map_u8(&mb->codes[i], codes, rows, K / 2, 128, (uint32_t)(kBN >> i), true)) return false;
+    return true;
+}
+
+// 2D fp16 map over [rows, cols] for TMA stores: box 128 columns x box_rows,
+// no swizzle (the smem image is row-major)
+static bool make_map_store16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {128, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I) {
     const int RB = (H > I ? H : I) / kBlkN;
@@ -1571,11 +1688,12 @@ cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E,
 // Block-scaled NVFP4 GEMM over the routed tiles; maps: A of gate (or down),
 // A of up, their scale tiles, B and its scale tiles.
 template <int MODE>
-static cudaError_t launch_fp4(const CUtensorMap (&m)[6], const GemmArgs& g, cudaStream_t st) {
+static cudaError_t launch_fp4(const CUtensorMap (&m)[2], const Fp4BMaps& mb, const OMaps& mo, const GemmArgs& g,
+                              cudaStream_t st) {
     constexpr int bytes = Fp4Cfg<MODE>::ALLOC;
     cudaError_t err = cudaFuncSetAttribute(k_fp4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (err != cudaSuccess) return err;
-    k_fp4_gemm<MODE><<<num_sms(), Fp4Cfg<MODE>::THREADS, bytes, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], g);
+    k_fp4_gemm<MODE><<<num_sms(), Fp4Cfg<MODE>::THREADS, bytes, st>>>(m[0], m[1], mb, mo, g);
     return cudaGetLastError();
 }
 
@@ -1592,18 +1710,16 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     uint8_t* a4 = reinterpret_cast<uint8_t*>(p.a_perm);               // [slots][I/2]
     uint8_t* as = a4 + (size_t)slots * I / 2;                          // [slots][I/16]
     {
-        k_x_fp4_perm<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, p.inv, T, H, k, ex.g_x, xc, xs, p.w,
-                                                   p.w_perm);
+        k_x_fp4_perm<<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)p.x, p.inv, T, H, k, ex.g_x, xc, xs,
+                                                   (long long)slots, p.w, p.w_perm);
     }
     // ---- gate / up
-    CUtensorMap m[6];
+    CUtensorMap m[2];
+    Fp4BMaps mb;
     BMaps m_shared;
     if (!make_map_u8(&m[0], p.fp4_codes[0], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
         !make_map_u8(&m[1], p.fp4_codes[1], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
-        !make_map_u8(&m[2], p.fp4_scales[0], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
-        !make_map_u8(&m[3], p.fp4_scales[1], (uint64_t)E * I, H / 16, 16, kBlkN, false) ||
-        !make_map_u8(&m[4], xc, (uint64_t)slots, H / 2, 128, kBN, true) ||
-        !make_map_u8(&m[5], xs, (uint64_t)slots, H / 16, 16, kBN, false) ||
+        !make_fp4_bmaps(&mb, xc, (uint64_t)slots, H) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
     k_build_tiles<<<2, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, H / kBlkN, has_sh ? 1 : 0, num_sms(),
@@ -1627,21 +1743,29 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.g_act = ex.g_x;
     g.g_req = ex.g_a;
     g.err = p.err;
+    g.sfa0 = p.fp4_scales[0];
+    g.sfa1 = p.fp4_scales[1];
+    g.sfb = xs;
+    g.sfa_rows = (long long)E * I;
+    g.sfb_rows = (long long)slots;
+    g.sfb_rows_out = (long long)slots;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
-    cudaError_t err = launch_fp4<0>(m, g, st);
+    OMaps mo;                         // the down GEMM's output maps (unused by gate/up)
+    for (int i = 0; i < 8; ++i) mo.m[i] = m[0];
+    cudaError_t err = launch_fp4<0>(m, mb, mo, g, st);
     if (err == cudaSuccess && p.ev_gu_r) cudaEventRecord(p.ev_gu_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
     if (!make_map_u8(&m[0], p.fp4_codes[2], (uint64_t)E * H, I / 2, 128, kBlkN, true) ||
-        !make_map_u8(&m[2], p.fp4_scales[2], (uint64_t)E * H, I / 16, 16, kBlkN, false) ||
-        !make_map_u8(&m[4], a4, (uint64_t)slots, I / 2, 128, kBN, true) ||
-        !make_map_u8(&m[5], as, (uint64_t)slots, I / 16, 16, kBN, false) ||
+        !make_fp4_bmaps(&mb, a4, (uint64_t)slots, I) ||
         !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
     m[1] = m[0];
-    m[3] = m[2];
+    g.sfa0 = g.sfa1 = p.fp4_scales[2];
+    g.sfb = as;
+    g.sfa_rows = (long long)E * H;
     g.tiles = p.tiles + p.tile_cap;          // the down list
     g.groups = p.groups + p.tile_cap;
     g.num_tiles = p.num_tiles + 4;
@@ -1658,7 +1782,10 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.g_w = ex.g_down;
     g.g_act = ex.g_a;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
-    err = launch_fp4<1>(m, g, st);
+    for (int i = 0; i < 8; ++i)
+        if (!make_map_store16(&mo.m[i], p.o, (uint64_t)slots, (uint64_t)H, (uint32_t)(kBN >> i)))
+            return cudaErrorInvalidValue;
+    err = launch_fp4<1>(m, mb, mo, g, st);
     if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;

@@ -28,7 +28,7 @@ struct moe_layer {
     uint8_t* router = nullptr;     // bf16 [E, H]
     uint8_t* shared[3] = {nullptr, nullptr, nullptr};   // bf16 device layout
     uint8_t* fp4_codes[3] = {nullptr, nullptr, nullptr};    // NVFP4: natural-layout images [E][N][K/2]
-    uint8_t* fp4_scales[3] = {nullptr, nullptr, nullptr};   //        and their block scales [E][N][K/16]
+    uint8_t* fp4_scales[3] = {nullptr, nullptr, nullptr};   //        and their block scales [K/256][E*N][16]
     float* g_gate = nullptr;       // NVFP4 global scales [E]
     float* g_down = nullptr;
     // workspace
@@ -178,7 +178,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
         for (int m = 0; m < 3; ++m) {
             const size_t nk = (size_t)h->geom[m].N * h->geom[m].K * E;
             img_off[m] = a; a = align_up(a + nk / 2, 256);
-            imgs_off[m] = a; a = align_up(a + nk / 16, 256);
+            imgs_off[m] = a; a = align_up(a + (size_t)((h->geom[m].K / 16 + 15) / 16) * 16 * h->geom[m].N * E, 256);
         }
     h->arena_bytes = a;
     if (cudaMalloc(&h->arena, h->arena_bytes) != cudaSuccess) {
@@ -196,7 +196,7 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     h->g_down = h->g_gate + E;
 
     // workspace
-    const int MT = 8;   // tokens per decode launch
+    const int MT = 16;  // tokens per launch of the two-kernel decode path
     size_t w = 0;
     auto carve = [&](size_t bytes) { size_t o = w; w = align_up(w + bytes, 256); return o; };
     const size_t o_logits = carve(sizeof(float) * (size_t)c.max_tokens * E);
@@ -319,7 +319,7 @@ moe_status moe_load_router(moe_handle h, const void* w_router_any, moe_stream_t 
 
 static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix& q, uint8_t* dst_codes,
                               uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st, uint8_t* img_codes = nullptr,
-                              uint8_t* img_scales = nullptr) {
+                              uint8_t* img_scales = nullptr, size_t img_rows = 0) {
     const size_t codes_in = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K * 2
                                                : (size_t)gm.N * gm.K /
                                                      (gm.quant == Q_INT2 ? 4 : ((gm.quant == Q_FP8 || gm.quant == Q_FP6) ? 1 : 2));
@@ -334,9 +334,19 @@ static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: copy");
     e = launch_relayout(gm, h->staging, h->staging + o_s, h->staging + o_z, dst_codes, dst_scales, dst_zeros, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: relayout");
-    if (img_codes) {   // NVFP4: the interchange layout is the prefill GEMM's operand image
+    if (img_codes) {
+        // NVFP4: the interchange codes are the prefill GEMM's operand image
+        // [E][N][K/2]; the block scales go to a stage-major image
+        // [K/256][E*N][16 B] (img_scales points at this expert's first row of
+        // stage 0, img_rows is E*N), so that one stage's scale tile of 128
+        // rows is one contiguous 2 KB bulk copy
         e = cudaMemcpyAsync(img_codes, h->staging, codes_in, cudaMemcpyDeviceToDevice, st);
-        if (e == cudaSuccess) e = cudaMemcpyAsync(img_scales, h->staging + o_s, scales_in, cudaMemcpyDeviceToDevice, st);
+        const int kb16 = gm.K / 16;
+        for (int ks = 0; e == cudaSuccess && ks * 16 < kb16; ++ks) {
+            const int w = kb16 - ks * 16 < 16 ? kb16 - ks * 16 : 16;
+            e = cudaMemcpy2DAsync(img_scales + (size_t)ks * img_rows * 16, 16, h->staging + o_s + ks * 16, (size_t)kb16,
+                                  (size_t)w, (size_t)gm.N, cudaMemcpyDeviceToDevice, st);
+        }
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: NVFP4 image");
     }
     return MOE_OK;
@@ -377,9 +387,9 @@ moe_status moe_load_expert_weights(moe_handle h, int32_t expert, const moe_exper
             uint8_t* base = h->experts + (size_t)expert * h->expert_stride;
             const size_t nk = (size_t)gm.N * gm.K;
             uint8_t* ic = h->fp4_codes[m] ? h->fp4_codes[m] + (size_t)expert * nk / 2 : nullptr;
-            uint8_t* is = h->fp4_scales[m] ? h->fp4_scales[m] + (size_t)expert * nk / 16 : nullptr;
+            uint8_t* is = h->fp4_scales[m] ? h->fp4_scales[m] + (size_t)expert * gm.N * 16 : nullptr;
             s = load_matrix(h, gm, *mats[m], base + h->off_codes[m], base + h->off_scales[m], base + h->off_zeros[m], st,
-                            ic, is);
+                            ic, is, (size_t)c.num_experts * gm.N);
         }
         if (s != MOE_OK) return s;
     }
@@ -503,7 +513,7 @@ static ExpertArgs expert_args(moe_layer* h) {
 static bool use_fused_decode(moe_layer* h, cudaStream_t st, cudaError_t* err) {
     *err = cudaSuccess;
     if (h->decode_path == MOE_DECODE_FUSED) return true;
-    if (h->decode_path == MOE_DECODE_KERNELS) return false;
+    if (h->decode_path == MOE_DECODE_KERNELS || h->decode_path == MOE_DECODE_GEMM) return false;
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     *err = cudaStreamIsCapturing(st, &cs);
     return *err == cudaSuccess && cs == cudaStreamCaptureStatusNone;
@@ -543,7 +553,11 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         return fail(h, MOE_ERR_STATE, "moe_forward: NVFP4 activation global scales not set");
     DeviceGuard dg(c.device);
     cudaStream_t st = (cudaStream_t)stream;
-    if (!decode_supported(T, c.top_k)) {       // more tokens than the GEMV path takes
+    // the grouped-GEMM path: more tokens than the GEMVs take, the GEMM path
+    // forced, or 9 to 16 tokens by default (measured: from 8 tokens per call
+    // the grouped GEMM is the faster of the two on the decode-b1 INT4 layer)
+    const bool gemv_ok = decode_supported(T, c.top_k) && (T <= 8 || h->decode_path == MOE_DECODE_KERNELS);
+    if (!gemv_ok || h->decode_path == MOE_DECODE_GEMM) {
         PrefillArgs p{};
         p.ex = expert_args(h);
         p.x = x; p.ids = topk_ids; p.w = topk_w; p.y = y; p.T = T;
@@ -601,7 +615,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
     a.ev_mid = h->prof[3];
     if (h->prof[2]) cudaEventRecord(h->prof[2], st);
     for (int t0 = 0; t0 < T;) {
-        int tc = T - t0 < 8 ? T - t0 : 8;
+        int tc = T - t0 < 16 ? T - t0 : 16;
         while (!decode_supported(tc, c.top_k)) --tc;
         a.x = reinterpret_cast<const uint8_t*>(x) + (size_t)t0 * c.hidden * 2;
         a.ids = topk_ids + (size_t)t0 * c.top_k;
@@ -806,9 +820,12 @@ moe_status moe_debug_get_act_nvfp4(moe_handle h, void* codes, void* scales, moe_
     DeviceGuard dg(h->cfg.device);
     cudaStream_t st = (cudaStream_t)stream;
     const size_t slots = (size_t)h->last_prefill_T * h->cfg.top_k, H = (size_t)h->cfg.hidden;
-    const uint8_t* xc = reinterpret_cast<const uint8_t*>(h->xp);    // [slots][H/2], then [slots][H/16]
+    // codes [slots][H/2], then the scales stage-major [H/256][slots][16 B]
+    const uint8_t* xc = reinterpret_cast<const uint8_t*>(h->xp);
     cudaError_t e = cudaMemcpyAsync(codes, xc, slots * H / 2, cudaMemcpyDefault, st);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(scales, xc + slots * H / 2, slots * H / 16, cudaMemcpyDefault, st);
+    for (size_t ks = 0; e == cudaSuccess && ks < H / 256; ++ks)
+        e = cudaMemcpy2DAsync(reinterpret_cast<uint8_t*>(scales) + ks * 16, H / 16, xc + slots * H / 2 + ks * slots * 16, 16,
+                              16, slots, cudaMemcpyDefault, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_debug_get_act_nvfp4");
     return MOE_OK;
 }
@@ -823,7 +840,7 @@ moe_status moe_debug_set_wait_test(moe_handle h, int32_t withhold_cta, int64_t w
 
 moe_status moe_set_decode_path(moe_handle h, int32_t path) {
     if (!h) return fail(nullptr, MOE_ERR_INVALID_ARG, "moe_set_decode_path: null handle");
-    if (path != MOE_DECODE_AUTO && path != MOE_DECODE_FUSED && path != MOE_DECODE_KERNELS)
+    if (path != MOE_DECODE_AUTO && path != MOE_DECODE_FUSED && path != MOE_DECODE_KERNELS && path != MOE_DECODE_GEMM)
         return fail(h, MOE_ERR_INVALID_ARG, "moe_set_decode_path: unknown path %d", path);
     h->decode_path = path;
     return MOE_OK;
