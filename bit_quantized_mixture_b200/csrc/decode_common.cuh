@@ -49,10 +49,10 @@ MOE_DEV void build_plan(const int32_t* __restrict__ ids, int n, Plan& p) {
 // input (distinct ids per token) there are at most T <= kDecMaxT; repeated
 // ids within a token are invalid input and the extra slots are dropped, so
 // no buffer is overrun.
-MOE_DEV int item_tokens(const int* __restrict__ ids, int n, int k, int s0, int* tok, int* slot) {
+MOE_DEV int item_tokens(const int* __restrict__ ids, int n, int k, int s0, int* tok, int* slot, int cap = kDecMaxT) {
     const int e0 = ids[s0];
     int c = 0;
-    for (int s = s0; s < n && c < kDecMaxT; ++s) {
+    for (int s = s0; s < n && c < cap; ++s) {
         if (ids[s] == e0) {
             if (threadIdx.x == 0) { tok[c] = s / k; slot[c] = s; }
             ++c;
@@ -275,11 +275,13 @@ MOE_DEV void mma_blk(float (&acc)[4], const Blk<Q>& o, const __nv_bfloat16* xrow
 }
 
 // One warp: 16 rows (rl, rl+8 per lane) of NM matrices over k-blocks
-// warp, warp + nwarps, ...
-template <int Q, int NM>
-MOE_DEV void warp_rows(float (&acc)[NM][4], const MatPtr (&mats)[NM], int nb, int rl, int KB, int G, int warp,
-                       int nwarps, const __nv_bfloat16* xrow, int c) {
-    constexpr int KPW = Fmt<Q>::KPW;
+// warp, warp + nwarps, ... against NG groups of 8 token columns (xrows[q]:
+// the lane's token row of group q); each k-block's weights are loaded once
+// for all groups.
+template <int Q, int NM, int NG = 1>
+MOE_DEV void warp_rows(float (&acc)[NM][NG][4], const MatPtr (&mats)[NM], int nb, int rl, int KB, int G, int warp,
+                       int nwarps, const __nv_bfloat16* const (&xrows)[NG], int c) {
+    constexpr int KPW = NG == 1 ? Fmt<Q>::KPW : 1;
     for (int kb0 = warp; kb0 < KB; kb0 += nwarps * KPW) {
         Blk<Q> blk[NM][KPW];
 #pragma unroll
@@ -295,7 +297,9 @@ MOE_DEV void warp_rows(float (&acc)[NM][4], const MatPtr (&mats)[NM], int nb, in
             const int kb = kb0 + i * nwarps;
             if (kb < KB) {
 #pragma unroll
-                for (int q = 0; q < NM; ++q) mma_blk<Q>(acc[q], blk[q][i], xrow + kb * kBlkK, c);
+                for (int q = 0; q < NM; ++q)
+#pragma unroll
+                    for (int gq = 0; gq < NG; ++gq) mma_blk<Q>(acc[q][gq], blk[q][i], xrows[gq] + kb * kBlkK, c);
             }
         }
     }
@@ -308,9 +312,9 @@ MOE_DEV void fp4_block_values(float (&v)[16], float g) { nvfp4_block16_values(v,
 // Stage rows (row_of[t], t < m) of a bf16 matrix [*, K] into smem rows of
 // ldx elements; rows m..7 are zero.  16-byte accesses, loads issued first.
 MOE_DEV void stage_rows_bf16(__nv_bfloat16* dst, int ldx, const __nv_bfloat16* src, int K, const int* row_of, int m,
-                             int tid, int nthreads) {
+                             int tid, int nthreads, int nrows = kDecMaxT) {
     const int per_row = K / 8;
-    const int total = kDecMaxT * per_row;
+    const int total = nrows * per_row;
     for (int i0 = tid; i0 < total; i0 += 4 * nthreads) {
         uint4 v[4];
 #pragma unroll
@@ -330,9 +334,10 @@ MOE_DEV void stage_rows_bf16(__nv_bfloat16* dst, int ldx, const __nv_bfloat16* s
 
 // Stage rows of bf16 activations [*, K] as W4A4 values (q * s_b).
 MOE_DEV void stage_rows_fp4_from_bf16(__nv_bfloat16* dst, int ldx, const __nv_bfloat16* src, int K,
-                                      const int* row_of, int m, float g, int tid, int nthreads) {
+                                      const int* row_of, int m, float g, int tid, int nthreads,
+                                      int nrows = kDecMaxT) {
     const int per_row = K / 16;
-    const int total = kDecMaxT * per_row;
+    const int total = nrows * per_row;
     for (int i = tid; i < total; i += nthreads) {
         const int t = i / per_row, b = i % per_row;
         float v[16];
@@ -358,9 +363,9 @@ MOE_DEV void stage_rows_fp4_from_bf16(__nv_bfloat16* dst, int ldx, const __nv_bf
 
 // Stage rows of fp32 intermediates [*, K] as bf16 (W4A4: as q * s_b).
 MOE_DEV void stage_rows_f32(__nv_bfloat16* dst, int ldx, const float* src, int K, const int* row_of, int m, bool fp4,
-                            float g, int tid, int nthreads) {
+                            float g, int tid, int nthreads, int nrows = kDecMaxT) {
     const int per_row = K / 16;
-    const int total = kDecMaxT * per_row;
+    const int total = nrows * per_row;
     for (int i = tid; i < total; i += nthreads) {
         const int t = i / per_row, b = i % per_row;
         float v[16];

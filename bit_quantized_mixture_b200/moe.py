@@ -190,8 +190,8 @@ class MoeLayer:
 
     def set_decode_path(self, path):
         """'auto' (fused kernel eagerly, three kernels inside a CUDA graph),
-        'fused' or 'kernels'."""
-        _check(lib().moe_set_decode_path(self.h, {"auto": 0, "fused": 1, "kernels": 2}[path]), self.h)
+        'fused', 'kernels' or 'gemm' (the grouped-GEMM path for every T)."""
+        _check(lib().moe_set_decode_path(self.h, {"auto": 0, "fused": 1, "kernels": 2, "gemm": 3}[path]), self.h)
 
     def expert_block_bytes(self):
         n = ctypes.c_size_t(0)

@@ -237,18 +237,25 @@ moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, in
                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                                moe_stream_t stream);
 
-/* Path of moe_route_forward and moe_forward for T <= 8 (decode):
- *   MOE_DECODE_AUTO     (default) the fused cooperative kernel for eager
- *                       calls; inside a stream capture (CUDA graph) the
+/* Path of moe_route_forward and moe_forward for T <= 16 (decode and the
+ * few-token verify steps of speculative decoding):
+ *   MOE_DECODE_AUTO     (default) T <= 8: the fused cooperative kernel for
+ *                       eager calls; inside a stream capture (CUDA graph) the
  *                       router kernel and the two GEMV kernels, which overlap
- *                       through programmatic launch and have no grid barriers
- *   MOE_DECODE_FUSED    always the fused kernel (where the format fits it)
- *   MOE_DECODE_KERNELS  always the router + two GEMV kernels
- * Both paths compute the same layer; their fp32 sums may round differently.
+ *                       through programmatic launch and have no grid
+ *                       barriers.  9 <= T <= 16: the grouped-GEMM path (the
+ *                       faster one there, measured on the decode-b1 layer)
+ *   MOE_DECODE_FUSED    the fused kernel for T <= 8 (where the format fits it)
+ *   MOE_DECODE_KERNELS  the router + two GEMV kernels for T <= 16 (two
+ *                       8-column MMA groups above 8 tokens)
+ *   MOE_DECODE_GEMM     the grouped-GEMM (prefill) path for every T, e.g. to
+ *                       find the token count where it overtakes the GEMVs
+ * All paths compute the same layer; their fp32 sums may round differently.
  * Errors: INVALID_ARG (unknown path). */
 #define MOE_DECODE_AUTO 0
 #define MOE_DECODE_FUSED 1
 #define MOE_DECODE_KERNELS 2
+#define MOE_DECODE_GEMM 3
 moe_status moe_set_decode_path(moe_handle h, int32_t path);
 
 /* ------------------------------------------------- expert address table

@@ -210,6 +210,48 @@ def test_decode_b4_int2_workload_all_steps():
     _decode_all_steps("decode-b4-int2")
 
 
+# ------------------------------------------- 9 to 16 tokens on the GEMV path
+@pytest.mark.parametrize("quant", ["int4", "int4g32", "int2", "nvfp4", "fp8", "fp6"])
+@pytest.mark.parametrize("T", [9, 12, 16])
+def test_decode_gemv_up_to_16_tokens(quant, T):
+    """9 to 16 tokens on the GEMV kernels (forced; two 8-column MMA groups)
+    and on the grouped-GEMM path, the default for these sizes."""
+    wl = SMALL[quant]
+    layer = get_layer(wl, max(T, 4))
+    layer.set_decode_path("kernels")
+    y, y_ref, layer, (x, ids, w) = _forward_case(wl, T)
+    assert_close_output(y, y_ref)
+    layer.set_decode_path("gemm")
+    y2 = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+    layer.forward(bf16_tensor(x, DEV), torch.from_numpy(ids).to(DEV), torch.from_numpy(w.astype(np.float32)).to(DEV), y2)
+    layer.sync_status()
+    layer.set_decode_path("auto")
+    assert_close_output(to_bits(y2), y_ref)
+
+
+def test_decode_b1_int4_16_tokens_full_size():
+    """The decode-b1 INT4 layer at full size with 16 tokens per call (a
+    speculative verify step), GEMV path and grouped-GEMM path."""
+    wl = synth.workload("decode-b1-int4")
+    layer, _ = build_layer(wl, 0, max_tokens=16)
+    xs = synth.activations_bf16(wl)[:16]
+    ids, w = O.route_topk(O.router_logits(xs, synth.router_bf16(wl)), wl.k)
+    ys = {}
+    for path in ("kernels", "gemm"):
+        layer.set_decode_path(path)
+        y = torch.empty((16, wl.H), dtype=torch.bfloat16, device=DEV)
+        layer.forward(bf16_tensor(xs, DEV), torch.from_numpy(ids).to(DEV), torch.from_numpy(w.astype(np.float32)).to(DEV), y)
+        layer.sync_status()
+        ys[path] = to_bits(y)
+    layer.close()
+    sx = StreamingExperts(wl)
+    sx.start(valid_experts(ids, wl.E))
+    y_ref = O.moe_forward(xs, ids, w, wl.quant, sx, shared=sx.shared())
+    sx.close()
+    for yb in ys.values():
+        assert_close_output(yb, y_ref)
+
+
 # ------------------------------------------------- slots without an expert
 @pytest.mark.parametrize("quant", ["int4", "int2", "nvfp4"])
 @pytest.mark.parametrize("T", [5, 300])
