@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "prefill-nvfp4"
-EXTRA_WORKLOADS = "decode-b1-int4,decode-b4-int2,prefill-int4-zipf"
+EXTRA_WORKLOADS = "decode-b1-int4,decode-b4-int2,prefill-int4-zipf,m-sweep"
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 roofline"
 UNIT = "tokens/s"
 
@@ -71,6 +71,14 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------- clock sampling
+class _NoClock:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
 
@@ -594,6 +602,67 @@ def run_decode(args, wl, dev, rank, world):
     }
 
 
+def run_m_sweep(args, dev, rank, world):
+    """Tokens per call M = 1, 2, 4, 8, 16 on the decode-b1 INT4 layer (H=2048,
+    I=512, E=512, top-10, bf16 shared expert): one CUDA graph of
+    moe_route_forward per seeded token batch on the GEMV path and on the
+    grouped-GEMM path, L2 flushed before every step; mean device time per
+    step and the smallest M at which the grouped GEMM is the faster."""
+    import torch
+
+    from bit_quantized_mixture_b200 import synth
+    from bit_quantized_mixture_b200.layer import build_layer
+    wl = synth.workload("decode-b1-int4")
+    layer, _ = build_layer(wl, dev.index, max_tokens=16)
+    xs = torch.from_numpy(synth.activations_bf16(wl).view(np.int16)).to(dev).view(torch.bfloat16)
+    flush = torch.empty(args.flush_mb * (1 << 20) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    nb = 6                       # distinct token batches per M (cycled)
+    table = {}
+    for M in (1, 2, 4, 8, 16):
+        row = {}
+        ids = torch.empty((M, wl.k), dtype=torch.int32, device=dev)
+        w = torch.empty((M, wl.k), dtype=torch.float32, device=dev)
+        y = torch.empty((M, wl.H), dtype=torch.bfloat16, device=dev)
+        for path in ("kernels", "gemm"):
+            layer.set_decode_path(path)
+            graphs = []
+            for b in range(nb):
+                xb = xs[(b * M) % (wl.steps - M + 1):][:M]
+                with torch.cuda.stream(stream):
+                    layer.route_forward(xb, ids, w, y)           # warm-up, uploads nothing new
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    layer.route_forward(xb, ids, w, y)
+                graphs.append(g)
+            steps = max(args.steps, 2 * nb)
+            e0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+            e1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+            with torch.cuda.stream(stream):
+                for s in range(nb):
+                    flush.zero_()
+                    graphs[s].replay()
+                for s in range(steps):
+                    flush.zero_()
+                    e0[s].record(stream)
+                    graphs[s % nb].replay()
+                    e1[s].record(stream)
+            stream.synchronize()
+            layer.sync_status(stream)
+            ms = allreduce_max(float(np.mean([a.elapsed_time(b) for a, b in zip(e0, e1)])), dev, world)
+            row["gemv_us" if path == "kernels" else "gemm_us"] = ms * 1e3
+            del graphs
+        row["tokens_per_s_gemv"] = M / (row["gemv_us"] * 1e-6)
+        table[str(M)] = row
+    layer.set_decode_path("auto")
+    layer.close()
+    cross = next((int(m) for m, r in table.items() if r["gemm_us"] < r["gemv_us"]), None)
+    return {"workload": "decode-b1-int4 layer, M tokens per call", "l2": "flushed between steps",
+            "us_per_step": table, "gemm_faster_from_M": cross,
+            "method": "one CUDA graph of moe_route_forward per token batch; decode path 'kernels' (GEMV) vs 'gemm'"}
+
+
 def prefill_flops(wl, slots):
     """Algorithmic FLOPs of the grouped GEMMs of one prefill step: gate/up
     2*m*H*2I and down 2*m*I*H over the routed slots and the shared rows."""
@@ -699,24 +768,39 @@ def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
             step(x, lg)
     layer.sync_status(stream)
 
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    clocks = ClockSampler(dev.index)
-    with clocks:
-        with torch.cuda.stream(stream):
-            for s in range(args.steps):
-                flush.zero_()
-                ev0[s].record(stream)
-                step(x, lg)
-                ev1[s].record(stream)
-        stream.synchronize()
-        torch.cuda.synchronize(dev)
-        barrier(world)
+    # the step as one CUDA graph (the layer's launches replayed without host
+    # launch gaps); the eager step is timed too and reported beside it
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(x, lg)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            graph.replay()
     layer.sync_status(stream)
-    total_ms = float(sum(a.elapsed_time(b) for a, b in zip(ev0, ev1)))
-    total_ms_max = allreduce_max(total_ms, dev, world)
+
+    def timed(run, clock=None):
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with (clock if clock is not None else _NoClock()):
+            with torch.cuda.stream(stream):
+                for s in range(args.steps):
+                    flush.zero_()
+                    e0[s].record(stream)
+                    run()
+                    e1[s].record(stream)
+            stream.synchronize()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+        layer.sync_status(stream)
+        return allreduce_max(float(sum(a.elapsed_time(b) for a, b in zip(e0, e1))), dev, world)
+
+    clocks = ClockSampler(dev.index)
+    total_ms_max = timed(graph.replay, clocks)
+    eager_ms_max = timed(lambda: step(x, lg))
+    del graph
 
     # ---- per-kernel breakdown: the library's profiling events
     pev = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(args.steps)]
@@ -772,6 +856,13 @@ def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
             lg_st[b].copy_(lg_pin, non_blocking=True)
             ev_in[s].record(h2d)
 
+    # one CUDA graph of the layer per staging buffer
+    g_st = []
+    for b in range(2):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(x_st[b], lg_st[b], y_st[b])
+        g_st.append(g)
     torch.cuda.synchronize(dev)
     t_first.record(h2d)
     copy_in(0)
@@ -783,7 +874,7 @@ def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
             stream.wait_event(ev_in[s])
             if s >= 2:
                 stream.wait_event(ev_out[s - 2])         # y_st[b] has been copied out
-            step(x_st[b], lg_st[b], y_st[b])
+            g_st[b].replay()
             ev_done[s].record(stream)
         with torch.cuda.stream(d2h):
             d2h.wait_event(ev_done[s])
@@ -796,6 +887,7 @@ def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
         raise RuntimeError("end-to-end prefill: the host copy of y differs from the device result")
     e2e_ms = float(t_first.elapsed_time(t_last))
     e2e_ms_max = allreduce_max(e2e_ms, dev, world)
+    del g_st
 
     fl_gu, fl_dn = prefill_flops(wl, T * k)
     peaks, peak_kind = measured_peaks()
@@ -806,14 +898,17 @@ def run_prefill(args, wl, dev, rank, world, tensor_peaks=None):
     roof["down_routed_tflops"] = 2.0 * T * k * wl.I * H / (kern["grouped_gemm_down_routed"] * 1e-3) / 1e12
     return {
         "total_ms": total_ms_max, "steps_tokens": args.steps * T, "e2e_ms": e2e_ms_max,
+        "eager_ms_per_step": eager_ms_max / args.steps,
         "clocks": clocks.summary(), "kernels_ms": kern, "roofline": roof,
         "e2e_method": ("chunks pipelined: inputs copied in and outputs copied out on two copy streams while the "
-                       "previous chunk computes; first input copy to last output copy"),
+                       "previous chunk computes (the layer as one CUDA graph per staging buffer); first input copy "
+                       "to last output copy"),
         # router GEMM, top-k, 3 permutation, 1 activation pass, 1 launch for
         # both tile lists, 2 routed GEMMs (+2 shared), combine
         "launches_per_step": 10 + (2 if wl.shared else 0), "h2d": T * H * 2 + T * E * 4, "d2h": T * H * 2,
-        "layer_tflops": (fl_gu + fl_dn) / (total_ms / args.steps * 1e-3) / 1e12,
-        "layer": prefill_layer_fractions(wl, experts_touched, total_ms / args.steps, peaks, roof["tensor_peak_tflops"]),
+        "layer_tflops": (fl_gu + fl_dn) / (total_ms_max / args.steps * 1e-3) / 1e12,
+        "layer": prefill_layer_fractions(wl, experts_touched, total_ms_max / args.steps, peaks,
+                                         roof["tensor_peak_tflops"]),
         "dtype": "e2m1" if wl.quant == "nvfp4" else "f16",
     }
 
@@ -883,7 +978,7 @@ def bench_line(args, wl, r, world, prefill):
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "quant": wl.quant,
                    "shared": wl.shared, "routing": wl.routing, "parallelism": f"replicas x{world}",
                    "l2": f"flushed ({args.flush_mb} MB write) between timed steps",
-                   "cuda_graph": not prefill,
+                   "cuda_graph": True,
                    "experts": "address table, shuffled pool" if args.expert_table else "arena"},
         "roofline": r["roofline"],
         "kernels_ms": r["kernels_ms"],
@@ -896,6 +991,8 @@ def bench_line(args, wl, r, world, prefill):
         line["layer_hbm_gbs"] = r["layer_gbs"]
     if "warm_ms_per_step" in r:      # decode without the L2 flush (a reported variant, not the value)
         line["warm_ms_per_step"] = r["warm_ms_per_step"]
+    if "eager_ms_per_step" in r:     # prefill launched eagerly (a reported variant, not the value)
+        line["eager_ms_per_step"] = r["eager_ms_per_step"]
     if "layer_tflops" in r:
         line["layer_tflops"] = r["layer_tflops"]
     if "layer" in r:
@@ -907,7 +1004,7 @@ def workload_entry(line):
     """A workload measured after the main one: its own value, step time,
     roofline, per-kernel times, end-to-end figure and clocks."""
     keep = ("value", "unit", "ms_per_step", "dtype", "config", "roofline", "layer", "kernels_ms", "e2e",
-            "gpu_launches", "clocks", "layer_hbm_gbs", "layer_tflops", "warm_ms_per_step")
+            "gpu_launches", "clocks", "layer_hbm_gbs", "layer_tflops", "warm_ms_per_step", "eager_ms_per_step")
     return {k: line[k] for k in keep if k in line}
 
 
@@ -938,7 +1035,8 @@ def run_ours(args):
         line["tensor_peaks_measured"] = tensor_peaks
     extras = [n for n in (args.extra_workloads or "").split(",") if n and n != "none" and n != wl.name]
     if extras:
-        line["workloads"] = {n: workload_entry(run_workload(n)[1]) for n in extras}
+        line["workloads"] = {n: (run_m_sweep(args, dev, rank, world) if n == "m-sweep" else
+                                 workload_entry(run_workload(n)[1])) for n in extras}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_tokens_per_s(wl, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",

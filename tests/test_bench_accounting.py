@@ -89,7 +89,7 @@ def test_default_line_is_the_largest_workload():
     args = bench.parse_args([])
     assert args.workload == "prefill-nvfp4"
     extra = args.extra_workloads.split(",")
-    assert set(extra) == {"decode-b1-int4", "decode-b4-int2", "prefill-int4-zipf"}
+    assert set(extra) == {"decode-b1-int4", "decode-b4-int2", "prefill-int4-zipf", "m-sweep"}
     line = {"value": 1.0, "unit": "tokens/s", "ms_per_step": 2.0, "config": {}, "roofline": {}, "metric": "m",
             "n_gpus": 1, "e2e": {}, "clocks": {}, "kernels_ms": {}, "layer": {}}
     e = bench.workload_entry(line)
