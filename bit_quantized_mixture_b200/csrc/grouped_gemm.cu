@@ -713,11 +713,12 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // stop decision is taken by one thread between two barriers.
         // token info of the next tile (scale factor, output row) is loaded
         // while the current one is processed
-        float nx_sc = 1.0f;
+        float nx_sc = 1.0f, nx_gw = 1.0f;
         int nx_row = 0;
         auto fetch = [&](int jn) {
             if (MODE == 2 || jn >= nseq) return;
             const GemmTile tn = tile_at(jn);
+            if (!SH && a.g_w) nx_gw = __ldg(a.g_w + tn.expert);     // the expert's global scale
             if (ej >= tn.count) return;
             if constexpr (SH) {
                 nx_sc = 1.0f;
@@ -738,8 +739,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
-            float gsc = 1.0f;
-            if (!SH && a.g_w) gsc = a.g_w[t.expert] * a.g_act;
+            const float gsc = (!SH && a.g_w) ? nx_gw * a.g_act : 1.0f;
             epi_sync();                                      // the previous tile's readers are done
             if (ej == 0) ep_stop = abort_flag;
             if (MODE != 2 && ej < t.count) {
@@ -1163,10 +1163,10 @@ struct Fp4Cfg {
     static constexpr int S = MODE == 0 ? 3 : 4;
     static constexpr int SF0 = kWarpMma + NMAT;                       // four scale-factor warps
     static constexpr int EPI0 = SF0 + 4;
-    // epilogue warps: four (down: three) per TMEM lane quarter, each taking
+    // epilogue warps: four per TMEM lane quarter, each taking
     // a part of the tile's token columns (the SwiGLU + requantization or the fp16
     // staging of a tile is the longest step of these kernels)
-    static constexpr int EPI_WARPS = MODE == 0 ? 16 : 12;
+    static constexpr int EPI_WARPS = 16;
     static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
     // accumulators: gate/up keeps one of 2 x 128 columns and a small one of
     // 2 x kFp4SmallN columns for tiles of at most kFp4SmallN tokens, so that
@@ -1345,11 +1345,14 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int ej = threadIdx.x - C::EPI0 * 32;
         const int cset = (warp - C::EPI0) >> 2;              // this warp's quarter of the token columns
         uint8_t* out_s = smem + C::OUT;
-        float nx_sc = 1.0f;                      // next tile's token info, loaded ahead
+        // the next tile's token info (routing weight, output row) and its
+        // expert's global scale, loaded while the current tile is processed
+        float nx_sc = 1.0f, nx_gw = 0.0f;
         int nx_row = 0;
         auto fetch = [&](int jn) {
             if (jn >= nseq) return;
             const GemmTile tn = tile_at(jn);
+            nx_gw = __ldg(a.g_w + tn.expert);
             if (ej >= tn.count) return;
             nx_sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
             nx_row = tn.seg + ej;
@@ -1361,7 +1364,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             const GemmTile t = tile_at(jt);
             const Fp4Acc acc = fp4_acc_next<MODE>(aseq, (t.count + 15) & ~15);
             const int ab = acc.buf;
-            const float gsc = a.g_w[t.expert] * a.g_act;
+            const float gsc = nx_gw * a.g_act;
             // down: this tile's staging buffer was last read by the TMA store
             // of the tile two back (one bulk group per tile)
             if (MODE == 1 && ej == 0) bulk_wait_read<1>();
@@ -1388,15 +1391,16 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             // start while this tile's SwiGLU / requantization or fp16
             // conversion runs.
             if constexpr (MODE == 1) {
-                static_assert(C::EPI_WARPS / 4 >= 2, "down: at most 64 columns per warp");
-                uint32_t r[64];
-                tmem_ld_chunks(lane_base + cbeg, nch, r);
+                static_assert(C::EPI_WARPS == 16, "down: at most 32 columns per warp");
+                uint32_t r[32];
+                if (nch == 2) tmem_ld_x32c(lane_base + cbeg, r);
+                else if (nch == 1) tmem_ld_x16c(lane_base + cbeg, r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
                 uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * kOutTile);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     if (q < nch) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
