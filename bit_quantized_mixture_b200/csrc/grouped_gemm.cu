@@ -27,16 +27,18 @@
 //   * every mbarrier wait is bounded: on timeout the CTA records an error
 //     code, stops all roles, frees TMEM and returns.
 #include <cuda.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tiles.cuh"
 
 namespace moe {
 
 using namespace sm100;
 
-constexpr int kBN = 128;            // tokens per tile (MMA N <= 128)
+constexpr int kBN = kTileTokens;    // tokens per tile (MMA N <= 128)
 constexpr int kEpiWarps = 8;        // two warps per TMEM lane quarter, 64 token columns each
 constexpr int kWarpProducer = 0, kWarpMma = 1;   // gate/up: warps 1 and 2 issue the MMAs
 constexpr uint32_t kTmemCols = 512;
@@ -92,8 +94,12 @@ struct Cfg {
     static constexpr int A = 0;                                           // SH: [S][NMAT][16 KB]
     static constexpr int B = A + (SH ? S * NMAT * kATile : 0);            // [S][KSTEP][16 KB]
     static constexpr int STG = B + S * KSTEP * kBTile;                    // routed: [SC][NMAT][STG_MAT]
-    static constexpr int OUT = STG + SC * NMAT * STG_MAT;                 // [128][128] 16-bit
-    static constexpr int BYTES = OUT + (MODE == 2 ? 0 : kOutTile);
+    static constexpr int OUT = STG + SC * NMAT * STG_MAT;                 // [OUT_BUFS][128][128] 16-bit
+    // down writes its staged rows with TMA stores: the shared-expert launch
+    // has room for two staging buffers (a tile's stores overlap the next
+    // tile's staging), the routed one for one
+    static constexpr int OUT_BUFS = (MODE == 1 && SH) ? 2 : 1;
+    static constexpr int BYTES = OUT + (MODE == 2 ? 0 : OUT_BUFS * kOutTile);
     static constexpr int ALLOC = BYTES + 1024;                            // slack for 1024-byte alignment
     static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
@@ -118,6 +124,30 @@ MOE_DEV uint32_t load_token_rows(uint8_t* dst, const BMaps& mb, int x, int y, in
             off += 16 << b;
         }
     return (uint32_t)off * 128u;
+}
+
+// Store maps of a 16-bit output [rows][H] (the per-slot outputs by permuted
+// position, the shared expert's output by token) with boxes of 128 / 2^i
+// rows x 128 columns: a tile's n consecutive rows leave as at most eight TMA
+// stores.
+struct OMaps {
+    CUtensorMap m[8];
+};
+// TMA stores of a tile's n staged rows ([n][128] 16-bit, row-major) to rows
+// y .. y+n-1, columns x .. x+127, as one bulk group (issued by one thread).
+MOE_DEV void store_tile_rows(const OMaps& mo, int x, int y, int n, const uint8_t* src) {
+    if (n == kBN) {
+        tma_store_2d(&mo.m[0], x, y, src);
+    } else {
+        int off = 0;
+#pragma unroll
+        for (int b = 6; b >= 0; --b)
+            if ((n >> b) & 1) {
+                tma_store_2d(&mo.m[7 - b], x, y + off, src + off * (kBlkN * 2));
+                off += 1 << b;
+            }
+    }
+    bulk_commit();
 }
 
 struct GemmArgs {
@@ -379,8 +409,6 @@ struct PermMeta {
 // gridDim.x, so that a CTA reads a weight block for its second token tile
 // while it is still in L2; otherwise (or when a CTA's tiles would not fit
 // the list) tiles go round robin, ti = first + j * gridDim.x.
-constexpr int kTileCache = 256;
-constexpr int kGroupTiles = 2;
 struct TileCache {
     GemmTile t[kTileCache];
     int n;          // tiles of this CTA
@@ -452,7 +480,8 @@ MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = null
 // shared-expert and router launches take Q_BF16.
 template <int MODE, bool SH, int Q>
 __global__ void __launch_bounds__(Cfg<MODE, SH>::THREADS, 1)
-k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUtensorMap map_a, GemmArgs a) {
+k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUtensorMap map_a,
+               const __grid_constant__ OMaps map_o, GemmArgs a) {
     using C = Cfg<MODE, SH>;
     constexpr int NMAT = C::NMAT, S = C::S, KSTEP = C::KSTEP;
     constexpr int SC = C::SC > 0 ? C::SC : 1;
@@ -713,40 +742,51 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         // stop decision is taken by one thread between two barriers.
         // token info of the next tile (scale factor, output row) is loaded
         // while the current one is processed
-        float nx_sc = 1.0f, nx_gw = 1.0f;
-        int nx_row = 0;
+        // (of the tiles two and one ahead)
+        struct TileInfo {
+            float sc, gw;
+            int row;
+        };
         auto fetch = [&](int jn) {
-            if (MODE == 2 || jn >= nseq) return;
+            TileInfo f{1.0f, 1.0f, 0};
+            if (MODE == 2 || jn >= nseq) return f;
             const GemmTile tn = tile_at(jn);
-            if (!SH && a.g_w) nx_gw = __ldg(a.g_w + tn.expert);     // the expert's global scale
-            if (ej >= tn.count) return;
+            if (!SH && a.g_w) f.gw = __ldg(a.g_w + tn.expert);     // the expert's global scale
+            if (ej >= tn.count) return f;
             if constexpr (SH) {
-                nx_sc = 1.0f;
-                nx_row = tn.seg + ej;
+                f.row = tn.seg + ej;
             } else if (MODE == 0) {
-                nx_sc = a.ts_perm ? __ldg(a.ts_perm + tn.seg + ej) : 1.0f;
-                nx_row = tn.seg + ej;
+                f.sc = a.ts_perm ? __ldg(a.ts_perm + tn.seg + ej) : 1.0f;
+                f.row = tn.seg + ej;
             } else {
                 // per-slot outputs are stored by permuted position (the
                 // combine finds them through the inverse permutation)
-                nx_sc = __ldg(a.w_perm + tn.seg + ej);
-                nx_row = tn.seg + ej;
+                f.sc = __ldg(a.w_perm + tn.seg + ej);
+                f.row = tn.seg + ej;
             }
+            return f;
         };
-        fetch(0);
+        TileInfo nx = fetch(0), nx2 = fetch(1);
         AccSeq aseq;
         for (int jt = 0; jt < nseq; ++jt) {
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
             const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
-            const float gsc = (!SH && a.g_w) ? nx_gw * a.g_act : 1.0f;
+            const float gsc = (!SH && a.g_w) ? nx.gw * a.g_act : 1.0f;
+            // down: the staging buffer of this tile was last read by the TMA
+            // stores of the tile OUT_BUFS back
+            if (MODE == 1 && ej == 0) {
+                if (C::OUT_BUFS == 2) bulk_wait_read<1>();
+                else bulk_wait_read<0>();
+            }
             epi_sync();                                      // the previous tile's readers are done
             if (ej == 0) ep_stop = abort_flag;
             if (MODE != 2 && ej < t.count) {
-                ep_scale[ej] = nx_sc * gsc;
-                ep_row[ej] = nx_row;
+                ep_scale[ej] = nx.sc * gsc;
+                ep_row[ej] = nx.row;
             }
-            fetch(jt + 1);
+            nx = nx2;
+            nx2 = fetch(jt + 2);
             epi_sync();
             if (ep_stop) break;
             // a failed wait sets abort_flag: this tile is skipped and all four
@@ -779,6 +819,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 uint32_t r[64];
                 const int nch = (cend - cbeg) >> 4;
                 tmem_ld_chunks(lane_base + cbeg, nch, r);
+                uint16_t* ob = out_s + (jt % C::OUT_BUFS) * (kOutTile / 2);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (q < nch) {
@@ -788,10 +829,11 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                         for (int i = 0; i < 16; ++i) {
                             const int col = cbeg + 16 * q + i;
                             const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                            out_s[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
+                            ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
                         }
                     }
                 }
+                fence_proxy_async_smem();                    // the TMA stores read what this thread wrote
             }
             if constexpr (MODE == 0) {
                 for (int c0 = cbeg; c0 < cend; c0 += 16) {
@@ -836,110 +878,28 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 if (au.mask & 2) mbar_arrive(&acc_empty[1]);
             }
             epi_sync();                                      // staging tile complete
-            uint16_t* dst = MODE == 0 ? reinterpret_cast<uint16_t*>(SH ? a.out_sh : a.out)
-                                      : reinterpret_cast<uint16_t*>(SH ? a.o16_sh : a.o16);
-            const int col0 = t.rb * kBlkN;
-            for (int i = ej; i < t.count * 16; i += kEpiWarps * 32) {
-                const int col = i >> 4, ch = i & 15;
-                const uint4 q = *reinterpret_cast<const uint4*>(out_s + col * kBlkN + ch * 8);
-                *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) = q;
+            if constexpr (MODE == 1) {
+                // the tile's rows (permuted positions, or tokens of the shared
+                // expert) are seg .. seg+count-1
+                if (ej == 0)
+                    store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count,
+                                    reinterpret_cast<const uint8_t*>(out_s + (jt % C::OUT_BUFS) * (kOutTile / 2)));
+            } else {
+                uint16_t* dst = reinterpret_cast<uint16_t*>(SH ? a.out_sh : a.out);
+                const int col0 = t.rb * kBlkN;
+                for (int i = ej; i < t.count * 16; i += kEpiWarps * 32) {
+                    const int col = i >> 4, ch = i & 15;
+                    const uint4 q = *reinterpret_cast<const uint4*>(out_s + col * kBlkN + ch * 8);
+                    *reinterpret_cast<uint4*>(dst + (size_t)ep_row[col] * a.out_ld + col0 + ch * 8) = q;
+                }
             }
         }
+        if (MODE == 1 && ej == 0) bulk_wait_all();          // every store done before the CTA leaves
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
-}
-
-// --------------------------------------------------------------- tile list
-// One CTA of 1024 threads. Tile order: by expert, then row block, then
-// token tile, so that the token tiles of one weight block are consecutive;
-// the shared expert's tiles (all T tokens) come last.
-__global__ void __launch_bounds__(1024) k_build_tiles(const int32_t* __restrict__ counts,
-                                                      const int32_t* __restrict__ offsets, int E, int T, int RB0,
-                                                      int RB1, int has_shared, int grid, GemmTile* __restrict__ tiles,
-                                                      int2* __restrict__ groups, int* __restrict__ num_tiles,
-                                                      size_t cap) {
-    // CTA b builds list b (row blocks RB0: gate/up, RB1: down) in its own
-    // part of the buffers, so both lists come from one launch
-    const int RB = blockIdx.x ? RB1 : RB0;
-    tiles += blockIdx.x * cap;
-    groups += blockIdx.x * cap;
-    num_tiles += 4 * blockIdx.x;
-    __shared__ int sc[1024], sg[1024], s_cnt[1024], s_off[1024];
-    const int e = threadIdx.x;
-    const int cnt = (e < E) ? counts[e] : 0;
-    s_cnt[e] = cnt;
-    s_off[e] = (e < E) ? offsets[e] : 0;
-    const int nt = (cnt + kBN - 1) / kBN;
-    const int mine = nt * RB;
-    sc[e] = mine;
-    sg[e] = ((nt + kGroupTiles - 1) / kGroupTiles) * RB;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        const int v = (e >= o) ? sc[e - o] : 0;
-        const int w = (e >= o) ? sg[e - o] : 0;
-        __syncthreads();
-        sc[e] += v;
-        sg[e] += w;
-        __syncthreads();
-    }
-    const int total = sc[1023], ngroups = sg[1023];
-    // groups: up to kGroupTiles consecutive token tiles of one (expert, row
-    // block), which read the same weight block
-    for (int i = e; i < ngroups; i += 1024) {
-        int lo = 0, hi = 1023;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (sg[mid] > i) hi = mid;
-            else lo = mid + 1;
-        }
-        const int ex = lo;
-        const int ntx = (s_cnt[ex] + kBN - 1) / kBN;
-        const int gpr = (ntx + kGroupTiles - 1) / kGroupTiles;     // groups per row block
-        const int j = i - (sg[ex] - gpr * RB);
-        const int rb = j / gpr, q = j % gpr;
-        groups[i] = make_int2(sc[ex] - ntx * RB + rb * ntx + q * kGroupTiles, min(kGroupTiles, ntx - q * kGroupTiles));
-    }
-    // all threads emit the routed tiles: tile i belongs to the expert whose
-    // inclusive prefix is the first one above i (binary search)
-    for (int i = e; i < total; i += 1024) {
-        int lo = 0, hi = 1023;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (sc[mid] > i) hi = mid;
-            else lo = mid + 1;
-        }
-        const int ex = lo;
-        const int c = s_cnt[ex];
-        const int ntx = (c + kBN - 1) / kBN;
-        const int j = i - (sc[ex] - ntx * RB);          // index within the expert's tiles
-        const int rb = j / ntx, tt = j % ntx;
-        GemmTile g;
-        g.expert = ex;
-        g.rb = rb;
-        g.seg = s_off[ex] + tt * kBN;
-        g.count = min(kBN, c - tt * kBN);
-        tiles[i] = g;
-    }
-    const int nts = has_shared ? (T + kBN - 1) / kBN : 0;
-    for (int i = e; i < nts * RB; i += 1024) {
-        const int rb = i / nts, tt = i % nts;
-        GemmTile g;
-        g.expert = -1;
-        g.rb = rb;
-        g.seg = tt * kBN;
-        g.count = min(kBN, T - tt * kBN);
-        tiles[total + i] = g;
-    }
-    if (e == 0) {
-        num_tiles[0] = total;               // routed tiles
-        num_tiles[1] = total + nts * RB;    // + shared-expert tiles
-        num_tiles[2] = ngroups;
-        // group order when every CTA's tiles fit its shared-memory list
-        num_tiles[3] = ((ngroups + grid - 1) / grid) * kGroupTiles <= kTileCache ? 1 : 0;
-    }
 }
 
 // --------------------------------------------------------------- combine
@@ -1116,11 +1076,6 @@ MOE_DEV void load_fp4_token_rows(uint8_t* dst_codes, const Fp4BMaps& mb, int x_c
         }
 }
 
-// Store maps of the per-slot output [slots][H] fp16 with boxes of 128 / 2^i
-// rows x 128 columns: a tile's n rows leave as at most eight TMA stores.
-struct OMaps {
-    CUtensorMap m[8];
-};
 
 constexpr int kFp4SmallN = 48;               // tokens of the gate/up small accumulator
 
@@ -1345,36 +1300,47 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         const int ej = threadIdx.x - C::EPI0 * 32;
         const int cset = (warp - C::EPI0) >> 2;              // this warp's quarter of the token columns
         uint8_t* out_s = smem + C::OUT;
-        // the next tile's token info (routing weight, output row) and its
-        // expert's global scale, loaded while the current tile is processed
-        float nx_sc = 1.0f, nx_gw = 0.0f;
-        int nx_row = 0;
-        auto fetch = [&](int jn) {
-            if (jn >= nseq) return;
-            const GemmTile tn = tile_at(jn);
-            nx_gw = __ldg(a.g_w + tn.expert);
-            if (ej >= tn.count) return;
-            nx_sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
-            nx_row = tn.seg + ej;
+        // token info (routing weight, output row) and expert global scale
+        // of the tiles two and one ahead, loaded while the current tile is
+        // processed (the routing weights are HBM reads by then)
+        struct TileInfo {
+            float sc, gw;
+            int row;
         };
-        fetch(0);
+        auto fetch = [&](int jn) {
+            TileInfo f{1.0f, 0.0f, 0};
+            if (jn >= nseq) return f;
+            const GemmTile tn = tile_at(jn);
+            f.gw = __ldg(a.g_w + tn.expert);
+            if (ej >= tn.count) return f;
+            f.sc = MODE == 0 ? 1.0f : __ldg(a.w_perm + tn.seg + ej);
+            f.row = tn.seg + ej;
+            return f;
+        };
+        // (gate/up reads only the small table of global scales: one tile ahead)
+        TileInfo nx = fetch(0), nx2 = MODE == 1 ? fetch(1) : TileInfo{1.0f, 0.0f, 0};
         int local = 0;
         Fp4AccSeq aseq;
         for (int jt = 0; jt < nseq; ++jt, ++local) {
             const GemmTile t = tile_at(jt);
             const Fp4Acc acc = fp4_acc_next<MODE>(aseq, (t.count + 15) & ~15);
             const int ab = acc.buf;
-            const float gsc = nx_gw * a.g_act;
+            const float gsc = nx.gw * a.g_act;
             // down: this tile's staging buffer was last read by the TMA store
             // of the tile two back (one bulk group per tile)
             if (MODE == 1 && ej == 0) bulk_wait_read<1>();
             epi_sync_n<C::EPI_WARPS>();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
-                ep_scale[ej] = nx_sc * gsc;
-                ep_row[ej] = nx_row;
+                ep_scale[ej] = nx.sc * gsc;
+                ep_row[ej] = nx.row;
             }
-            fetch(jt + 1);
+            if constexpr (MODE == 1) {
+                nx = nx2;
+                nx2 = fetch(jt + 2);
+            } else {
+                nx = fetch(jt + 1);
+            }
             epi_sync_n<C::EPI_WARPS>();
             if (ep_stop) break;
             if (!warp_wait(&acc_full[ab], acc.parity, &abort_flag, a.err, 16)) continue;
@@ -1487,19 +1453,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
             } else if (ej == 0) {
                 // the tile's rows are the permuted positions seg .. seg+count-1:
                 // TMA stores of boxes of 128, 64, ..., 1 rows, one bulk group
-                const uint8_t* ob = out_s + (local & 1) * kOutTile;
-                if (t.count == kBN) {
-                    tma_store_2d(&map_o.m[0], t.rb * kBlkN, t.seg, ob);
-                } else {
-                    int off = 0;
-#pragma unroll
-                    for (int b = 6; b >= 0; --b)
-                        if ((t.count >> b) & 1) {
-                            tma_store_2d(&map_o.m[7 - b], t.rb * kBlkN, t.seg + off, ob + off * (kBlkN * 2));
-                            off += 1 << b;
-                        }
-                }
-                bulk_commit();
+                store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count, out_s + (local & 1) * kOutTile);
             }
         }
         if (MODE == 1 && ej == 0) bulk_wait_all();     // every store done before the CTA leaves
@@ -1623,6 +1577,13 @@ static bool make_map_store16(CUtensorMap* m, const void* base, uint64_t rows, ui
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The eight store maps (boxes of 128 / 2^i rows) of a 16-bit [rows][cols] output.
+static bool make_omaps(OMaps* mo, const void* base, uint64_t rows, uint64_t cols) {
+    for (int i = 0; i < 8; ++i)
+        if (!make_map_store16(&mo->m[i], base, rows, cols, (uint32_t)(kBN >> i))) return false;
+    return true;
+}
+
 size_t prefill_tile_capacity(int max_tokens, int k, int E, int H, int I) {
     const int RB = (H > I ? H : I) / kBlkN;
     return (size_t)((max_tokens * (size_t)k + kBN - 1) / kBN + E + (max_tokens + kBN - 1) / kBN + 1) * RB;
@@ -1641,31 +1602,36 @@ static int num_sms() {
 
 // One persistent CTA per SM over the routed (SH = false) or the shared (SH =
 // true) tiles of the list.
+// map_o: the down launches' output store maps (unused by the others).
 template <int MODE, bool SH, int Q>
 static cudaError_t launch_gemm_q(const BMaps& map_b, const GemmArgs& g, cudaStream_t st, const CUtensorMap* map_a,
-                                 int grid) {
+                                 int grid, const OMaps& map_o) {
     constexpr int bytes = Cfg<MODE, SH>::ALLOC;
     cudaError_t err =
         cudaFuncSetAttribute(k_grouped_gemm<MODE, SH, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (err != cudaSuccess) return err;
     k_grouped_gemm<MODE, SH, Q><<<grid > 0 ? grid : num_sms(), Cfg<MODE, SH>::THREADS, bytes, st>>>(
-        map_b, map_a ? *map_a : map_b.m[0], g);
+        map_b, map_a ? *map_a : map_b.m[0], map_o, g);
     return cudaGetLastError();
 }
 
 template <int MODE, bool SH>
 static cudaError_t launch_gemm(const BMaps& map_b, const GemmArgs& g, cudaStream_t st,
-                               const CUtensorMap* map_a = nullptr, int grid = 0) {
+                               const CUtensorMap* map_a = nullptr, int grid = 0, const OMaps* map_o = nullptr) {
+    OMaps none;
+    memset(&none, 0, sizeof(none));
+    const OMaps& mo = map_o ? *map_o : none;
+    if (MODE == 1 && !map_o) return cudaErrorInvalidValue;
     if constexpr (SH) {
-        return launch_gemm_q<MODE, true, Q_BF16>(map_b, g, st, map_a, grid);
+        return launch_gemm_q<MODE, true, Q_BF16>(map_b, g, st, map_a, grid, mo);
     } else {
         switch (g.quant) {
-            case Q_INT4: return launch_gemm_q<MODE, false, Q_INT4>(map_b, g, st, map_a, grid);
-            case Q_INT4G32: return launch_gemm_q<MODE, false, Q_INT4G32>(map_b, g, st, map_a, grid);
-            case Q_INT2: return launch_gemm_q<MODE, false, Q_INT2>(map_b, g, st, map_a, grid);
-            case Q_NVFP4: return launch_gemm_q<MODE, false, Q_NVFP4>(map_b, g, st, map_a, grid);
-            case Q_FP8: return launch_gemm_q<MODE, false, Q_FP8>(map_b, g, st, map_a, grid);
-            case Q_FP6: return launch_gemm_q<MODE, false, Q_FP6>(map_b, g, st, map_a, grid);
+            case Q_INT4: return launch_gemm_q<MODE, false, Q_INT4>(map_b, g, st, map_a, grid, mo);
+            case Q_INT4G32: return launch_gemm_q<MODE, false, Q_INT4G32>(map_b, g, st, map_a, grid, mo);
+            case Q_INT2: return launch_gemm_q<MODE, false, Q_INT2>(map_b, g, st, map_a, grid, mo);
+            case Q_NVFP4: return launch_gemm_q<MODE, false, Q_NVFP4>(map_b, g, st, map_a, grid, mo);
+            case Q_FP8: return launch_gemm_q<MODE, false, Q_FP8>(map_b, g, st, map_a, grid, mo);
+            case Q_FP6: return launch_gemm_q<MODE, false, Q_FP6>(map_b, g, st, map_a, grid, mo);
             default: return cudaErrorInvalidValue;
         }
     }
@@ -1726,8 +1692,6 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
         !make_fp4_bmaps(&mb, xc, (uint64_t)slots, H) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<2, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, H / kBlkN, has_sh ? 1 : 0, num_sms(),
-                                     p.tiles, p.groups, p.num_tiles, p.tile_cap);
     GemmArgs g{};
     g.quant = ex.quant;
     g.sh0 = ex.sh_gate;
@@ -1786,12 +1750,13 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.g_w = ex.g_down;
     g.g_act = ex.g_a;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
-    for (int i = 0; i < 8; ++i)
-        if (!make_map_store16(&mo.m[i], p.o, (uint64_t)slots, (uint64_t)H, (uint32_t)(kBN >> i)))
-            return cudaErrorInvalidValue;
+    OMaps mo_sh;
+    if (!make_omaps(&mo, p.o, (uint64_t)slots, (uint64_t)H) ||
+        (has_sh && !make_omaps(&mo_sh, p.o_sh, (uint64_t)T, (uint64_t)H)))
+        return cudaErrorInvalidValue;
     err = launch_fp4<1>(m, mb, mo, g, st);
     if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
-    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st, nullptr, 0, &mo_sh);
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     const long long threads = (long long)T * (H / 8);
@@ -1804,7 +1769,19 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const ExpertArgs& ex = p.ex;
     const int T = p.T, k = ex.k, H = ex.H, I = ex.I, E = ex.E;
     const int slots = T * k;
-    cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st);
+    // the permutation launch also builds both tile lists (gate/up: I / 128
+    // row blocks, down: H / 128)
+    TileListArgs tl{};
+    tl.tiles = p.tiles;
+    tl.groups = p.groups;
+    tl.num_tiles = p.num_tiles;
+    tl.cap = p.tile_cap;
+    tl.T = T;
+    tl.RB0 = I / kBlkN;
+    tl.RB1 = H / kBlkN;
+    tl.has_shared = ex.sh_gate != nullptr ? 1 : 0;
+    tl.grid = num_sms();
+    cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st, &tl);
     if (err != cudaSuccess) return err;
     const bool fp4 = ex.quant == Q_NVFP4;
     // NVFP4 W4A4 on the block-scaled tensor cores when the shapes allow
@@ -1834,8 +1811,6 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (!make_bmaps(&m_routed, p.xp, (uint64_t)slots, (uint64_t)H, xdt) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
-    k_build_tiles<<<2, 1024, 0, st>>>(p.counts, p.offsets, E, T, I / kBlkN, H / kBlkN, has_sh ? 1 : 0, num_sms(),
-                                     p.tiles, p.groups, p.num_tiles, p.tile_cap);
     GemmArgs g{};
     g.quant = ex.quant;
     g.w0 = ex.gate;
@@ -1886,10 +1861,14 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     g.g_act = fp4 ? ex.g_a : 1.0f;
     g.tok_scale = nullptr;
     g.ts_perm = nullptr;
+    OMaps mo, mo_sh;
+    if (!make_omaps(&mo, p.o, (uint64_t)slots, (uint64_t)H) ||
+        (has_sh && !make_omaps(&mo_sh, p.o_sh, (uint64_t)T, (uint64_t)H)))
+        return cudaErrorInvalidValue;
     if (p.ev_dn0) cudaEventRecord(p.ev_dn0, st);
-    err = launch_gemm<1, false>(m_routed, g, st);
+    err = launch_gemm<1, false>(m_routed, g, st, nullptr, 0, &mo);
     if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
-    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st);
+    if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st, nullptr, 0, &mo_sh);
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     // ---- combine

@@ -46,8 +46,30 @@ cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E,
 void set_thread_error(const char* msg);
 
 // permute.cu
+// One tile of a grouped GEMM: (expert, 128-row weight block, up to 128
+// consecutive permuted positions).
+struct GemmTile {
+    int expert;   // routed expert, or -1 for the shared expert
+    int rb;       // 128-row block of the weight matrix
+    int seg;      // first row of the segment (permuted position, or token for shared)
+    int count;    // tokens in this tile
+};
+// The grouped GEMMs' tile lists, built by the permutation launch from the
+// expert counts it computes: list 0 (gate/up, RB0 row blocks) and list 1
+// (down, RB1 row blocks), each of cap entries with its group list and four
+// counts (routed tiles, all tiles, routed groups, group order).
+struct TileListArgs {
+    GemmTile* tiles;               // [2][cap]
+    int2* groups;                  // [2][cap]
+    int* num_tiles;                // [2][4]
+    size_t cap;
+    int T, RB0, RB1, has_shared;
+    int grid;                      // CTAs of the GEMM launches
+};
+// tl may be null (permutation only)
 cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* perm, int32_t* inv, int32_t* chunk_scratch, cudaStream_t st);
+                           int32_t* perm, int32_t* inv, int32_t* chunk_scratch, cudaStream_t st,
+                           const TileListArgs* tl = nullptr);
 size_t permute_scratch_ints(int slots, int E);
 
 // decode.cu (small-T path) and segment path
@@ -99,12 +121,6 @@ cudaError_t launch_decode_fused(const FusedArgs& f, cudaStream_t st);   // cudaE
 bool fused_supported(int T, int H, int I, int quant);
 
 // grouped_gemm.cu (prefill path)
-struct GemmTile {
-    int expert;   // routed expert, or -1 for the shared expert
-    int rb;       // 128-row block of the weight matrix
-    int seg;      // first row of the segment (permuted position, or token for shared)
-    int count;    // tokens in this tile
-};
 struct PrefillArgs {
     ExpertArgs ex;
     const void* x;                 // bf16 [T, H]

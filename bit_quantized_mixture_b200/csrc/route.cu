@@ -23,15 +23,30 @@ MOE_DEV uint32_t order_key(float v) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Inverse of order_key.
+MOE_DEV float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+constexpr int kTopkWarps = 8;        // warps of a CTA with shared candidate lists
+
 // One warp selects the top-k of one token's logits (E <= 1024 values read
-// through L2, expert e held by lane e % 32) and writes ids / weights.  Each
-// lane keeps the best of its own live keys (largest key, smallest expert on
-// equal keys); a round takes the warp maximum of those with one
-// max-reduction and, among lanes holding it, the smallest expert with one
-// min-reduction; only the lane that lost its key rescans its slots.
+// through L2, expert e held by lane e % 32) and writes ids / weights, in the
+// order key descending, expert ascending on equal keys.
+//
+// Threshold selection: the k-th largest of the 32 lanes' own maxima, t, is
+// reached by at least k logits, so every selected expert is among the
+// logits >= t (about 12 of 512 for continuous logits).  Those candidates are
+// gathered into the warp's shared list and each is ranked exactly by
+// counting the candidates ahead of it.  With more than 32 candidates (many
+// equal logits), or without a shared list, selection rounds run instead:
+// each lane keeps the best of its own live keys, a round takes the warp
+// maximum with one max-reduction and, among lanes holding it, the smallest
+// expert with one min-reduction; only the lane that lost its key rescans.
+// sk / se: 64 entries of this warp's shared memory each, or null.
 template <int SLOTS>
 MOE_DEV void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                         float* __restrict__ wout) {
+                         float* __restrict__ wout, uint32_t* sk, int* se) {
     const int lane = threadIdx.x & 31;
     uint32_t key[SLOTS];
 #pragma unroll
@@ -42,33 +57,93 @@ MOE_DEV void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* _
     uint32_t live = 0;
 #pragma unroll
     for (int i = 0; i < SLOTS; ++i) live |= ((lane + 32 * i) < E ? 1u : 0u) << i;
-    // best live key of this lane and its slot (first slot on equal keys)
-    auto rescan = [&](uint32_t& best, int& slot) {
-        best = 0;
-        slot = -1;
-#pragma unroll
-        for (int i = 0; i < SLOTS; ++i)
-            if (((live >> i) & 1u) && (slot < 0 || key[i] > best)) {
-                best = key[i];
-                slot = i;
-            }
-    };
-    uint32_t best;
-    int slot;
-    rescan(best, slot);
     float my_val = 0.0f, lmax = 0.0f;
     int my_idx = 0;
-    for (int j = 0; j < k; ++j) {
-        const uint32_t top = __reduce_max_sync(0xffffffffu, slot >= 0 ? best : 0u);
-        const uint32_t mine = (slot >= 0 && best == top) ? (uint32_t)(lane + 32 * slot) : 0xffffffffu;
-        const uint32_t e = __reduce_min_sync(0xffffffffu, mine);
-        if ((int)(e & 31u) == lane) {
-            live &= ~(1u << (e >> 5));
-            rescan(best, slot);
+    bool done = false;
+    if (sk != nullptr) {
+        uint32_t m = 0;                      // the lane's largest key
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i)
+            if ((live >> i) & 1u) m = max(m, key[i]);
+        // t: the k-th largest lane maximum (each round retires the lowest
+        // lane holding the current maximum)
+        bool alive = live != 0;
+        uint32_t t = 0;
+        for (int r = 0; r < k; ++r) {
+            t = __reduce_max_sync(0xffffffffu, alive ? m : 0u);
+            const unsigned hold = __ballot_sync(0xffffffffu, alive && m == t);
+            if (lane == __ffs(hold) - 1) alive = false;
         }
-        const float v = __uint_as_float((top & 0x80000000u) ? (top & 0x7fffffffu) : ~top);   // key -> value
-        if (j == 0) lmax = v;
-        if (lane == j) { my_val = v; my_idx = (int)e; }
+        unsigned cm = 0;                     // the lane's candidates
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i) cm |= (((live >> i) & 1u) && key[i] >= t) ? (1u << i) : 0u;
+        const int cl = __popc(cm);
+        int incl = cl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const int C = __shfl_sync(0xffffffffu, incl, 31);
+        if (C <= 32) {
+            int p = incl - cl;
+#pragma unroll
+            for (int i = 0; i < SLOTS; ++i)
+                if ((cm >> i) & 1u) {
+                    sk[p] = key[i];
+                    se[p] = lane + 32 * i;
+                    ++p;
+                }
+            __syncwarp();
+            const uint32_t mk = lane < C ? sk[lane] : 0u;
+            const int me = lane < C ? se[lane] : 0x7fffffff;
+            int rank = 0;                    // candidates ahead of this lane's
+            for (int j = 0; j < C; ++j) {
+                const uint32_t kj = sk[j];
+                const int ej = se[j];
+                rank += (kj > mk || (kj == mk && ej < me)) ? 1 : 0;
+            }
+            if (lane < C && rank < k) {
+                sk[32 + rank] = mk;
+                se[32 + rank] = me;
+            }
+            __syncwarp();
+            if (lane < k) {
+                my_val = key_value(sk[32 + lane]);
+                my_idx = se[32 + lane];
+            }
+            lmax = key_value(sk[32]);
+            __syncwarp();                    // the list is free for the warp's next token
+            done = true;
+        }
+    }
+    if (!done) {
+        // best live key of this lane and its slot (first slot on equal keys)
+        auto rescan = [&](uint32_t& best, int& slot) {
+            best = 0;
+            slot = -1;
+#pragma unroll
+            for (int i = 0; i < SLOTS; ++i)
+                if (((live >> i) & 1u) && (slot < 0 || key[i] > best)) {
+                    best = key[i];
+                    slot = i;
+                }
+        };
+        uint32_t best;
+        int slot;
+        rescan(best, slot);
+        for (int j = 0; j < k; ++j) {
+            const uint32_t top = __reduce_max_sync(0xffffffffu, slot >= 0 ? best : 0u);
+            const uint32_t mine = (slot >= 0 && best == top) ? (uint32_t)(lane + 32 * slot) : 0xffffffffu;
+            const uint32_t e = __reduce_min_sync(0xffffffffu, mine);
+            if ((int)(e & 31u) == lane) {
+                live &= ~(1u << (e >> 5));
+                rescan(best, slot);
+            }
+            const float v = key_value(top);
+            if (j == 0) lmax = v;
+            if (lane == j) { my_val = v; my_idx = (int)e; }
+        }
     }
     const float ex = (lane < k) ? expf(my_val - lmax) : 0.0f;
     const float sum = warp_sum(ex);
@@ -78,11 +153,17 @@ MOE_DEV void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* _
     }
 }
 
-// E <= 512: 16 slots per lane; E <= 1024: 32
+// E <= 512: 16 slots per lane; E <= 1024: 32.  Warps beyond kTopkWarps of
+// their CTA take the selection rounds.
 MOE_DEV void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
                        float* __restrict__ wout) {
-    if (E <= 512) warp_topk_n<16>(row, E, k, ids, wout);
-    else warp_topk_n<32>(row, E, k, ids, wout);
+    __shared__ uint32_t s_key[kTopkWarps][64];
+    __shared__ int s_exp[kTopkWarps][64];
+    const int w = threadIdx.x >> 5;
+    uint32_t* sk = w < kTopkWarps ? s_key[w] : nullptr;
+    int* se = w < kTopkWarps ? s_exp[w] : nullptr;
+    if (E <= 512) warp_topk_n<16>(row, E, k, ids, wout, sk, se);
+    else warp_topk_n<32>(row, E, k, ids, wout, sk, se);
 }
 
 // Decode router (T <= 8): one warp per expert row, a grid-wide ticket lets

@@ -213,7 +213,9 @@ moe_status moe_quantize_act_nvfp4(const void* x, int32_t T, int32_t K, float g,
 /* Token permutation of the flat slots s = t*k + j into expert-major order,
  * stable in s: counts int32 [E], offsets int32 [E+1], perm int32 [T*k]
  * (slot at each permuted position), inv int32 [T*k] (position of each slot).
- * ids must lie in [0, E).  Uses no handle; deterministic. */
+ * A slot whose id lies outside [0, E) gets no position: its inv entry is -1,
+ * it is not counted, and only the first offsets[E] entries of perm are
+ * written.  T*k <= 2^30, 1 <= E <= 1024.  Uses no handle; deterministic. */
 moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                        moe_stream_t stream);

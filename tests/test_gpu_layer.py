@@ -89,6 +89,37 @@ def test_route_from_logits_ties_and_order():
     layer.close()
 
 
+# the threshold selection (candidates ranked in a shared list) and its
+# fallback to selection rounds (more than 32 candidates): continuous logits,
+# coarse grids with ties at the threshold, all logits equal, the smallest and
+# largest E and k, and E = 1024 (32 logits per lane)
+@pytest.mark.parametrize("E,k,kind", [(512, 10, "normal"), (512, 10, "grid"), (512, 10, "fine"), (512, 10, "equal"),
+                                      (512, 1, "normal"),
+                                      (1024, 10, "normal"), (1024, 32, "grid"), (32, 32, "normal"), (7, 3, "grid"),
+                                      (600, 10, "normal")])
+def test_route_from_logits_selection_paths(E, k, kind):
+    T = 333
+    wl = synth.custom("tiny-int4", T=T, E=E, k=k)
+    layer = moe.MoeLayer(wl.H, wl.I, wl.E, wl.k, "int4", False, T, 0)
+    rng = np.random.default_rng(E * 37 + k)
+    if kind == "normal":
+        L = rng.standard_normal((T, E)).astype(np.float32)
+    elif kind == "grid":
+        L = rng.integers(-6, 7, size=(T, E)).astype(np.float32) * np.float32(0.25)
+    elif kind == "fine":
+        L = rng.integers(-100, 101, size=(T, E)).astype(np.float32) * np.float32(0.03125)
+    else:
+        L = np.full((T, E), 0.5, dtype=np.float32)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    layer.route_from_logits(torch.from_numpy(L).to(DEV), ids, w)
+    torch.cuda.synchronize()
+    rid, rw = O.route_topk(L, k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+    layer.close()
+
+
 @pytest.mark.parametrize("wl_name", ["prefill-int4-zipf", "prefill-nvfp4"])
 def test_route_from_logits_full_size(wl_name):
     wl = synth.workload(wl_name)
@@ -115,6 +146,37 @@ def test_permute_bit_exact(T, k, E):
     assert np.array_equal(counts.cpu().numpy(), rc)
     assert np.array_equal(offsets.cpu().numpy(), ro)
     assert np.array_equal(perm.cpu().numpy(), rp)
+    assert np.array_equal(inv.cpu().numpy(), ri)
+
+
+# chunks of 2048 slots (more than 128 x 1024 slots), the largest E, an E
+# that is not a multiple of 32, every token on the same k experts (one
+# segment spans all warps and chunks), and ids outside [0, E) (dropped)
+@pytest.mark.parametrize("case", ["chunk2048", "e1024", "e7", "same_experts", "invalid_ids"])
+def test_permute_bit_exact_edge_cases(case):
+    rng = np.random.default_rng(7)
+    if case == "chunk2048":
+        T, k, E = 20000, 10, 512
+    elif case == "e1024":
+        T, k, E = 3000, 8, 1024
+    elif case == "e7":
+        T, k, E = 1000, 3, 7
+    else:
+        T, k, E = 5000, 10, 512
+    if case == "same_experts":
+        ids = np.tile(np.arange(k, dtype=np.int32)[::-1], (T, 1))
+    else:
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    if case == "invalid_ids":
+        mask = rng.random(ids.shape) < 0.05
+        ids[mask] = rng.choice(np.array([-1, E, E + 100, -(1 << 30)], dtype=np.int32), int(mask.sum()))
+    counts, offsets, perm, inv = moe.permute(torch.from_numpy(ids).to(DEV), E)
+    torch.cuda.synchronize()
+    rc, ro, rp, ri = O.permute(ids, E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    n = int(ro[-1])
+    assert np.array_equal(perm.cpu().numpy()[:n], rp[:n])
     assert np.array_equal(inv.cpu().numpy(), ri)
 
 
