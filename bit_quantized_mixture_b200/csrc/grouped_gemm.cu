@@ -179,13 +179,13 @@ struct GemmArgs {
     const float* ts_perm;     // INT4/INT2 gate/up: token scale of each permuted position
     uint8_t* out4;            // NVFP4 gate/up: e2m1 intermediate [slots, I/2] (permuted rows)
     uint8_t* out_sf;          // NVFP4 gate/up: its e4m3 block scales, stage-major [I/256][slots][16]
-    // NVFP4 block-scaled GEMMs: the e4m3 scales of the weights (per matrix)
-    // and of the token operand, stage-major [K/256][rows][16 B] with
-    // sfa_rows = E * N and sfb_rows = slots rows per stage
-    const uint8_t* sfa0;
-    const uint8_t* sfa1;
+    // NVFP4 block-scaled GEMMs: the weight image (per expert, 128-row block
+    // and 256-value stage one block of NMAT swizzled 16 KB code tiles and
+    // NMAT 2 KB scale tiles), and the e4m3 scales of the token operand,
+    // stage-major [K/256][rows][16 B] with sfb_rows = slots rows per stage
+    const uint8_t* wimg;
     const uint8_t* sfb;
-    long long sfa_rows, sfb_rows;
+    long long sfb_rows;
     long long sfb_rows_out;   // NVFP4 gate/up: rows per stage of out_sf (the slots)
     int* err;
 };
@@ -1056,28 +1056,21 @@ constexpr int kFp4Tile = 128 * 128;          // 16 KB: 128 rows x 128 bytes
 constexpr int kFp4SfTile = 128 * 16;         // 2 KB: 128 rows x 16 scale bytes
 
 // Token-operand maps of the block-scaled GEMM (e2m1 codes, 128-byte rows,
-// 128-byte swizzle) with boxes of 128, 64, 32 and 16 rows: a tile of n (a
-// multiple of 16) tokens loads only its rows.
+// 128-byte swizzle) with boxes of 16, 32, ..., 176 rows: a tile of n (a
+// multiple of 16) tokens loads exactly its rows with one TMA request (the
+// copy engine's requests per SM, not bytes, bound these GEMMs' streaming).
 struct Fp4BMaps {
-    CUtensorMap codes[4];
+    CUtensorMap codes[11];  // box rows 16 (i + 1), up to a gate/up tile's 176
 };
 MOE_DEV void load_fp4_token_rows(uint8_t* dst_codes, const Fp4BMaps& mb, int x_codes, int y, int n, uint64_t* bar) {
-    const int n16 = n >> 4;
-    if (n16 >= 8) {
-        tma_load_2d(dst_codes, &mb.codes[0], x_codes, y, bar);
-        return;
-    }
-    int off = 0;
-#pragma unroll
-    for (int b = 2; b >= 0; --b)
-        if (n16 & (1 << b)) {
-            tma_load_2d(dst_codes + off * 128, &mb.codes[3 - b], x_codes, y + off, bar);
-            off += 16 << b;
-        }
+    tma_load_2d(dst_codes, &mb.codes[(n >> 4) - 1], x_codes, y, bar);
 }
 
 
-constexpr int kFp4SmallN = 48;               // tokens of the gate/up small accumulator
+// Tokens per gate/up tile (the MMA's N, at most 256): an expert's ~160 tokens
+// of the uniform workload are one tile, so each weight block streams once.
+// (Down keeps 128: its accumulators alternate between two tiles.)
+constexpr int kFp4GuN = 176;
 
 // The accumulator of the next tile, walked identically by the MMA warps and
 // the epilogue: buffer, first column, matrix stride and phase parity.
@@ -1092,18 +1085,15 @@ struct Fp4AccSeq {
 template <int MODE>
 MOE_DEV Fp4Acc fp4_acc_next(Fp4AccSeq& q, int n_mma) {
     Fp4Acc a;
+    (void)n_mma;
     if (MODE == 1) {
         a.buf = q.local & 1;
         a.col = (uint32_t)(a.buf * kBN);
         a.mat_stride = kBN;
-    } else if (n_mma <= kFp4SmallN) {
-        a.buf = 1;
-        a.col = 2 * kBN;
-        a.mat_stride = kFp4SmallN;
     } else {
         a.buf = 0;
         a.col = 0;
-        a.mat_stride = kBN;
+        a.mat_stride = kFp4GuN;
     }
     a.parity = (a.buf ? q.uses1 : q.uses0) & 1u;
     q.uses0 += a.buf == 0 ? 1u : 0u;
@@ -1123,39 +1113,52 @@ struct Fp4Cfg {
     // staging of a tile is the longest step of these kernels)
     static constexpr int EPI_WARPS = 16;
     static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
-    // accumulators: gate/up keeps one of 2 x 128 columns and a small one of
-    // 2 x kFp4SmallN columns for tiles of at most kFp4SmallN tokens, so that
-    // such a tile and its neighbours take turns; down alternates two of 128
-    static constexpr int ACC_BUFS = 2;
-    static constexpr int ACC_COLS = NMAT * kBN;
-    static constexpr int SF_COL0 = MODE == 0 ? ACC_COLS + 2 * kFp4SmallN : 2 * ACC_COLS;
-    static constexpr int SF_STAGE_COLS = (NMAT + 1) * 16;             // A per matrix, then B; 4 MMAs x 4 columns
-    static_assert(SF_COL0 + S * SF_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
-    static constexpr int A = 0;                                       // [S][NMAT][16 KB]
-    static constexpr int B = A + S * NMAT * kFp4Tile;                 // [S][16 KB]
-    static constexpr int SFA = B + S * kFp4Tile;                      // [S][NMAT][2 KB]
-    static constexpr int SFB = SFA + S * NMAT * kFp4SfTile;           // [S][2 KB]
-    static constexpr int OUT = SFB + S * kFp4SfTile;                  // gate/up: [128][80 B]; down: 2 x [128][128] fp16
-    static constexpr int OUT_BYTES = MODE == 0 ? kBN * 80 : 2 * kOutTile;
-    static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [16 tok][32] fp32
-    static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 16 * 32 * 4 : 0;
+    // token rows per tile: gate/up kFp4GuN, down 128
+    static constexpr int BROWS = MODE == 0 ? kFp4GuN : kBN;
+    // accumulators: gate/up one of 2 x kFp4GuN columns (the epilogue reads
+    // it and releases it before the requantization); down alternates two of
+    // 128
+    static constexpr int ACC_COLS = NMAT * BROWS;
+    // scale factors in TMEM: per slot, A (4 columns per MMA and matrix), then
+    // B (ceil(rows / 32) columns per MMA, at 8-column steps for 176 rows);
+    // gate/up keeps two slots (released by their own MMA commits), down one
+    // per stage
+    static constexpr int SFB_KK = MODE == 0 ? 8 : 4;
+    static constexpr int SF_STAGE_COLS = NMAT * 16 + 4 * SFB_KK;
+    static constexpr int SF_SLOTS = MODE == 0 ? 2 : S;
+    static constexpr int SF_COL0 = MODE == 0 ? ACC_COLS : 2 * ACC_COLS;
+    static_assert(SF_COL0 + SF_SLOTS * SF_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
+    // weights: per stage one block of the image, [NMAT][16 KB codes] then
+    // [NMAT][2 KB scales] (a multiple of 1 KB: every code tile stays aligned
+    // for the 128-byte swizzle)
+    static constexpr int W_STAGE = NMAT * (kFp4Tile + kFp4SfTile);
+    static constexpr int B_STAGE = BROWS * 128;                       // a multiple of 1 KB
+    // token scales: rows 32c + lane of each 32-row column group are read, so
+    // a stage's tile spans whole groups
+    static constexpr int SFB_STAGE = ((BROWS + 31) / 32) * 32 * 16;
+    static constexpr int W = 0;                                       // [S][W_STAGE]
+    static constexpr int B = W + S * W_STAGE;                         // [S][B_STAGE]
+    static constexpr int SFB = B + S * B_STAGE;                       // [S][SFB_STAGE]
+    static constexpr int OUT = SFB + S * SFB_STAGE;                   // gate/up: [BROWS][80 B]; down: 2 x [128][128] fp16
+    static constexpr int OUT_BYTES = MODE == 0 ? BROWS * 80 : 2 * kOutTile;
+    static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [8 tok][32] fp32
+    static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 8 * 32 * 4 : 0;
     static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
     static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
 
 template <int MODE>
 __global__ void __launch_bounds__(Fp4Cfg<MODE>::THREADS, 1)
-k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
-           const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps map_o, GemmArgs a) {
+k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps map_o, GemmArgs a) {
     using C = Fp4Cfg<MODE>;
     constexpr int NMAT = C::NMAT, S = C::S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[S], sfready[S], empty[S], acc_full[2], acc_empty[2];
+    __shared__ uint64_t full[S], sfready[S], empty[S], acc_full[2], acc_empty[2], sffree[2];
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
-    __shared__ float ep_scale[kBN];
-    __shared__ int ep_row[kBN];
+    __shared__ float ep_scale[kFp4GuN];
+    __shared__ int ep_row[kFp4GuN];
     __shared__ int ep_stop;
     __shared__ float rcp_tab[256];              // gate/up: 1 / (e4m3(code) * g_req), IEEE division, 0 for zero
     __shared__ TileCache tcache;
@@ -1177,6 +1180,7 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], NMAT);
             mbar_init(&acc_empty[b], C::EPI_WARPS);
+            mbar_init(&sffree[b], NMAT);                  // gate/up: one commit per MMA warp
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -1196,28 +1200,25 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
         int g = 0;
         for (int jt = 0; jt < nseq && !abort_flag; ++jt) {
             const GemmTile t = tile_at(jt);
-            const int arow = t.expert * a.n_rows + t.rb * kBlkN;
+            // this (expert, row block)'s NS consecutive image blocks
+            const uint8_t* wblk = a.wimg + ((size_t)t.expert * (a.n_rows / kBlkN) + t.rb) * NS * C::W_STAGE;
             bool ok = true;
             for (int ks = 0; ks < NS; ++ks, ++g) {
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
                 if (!warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 11)) { ok = false; break; }
                 if (lane == 0) {
-                    // the weight tiles and their scales, then the tile's token rows
+                    // the stage's weight codes and scales (one bulk copy),
+                    // then the tile's token rows and their scales
                     const int n_mma = (t.count + 15) & ~15;
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * (kFp4Tile + kFp4SfTile)) + (uint32_t)n_mma * 144u);
-                    for (int m = 0; m < NMAT; ++m) {
-                        tma_load_2d(smem + C::A + (s * NMAT + m) * kFp4Tile, m == 0 ? &map_a0 : &map_a1, ks * 128, arow,
-                                    &full[s]);
-                        // the stage's scale tile: 128 rows x 16 B, contiguous (stage-major)
-                        bulk_g2s(smem + C::SFA + (s * NMAT + m) * kFp4SfTile,
-                                 (m == 0 ? a.sfa0 : a.sfa1) + ((size_t)ks * a.sfa_rows + arow) * 16, kFp4SfTile, &full[s]);
-                    }
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)C::W_STAGE + (uint32_t)n_mma * 144u);
+                    bulk_g2s(smem + C::W + s * C::W_STAGE, wblk + (size_t)ks * C::W_STAGE, (uint32_t)C::W_STAGE,
+                             &full[s]);
                     // the token rows' scales: n_mma x 16 B, contiguous (rows past
                     // the end of the slots read workspace slack, never used)
-                    bulk_g2s(smem + C::SFB + s * kFp4SfTile, a.sfb + ((size_t)ks * a.sfb_rows + t.seg) * 16,
+                    bulk_g2s(smem + C::SFB + s * C::SFB_STAGE, a.sfb + ((size_t)ks * a.sfb_rows + t.seg) * 16,
                              (uint32_t)n_mma * 16u, &full[s]);
-                    load_fp4_token_rows(smem + C::B + s * kFp4Tile, map_b, ks * 128, t.seg, n_mma, &full[s]);
+                    load_fp4_token_rows(smem + C::B + s * C::B_STAGE, map_b, ks * 128, t.seg, n_mma, &full[s]);
                 }
                 __syncwarp();
             }
@@ -1245,14 +1246,16 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 if (!warp_wait(&sfready[s], r & 1u, &abort_flag, a.err, 14)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t adesc = desc_kmajor_sw128(smem_u32(smem + C::A + (s * NMAT + mi) * kFp4Tile));
-                    const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + s * kFp4Tile));
-                    const uint32_t sf = tmem + C::SF_COL0 + s * C::SF_STAGE_COLS;
+                    const uint64_t adesc = desc_kmajor_sw128(smem_u32(smem + C::W + s * C::W_STAGE + mi * kFp4Tile));
+                    const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + s * C::B_STAGE));
+                    const int slot = g % C::SF_SLOTS;
+                    const uint32_t sf = tmem + C::SF_COL0 + slot * C::SF_STAGE_COLS;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_fp4_block16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, sf + mi * 16 + kk * 4,
-                                        sf + NMAT * 16 + kk * 4, (ks | kk) != 0);
+                                        sf + NMAT * 16 + kk * C::SFB_KK, (ks | kk) != 0);
                     mma_commit(&empty[s]);
+                    if (MODE == 0) mma_commit(&sffree[slot]);     // this slot's scales are consumed
                     if (ks == NS - 1) mma_commit(&acc_full[ab]);
                 }
                 __syncwarp();
@@ -1270,21 +1273,52 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
                 if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 15)) { ok = false; break; }
+                // gate/up: the TMEM slot is free once the MMAs of stage g - 2 are done
+                const int slot = g % C::SF_SLOTS;
+                if (MODE == 0 && g >= C::SF_SLOTS &&
+                    !warp_wait(&sffree[slot], (uint32_t)((g / C::SF_SLOTS - 1) & 1), &abort_flag, a.err, 17)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t sf = tmem + lane_addr + C::SF_COL0 + s * C::SF_STAGE_COLS;
+                const uint32_t sf = tmem + lane_addr + C::SF_COL0 + slot * C::SF_STAGE_COLS;
+                // column 4 kk + cc (A) / SFB_KK kk + cc (B): the scales of
+                // K-blocks 4kk..4kk+3 of row 32cc + lane
 #pragma unroll
-                for (int q = 0; q <= NMAT; ++q) {
-                    const uint8_t* tile = q < NMAT ? smem + C::SFA + (s * NMAT + q) * kFp4SfTile : smem + C::SFB + s * kFp4SfTile;
+                for (int q = 0; q < NMAT; ++q) {
+                    const uint8_t* tile = smem + C::W + s * C::W_STAGE + NMAT * kFp4Tile + q * kFp4SfTile;
                     uint32_t v[16];
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
                         const uint4 w = *reinterpret_cast<const uint4*>(tile + (32 * cc + lane) * 16);
-                        v[0 * 4 + cc] = w.x;      // column 4 kk + cc: scales of K-blocks 4kk..4kk+3 of row 32cc + lane
+                        v[0 * 4 + cc] = w.x;
                         v[1 * 4 + cc] = w.y;
                         v[2 * 4 + cc] = w.z;
                         v[3 * 4 + cc] = w.w;
                     }
                     tmem_st16(sf + q * 16, v);
+                }
+                {
+                    const uint8_t* tile = smem + C::SFB + s * C::SFB_STAGE;
+                    constexpr int CB = C::SFB_STAGE / (32 * 16);           // 32-row groups of the B tile
+                    uint32_t v[4 * C::SFB_KK];
+#pragma unroll
+                    for (int i = 0; i < 4 * C::SFB_KK; ++i) v[i] = 0u;
+#pragma unroll
+                    for (int cc = 0; cc < CB; ++cc) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(tile + (32 * cc + lane) * 16);
+                        v[0 * C::SFB_KK + cc] = w.x;
+                        v[1 * C::SFB_KK + cc] = w.y;
+                        v[2 * C::SFB_KK + cc] = w.z;
+                        v[3 * C::SFB_KK + cc] = w.w;
+                    }
+#pragma unroll
+                    for (int h = 0; h < C::SFB_KK / 4; ++h) {
+                        uint32_t u[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) u[i] = v[16 * h + i];
+                        tmem_st16(sf + NMAT * 16 + 16 * h, u);
+                    }
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -1378,12 +1412,12 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 }
                 fence_proxy_async_smem();        // the TMA store reads what this thread wrote
             } else {
-                static_assert(C::EPI_WARPS == 16, "gate/up: at most 32 columns per warp");
-                // SwiGLU as each 16-column chunk is read: only the 2 x 16
+                static_assert(C::EPI_WARPS == 16 && kFp4GuN <= 192, "gate/up: at most 48 columns per warp");
+                // SwiGLU as each 16-column chunk is read: only the 3 x 16
                 // results stay live across the release
-                float act[2][16];
+                float act[3][16];
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < 3; ++q) {
                     if (q < nch) {
                         const int c0 = cbeg + 16 * q;
                         float vg[16], vu[16];
@@ -1398,41 +1432,45 @@ k_fp4_gemm(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ C
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                // the warp's scratch [16 tokens][32 outputs] turns the results
-                // into 16-output blocks per lane for the requantization
-                float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 16 * 32;
+                // the warp's scratch [8 tokens][32 outputs] turns the results
+                // into 16-output blocks per lane for the requantization, eight
+                // tokens at a time (lanes 0..15: token i, block b)
+                float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 8 * 32;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < 3; ++q) {
                     if (q < nch) {
-                        const int c0 = cbeg + 16 * q;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) scr[i * 32 + lane] = act[q][i];
-                        __syncwarp();
-                        // lane = (token i, 16-output block b): NVFP4 with the static global
-                        // scale; code decisions in fp32 as the format defines them
-                        {
-                            const int i = lane & 15, b = lane >> 4;
-                            const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
-                            float v[16];
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c0 = cbeg + 16 * q + 8 * hh;
 #pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                const float4 f4 = src[qq];
-                                v[4 * qq] = f4.x; v[4 * qq + 1] = f4.y; v[4 * qq + 2] = f4.z; v[4 * qq + 3] = f4.w;
+                            for (int i = 0; i < 8; ++i) scr[i * 32 + lane] = act[q][8 * hh + i];
+                            __syncwarp();
+                            // lane = (token i, 16-output block b): NVFP4 with the static global
+                            // scale; code decisions in fp32 as the format defines them
+                            if (lane < 16) {
+                                const int i = lane & 7, b = lane >> 3;
+                                const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
+                                float v[16];
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const float4 f4 = src[qq];
+                                    v[4 * qq] = f4.x; v[4 * qq + 1] = f4.y; v[4 * qq + 2] = f4.z; v[4 * qq + 3] = f4.w;
+                                }
+                                float amax = 0.0f;
+#pragma unroll
+                                for (int qq = 0; qq < 16; ++qq) amax = fmaxf(amax, fabsf(v[qq]));
+                                const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
+                                const float rcp = rcp_tab[sbc];
+                                uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                                for (int qq = 0; qq < 8; ++qq)
+                                    w[qq >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * qq], rcp), __fmul_rn(v[2 * qq + 1], rcp)) << (8 * (qq & 3));
+                                const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
+                                *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
+                                out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
                             }
-                            float amax = 0.0f;
-#pragma unroll
-                            for (int qq = 0; qq < 16; ++qq) amax = fmaxf(amax, fabsf(v[qq]));
-                            const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
-                            const float rcp = rcp_tab[sbc];
-                            uint32_t w[2] = {0u, 0u};
-#pragma unroll
-                            for (int qq = 0; qq < 8; ++qq)
-                                w[qq >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * qq], rcp), __fmul_rn(v[2 * qq + 1], rcp)) << (8 * (qq & 3));
-                            const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
-                            *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
-                            out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
+                            __syncwarp();
                         }
-                        __syncwarp();
                     }
                 }
             }
@@ -1556,10 +1594,10 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 bool prefill_native_fp4(int H, int I) { return H % kFp4KS == 0 && I % kFp4KS == 0; }
 
 // Token-operand maps of the block-scaled GEMM over codes [rows][K/2], boxes
-// of 128 / 64 / 32 / 16 rows
+// of 16, 32, ..., 176 rows
 static bool make_fp4_bmaps(Fp4BMaps* mb, const void* codes, uint64_t rows, int K) {
-    for (int i = 0; i < 4; ++i)
-        if (!make_map_u8(&mb->codes[i], codes, rows, K / 2, 128, (uint32_t)(kBN >> i), true)) return false;
+    for (int i = 0; i < 11; ++i)
+        if (!make_map_u8(&mb->codes[i], codes, rows, K / 2, 128, (uint32_t)(16 * (i + 1)), true)) return false;
     return true;
 }
 
@@ -1658,12 +1696,11 @@ cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E,
 // Block-scaled NVFP4 GEMM over the routed tiles; maps: A of gate (or down),
 // A of up, their scale tiles, B and its scale tiles.
 template <int MODE>
-static cudaError_t launch_fp4(const CUtensorMap (&m)[2], const Fp4BMaps& mb, const OMaps& mo, const GemmArgs& g,
-                              cudaStream_t st) {
+static cudaError_t launch_fp4(const Fp4BMaps& mb, const OMaps& mo, const GemmArgs& g, cudaStream_t st) {
     constexpr int bytes = Fp4Cfg<MODE>::ALLOC;
     cudaError_t err = cudaFuncSetAttribute(k_fp4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (err != cudaSuccess) return err;
-    k_fp4_gemm<MODE><<<num_sms(), Fp4Cfg<MODE>::THREADS, bytes, st>>>(m[0], m[1], mb, mo, g);
+    k_fp4_gemm<MODE><<<num_sms(), Fp4Cfg<MODE>::THREADS, bytes, st>>>(mb, mo, g);
     return cudaGetLastError();
 }
 
@@ -1684,12 +1721,9 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
                                                    (long long)slots, p.w, p.w_perm);
     }
     // ---- gate / up
-    CUtensorMap m[2];
     Fp4BMaps mb;
     BMaps m_shared;
-    if (!make_map_u8(&m[0], p.fp4_codes[0], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
-        !make_map_u8(&m[1], p.fp4_codes[1], (uint64_t)E * I, H / 2, 128, kBlkN, true) ||
-        !make_fp4_bmaps(&mb, xc, (uint64_t)slots, H) ||
+    if (!make_fp4_bmaps(&mb, xc, (uint64_t)slots, H) ||
         !make_bmaps(&m_shared, p.x, (uint64_t)T, (uint64_t)H))
         return cudaErrorInvalidValue;
     GemmArgs g{};
@@ -1711,29 +1745,24 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     g.g_act = ex.g_x;
     g.g_req = ex.g_a;
     g.err = p.err;
-    g.sfa0 = p.fp4_scales[0];
-    g.sfa1 = p.fp4_scales[1];
+    g.wimg = p.fp4_img[0];
     g.sfb = xs;
-    g.sfa_rows = (long long)E * I;
     g.sfb_rows = (long long)slots;
     g.sfb_rows_out = (long long)slots;
     if (p.ev_gu0) cudaEventRecord(p.ev_gu0, st);
     OMaps mo;                         // the down GEMM's output maps (unused by gate/up)
-    for (int i = 0; i < 8; ++i) mo.m[i] = m[0];
-    cudaError_t err = launch_fp4<0>(m, mb, mo, g, st);
+    memset(&mo, 0, sizeof(mo));
+    cudaError_t err = launch_fp4<0>(mb, mo, g, st);
     if (err == cudaSuccess && p.ev_gu_r) cudaEventRecord(p.ev_gu_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<0, true>(m_shared, g, st);
     if (err != cudaSuccess) return err;
     if (p.ev_gu1) cudaEventRecord(p.ev_gu1, st);
     // ---- down
-    if (!make_map_u8(&m[0], p.fp4_codes[2], (uint64_t)E * H, I / 2, 128, kBlkN, true) ||
-        !make_fp4_bmaps(&mb, a4, (uint64_t)slots, I) ||
+    if (!make_fp4_bmaps(&mb, a4, (uint64_t)slots, I) ||
         !make_bmaps(&m_shared, p.a_sh, (uint64_t)T, (uint64_t)I))
         return cudaErrorInvalidValue;
-    m[1] = m[0];
-    g.sfa0 = g.sfa1 = p.fp4_scales[2];
+    g.wimg = p.fp4_img[1];
     g.sfb = as;
-    g.sfa_rows = (long long)E * H;
     g.tiles = p.tiles + p.tile_cap;          // the down list
     g.groups = p.groups + p.tile_cap;
     g.num_tiles = p.num_tiles + 4;
@@ -1754,7 +1783,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     if (!make_omaps(&mo, p.o, (uint64_t)slots, (uint64_t)H) ||
         (has_sh && !make_omaps(&mo_sh, p.o_sh, (uint64_t)T, (uint64_t)H)))
         return cudaErrorInvalidValue;
-    err = launch_fp4<1>(m, mb, mo, g, st);
+    err = launch_fp4<1>(mb, mo, g, st);
     if (err == cudaSuccess && p.ev_dn_r) cudaEventRecord(p.ev_dn_r, st);
     if (err == cudaSuccess && has_sh) err = launch_gemm<1, true>(m_shared, g, st, nullptr, 0, &mo_sh);
     if (err != cudaSuccess) return err;
@@ -1769,6 +1798,10 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     const ExpertArgs& ex = p.ex;
     const int T = p.T, k = ex.k, H = ex.H, I = ex.I, E = ex.E;
     const int slots = T * k;
+    const bool fp4 = ex.quant == Q_NVFP4;
+    // NVFP4 W4A4 on the block-scaled tensor cores when the shapes allow
+    // 256-value stages (else the exact bf16 dequantization path below)
+    const bool native = fp4 && p.fp4_img[0] && p.fp4_img[1] && prefill_native_fp4(H, I);
     // the permutation launch also builds both tile lists (gate/up: I / 128
     // row blocks, down: H / 128)
     TileListArgs tl{};
@@ -1780,13 +1813,11 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     tl.RB0 = I / kBlkN;
     tl.RB1 = H / kBlkN;
     tl.has_shared = ex.sh_gate != nullptr ? 1 : 0;
+    tl.tok0 = native ? kFp4GuN : kBN;        // the block-scaled gate/up takes wider tiles
+    tl.tok1 = kBN;
     tl.grid = num_sms();
     cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st, &tl);
     if (err != cudaSuccess) return err;
-    const bool fp4 = ex.quant == Q_NVFP4;
-    // NVFP4 W4A4 on the block-scaled tensor cores when the shapes allow
-    // 256-value stages (else the exact bf16 dequantization path below)
-    const bool native = fp4 && p.fp4_codes[0] && prefill_native_fp4(H, I);
     if (native) return launch_prefill_fp4(p, st);
     const __nv_bfloat16* xin = nullptr;
     CUtensorMapDataType xdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

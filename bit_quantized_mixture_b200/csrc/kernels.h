@@ -18,6 +18,14 @@ cudaError_t launch_quantize_act_nvfp4(const void* x, int T, int K, float g, void
 cudaError_t launch_absmax(const float* x, long long n, float* out, cudaStream_t st);
 // g[e] = gate/up and g[E + e] = down global scale read from each table block at offset off
 cudaError_t launch_gather_global_scales(const uint8_t* const* table, size_t off, int E, float* g, cudaStream_t st);
+// NVFP4 block-scaled GEMM weight image (see k_fp4_block_image): one matrix of
+// one expert into slot `slot` of its nmat-matrix blocks (N % 128 == 0, K % 256 == 0)
+cudaError_t launch_fp4_block_image(const uint8_t* codes, const uint8_t* scales, int N, int K, int slot, int nmat,
+                                   uint8_t* dst, cudaStream_t st);
+// bytes of one expert's image of nmat matrices of N rows and K columns
+inline size_t fp4_block_image_bytes(int N, int K, int nmat) {
+    return (size_t)(N / 128) * (K / 256) * nmat * (16384 + 2048);
+}
 cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const uint8_t* src_scales,
                             const uint8_t* src_zeros, uint8_t* dst_codes, uint8_t* dst_scales,
                             uint8_t* dst_zeros, cudaStream_t st);
@@ -64,6 +72,7 @@ struct TileListArgs {
     int* num_tiles;                // [2][4]
     size_t cap;
     int T, RB0, RB1, has_shared;
+    int tok0, tok1;                // tokens per routed tile of each list
     int grid;                      // CTAs of the GEMM launches
 };
 // tl may be null (permutation only)
@@ -138,8 +147,9 @@ struct PrefillArgs {
     __nv_bfloat16* xp;             // [T*k, H]: rows of xq in permuted (expert-major) order
     float* w_perm;                 // [T*k]: routing weight of each permuted position
     float* ts_perm;                // [T*k]: token scale of each permuted position (INT4/INT2)
-    const uint8_t* fp4_codes[3];   // NVFP4: natural-layout weight images (gate, up, down) or null
-    const uint8_t* fp4_scales[3];
+    // NVFP4: block-scaled GEMM weight images (k_fp4_block_image), gate/up
+    // (two matrices per block) and down, or null
+    const uint8_t* fp4_img[2];
     __nv_bfloat16* a_perm;         // [T*k, I] intermediate in permuted order
     __nv_bfloat16* a_sh;           // [T, I] shared-expert intermediate
     __half* o;                     // [T*k, H] weighted expert outputs by slot (fp16)

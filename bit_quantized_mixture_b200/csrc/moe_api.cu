@@ -27,8 +27,9 @@ struct moe_layer {
     uint8_t* experts = nullptr;    // expert e at experts + e * expert_stride
     uint8_t* router = nullptr;     // bf16 [E, H]
     uint8_t* shared[3] = {nullptr, nullptr, nullptr};   // bf16 device layout
-    uint8_t* fp4_codes[3] = {nullptr, nullptr, nullptr};    // NVFP4: natural-layout images [E][N][K/2]
-    uint8_t* fp4_scales[3] = {nullptr, nullptr, nullptr};   //        and their block scales [K/256][E*N][16]
+    // NVFP4: the block-scaled prefill GEMM's weight images (gate/up, down),
+    // when H and I allow 256-value stages
+    uint8_t* fp4_img[2] = {nullptr, nullptr};
     float* g_gate = nullptr;       // NVFP4 global scales [E]
     float* g_down = nullptr;
     // workspace
@@ -171,15 +172,15 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
     if (c.has_shared)
         for (int m = 0; m < 3; ++m) { shared_off[m] = a; a = align_up(a + (size_t)H * I * 2, 256); }
     const size_t g_off = a; a = align_up(a + sizeof(float) * 2 * E, 256);
-    // NVFP4: the interchange codes and scales kept as natural-layout images,
-    // the operands of the block-scaled prefill GEMM (TMA tiles)
-    size_t img_off[3] = {0, 0, 0}, imgs_off[3] = {0, 0, 0};
-    if (c.quant == MOE_Q_NVFP4)
-        for (int m = 0; m < 3; ++m) {
-            const size_t nk = (size_t)h->geom[m].N * h->geom[m].K * E;
-            img_off[m] = a; a = align_up(a + nk / 2, 256);
-            imgs_off[m] = a; a = align_up(a + (size_t)((h->geom[m].K / 16 + 15) / 16) * 16 * h->geom[m].N * E, 256);
-        }
+    // NVFP4: the interchange codes and scales, kept again as the block-scaled
+    // prefill GEMM's weight images (per 128-row block and 256-value stage one
+    // contiguous block of swizzled codes and scales; gate and up share blocks)
+    const bool fp4_images = c.quant == MOE_Q_NVFP4 && prefill_native_fp4(H, I);
+    size_t img_off[2] = {0, 0};
+    if (fp4_images) {
+        img_off[0] = a; a = align_up(a + (size_t)E * fp4_block_image_bytes(I, H, 2), 256);
+        img_off[1] = a; a = align_up(a + (size_t)E * fp4_block_image_bytes(H, I, 1), 256);
+    }
     h->arena_bytes = a;
     if (cudaMalloc(&h->arena, h->arena_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -187,8 +188,8 @@ moe_status moe_create(const moe_config* cfg, moe_handle* out) {
         return fail(nullptr, MOE_ERR_OOM, "moe_create: arena of %zu bytes", a);
     }
     h->experts = h->arena + experts_off;
-    if (c.quant == MOE_Q_NVFP4)
-        for (int m = 0; m < 3; ++m) { h->fp4_codes[m] = h->arena + img_off[m]; h->fp4_scales[m] = h->arena + imgs_off[m]; }
+    if (fp4_images)
+        for (int i = 0; i < 2; ++i) h->fp4_img[i] = h->arena + img_off[i];
     h->router = h->arena + router_off;
     if (c.has_shared)
         for (int m = 0; m < 3; ++m) h->shared[m] = h->arena + shared_off[m];
@@ -318,8 +319,8 @@ moe_status moe_load_router(moe_handle h, const void* w_router_any, moe_stream_t 
 }
 
 static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix& q, uint8_t* dst_codes,
-                              uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st, uint8_t* img_codes = nullptr,
-                              uint8_t* img_scales = nullptr, size_t img_rows = 0) {
+                              uint8_t* dst_scales, uint8_t* dst_zeros, cudaStream_t st, uint8_t* img = nullptr,
+                              int img_slot = 0, int img_nmat = 1) {
     const size_t codes_in = gm.quant == Q_BF16 ? (size_t)gm.N * gm.K * 2
                                                : (size_t)gm.N * gm.K /
                                                      (gm.quant == Q_INT2 ? 4 : ((gm.quant == Q_FP8 || gm.quant == Q_FP6) ? 1 : 2));
@@ -334,19 +335,10 @@ static moe_status load_matrix(moe_layer* h, const MatGeom& gm, const moe_qmatrix
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: copy");
     e = launch_relayout(gm, h->staging, h->staging + o_s, h->staging + o_z, dst_codes, dst_scales, dst_zeros, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: relayout");
-    if (img_codes) {
-        // NVFP4: the interchange codes are the prefill GEMM's operand image
-        // [E][N][K/2]; the block scales go to a stage-major image
-        // [K/256][E*N][16 B] (img_scales points at this expert's first row of
-        // stage 0, img_rows is E*N), so that one stage's scale tile of 128
-        // rows is one contiguous 2 KB bulk copy
-        e = cudaMemcpyAsync(img_codes, h->staging, codes_in, cudaMemcpyDeviceToDevice, st);
-        const int kb16 = gm.K / 16;
-        for (int ks = 0; e == cudaSuccess && ks * 16 < kb16; ++ks) {
-            const int w = kb16 - ks * 16 < 16 ? kb16 - ks * 16 : 16;
-            e = cudaMemcpy2DAsync(img_scales + (size_t)ks * img_rows * 16, 16, h->staging + o_s + ks * 16, (size_t)kb16,
-                                  (size_t)w, (size_t)gm.N, cudaMemcpyDeviceToDevice, st);
-        }
+    if (img) {
+        // NVFP4: the prefill GEMM's weight image, built from the interchange
+        // codes and scales still in the staging buffer
+        e = launch_fp4_block_image(h->staging, h->staging + o_s, gm.N, gm.K, img_slot, img_nmat, img, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "moe_load_expert_weights: NVFP4 image");
     }
     return MOE_OK;
@@ -385,11 +377,12 @@ moe_status moe_load_expert_weights(moe_handle h, int32_t expert, const moe_exper
             s = load_matrix(h, gm, *mats[m], h->shared[m], nullptr, nullptr, st);
         } else {
             uint8_t* base = h->experts + (size_t)expert * h->expert_stride;
-            const size_t nk = (size_t)gm.N * gm.K;
-            uint8_t* ic = h->fp4_codes[m] ? h->fp4_codes[m] + (size_t)expert * nk / 2 : nullptr;
-            uint8_t* is = h->fp4_scales[m] ? h->fp4_scales[m] + (size_t)expert * gm.N * 16 : nullptr;
+            // gate and up fill slots 0 and 1 of the gate/up image's blocks
+            const int im = m == 2 ? 1 : 0, nmat = m == 2 ? 1 : 2;
+            uint8_t* img = h->fp4_img[im] ? h->fp4_img[im] + (size_t)expert * fp4_block_image_bytes(gm.N, gm.K, nmat)
+                                          : nullptr;
             s = load_matrix(h, gm, *mats[m], base + h->off_codes[m], base + h->off_scales[m], base + h->off_zeros[m], st,
-                            ic, is, (size_t)c.num_experts * gm.N);
+                            img, m == 1 ? 1 : 0, nmat);
         }
         if (s != MOE_OK) return s;
     }
@@ -569,10 +562,7 @@ moe_status moe_forward(moe_handle h, const void* x, int32_t T, const int32_t* to
         p.err = h->dev_err;
         // the block-scaled NVFP4 images live in the arena: with an address
         // table the exact bf16-dequantization path reads the table's blocks
-        for (int m = 0; m < 3; ++m) {
-            p.fp4_codes[m] = h->table_set ? nullptr : h->fp4_codes[m];
-            p.fp4_scales[m] = h->table_set ? nullptr : h->fp4_scales[m];
-        }
+        for (int i = 0; i < 2; ++i) p.fp4_img[i] = h->table_set ? nullptr : h->fp4_img[i];
         p.ev_gu0 = h->prof[5]; p.ev_gu1 = h->prof[3]; p.ev_dn0 = h->prof[6]; p.ev_dn1 = h->prof[7];
         p.ev_gu_r = h->prof[8]; p.ev_dn_r = h->prof[9];
         h->last_prefill_T = T;

@@ -86,12 +86,13 @@ k_perm_place(const int32_t* __restrict__ ids, int n, int E, int chunk, int chunk
         if (e == kPlaceThreads - 1) offsets[E] = incl;    // all placed slots
     }
     if (tl.tiles) {                          // both tile lists, entries spread over all CTAs
-        tile_list_prefix(s_cnt, tl.RB0, s_sc[0], s_sg[0], wsum);
-        tile_list_prefix(s_cnt, tl.RB1, s_sc[1], s_sg[1], wsum);
+        tile_list_prefix(s_cnt, tl.RB0, tl.tok0, s_sc[0], s_sg[0], wsum);
+        tile_list_prefix(s_cnt, tl.RB1, tl.tok1, s_sc[1], s_sg[1], wsum);
         __syncthreads();
         const long long first = (long long)c * kPlaceThreads + e, stride = (long long)gridDim.x * kPlaceThreads;
         for (int list = 0; list < 2; ++list)
-            emit_tile_list(s_cnt, s_off, s_sc[list], s_sg[list], tl.T, list ? tl.RB1 : tl.RB0, tl.has_shared,
+            emit_tile_list(s_cnt, s_off, s_sc[list], s_sg[list], tl.T, list ? tl.RB1 : tl.RB0,
+                           list ? tl.tok1 : tl.tok0, tl.has_shared,
                            tl.grid, first, stride, tl.tiles + (size_t)list * tl.cap,
                            tl.groups + (size_t)list * tl.cap, tl.num_tiles + 4 * list, c == 0);
     }

@@ -448,6 +448,39 @@ cudaError_t launch_relayout(const MatGeom& gm, const uint8_t* src_codes, const u
     return cudaGetLastError();
 }
 
+// Block-scaled GEMM weight image of one NVFP4 matrix of one expert (codes
+// [N][K/2], scales [N][K/16] in the interchange layout): for each 128-row
+// block rb and 256-value stage ks, one contiguous block of nmat x 16 KB of
+// codes followed by nmat x 2 KB of scales, at dst + (rb * K/256 + ks) *
+// nmat * 18 KB.  This matrix fills slot `slot` of each block (gate 0 and up 1
+// share the blocks of the gate/up image; down has nmat = 1).  The codes tile
+// (128 rows x 128 bytes) is stored in the 128-byte swizzled order the tensor
+// core reads from shared memory (16-byte chunk c of row r at chunk c ^ (r % 8)
+// of its row), so a stage's weights and scales arrive in one bulk copy.
+__global__ void k_fp4_block_image(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int N, int K,
+                                  int slot, int nmat, uint8_t* __restrict__ dst) {
+    const int NS = K / 256;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;     // (row n, stage ks)
+    if (i >= (long long)N * NS) return;
+    const int n = (int)(i / NS), ks = (int)(i % NS);
+    const int rb = n >> 7, r = n & 127;
+    uint8_t* blk = dst + ((size_t)rb * NS + ks) * (size_t)nmat * (16384 + 2048);
+    const uint4* src = reinterpret_cast<const uint4*>(codes + (size_t)n * (K / 2) + ks * 128);
+    uint8_t* tile = blk + slot * 16384 + r * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(tile + ((c ^ (r & 7)) << 4)) = src[c];
+    *reinterpret_cast<uint4*>(blk + nmat * 16384 + slot * 2048 + r * 16) =
+        *reinterpret_cast<const uint4*>(scales + (size_t)n * (K / 16) + ks * 16);
+}
+
+cudaError_t launch_fp4_block_image(const uint8_t* codes, const uint8_t* scales, int N, int K, int slot, int nmat,
+                                   uint8_t* dst, cudaStream_t st) {
+    if (N % 128 || K % 256 || slot < 0 || slot >= nmat || nmat < 1 || nmat > 2) return cudaErrorInvalidValue;
+    const size_t n = (size_t)N * (K / 256);
+    k_fp4_block_image<<<blocks_for(n, 256), 256, 0, st>>>(codes, scales, N, K, slot, nmat, dst);
+    return cudaGetLastError();
+}
+
 __global__ void k_gather_global_scales(const uint8_t* const* __restrict__ table, size_t off, int E,
                                        float* __restrict__ g) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;

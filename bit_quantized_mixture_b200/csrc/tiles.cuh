@@ -2,10 +2,11 @@
 // counts and segment offsets of the token permutation.
 //
 // A routed tile is (expert e, 128-row block rb of the weight matrix, up to
-// kTileTokens consecutive permuted positions of e's segment); the list holds
+// `tok` consecutive permuted positions of e's segment: kTileTokens, or more
+// for a GEMM whose MMA takes wider tiles); the list holds
 // every expert's tiles expert by expert, row block by row block, then (when
 // the layer has a shared expert) the shared-expert tiles (expert -1, token
-// rows instead of positions).  A group is up to kGroupTiles consecutive token
+// rows instead of positions, kTileTokens per tile).  A group is up to kGroupTiles consecutive token
 // tiles of one (expert, row block), which read the same weight block.
 #pragma once
 
@@ -47,9 +48,9 @@ MOE_DEV int block_incl_scan_1024(int v, int* wsum) {
 // sc and sg (1024 ints of shared memory each; thread e takes expert e).
 // s_cnt: 1024 expert counts, zero beyond E.  A CTA of 1024 threads; the
 // caller synchronizes before reading sc / sg.
-MOE_DEV void tile_list_prefix(const int* s_cnt, int RB, int* sc, int* sg, int* wsum) {
+MOE_DEV void tile_list_prefix(const int* s_cnt, int RB, int tok, int* sc, int* sg, int* wsum) {
     const int e = threadIdx.x;
-    const int nt = (s_cnt[e] + kTileTokens - 1) / kTileTokens;
+    const int nt = (s_cnt[e] + tok - 1) / tok;
     const int ci = block_incl_scan_1024(nt * RB, wsum);
     const int gi = block_incl_scan_1024(((nt + kGroupTiles - 1) / kGroupTiles) * RB, wsum);
     sc[e] = ci;
@@ -73,14 +74,14 @@ MOE_DEV int tile_owner(const int* pre, int i) {
 // write_counts sets num_tiles[0..3] = routed tiles, routed + shared tiles,
 // routed groups, and 1 when every GEMM CTA's groups fit its shared-memory
 // tile list (group order), else 0.
-MOE_DEV void emit_tile_list(const int* s_cnt, const int* s_off, const int* sc, const int* sg, int T, int RB,
+MOE_DEV void emit_tile_list(const int* s_cnt, const int* s_off, const int* sc, const int* sg, int T, int RB, int tok,
                             int has_shared, int grid, long long first, long long stride, GemmTile* __restrict__ tiles,
                             int2* __restrict__ groups, int* __restrict__ num_tiles, bool write_counts) {
     const int total = sc[1023], ngroups = sg[1023];
     for (long long ii = first; ii < ngroups; ii += stride) {
         const int i = (int)ii;
         const int ex = tile_owner(sg, i);
-        const int ntx = (s_cnt[ex] + kTileTokens - 1) / kTileTokens;
+        const int ntx = (s_cnt[ex] + tok - 1) / tok;
         const int gpr = (ntx + kGroupTiles - 1) / kGroupTiles;     // groups per row block
         const int j = i - (sg[ex] - gpr * RB);
         const int rb = j / gpr, q = j % gpr;
@@ -90,14 +91,14 @@ MOE_DEV void emit_tile_list(const int* s_cnt, const int* s_off, const int* sc, c
         const int i = (int)ii;
         const int ex = tile_owner(sc, i);
         const int c = s_cnt[ex];
-        const int ntx = (c + kTileTokens - 1) / kTileTokens;
+        const int ntx = (c + tok - 1) / tok;
         const int j = i - (sc[ex] - ntx * RB);          // index within the expert's tiles
         const int rb = j / ntx, tt = j % ntx;
         GemmTile g;
         g.expert = ex;
         g.rb = rb;
-        g.seg = s_off[ex] + tt * kTileTokens;
-        g.count = min(kTileTokens, c - tt * kTileTokens);
+        g.seg = s_off[ex] + tt * tok;
+        g.count = min(tok, c - tt * tok);
         tiles[i] = g;
     }
     const int nts = has_shared ? (T + kTileTokens - 1) / kTileTokens : 0;

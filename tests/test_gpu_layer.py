@@ -406,11 +406,33 @@ def test_prefill_matches_oracle(quant, T):
 NATIVE_FP4 = synth.custom("tiny-int4", quant="nvfp4", H=512, I=256, E=24, k=6, shared=True)
 
 
-@pytest.mark.parametrize("T", [5, 37, 300])
+# T = 700 and 1500: experts with 129..176 tokens (one wide gate/up tile) and
+# with more (several tiles, the last a ragged one)
+@pytest.mark.parametrize("T", [5, 37, 300, 700, 1500])
 def test_prefill_nvfp4_block_scaled_matches_oracle(T):
     y, y_ref, layer, _ = _forward_case(NATIVE_FP4, T)
     layer.sync_status()
     assert_close_output(y, y_ref)
+
+
+def test_prefill_nvfp4_block_scaled_one_expert_takes_many_tokens():
+    """Every token on the same six experts: gate/up tiles of 176 tokens and a
+    ragged last tile, down tiles of 128."""
+    wl = NATIVE_FP4
+    T = 700
+    ox = OracleExperts(wl)
+    layer = get_layer(wl, T)
+    x = synth.activations_bf16(wl, steps=T // wl.T + 1)[:T]
+    ids = np.tile(np.array([3, 7, 0, 23, 11, 5], np.int32), (T, 1))
+    w = np.tile(np.array([0.3, 0.2, 0.15, 0.15, 0.1, 0.1]), (T, 1))
+    g_x = O.nvfp4_global_scale(np.abs(O.bf16_bits_to_f32(x)).max())
+    g_a = O.nvfp4_global_scale(O.intermediate_amax(x, ids, "nvfp4", ox, g_x))
+    layer.set_act_global_scales(g_x, g_a)
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=DEV)
+    layer.forward(bf16_tensor(x, DEV), torch.from_numpy(ids).to(DEV), torch.from_numpy(w.astype(np.float32)).to(DEV), y)
+    layer.sync_status()
+    y_ref = O.moe_forward(x, ids, w, "nvfp4", ox, shared=ox.shared(), act_scales=(g_x, g_a))
+    assert_close_output(to_bits(y), y_ref)
 
 
 def test_prefill_one_expert_takes_many_tokens():
