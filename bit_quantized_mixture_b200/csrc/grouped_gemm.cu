@@ -136,17 +136,13 @@ struct OMaps {
 // TMA stores of a tile's n staged rows ([n][128] 16-bit, row-major) to rows
 // y .. y+n-1, columns x .. x+127, as one bulk group (issued by one thread).
 MOE_DEV void store_tile_rows(const OMaps& mo, int x, int y, int n, const uint8_t* src) {
-    if (n == kBN) {
-        tma_store_2d(&mo.m[0], x, y, src);
-    } else {
-        int off = 0;
+    int off = 0;
 #pragma unroll
-        for (int b = 6; b >= 0; --b)
-            if ((n >> b) & 1) {
-                tma_store_2d(&mo.m[7 - b], x, y + off, src + off * (kBlkN * 2));
-                off += 1 << b;
-            }
-    }
+    for (int b = 7; b >= 0; --b)
+        if ((n >> b) & 1) {
+            tma_store_2d(&mo.m[7 - b], x, y + off, src + off * (kBlkN * 2));
+            off += 1 << b;
+        }
     bulk_commit();
 }
 
@@ -1067,9 +1063,9 @@ MOE_DEV void load_fp4_token_rows(uint8_t* dst_codes, const Fp4BMaps& mb, int x_c
 }
 
 
-// Tokens per gate/up tile (the MMA's N, at most 256): an expert's ~160 tokens
-// of the uniform workload are one tile, so each weight block streams once.
-// (Down keeps 128: its accumulators alternate between two tiles.)
+// Tokens per tile of the block-scaled GEMMs (the MMA's N, at most 256): an
+// expert's ~160 tokens of the uniform workload are one tile, so each weight
+// block streams once and each (expert, row block) pays one epilogue.
 constexpr int kFp4GuN = 176;
 
 // The accumulator of the next tile, walked identically by the MMA warps and
@@ -1088,8 +1084,8 @@ MOE_DEV Fp4Acc fp4_acc_next(Fp4AccSeq& q, int n_mma) {
     (void)n_mma;
     if (MODE == 1) {
         a.buf = q.local & 1;
-        a.col = (uint32_t)(a.buf * kBN);
-        a.mat_stride = kBN;
+        a.col = (uint32_t)(a.buf * kFp4GuN);
+        a.mat_stride = kFp4GuN;
     } else {
         a.buf = 0;
         a.col = 0;
@@ -1105,7 +1101,7 @@ MOE_DEV Fp4Acc fp4_acc_next(Fp4AccSeq& q, int n_mma) {
 template <int MODE>
 struct Fp4Cfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
-    static constexpr int S = MODE == 0 ? 3 : 4;
+    static constexpr int S = 3;
     static constexpr int SF0 = kWarpMma + NMAT;                       // four scale-factor warps
     static constexpr int EPI0 = SF0 + 4;
     // epilogue warps: four per TMEM lane quarter, each taking
@@ -1113,19 +1109,18 @@ struct Fp4Cfg {
     // staging of a tile is the longest step of these kernels)
     static constexpr int EPI_WARPS = 16;
     static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
-    // token rows per tile: gate/up kFp4GuN, down 128
-    static constexpr int BROWS = MODE == 0 ? kFp4GuN : kBN;
-    // accumulators: gate/up one of 2 x kFp4GuN columns (the epilogue reads
-    // it and releases it before the requantization); down alternates two of
-    // 128
+    // token rows per tile
+    static constexpr int BROWS = kFp4GuN;
+    // accumulators: gate/up one of 2 x BROWS columns (the epilogue reads it
+    // and releases it before the requantization); down alternates two of
+    // BROWS
     static constexpr int ACC_COLS = NMAT * BROWS;
     // scale factors in TMEM: per slot, A (4 columns per MMA and matrix), then
-    // B (ceil(rows / 32) columns per MMA, at 8-column steps for 176 rows);
-    // gate/up keeps two slots (released by their own MMA commits), down one
-    // per stage
-    static constexpr int SFB_KK = MODE == 0 ? 8 : 4;
+    // B (ceil(rows / 32) columns per MMA, at 8-column steps); two slots, each
+    // released by its own MMA commits
+    static constexpr int SFB_KK = 8;
     static constexpr int SF_STAGE_COLS = NMAT * 16 + 4 * SFB_KK;
-    static constexpr int SF_SLOTS = MODE == 0 ? 2 : S;
+    static constexpr int SF_SLOTS = 2;
     static constexpr int SF_COL0 = MODE == 0 ? ACC_COLS : 2 * ACC_COLS;
     static_assert(SF_COL0 + SF_SLOTS * SF_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
     // weights: per stage one block of the image, [NMAT][16 KB codes] then
@@ -1139,8 +1134,8 @@ struct Fp4Cfg {
     static constexpr int W = 0;                                       // [S][W_STAGE]
     static constexpr int B = W + S * W_STAGE;                         // [S][B_STAGE]
     static constexpr int SFB = B + S * B_STAGE;                       // [S][SFB_STAGE]
-    static constexpr int OUT = SFB + S * SFB_STAGE;                   // gate/up: [BROWS][80 B]; down: 2 x [128][128] fp16
-    static constexpr int OUT_BYTES = MODE == 0 ? BROWS * 80 : 2 * kOutTile;
+    static constexpr int OUT = SFB + S * SFB_STAGE;                   // gate/up: [BROWS][80 B]; down: [BROWS][128] fp16
+    static constexpr int OUT_BYTES = MODE == 0 ? BROWS * 80 : BROWS * kBlkN * 2;
     static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [8 tok][32] fp32
     static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 8 * 32 * 4 : 0;
     static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
@@ -1180,7 +1175,7 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], NMAT);
             mbar_init(&acc_empty[b], C::EPI_WARPS);
-            mbar_init(&sffree[b], NMAT);                  // gate/up: one commit per MMA warp
+            mbar_init(&sffree[b], NMAT);                  // one commit per MMA warp
         }
         abort_flag = 0;
         fence_barrier_init();
@@ -1255,7 +1250,7 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
                         mma_fp4_block16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, sf + mi * 16 + kk * 4,
                                         sf + NMAT * 16 + kk * C::SFB_KK, (ks | kk) != 0);
                     mma_commit(&empty[s]);
-                    if (MODE == 0) mma_commit(&sffree[slot]);     // this slot's scales are consumed
+                    mma_commit(&sffree[slot]);                    // this slot's scales are consumed
                     if (ks == NS - 1) mma_commit(&acc_full[ab]);
                 }
                 __syncwarp();
@@ -1273,9 +1268,9 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
                 const int s = g % S;
                 const uint32_t r = (uint32_t)(g / S);
                 if (!warp_wait(&full[s], r & 1u, &abort_flag, a.err, 15)) { ok = false; break; }
-                // gate/up: the TMEM slot is free once the MMAs of stage g - 2 are done
+                // the TMEM slot is free once the MMAs of stage g - 2 are done
                 const int slot = g % C::SF_SLOTS;
-                if (MODE == 0 && g >= C::SF_SLOTS &&
+                if (g >= C::SF_SLOTS &&
                     !warp_wait(&sffree[slot], (uint32_t)((g / C::SF_SLOTS - 1) & 1), &abort_flag, a.err, 17)) {
                     ok = false;
                     break;
@@ -1360,9 +1355,9 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             const Fp4Acc acc = fp4_acc_next<MODE>(aseq, (t.count + 15) & ~15);
             const int ab = acc.buf;
             const float gsc = nx.gw * a.g_act;
-            // down: this tile's staging buffer was last read by the TMA store
-            // of the tile two back (one bulk group per tile)
-            if (MODE == 1 && ej == 0) bulk_wait_read<1>();
+            // down: the staging buffer was last read by the previous tile's
+            // TMA stores (one bulk group per tile)
+            if (MODE == 1 && ej == 0) bulk_wait_read<0>();
             epi_sync_n<C::EPI_WARPS>();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
@@ -1391,22 +1386,25 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             // start while this tile's SwiGLU / requantization or fp16
             // conversion runs.
             if constexpr (MODE == 1) {
-                static_assert(C::EPI_WARPS == 16, "down: at most 32 columns per warp");
-                uint32_t r[32];
-                if (nch == 2) tmem_ld_x32c(lane_base + cbeg, r);
-                else if (nch == 1) tmem_ld_x16c(lane_base + cbeg, r);
+                static_assert(C::EPI_WARPS == 16 && kFp4GuN <= 192, "down: at most 48 columns per warp");
+                // (at most 32 registers per TMEM load: the third chunk separately)
+                uint32_t r0[32], r1[32];
+                if (nch >= 2) tmem_ld_x32c(lane_base + cbeg, r0);
+                else if (nch == 1) tmem_ld_x16c(lane_base + cbeg, r0);
+                if (nch == 3) tmem_ld_x16c(lane_base + cbeg + 32, r1);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * kOutTile);
+                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < 3; ++q) {
                     if (q < nch) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int col = cbeg + 16 * q + i;
                             const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                            ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[16 * q + i]) * sc));
+                            const uint32_t v = q < 2 ? r0[16 * q + i] : r1[i];
+                            ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(v) * sc));
                         }
                     }
                 }
@@ -1491,7 +1489,7 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             } else if (ej == 0) {
                 // the tile's rows are the permuted positions seg .. seg+count-1:
                 // TMA stores of boxes of 128, 64, ..., 1 rows, one bulk group
-                store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count, out_s + (local & 1) * kOutTile);
+                store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count, out_s);
             }
         }
         if (MODE == 1 && ej == 0) bulk_wait_all();     // every store done before the CTA leaves
@@ -1813,8 +1811,8 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     tl.RB0 = I / kBlkN;
     tl.RB1 = H / kBlkN;
     tl.has_shared = ex.sh_gate != nullptr ? 1 : 0;
-    tl.tok0 = native ? kFp4GuN : kBN;        // the block-scaled gate/up takes wider tiles
-    tl.tok1 = kBN;
+    tl.tok0 = native ? kFp4GuN : kBN;        // the block-scaled GEMMs take wider tiles
+    tl.tok1 = native ? kFp4GuN : kBN;
     tl.grid = num_sms();
     cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st, &tl);
     if (err != cudaSuccess) return err;
