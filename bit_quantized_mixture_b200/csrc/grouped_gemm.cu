@@ -1101,7 +1101,9 @@ MOE_DEV Fp4Acc fp4_acc_next(Fp4AccSeq& q, int n_mma) {
 template <int MODE>
 struct Fp4Cfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
-    static constexpr int S = 3;
+    // stages: down takes two (a tile is two stages) so that two staging
+    // buffers fit, which let a tile's TMA stores overlap the next staging
+    static constexpr int S = MODE == 0 ? 3 : 2;
     static constexpr int SF0 = kWarpMma + NMAT;                       // four scale-factor warps
     static constexpr int EPI0 = SF0 + 4;
     // epilogue warps: four per TMEM lane quarter, each taking
@@ -1134,8 +1136,9 @@ struct Fp4Cfg {
     static constexpr int W = 0;                                       // [S][W_STAGE]
     static constexpr int B = W + S * W_STAGE;                         // [S][B_STAGE]
     static constexpr int SFB = B + S * B_STAGE;                       // [S][SFB_STAGE]
-    static constexpr int OUT = SFB + S * SFB_STAGE;                   // gate/up: [BROWS][80 B]; down: [BROWS][128] fp16
-    static constexpr int OUT_BYTES = MODE == 0 ? BROWS * 80 : BROWS * kBlkN * 2;
+    static constexpr int OUT = SFB + S * SFB_STAGE;                   // gate/up: [BROWS][80 B]; down: 2 x [BROWS][128] fp16
+    static constexpr int OUT_TILE = BROWS * kBlkN * 2;
+    static constexpr int OUT_BYTES = MODE == 0 ? BROWS * 80 : 2 * OUT_TILE;
     static constexpr int SCR = OUT + OUT_BYTES;                       // gate/up: per epilogue warp [8 tok][32] fp32
     static constexpr int SCR_BYTES = MODE == 0 ? EPI_WARPS * 8 * 32 * 4 : 0;
     static constexpr int ALLOC = SCR + SCR_BYTES + 1024;
@@ -1355,9 +1358,9 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             const Fp4Acc acc = fp4_acc_next<MODE>(aseq, (t.count + 15) & ~15);
             const int ab = acc.buf;
             const float gsc = nx.gw * a.g_act;
-            // down: the staging buffer was last read by the previous tile's
-            // TMA stores (one bulk group per tile)
-            if (MODE == 1 && ej == 0) bulk_wait_read<0>();
+            // down: this tile's staging buffer was last read by the TMA
+            // stores of the tile two back (one bulk group per tile)
+            if (MODE == 1 && ej == 0) bulk_wait_read<1>();
             epi_sync_n<C::EPI_WARPS>();
             if (ej == 0) ep_stop = abort_flag;
             if (ej < t.count) {
@@ -1395,7 +1398,7 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s);
+                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * C::OUT_TILE);
 #pragma unroll
                 for (int q = 0; q < 3; ++q) {
                     if (q < nch) {
@@ -1420,9 +1423,12 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
                         const int c0 = cbeg + 16 * q;
                         float vg[16], vu[16];
                         tmem_ld16x2(lane_base + c0, lane_base + acc.mat_stride + c0, vg, vu);
+                        // one scale for the whole tile (the expert's and the
+                        // activations' global scales); padding columns give 0
+                        const float sct = ep_scale[0];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float sc = c0 + i < t.count ? ep_scale[c0 + i] : 0.0f;
+                            const float sc = c0 + i < t.count ? sct : 0.0f;
                             act[q][i] = swiglu_fast(vg[i] * sc, vu[i] * sc);
                         }
                     }
@@ -1431,8 +1437,9 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
                 // the warp's scratch [8 tokens][32 outputs] turns the results
-                // into 16-output blocks per lane for the requantization, eight
-                // tokens at a time (lanes 0..15: token i, block b)
+                // into 16-output blocks for the requantization, eight tokens
+                // at a time: lane = (token i, block b, half hf) takes eight
+                // values of the block, the two halves share the block's amax
                 float* scr = reinterpret_cast<float*>(smem + C::SCR) + (warp - C::EPI0) * 8 * 32;
 #pragma unroll
                 for (int q = 0; q < 3; ++q) {
@@ -1443,29 +1450,26 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
 #pragma unroll
                             for (int i = 0; i < 8; ++i) scr[i * 32 + lane] = act[q][8 * hh + i];
                             __syncwarp();
-                            // lane = (token i, 16-output block b): NVFP4 with the static global
-                            // scale; code decisions in fp32 as the format defines them
-                            if (lane < 16) {
-                                const int i = lane & 7, b = lane >> 3;
-                                const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16);
-                                float v[16];
-#pragma unroll
-                                for (int qq = 0; qq < 4; ++qq) {
-                                    const float4 f4 = src[qq];
-                                    v[4 * qq] = f4.x; v[4 * qq + 1] = f4.y; v[4 * qq + 2] = f4.z; v[4 * qq + 3] = f4.w;
-                                }
+                            // NVFP4 with the static global scale; code decisions in
+                            // fp32 as the format defines them
+                            {
+                                const int i = lane & 7, b = (lane >> 3) & 1, hf = lane >> 4;
+                                const float4* src = reinterpret_cast<const float4*>(scr + i * 32 + b * 16 + hf * 8);
+                                const float4 f0 = src[0], f1 = src[1];
+                                const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
                                 float amax = 0.0f;
 #pragma unroll
-                                for (int qq = 0; qq < 16; ++qq) amax = fmaxf(amax, fabsf(v[qq]));
+                                for (int qq = 0; qq < 8; ++qq) amax = fmaxf(amax, fabsf(v[qq]));
+                                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
                                 const uint32_t sbc = a.g_req != 0.0f ? f32_to_e4m3(__fdiv_rn(amax, __fmul_rn(6.0f, a.g_req))) : 0u;
                                 const float rcp = rcp_tab[sbc];
-                                uint32_t w[2] = {0u, 0u};
+                                uint32_t w = 0u;
 #pragma unroll
-                                for (int qq = 0; qq < 8; ++qq)
-                                    w[qq >> 2] |= f32x2_to_e2m1(__fmul_rn(v[2 * qq], rcp), __fmul_rn(v[2 * qq + 1], rcp)) << (8 * (qq & 3));
+                                for (int qq = 0; qq < 4; ++qq)
+                                    w |= f32x2_to_e2m1(__fmul_rn(v[2 * qq], rcp), __fmul_rn(v[2 * qq + 1], rcp)) << (8 * qq);
                                 const int col = c0 + i, o0 = (quarter * 32 + b * 16) >> 1;   // byte of output row quarter*32 + 16b
-                                *reinterpret_cast<uint2*>(out_s + col * 80 + o0) = make_uint2(w[0], w[1]);
-                                out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
+                                *reinterpret_cast<uint32_t*>(out_s + col * 80 + o0 + 4 * hf) = w;
+                                if (hf == 0) out_s[col * 80 + 64 + quarter * 2 + b] = (uint8_t)sbc;
                             }
                             __syncwarp();
                         }
@@ -1489,7 +1493,7 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             } else if (ej == 0) {
                 // the tile's rows are the permuted positions seg .. seg+count-1:
                 // TMA stores of boxes of 128, 64, ..., 1 rows, one bulk group
-                store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count, out_s);
+                store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count, out_s + (local & 1) * C::OUT_TILE);
             }
         }
         if (MODE == 1 && ej == 0) bulk_wait_all();     // every store done before the CTA leaves
