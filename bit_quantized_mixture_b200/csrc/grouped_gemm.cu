@@ -58,6 +58,12 @@ struct Cfg {
     // k-blocks (64 columns) per pipeline stage: routed stages cover 128
     // columns, which halves the barrier round trips and commits per MMA
     static constexpr int KSTEP = SH ? 1 : 2;
+    // tokens per tile: the router launch takes 256 (each Wr byte it streams
+    // serves twice the tokens: 31 -> 21 us at T = 8192); the shared-expert
+    // launches measured slower with 256 (one accumulator, two stages) and
+    // keep 128, as the routed ones
+    static constexpr int TN = MODE == 2 ? 2 * kBN : kBN;
+    static constexpr int B_TILE = TN * 128;           // one k-block of the token operand
     // S: stages of the token operand ring, which for routed tiles are also
     // the TMEM slots of the dequantized weights (a slot and its token tile
     // are released by the same MMA commit)
@@ -79,10 +85,11 @@ struct Cfg {
     static constexpr int DEQ_WARPS = SH ? 0 : 4 * NMAT * KSTEP;
     static constexpr int EPI0 = DEQ0 + DEQ_WARPS;                    // first epilogue warp
     static constexpr int THREADS = (EPI0 + kEpiWarps) * 32;
-    // accumulators: NMAT x 128 columns per buffer; routed gate/up keeps one
+    // accumulators: NMAT x TN columns per buffer; routed gate/up keeps one
     // buffer so that its A slots fit in the 512 columns
     static constexpr int ACC_BUFS = (SH || MODE == 1) ? 2 : 1;
-    static constexpr int ACC_COLS = NMAT * kBN;
+    static constexpr bool ACC_SPLIT = MODE == 0 && !SH;   // routed gate/up: halves for small tiles
+    static constexpr int ACC_COLS = NMAT * TN;
     static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;   // TMEM column of A slot 0 (routed)
     static constexpr int A_STAGE_COLS = NMAT * KSTEP * 32;
     static_assert(SH || A_COL0 + S * A_STAGE_COLS <= (int)kTmemCols, "TMEM budget");
@@ -92,14 +99,15 @@ struct Cfg {
     static constexpr int STG_MAT = KSTEP * 4096 + KSTEP * 512;
     // shared memory
     static constexpr int A = 0;                                           // SH: [S][NMAT][16 KB]
-    static constexpr int B = A + (SH ? S * NMAT * kATile : 0);            // [S][KSTEP][16 KB]
-    static constexpr int STG = B + S * KSTEP * kBTile;                    // routed: [SC][NMAT][STG_MAT]
-    static constexpr int OUT = STG + SC * NMAT * STG_MAT;                 // [OUT_BUFS][128][128] 16-bit
+    static constexpr int B = A + (SH ? S * NMAT * kATile : 0);            // [S][KSTEP][B_TILE]
+    static constexpr int STG = B + S * KSTEP * B_TILE;                    // routed: [SC][NMAT][STG_MAT]
+    static constexpr int OUT = STG + SC * NMAT * STG_MAT;                 // [OUT_BUFS][TN][128] 16-bit
+    static constexpr int OUT_TILE = TN * kBlkN * 2;
     // down writes its staged rows with TMA stores: the shared-expert launch
     // has room for two staging buffers (a tile's stores overlap the next
     // tile's staging), the routed one for one
     static constexpr int OUT_BUFS = (MODE == 1 && SH) ? 2 : 1;
-    static constexpr int BYTES = OUT + (MODE == 2 ? 0 : OUT_BUFS * kOutTile);
+    static constexpr int BYTES = OUT + (MODE == 2 ? 0 : OUT_BUFS * OUT_TILE);
     static constexpr int ALLOC = BYTES + 1024;                            // slack for 1024-byte alignment
     static_assert(ALLOC <= 227 * 1024 - 8192, "shared memory budget (static arrays take up to 8 KB)");
 };
@@ -111,12 +119,9 @@ struct BMaps {
     CUtensorMap m[4];
 };
 MOE_DEV uint32_t load_token_rows(uint8_t* dst, const BMaps& mb, int x, int y, int n, uint64_t* bar) {
-    const int n16 = n >> 4;
-    if (n16 >= 8) {
-        tma_load_2d(dst, &mb.m[0], x, y, bar);
-        return 128u * 128u;
-    }
     int off = 0;
+    for (; n - off >= 128; off += 128) tma_load_2d(dst + off * 128, &mb.m[0], x, y + off, bar);
+    const int n16 = (n - off) >> 4;
 #pragma unroll
     for (int b = 2; b >= 0; --b)
         if (n16 & (1 << b)) {
@@ -137,9 +142,11 @@ struct OMaps {
 // y .. y+n-1, columns x .. x+127, as one bulk group (issued by one thread).
 MOE_DEV void store_tile_rows(const OMaps& mo, int x, int y, int n, const uint8_t* src) {
     int off = 0;
+    for (; n - off >= 128; off += 128) tma_store_2d(&mo.m[0], x, y + off, src + off * (kBlkN * 2));
+    const int rem = n - off;                     // < 128: one box per set bit
 #pragma unroll
-    for (int b = 7; b >= 0; --b)
-        if ((n >> b) & 1) {
+    for (int b = 6; b >= 0; --b)
+        if ((rem >> b) & 1) {
             tma_store_2d(&mo.m[7 - b], x, y + off, src + off * (kBlkN * 2));
             off += 1 << b;
         }
@@ -367,13 +374,17 @@ struct AccUse {
     uint32_t mat_stride;    // columns from matrix 0 to matrix 1
     uint32_t par0, par1;    // phase parity of this use of buffer 0 / 1
 };
-template <int ACC_BUFS, int ACC_COLS>
+template <int ACC_BUFS, int ACC_COLS, int TN, bool SPLIT>
 MOE_DEV AccUse acc_next(AccSeq& q, int n_mma) {
     AccUse u;
     if (ACC_BUFS == 2) {
         u.mask = 1 << q.next;
         u.col = (uint32_t)(q.next * ACC_COLS);
-        u.mat_stride = kBN;
+        u.mat_stride = TN;
+    } else if (!SPLIT) {
+        u.mask = 1;                              // one buffer, gate at 0 and up at TN
+        u.col = 0;
+        u.mat_stride = TN;
     } else if (n_mma > 64) {
         u.mask = 3;
         u.col = 0;
@@ -387,7 +398,7 @@ MOE_DEV AccUse acc_next(AccSeq& q, int n_mma) {
     u.par1 = q.uses1 & 1u;
     q.uses0 += (uint32_t)(u.mask & 1);
     q.uses1 += (uint32_t)(u.mask >> 1);
-    q.next = u.mask == 3 ? 0 : (q.next ^ 1);
+    q.next = (u.mask == 3 || (ACC_BUFS == 1 && !SPLIT)) ? 0 : (q.next ^ 1);
     return u;
 }
 
@@ -456,12 +467,13 @@ MOE_DEV void cache_groups(TileCache& tc, const GemmTile* tiles, const int2* grou
 template <int MODE>
 MOE_DEV GemmTile load_tile(const GemmArgs& a, int ti, const TileCache* tc = nullptr, int first = 0, int j = -1) {
     if constexpr (MODE == 2) {
+        constexpr int TN = 2 * kBN;              // the router launch's token tiles
         const int RB = (a.n_rows + kBlkN - 1) / kBlkN;
         GemmTile t;
         t.expert = -1;
         t.rb = ti % RB;
-        t.seg = (ti / RB) * kBN;
-        t.count = min(kBN, a.n_tok - t.seg);
+        t.seg = (ti / RB) * TN;
+        t.count = min(TN, a.n_tok - t.seg);
         return t;
     } else {
         if (tc && tc->grouped) return tc->t[j];
@@ -486,8 +498,8 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
     __shared__ uint64_t cfull[SC], cempty[SC], full[S], empty[S], acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
-    __shared__ float ep_scale[kBN];             // epilogue: per token column of the current tile
-    __shared__ int ep_row[kBN];
+    __shared__ float ep_scale[C::TN];           // epilogue: per token column of the current tile
+    __shared__ int ep_row[C::TN];
     __shared__ int ep_stop;
     __shared__ TileCache tcache;
 
@@ -595,7 +607,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 if (!warp_wait(&empty[s], (r & 1u) ^ 1u, &abort_flag, a.err, 1)) { ok = false; break; }
                 if (lane == 0) {
                     const int kb0 = ks * KSTEP;
-                    uint8_t* B = smem + C::B + s * KSTEP * kBTile;
+                    uint8_t* B = smem + C::B + s * KSTEP * C::B_TILE;
                     const uint32_t tb = (uint32_t)KSTEP * (uint32_t)n_mma * 128u;
                     if constexpr (MODE == 2) {
                         mbar_arrive_expect_tx(&full[s], tb + kATile);
@@ -613,7 +625,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                     // token rows t.seg .. t.seg + n_mma - 1 (rows past the
                     // end of the operand read as zero)
                     for (int j = 0; j < KSTEP; ++j)
-                        load_token_rows(B + j * kBTile, map_b, (kb0 + j) * kBlkK, t.seg, n_mma, &full[s]);
+                        load_token_rows(B + j * C::B_TILE, map_b, (kb0 + j) * kBlkK, t.seg, n_mma, &full[s]);
                 }
                 __syncwarp();
             }
@@ -631,7 +643,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
             // INT/FP8/FP6 routed tiles, gate/up and down: fp16 operands
             constexpr bool f16 = MODE != 2 && !SH && Q != Q_NVFP4;
             const uint32_t idesc = f16 ? idesc_f16_f32(128, n_mma) : idesc_bf16_f32(128, n_mma);
-            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
+            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS, C::TN, C::ACC_SPLIT>(aseq, n_mma);
             if ((au.mask & 1) && !warp_wait(&acc_empty[0], au.par0 ^ 1u, &abort_flag, a.err, 2)) break;
             if ((au.mask & 2) && !warp_wait(&acc_empty[1], au.par1 ^ 1u, &abort_flag, a.err, 2)) break;
             tc_fence_after();
@@ -645,7 +657,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 if (lane == 0) {
 #pragma unroll
                     for (int j = 0; j < KSTEP; ++j) {
-                        const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + (s * KSTEP + j) * kBTile));
+                        const uint64_t bdesc = desc_kmajor_sw128(smem_u32(smem + C::B + (s * KSTEP + j) * C::B_TILE));
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t acc = (ks | j | kk) != 0;
@@ -767,7 +779,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
         for (int jt = 0; jt < nseq; ++jt) {
             const GemmTile t = tile_at(jt);
             const int n_mma = (t.count + 15) & ~15;
-            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS>(aseq, n_mma);
+            const AccUse au = acc_next<C::ACC_BUFS, C::ACC_COLS, C::TN, C::ACC_SPLIT>(aseq, n_mma);
             const float gsc = (!SH && a.g_w) ? nx.gw * a.g_act : 1.0f;
             // down: the staging buffer of this tile was last read by the TMA
             // stores of the tile OUT_BUFS back
@@ -815,7 +827,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 uint32_t r[64];
                 const int nch = (cend - cbeg) >> 4;
                 tmem_ld_chunks(lane_base + cbeg, nch, r);
-                uint16_t* ob = out_s + (jt % C::OUT_BUFS) * (kOutTile / 2);
+                uint16_t* ob = out_s + (jt % C::OUT_BUFS) * (C::OUT_TILE / 2);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (q < nch) {
@@ -879,7 +891,7 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
                 // expert) are seg .. seg+count-1
                 if (ej == 0)
                     store_tile_rows(map_o, t.rb * kBlkN, t.seg, t.count,
-                                    reinterpret_cast<const uint8_t*>(out_s + (jt % C::OUT_BUFS) * (kOutTile / 2)));
+                                    reinterpret_cast<const uint8_t*>(out_s + (jt % C::OUT_BUFS) * (C::OUT_TILE / 2)));
             } else {
                 uint16_t* dst = reinterpret_cast<uint16_t*>(SH ? a.out_sh : a.out);
                 const int col0 = t.rb * kBlkN;
@@ -1690,7 +1702,8 @@ cudaError_t launch_router_tc(const void* x, const void* wr, int T, int H, int E,
     g.logits = logits;
     g.n_tok = T;
     g.n_rows = E;
-    g.n_tiles = ((E + kBlkN - 1) / kBlkN) * ((T + kBN - 1) / kBN);
+    constexpr int TN = Cfg<2, true>::TN;
+    g.n_tiles = ((E + kBlkN - 1) / kBlkN) * ((T + TN - 1) / TN);
     g.err = err;
     return launch_gemm<2, true>(m_x, g, st, &m_w, g.n_tiles < num_sms() ? g.n_tiles : num_sms());
 }
@@ -1817,6 +1830,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     tl.has_shared = ex.sh_gate != nullptr ? 1 : 0;
     tl.tok0 = native ? kFp4GuN : kBN;        // the block-scaled GEMMs take wider tiles
     tl.tok1 = native ? kFp4GuN : kBN;
+    tl.tok_sh = Cfg<0, true>::TN;            // the shared expert's launches
     tl.grid = num_sms();
     cudaError_t err = launch_permute(p.ids, T, k, E, p.counts, p.offsets, p.perm, p.inv, p.perm_scratch, st, &tl);
     if (err != cudaSuccess) return err;

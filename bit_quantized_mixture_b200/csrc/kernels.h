@@ -73,6 +73,7 @@ struct TileListArgs {
     size_t cap;
     int T, RB0, RB1, has_shared;
     int tok0, tok1;                // tokens per routed tile of each list
+    int tok_sh;                    // tokens per shared-expert tile
     int grid;                      // CTAs of the GEMM launches
 };
 // tl may be null (permutation only)

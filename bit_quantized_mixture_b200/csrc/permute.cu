@@ -92,7 +92,7 @@ k_perm_place(const int32_t* __restrict__ ids, int n, int E, int chunk, int chunk
         const long long first = (long long)c * kPlaceThreads + e, stride = (long long)gridDim.x * kPlaceThreads;
         for (int list = 0; list < 2; ++list)
             emit_tile_list(s_cnt, s_off, s_sc[list], s_sg[list], tl.T, list ? tl.RB1 : tl.RB0,
-                           list ? tl.tok1 : tl.tok0, tl.has_shared,
+                           list ? tl.tok1 : tl.tok0, tl.tok_sh, tl.has_shared,
                            tl.grid, first, stride, tl.tiles + (size_t)list * tl.cap,
                            tl.groups + (size_t)list * tl.cap, tl.num_tiles + 4 * list, c == 0);
     }

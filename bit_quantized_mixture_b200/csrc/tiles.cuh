@@ -6,7 +6,7 @@
 // for a GEMM whose MMA takes wider tiles); the list holds
 // every expert's tiles expert by expert, row block by row block, then (when
 // the layer has a shared expert) the shared-expert tiles (expert -1, token
-// rows instead of positions, kTileTokens per tile).  A group is up to kGroupTiles consecutive token
+// rows instead of positions, tok_sh per tile).  A group is up to kGroupTiles consecutive token
 // tiles of one (expert, row block), which read the same weight block.
 #pragma once
 
@@ -75,7 +75,7 @@ MOE_DEV int tile_owner(const int* pre, int i) {
 // routed groups, and 1 when every GEMM CTA's groups fit its shared-memory
 // tile list (group order), else 0.
 MOE_DEV void emit_tile_list(const int* s_cnt, const int* s_off, const int* sc, const int* sg, int T, int RB, int tok,
-                            int has_shared, int grid, long long first, long long stride, GemmTile* __restrict__ tiles,
+                            int tok_sh, int has_shared, int grid, long long first, long long stride, GemmTile* __restrict__ tiles,
                             int2* __restrict__ groups, int* __restrict__ num_tiles, bool write_counts) {
     const int total = sc[1023], ngroups = sg[1023];
     for (long long ii = first; ii < ngroups; ii += stride) {
@@ -101,15 +101,15 @@ MOE_DEV void emit_tile_list(const int* s_cnt, const int* s_off, const int* sc, c
         g.count = min(tok, c - tt * tok);
         tiles[i] = g;
     }
-    const int nts = has_shared ? (T + kTileTokens - 1) / kTileTokens : 0;
+    const int nts = has_shared ? (T + tok_sh - 1) / tok_sh : 0;
     for (long long ii = first; ii < (long long)nts * RB; ii += stride) {
         const int i = (int)ii;
         const int rb = i / nts, tt = i % nts;
         GemmTile g;
         g.expert = -1;
         g.rb = rb;
-        g.seg = tt * kTileTokens;
-        g.count = min(kTileTokens, T - tt * kTileTokens);
+        g.seg = tt * tok_sh;
+        g.count = min(tok_sh, T - tt * tok_sh);
         tiles[total + i] = g;
     }
     if (write_counts && threadIdx.x == 0) {
