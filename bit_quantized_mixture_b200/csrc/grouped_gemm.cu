@@ -918,6 +918,11 @@ k_grouped_gemm(const __grid_constant__ BMaps map_b, const __grid_constant__ CUte
 MOE_DEV float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 MOE_DEV float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
+// Slot rows per batch of loads: the top-10 workloads issue every slot row
+// and the shared row at once (one round trip per thread; 70.4 -> 67.3 us
+// against batches of 8 at T = 8192).
+constexpr int kCombineBatch = 12;
+template <int KB>
 __global__ void k_combine(const __half* __restrict__ O, const __half* __restrict__ S, const int32_t* __restrict__ inv,
                           int T, int H, int k, __nv_bfloat16* __restrict__ y) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one thread per 8 columns
@@ -925,31 +930,33 @@ __global__ void k_combine(const __half* __restrict__ O, const __half* __restrict
     if (i >= (long long)T * per_row) return;
     const int t = (int)(i / per_row), c = (int)(i % per_row) * 8;
     // the permuted position of each of the token's slots (-1: no expert
-    // output); eight 16-byte slot rows in flight per thread, summed in the
-    // fixed j order
+    // output); KB 16-byte slot rows and the shared row in flight per thread,
+    // summed in the fixed j order
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j0 = 0; j0 < k; j0 += 8) {
-        int pos[8];
+    for (int j0 = 0; j0 < k; j0 += KB) {
+        int pos[KB];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) pos[u] = j0 + u < k ? __ldg(inv + (size_t)t * k + j0 + u) : -1;
-        uint4 q[8];
+        for (int u = 0; u < KB; ++u) pos[u] = j0 + u < k ? __ldg(inv + (size_t)t * k + j0 + u) : -1;
+        uint4 q[KB];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < KB; ++u)
             q[u] = pos[u] >= 0 ? ldg_stream_v4(O + (size_t)pos[u] * H + c) : make_uint4(0, 0, 0, 0);
+        uint4 sq = make_uint4(0, 0, 0, 0);
+        const bool last = j0 + KB >= k;
+        if (S && last) sq = ldg_stream_v4(S + (size_t)t * H + c);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < KB; ++u) {
             if (pos[u] >= 0) {
                 const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
             }
         }
-    }
-    if (S) {
-        const uint4 q = ldg_stream_v4(S + (size_t)t * H + c);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        if (S && last) {
+            const uint32_t w[4] = {sq.x, sq.y, sq.z, sq.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
+            for (int p = 0; p < 4; ++p) { acc[2 * p] += h_lo(w[p]); acc[2 * p + 1] += h_hi(w[p]); }
+        }
     }
     uint4 out;
     out.x = pack_bf16x2(acc[0], acc[1]);
@@ -1804,7 +1811,7 @@ static cudaError_t launch_prefill_fp4(const PrefillArgs& p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     const long long threads = (long long)T * (H / 8);
-    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
+    k_combine<kCombineBatch><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
                                                                (__nv_bfloat16*)p.y);
     return cudaGetLastError();
 }
@@ -1920,7 +1927,7 @@ cudaError_t launch_prefill(const PrefillArgs& p, cudaStream_t st) {
     if (p.ev_dn1) cudaEventRecord(p.ev_dn1, st);
     // ---- combine
     const long long threads = (long long)T * (H / 8);
-    k_combine<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
+    k_combine<kCombineBatch><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p.o, has_sh ? p.o_sh : nullptr, p.inv, T, H, k,
                                                                (__nv_bfloat16*)p.y);
     return cudaGetLastError();
 }
