@@ -44,8 +44,6 @@ constexpr int kWarpProducer = 0, kWarpMma = 1;   // gate/up: warps 1 and 2 issue
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kATile = kBlkN * 128;          // 16 KB: 128 rows x 64 16-bit
-constexpr int kBTile = kBN * 128;            // 16 KB: 128 tokens x 64 16-bit
-constexpr int kOutTile = kBN * kBlkN * 2;    // 32 KB: epilogue staging, [token][128] 16-bit
 
 // MODE 0: gate + up (two matrices, SwiGLU epilogue); MODE 1: down; MODE 2:
 // the router logits x . Wr^T (fp32 out, A = Wr rows by TMA, no tile list).

@@ -79,14 +79,6 @@ MOE_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;"
 // all of the thread's bulk groups are complete (their global writes done)
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// TMA gather of four rows r0..r3 at inner coordinate c0 (box one row high)
-MOE_DEV void tma_gather4(void* dst, const CUtensorMap* map, int c0, int r0, int r1, int r2, int r3, uint64_t* bar) {
-    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-                 " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-                 ::"r"(smem_u32(dst)), "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-                   "r"(r3) : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 MOE_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
