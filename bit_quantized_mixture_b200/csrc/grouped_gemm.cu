@@ -1407,27 +1407,23 @@ k_fp4_gemm(const __grid_constant__ Fp4BMaps map_b, const __grid_constant__ OMaps
             // conversion runs.
             if constexpr (MODE == 1) {
                 static_assert(C::EPI_WARPS == 16 && kFp4GuN <= 192, "down: at most 48 columns per warp");
-                // (at most 32 registers per TMEM load: the third chunk separately)
-                uint32_t r0[32], r1[32];
-                if (nch >= 2) tmem_ld_x32c(lane_base + cbeg, r0);
-                else if (nch == 1) tmem_ld_x16c(lane_base + cbeg, r0);
-                if (nch == 3) tmem_ld_x16c(lane_base + cbeg + 32, r1);
+                // 16 columns at a time (the two accumulators alternate, so
+                // this one is released after the conversion)
+                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * C::OUT_TILE);
+#pragma unroll 1
+                for (int q = 0; q < nch; ++q) {
+                    uint32_t r[32];
+                    tmem_ld_x16c(lane_base + cbeg + 16 * q, r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = cbeg + 16 * q + i;
+                        const float sc = col < t.count ? ep_scale[col] : 0.0f;
+                        ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(r[i]) * sc));
+                    }
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                uint16_t* ob = reinterpret_cast<uint16_t*>(out_s + (local & 1) * C::OUT_TILE);
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    if (q < nch) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int col = cbeg + 16 * q + i;
-                            const float sc = col < t.count ? ep_scale[col] : 0.0f;
-                            const uint32_t v = q < 2 ? r0[16 * q + i] : r1[i];
-                            ob[col * kBlkN + row] = __half_as_ushort(f16_sat(__uint_as_float(v) * sc));
-                        }
-                    }
-                }
                 fence_proxy_async_smem();        // the TMA store reads what this thread wrote
             } else {
                 static_assert(C::EPI_WARPS == 16 && kFp4GuN <= 192, "gate/up: at most 48 columns per warp");
