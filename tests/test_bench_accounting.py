@@ -94,3 +94,25 @@ def test_default_line_is_the_largest_workload():
             "n_gpus": 1, "e2e": {}, "clocks": {}, "kernels_ms": {}, "layer": {}}
     e = bench.workload_entry(line)
     assert "metric" not in e and "n_gpus" not in e and e["roofline"] == {} and e["layer"] == {}
+
+
+def test_traffic_is_reported_only_for_the_source_it_was_measured_on(tmp_path, monkeypatch):
+    """The ncu DRAM bytes of a kernel key the sha256 of its source file: the
+    bench reports them while that file is unchanged and null after an edit."""
+    import hashlib
+    import json
+
+    src_dir = tmp_path / "bit_quantized_mixture_b200" / "csrc"
+    src_dir.mkdir(parents=True)
+    src = src_dir / "kernel.cu"
+    src.write_text("// one kernel\n")
+    (tmp_path / "profiles").mkdir()
+    table = {"work-a:k_one": {"source": "kernel.cu", "sha256": hashlib.sha256(src.read_bytes()).hexdigest(),
+                              "dram_bytes_per_launch": 123456, "from": "profiles/k_one.md"}}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_traffic("k_one", "work-a") == 123456
+    assert bench.load_traffic("k_one", "work-b") is None          # another workload
+    assert bench.load_traffic("k_two", "work-a") is None          # another kernel
+    src.write_text("// one kernel, edited\n")
+    assert bench.load_traffic("k_one", "work-a") is None
