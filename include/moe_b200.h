@@ -130,6 +130,10 @@ typedef struct {
 
 /* Validate cfg, allocate the weight arena and the workspace for max_tokens on
  * cfg->device.  On success *out owns all device memory until moe_destroy.
+ * NVFP4 layers whose hidden and inter sizes are multiples of 256 also keep,
+ * in the arena, the block-scaled prefill GEMM's weight images: a second copy
+ * of the routed experts' codes and scales (the same number of bytes), laid
+ * out per 128-row block and 256-value stage.
  * Errors: INVALID_ARG (bad cfg/null), UNSUPPORTED (shape), OOM, CUDA. */
 moe_status moe_create(const moe_config* cfg, moe_handle* out);
 
@@ -140,7 +144,8 @@ moe_status moe_destroy(moe_handle h);
 moe_status moe_load_router(moe_handle h, const void* w_router_any, moe_stream_t stream);
 
 /* Copy one expert's three matrices (host or device, interchange layout) into
- * the arena, re-laid for the kernels.  expert in [0, E) takes the routed
+ * the arena, re-laid for the kernels (NVFP4: and into the block-scaled weight
+ * images described at moe_create).  expert in [0, E) takes the routed
  * format of the handle; MOE_SHARED_EXPERT takes BF16 codes.  The caller may
  * free its arrays once the stream has passed this call.  Errors:
  * INVALID_ARG (index, null codes/scales/zeros for the format). */
